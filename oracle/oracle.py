@@ -1,0 +1,262 @@
+"""CPU oracle for the FP8 scaled-quantization path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  The product path (the CUDA library and
+its Python binding) never imports it and shares no code with it.
+
+This is a thin ctypes wrapper over ``fp8_oracle.c`` (plain C, fp64 sums,
+fp32 where the method fixes fp32).  Arrays are numpy: bf16 tensors are passed
+as their raw ``uint16`` bit patterns, FP8 tensors as ``uint8`` codes.
+Which page and section each function follows is stated in the C file.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp8_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+E4M3 = 0
+E5M2 = 1
+SCALE_TENSOR = 0
+SCALE_ROW = 1
+SCALE_BLOCK = 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (IEEE arithmetic: no fast-math, no FMA
+    contraction) into ``oracle/liboracle.so``."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+               "-fno-fast-math", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I = ctypes.c_int
+        F = ctypes.c_float
+        L.orc_decode.restype = ctypes.c_double
+        L.orc_decode.argtypes = [ctypes.c_uint8, I]
+        L.orc_encode.restype = ctypes.c_uint8
+        L.orc_encode.argtypes = [F, I]
+        L.orc_fmax.restype = ctypes.c_double
+        L.orc_fmax.argtypes = [I]
+        L.orc_f32_to_bf16.restype = ctypes.c_uint16
+        L.orc_f32_to_bf16.argtypes = [F]
+        L.orc_amax_bf16.restype = F
+        L.orc_amax_bf16.argtypes = [P, I64, P]
+        L.orc_scale_from_amax.restype = F
+        L.orc_scale_from_amax.argtypes = [F, I]
+        L.orc_scale_pow2_from_amax.restype = F
+        L.orc_scale_pow2_from_amax.argtypes = [F, I]
+        L.orc_inverse.restype = F
+        L.orc_inverse.argtypes = [F]
+        L.orc_quantize_tensorwise.restype = None
+        L.orc_quantize_tensorwise.argtypes = [P, I64, I64, I, P, I, P, P, P, P]
+        L.orc_quantize_rowwise.restype = None
+        L.orc_quantize_rowwise.argtypes = [P, I64, I64, I64, I, I, P, P]
+        L.orc_quantize_blockwise.restype = None
+        L.orc_quantize_blockwise.argtypes = [P, I64, I64, I64, I, I, I, P, P]
+        L.orc_gemm_scaled.restype = None
+        L.orc_gemm_scaled.argtypes = [P, I, P, I, I64, I64, I64, I, P, P, P, P]
+        L.orc_gemm_scaled_sampled.restype = None
+        L.orc_gemm_scaled_sampled.argtypes = [P, I, P, I, I64, I64, I64, I, P, P, P, P, I64, P, P]
+        L.orc_amax_history_update.restype = None
+        L.orc_amax_history_update.argtypes = [P, P, I, F, I, P, P, P]
+        L.orc_kv_quant.restype = None
+        L.orc_kv_quant.argtypes = [P, I64, I64, I, P, P]
+        L.orc_kv_dequant.restype = None
+        L.orc_kv_dequant.argtypes = [P, P, I64, I64, I, P]
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _u16(x) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    assert x.dtype == np.uint16, "bf16 inputs are passed as uint16 bit patterns"
+    return x
+
+
+# ------------------------------------------------------------------ formats --
+
+def decode(code: int, fmt: int) -> float:
+    return lib().orc_decode(code, fmt)
+
+
+def decode_table(fmt: int) -> np.ndarray:
+    """All 256 code values of a format (fp64), index == code."""
+    return np.array([decode(c, fmt) for c in range(256)], dtype=np.float64)
+
+
+def encode(y: float, fmt: int) -> int:
+    return int(lib().orc_encode(float(y), fmt))
+
+
+def encode_array(y: np.ndarray, fmt: int) -> np.ndarray:
+    y = np.asarray(y, dtype=np.float32).ravel()
+    return np.array([encode(v, fmt) for v in y], dtype=np.uint8)
+
+
+def fmax(fmt: int) -> float:
+    return lib().orc_fmax(fmt)
+
+
+def f32_to_bf16(f: float) -> int:
+    return int(lib().orc_f32_to_bf16(float(f)))
+
+
+# ------------------------------------------------------------ amax / scale --
+
+def amax(x_bits: np.ndarray) -> tuple[float, int]:
+    x = _u16(x_bits)
+    nf = ctypes.c_uint64(0)
+    a = lib().orc_amax_bf16(_p(x), x.size, ctypes.byref(nf))
+    return float(np.float32(a)), int(nf.value)
+
+
+def scale_from_amax(a: float, fmt: int) -> float:
+    return float(np.float32(lib().orc_scale_from_amax(a, fmt)))
+
+
+def scale_pow2_from_amax(a: float, fmt: int) -> float:
+    return float(np.float32(lib().orc_scale_pow2_from_amax(a, fmt)))
+
+
+def inverse(s: float) -> float:
+    return float(np.float32(lib().orc_inverse(s)))
+
+
+# ---------------------------------------------------------------- quantize --
+
+def quantize_tensorwise(x_bits: np.ndarray, fmt: int, scale_in: float | None = None,
+                        transpose_out: bool = False):
+    """Returns (q [rows, cols] or [cols, rows], scale_inv, amax, (nonfinite, saturated))."""
+    x = _u16(x_bits)
+    rows, cols = (1, x.size) if x.ndim == 1 else x.shape
+    q = np.empty((cols, rows) if transpose_out else (rows, cols), dtype=np.uint8)
+    sinv = np.zeros(1, np.float32)
+    am = np.zeros(1, np.float32)
+    counts = np.zeros(2, np.uint64)
+    s_in = None if scale_in is None else np.array([scale_in], np.float32)
+    lib().orc_quantize_tensorwise(_p(x), rows, cols, fmt, None if s_in is None else _p(s_in),
+                                  int(transpose_out), _p(q), _p(sinv), _p(am), _p(counts))
+    return q, float(sinv[0]), float(am[0]), (int(counts[0]), int(counts[1]))
+
+
+def quantize_rowwise(x_bits: np.ndarray, fmt: int, pow2: bool = True):
+    x = _u16(x_bits)
+    rows, cols = x.shape
+    q = np.empty((rows, cols), np.uint8)
+    sinv = np.empty(rows, np.float32)
+    lib().orc_quantize_rowwise(_p(x), rows, cols, cols, fmt, int(pow2), _p(q), _p(sinv))
+    return q, sinv
+
+
+def quantize_blockwise(x_bits: np.ndarray, fmt: int, block_rows: int, pow2: bool = False):
+    """block_rows 1: scales [ceil(cols/128), rows]; block_rows 128: scales
+    [ceil(rows/128), ceil(cols/128)]."""
+    x = _u16(x_bits)
+    rows, cols = x.shape
+    nkb = (cols + 127) // 128
+    q = np.empty((rows, cols), np.uint8)
+    if block_rows == 1:
+        sinv = np.empty((nkb, rows), np.float32)
+    else:
+        sinv = np.empty(((rows + block_rows - 1) // block_rows, nkb), np.float32)
+    lib().orc_quantize_blockwise(_p(x), rows, cols, cols, fmt, block_rows, int(pow2), _p(q), _p(sinv))
+    return q, sinv
+
+
+# -------------------------------------------------------------------- GEMM --
+
+def gemm_scaled(A: np.ndarray, fa: int, B: np.ndarray, fb: int, mode: int,
+                da: np.ndarray, db: np.ndarray):
+    """Full reference D (fp64 [M, N]) and magnitude mag (fp64 [M, N])."""
+    A = np.ascontiguousarray(A, np.uint8)
+    B = np.ascontiguousarray(B, np.uint8)
+    M, K = A.shape
+    N, K2 = B.shape
+    assert K == K2
+    da = np.ascontiguousarray(da, np.float32)
+    db = np.ascontiguousarray(db, np.float32)
+    D = np.empty((M, N), np.float64)
+    mag = np.empty((M, N), np.float64)
+    lib().orc_gemm_scaled(_p(A), fa, _p(B), fb, M, N, K, mode, _p(da), _p(db), _p(D), _p(mag))
+    return D, mag
+
+
+def gemm_scaled_sampled(A: np.ndarray, fa: int, B: np.ndarray, fb: int, mode: int,
+                        da: np.ndarray, db: np.ndarray, idx_m: np.ndarray, idx_n: np.ndarray):
+    A = np.ascontiguousarray(A, np.uint8)
+    B = np.ascontiguousarray(B, np.uint8)
+    M, K = A.shape
+    N, _ = B.shape
+    da = np.ascontiguousarray(da, np.float32)
+    db = np.ascontiguousarray(db, np.float32)
+    im = np.ascontiguousarray(idx_m, np.int64)
+    inn = np.ascontiguousarray(idx_n, np.int64)
+    val = np.empty(im.size, np.float64)
+    mag = np.empty(im.size, np.float64)
+    lib().orc_gemm_scaled_sampled(_p(A), fa, _p(B), fb, M, N, K, mode, _p(da), _p(db),
+                                  _p(im), _p(inn), im.size, _p(val), _p(mag))
+    return val, mag
+
+
+# --------------------------------------------------------- delayed scaling --
+
+class AmaxHistory:
+    """Host-side delayed-scaling state: history ring, position, scale."""
+
+    def __init__(self, length: int, fmt: int):
+        self.history = np.zeros(length, np.float32)
+        self.pos = np.zeros(1, np.int32)
+        self.scale = np.ones(1, np.float32)
+        self.scale_inv = np.ones(1, np.float32)
+        self.fmt = fmt
+
+    def update(self, amax_cur: float) -> int:
+        sat = np.zeros(1, np.uint32)
+        lib().orc_amax_history_update(_p(self.history), _p(self.pos), self.history.size,
+                                      float(amax_cur), self.fmt, _p(self.scale),
+                                      _p(self.scale_inv), _p(sat))
+        return int(sat[0])
+
+
+# ---------------------------------------------------------------- KV cache --
+
+def kv_quant(x_bits: np.ndarray, fmt: int = E4M3):
+    """x [B, H, S, Dh] bf16 bits -> (q same shape, scale_inv [B*H])."""
+    x = _u16(x_bits)
+    B, H, S, Dh = x.shape
+    q = np.empty(x.shape, np.uint8)
+    sinv = np.empty(B * H, np.float32)
+    lib().orc_kv_quant(_p(x), B * H, S * Dh, fmt, _p(q), _p(sinv))
+    return q, sinv
+
+
+def kv_dequant(q: np.ndarray, scale_inv: np.ndarray, fmt: int = E4M3) -> np.ndarray:
+    q = np.ascontiguousarray(q, np.uint8)
+    B, H, S, Dh = q.shape
+    sinv = np.ascontiguousarray(scale_inv, np.float32)
+    out = np.empty(q.shape, np.uint16)
+    lib().orc_kv_dequant(_p(q), _p(sinv), B * H, S * Dh, fmt, _p(out))
+    return out

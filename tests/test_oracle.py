@@ -1,0 +1,443 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- values the pages print, the format definition's fixed points,
+library routines that compute a special case (torch's CPU float8 / bf16
+casts, numpy / integer matmul), closed forms, invariants and brute force.
+
+Pages cited:
+  "DeepL押注FP8：大模型训练与推理统一精度实战解析" (§2.1 formats, §2.3 scaling
+  granularity and delayed scaling, §3.1 FP8 KV cache, §4.2 amax statistics);
+  "H100 FP8加速实测：新一代计算架构的飞跃" (E5M2 range +-57344);
+  "FP8训练与QAT量化感知训练：…用Soup把大模型微调提速2倍", section
+  "FP8 三种缩放配方怎么选" (rowwise power-of-two scales).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_scaled_quantization_amax_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+FMTS = {"e4m3": 0, "e5m2": 1}
+TORCH_FP8 = {0: torch.float8_e4m3fn, 1: torch.float8_e5m2}
+
+
+def _golden(name):
+    rows = []
+    for line in open(os.path.join(GOLDEN, name)):
+        if line.startswith("#") or not line.strip():
+            continue
+        rows.append(line.split())
+    return rows
+
+
+def _bits(x: torch.Tensor) -> np.ndarray:
+    return inputs.bf16_bits(x)
+
+
+# ----------------------------------------------------------------- decode --
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_decode_matches_torch_float8_views(orc, fmt):
+    """All 256 codes against torch's own float8 dtypes (a library decode)."""
+    ours = orc.decode_table(fmt)
+    lib = torch.arange(256, dtype=torch.uint8).view(TORCH_FP8[fmt]).to(torch.float64).numpy()
+    nan = np.isnan(lib)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], lib[~nan])
+    # signed zero survives
+    assert math.copysign(1.0, ours[0x80]) == -1.0
+
+
+def test_decode_code_counts(orc):
+    """E4M3: 254 finite (with +-0) + 2 NaN, no Inf.  E5M2: 248 finite + 2 Inf + 6 NaN."""
+    e4 = orc.decode_table(0)
+    e5 = orc.decode_table(1)
+    assert np.isfinite(e4).sum() == 254 and np.isnan(e4).sum() == 2 and np.isinf(e4).sum() == 0
+    assert np.isfinite(e5).sum() == 248 and np.isnan(e5).sum() == 6 and np.isinf(e5).sum() == 2
+
+
+def test_decode_golden_points(orc):
+    """Fixed points of the formats, incl. the E5M2 range the H100 page prints."""
+    for fmt_s, code, val, *_ in _golden("fp8_format_points.txt"):
+        got = orc.decode(int(code, 16), FMTS[fmt_s])
+        exp = float(val)
+        if math.isnan(exp):
+            assert math.isnan(got), (fmt_s, code)
+        else:
+            assert got == exp and math.copysign(1, got) == math.copysign(1, exp), (fmt_s, code, got)
+    assert orc.fmax(1) == 57344.0 and orc.fmax(0) == 448.0
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_decode_monotone_positive_codes(orc, fmt):
+    t = orc.decode_table(fmt)
+    top = 0x7E if fmt == 0 else 0x7B
+    pos = t[: top + 1]
+    assert np.all(np.diff(pos) > 0)
+    assert np.array_equal(t[0x80: 0x80 + top + 1], -pos)
+
+
+# ----------------------------------------------------------------- encode --
+
+def test_encode_golden_cases(orc):
+    for fmt_s, x, code, *_ in _golden("fp8_encode_cases.txt"):
+        assert orc.encode(float(x), FMTS[fmt_s]) == int(code, 16), (fmt_s, x)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_encode_roundtrip_all_finite_codes(orc, fmt):
+    t = orc.decode_table(fmt)
+    for c in range(256):
+        if np.isfinite(t[c]):
+            assert orc.encode(t[c], fmt) == c, hex(c)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_encode_matches_torch_in_range(orc, fmt):
+    """In range, torch's CPU fp32 -> float8 conversion is RNE; it only differs
+    from the saturating cast above fmax (it overflows to NaN / Inf there)."""
+    rng = np.random.default_rng(11 + fmt)
+    fm = orc.fmax(fmt)
+    # log-uniform magnitudes across the whole range incl. subnormals, both signs
+    e = rng.uniform(-20 if fmt == 0 else -19, math.log2(fm), 20000)
+    y = (np.exp2(e) * rng.choice([-1.0, 1.0], e.size)).astype(np.float32)
+    # plus exact midpoints between neighbouring codes (ties)
+    t = orc.decode_table(fmt)
+    top = 0x7E if fmt == 0 else 0x7B
+    mids = ((t[: top] + t[1: top + 1]) / 2).astype(np.float32)
+    y = np.concatenate([y, mids, -mids])
+    y = y[np.abs(y) <= fm]
+    ours = orc.encode_array(y, fmt)
+    lib = torch.from_numpy(y).to(TORCH_FP8[fmt]).view(torch.uint8).numpy()
+    assert np.array_equal(ours, lib)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_encode_is_nearest_by_brute_force(orc, fmt):
+    """Brute force over all finite codes: the chosen code is a nearest one."""
+    rng = np.random.default_rng(5)
+    t = orc.decode_table(fmt)
+    fin = np.isfinite(t)
+    fm = orc.fmax(fmt)
+    y = (rng.standard_normal(3000) * rng.choice([1e-4, 1e-2, 1.0, 100.0], 3000)).astype(np.float32)
+    for v in y:
+        c = orc.encode(v, fmt)
+        if abs(v) >= fm:
+            assert abs(t[c]) == fm
+            continue
+        best = np.min(np.abs(t[fin] - np.float64(v)))
+        assert abs(t[c] - np.float64(v)) == best
+
+
+def test_bf16_rounding_matches_torch(orc):
+    rng = np.random.default_rng(3)
+    f = (rng.standard_normal(20000) * 10.0 ** rng.uniform(-30, 30, 20000)).astype(np.float32)
+    # exact ties: bf16 values plus half an ulp
+    base = torch.from_numpy(rng.standard_normal(2000).astype(np.float32)).to(torch.bfloat16)
+    bb = base.float().numpy().view(np.uint32)
+    ties = (bb | np.uint32(0x8000)).view(np.float32)
+    f = np.concatenate([f, ties, np.array([3.3895e38, 3.4e38], np.float32)])
+    ours = np.array([orc.f32_to_bf16(v) for v in f], np.uint16)
+    lib = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, lib)
+
+
+# ------------------------------------------------------------ amax, scale --
+
+def test_amax_against_numpy_and_nonfinite(orc):
+    x = inputs.normal_bf16((1000,), 3.0, seed=1)
+    bits = _bits(x).copy()
+    assert orc.amax(bits)[0] == np.abs(x.float().numpy()).max()
+    bits[[3, 50, 700]] = [0x7FC0, 0x7F80, 0xFF80]   # NaN, +Inf, -Inf
+    ref = np.abs(x.float().numpy())
+    ref[[3, 50, 700]] = 0
+    a, nf = orc.amax(bits)
+    assert a == ref.max() and nf == 3
+    assert orc.amax(np.zeros(17, np.uint16))[0] == 0.0
+    assert orc.amax(np.array([0x8000, 0x0000], np.uint16))[0] == 0.0
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_scale_closed_forms(orc, fmt):
+    fm = orc.fmax(fmt)
+    assert orc.scale_from_amax(0.0, fmt) == 1.0
+    assert orc.scale_from_amax(1.0, fmt) == fm
+    assert orc.scale_from_amax(fm, fmt) == 1.0
+    assert orc.scale_from_amax(1e-38, fmt) == np.finfo(np.float32).max   # overflow clamps
+    assert orc.scale_pow2_from_amax(1.0, fmt) == (256.0 if fmt == 0 else 32768.0)
+    assert orc.scale_pow2_from_amax(fm, fmt) == 1.0
+    assert orc.scale_pow2_from_amax(0.0, fmt) == 1.0
+    assert orc.scale_pow2_from_amax(float(np.nextafter(np.float32(fm), np.float32(1e9))), fmt) == 0.5
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_pow2_scale_property_on_bf16_amax(orc, fmt):
+    """s is a power of two with amax*s <= fmax < amax*2s (the largest such)."""
+    fm = orc.fmax(fmt)
+    x = inputs.normal_bf16((4000,), 1.0, seed=2)
+    vals = np.abs(x.float().numpy()) * 10.0 ** np.random.default_rng(0).uniform(-30, 30, 4000)
+    vals = torch.from_numpy(vals.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    for a in vals[vals > 0]:
+        s = orc.scale_pow2_from_amax(float(a), fmt)
+        m, e = math.frexp(s)
+        assert m == 0.5
+        if s < 2.0 ** 127:
+            assert np.float64(a) * s <= fm < np.float64(a) * 2 * s
+
+
+# --------------------------------------------------------------- quantize --
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_tensorwise_invariants(orc, fmt):
+    """The amax element maps to +-fmax; every element is the cast of x*s, and
+    the dequantized value is within half a code step of x."""
+    x = inputs.normal_bf16((96, 80), 2.0, seed=3)
+    bits = _bits(x)
+    q, sinv, amax, (nf, sat) = orc.quantize_tensorwise(bits, fmt)
+    xf = x.float().numpy()
+    assert amax == np.abs(xf).max() and nf == 0 and sat == 0
+    s = np.float32(orc.fmax(fmt)) / np.float32(amax)
+    assert sinv == np.float32(1.0) / s
+    t = orc.decode_table(fmt)
+    i = np.unravel_index(np.argmax(np.abs(xf)), xf.shape)
+    assert abs(t[q[i]]) == orc.fmax(fmt)
+    # relative error of the dequantized tensor: at most half a mantissa step
+    deq = t[q].astype(np.float64) * sinv
+    rel = 2.0 ** -(4 if fmt == 0 else 3)
+    tiny = orc.decode(1, fmt) * sinv
+    assert np.all(np.abs(deq - xf) <= rel * np.abs(xf) + tiny)
+    # transposed output is the transpose
+    qt, *_ = orc.quantize_tensorwise(bits, fmt, transpose_out=True)
+    assert np.array_equal(qt, q.T)
+    # lib cross-check of the whole cast (values in range, no saturation)
+    y = (xf * s).astype(np.float32)
+    lib = torch.from_numpy(y).to(TORCH_FP8[fmt]).view(torch.uint8).numpy()
+    assert np.array_equal(q, lib)
+
+
+def test_tensorwise_delayed_scale_saturation(orc):
+    x = inputs.normal_bf16((64, 64), 1.0, seed=4)
+    bits = _bits(x)
+    q, sinv, amax, (nf, sat) = orc.quantize_tensorwise(bits, 0, scale_in=1000.0)
+    xf = x.float().numpy()
+    assert sat == int((np.abs(xf.astype(np.float32) * np.float32(1000.0)) > 448).sum()) > 0
+    assert sinv == np.float32(1.0) / np.float32(1000.0)
+    assert amax == np.abs(xf).max()
+    t = orc.decode_table(0)
+    assert np.all(np.abs(t[q]) <= 448)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_rowwise_pow2_per_row(orc, fmt):
+    """Per-row pow2 scales; with outlier rows the per-row scale keeps the
+    ordinary rows precise where a per-tensor scale would not (the outlier
+    claim of the DeepL page §2.3)."""
+    x = inputs.outlier_activations_bf16((64, 256), seed=5, frac=2e-3)
+    bits = _bits(x)
+    q, sinv = orc.quantize_rowwise(bits, fmt, pow2=True)
+    xf = x.float().numpy()
+    t = orc.decode_table(fmt)
+    fm = orc.fmax(fmt)
+    for r in range(64):
+        a = np.abs(xf[r]).max()
+        s = 1.0 / sinv[r]
+        assert math.frexp(s)[0] == 0.5 and a * s <= fm < a * 2 * s
+        row = torch.from_numpy((xf[r] * np.float32(s)).astype(np.float32))
+        assert np.array_equal(q[r], row.to(TORCH_FP8[fmt]).view(torch.uint8).numpy())
+    # one extreme outlier row: under one tensor scale the ordinary rows fall
+    # into the subnormal range and lose precision; per-row scales keep them
+    xo = inputs.normal_bf16((64, 256), 1.0, seed=15).float()
+    xo[0, 7] = 1.0e5 if fmt == 0 else 1.0e11   # pushes ordinary values to subnormals
+    ob = _bits(xo.to(torch.bfloat16))
+    xof = xo.to(torch.bfloat16).float().numpy()
+    qr, sr = orc.quantize_rowwise(ob, fmt, pow2=True)
+    qt, st, *_ = orc.quantize_tensorwise(ob, fmt)
+    err_row = np.abs(t[qr[1:]] * sr[1:, None] - xof[1:]).sum()
+    err_ten = np.abs(t[qt[1:]] * st - xof[1:]).sum()
+    assert err_row < 0.5 * err_ten
+
+
+@pytest.mark.parametrize("block_rows", [1, 128])
+def test_blockwise_layout_and_invariants(orc, block_rows):
+    """Blocks with very different magnitudes: each block's scale follows its
+    own amax (checked against a numpy reshape-max), the block's amax element
+    maps to fmax, and the scale layout is the documented one."""
+    rows, cols = (200, 300) if block_rows == 128 else (7, 400)
+    rng = np.random.default_rng(6)
+    xf = rng.standard_normal((rows, cols)).astype(np.float32)
+    nrb, nkb = -(-rows // block_rows), -(-cols // 128)
+    mult = 10.0 ** rng.integers(-3, 4, (nrb, nkb))
+    xf *= np.kron(mult, np.ones((block_rows, 128)))[:rows, :cols]
+    x = torch.from_numpy(xf).to(torch.bfloat16)
+    bits = _bits(x)
+    q, sinv = orc.quantize_blockwise(bits, 0, block_rows)
+    xb = x.float().numpy()
+    pad = np.zeros((nrb * block_rows, nkb * 128), np.float32)
+    pad[:rows, :cols] = np.abs(xb)
+    bam = pad.reshape(nrb, block_rows, nkb, 128).max(axis=(1, 3))
+    exp_s = np.float32(448.0) / bam.astype(np.float32)
+    exp_inv = (np.float32(1.0) / exp_s).astype(np.float32)
+    if block_rows == 1:
+        assert sinv.shape == (nkb, rows)
+        assert np.array_equal(sinv, exp_inv.T)
+    else:
+        assert sinv.shape == (nrb, nkb)
+        assert np.array_equal(sinv, exp_inv)
+    t = orc.decode_table(0)
+    deq = np.abs(t[q])
+    dpad = np.zeros_like(pad)
+    dpad[:rows, :cols] = deq
+    assert np.all(dpad.reshape(nrb, block_rows, nkb, 128).max(axis=(1, 3)) == 448.0)
+
+
+# -------------------------------------------------------------------- GEMM --
+
+def _int_codes(rng, shape, fmt):
+    """Codes of small integers (exactly representable): |v| <= 16 (E4M3), <= 8 (E5M2)."""
+    top = 16 if fmt == 0 else 8
+    vals = rng.integers(-top, top + 1, shape)
+    enc = np.vectorize(lambda v: _enc_cache(fmt, int(v)))
+    return vals, enc(vals).astype(np.uint8)
+
+
+_CACHE = {}
+
+
+def _enc_cache(fmt, v):
+    from oracle import oracle
+    k = (fmt, v)
+    if k not in _CACHE:
+        _CACHE[k] = oracle.encode(float(v), fmt)
+    return _CACHE[k]
+
+
+@pytest.mark.parametrize("fa,fb", [(0, 0), (1, 0)])
+def test_gemm_integer_special_case(orc, fa, fb):
+    """Codes of small integers with unit scales give an exact integer GEMM."""
+    rng = np.random.default_rng(7)
+    M, N, K = 24, 40, 72
+    va, A = _int_codes(rng, (M, K), fa)
+    vb, B = _int_codes(rng, (N, K), fb)
+    one = np.ones(1, np.float32)
+    D, mag = orc.gemm_scaled(A, fa, B, fb, orc.SCALE_TENSOR, one, one)
+    exact = va.astype(np.int64) @ vb.astype(np.int64).T
+    assert np.array_equal(D, exact.astype(np.float64))
+    assert np.array_equal(mag, (np.abs(va) @ np.abs(vb).T).astype(np.float64))
+
+
+def test_gemm_random_codes_against_numpy(orc):
+    """Non-square shapes so a transposed operand fails; rowwise scales."""
+    rng = np.random.default_rng(8)
+    M, N, K = 19, 33, 100
+    t = orc.decode_table(0)
+    fin = np.where(np.isfinite(t))[0]
+    A = rng.choice(fin, (M, K)).astype(np.uint8)
+    B = rng.choice(fin, (N, K)).astype(np.uint8)
+    da = rng.uniform(0.5, 2, M).astype(np.float32)
+    db = rng.uniform(0.5, 2, N).astype(np.float32)
+    D, mag = orc.gemm_scaled(A, 0, B, 0, orc.SCALE_ROW, da, db)
+    ref = (t[A] @ t[B].T) * da[:, None].astype(np.float64) * db[None, :].astype(np.float64)
+    assert np.allclose(D, ref, rtol=1e-12, atol=1e-9)
+    ref_mag = (np.abs(t[A]) @ np.abs(t[B]).T) * da[:, None] * db[None, :]
+    assert np.allclose(mag, ref_mag, rtol=1e-12)
+    # identity B: D = A's values times the scales
+    Bi = np.zeros((K, K), np.uint8)
+    Bi[np.arange(K), np.arange(K)] = 0x38
+    Di, _ = orc.gemm_scaled(A, 0, Bi, 0, orc.SCALE_TENSOR, np.float32([0.5]), np.float32([1.0]))
+    assert np.array_equal(Di, t[A] * 0.5)
+    # sampled entries equal the full product
+    im = rng.integers(0, M, 50)
+    inn = rng.integers(0, N, 50)
+    v, mg = orc.gemm_scaled_sampled(A, 0, B, 0, orc.SCALE_ROW, da, db, im, inn)
+    assert np.array_equal(v, D[im, inn]) and np.array_equal(mg, mag[im, inn])
+
+
+def test_gemm_blockwise_against_numpy(orc):
+    """Per-(row, 128-K block) A scales and per-(128x128) B scales, ragged K."""
+    rng = np.random.default_rng(9)
+    M, N, K = 9, 260, 300
+    nkb = -(-K // 128)
+    t = orc.decode_table(0)
+    fin = np.where(np.isfinite(t))[0]
+    A = rng.choice(fin, (M, K)).astype(np.uint8)
+    B = rng.choice(fin, (N, K)).astype(np.uint8)
+    da = rng.uniform(0.1, 3, (nkb, M)).astype(np.float32)
+    db = rng.uniform(0.1, 3, (-(-N // 128), nkb)).astype(np.float32)
+    D, _ = orc.gemm_scaled(A, 0, B, 0, orc.SCALE_BLOCK, da, db)
+    sa = np.repeat(da.T.astype(np.float64), 128, axis=1)[:, :K]          # [M, K]
+    sb = np.repeat(np.repeat(db.astype(np.float64), 128, axis=0)[:N], 128, axis=1)[:, :K]  # [N, K]
+    ref = np.einsum("mk,nk->mn", t[A] * sa, t[B] * sb)
+    assert np.allclose(D, ref, rtol=1e-12, atol=1e-9)
+    # with all scales equal it is the tensorwise GEMM
+    D1, _ = orc.gemm_scaled(A, 0, B, 0, orc.SCALE_BLOCK, np.ones_like(da), np.ones_like(db))
+    D2, _ = orc.gemm_scaled(A, 0, B, 0, orc.SCALE_TENSOR, np.ones(1, np.float32), np.ones(1, np.float32))
+    assert np.allclose(D1, D2, rtol=1e-13)
+
+
+# --------------------------------------------------------- delayed scaling --
+
+def test_history_constant_amax_and_spike_window(orc):
+    """Constant amax: step 0 uses s = 1 (empty history), then s = fmax/amax.
+    A spike stays in the window for exactly `len` steps."""
+    h = orc.AmaxHistory(16, 0)
+    assert h.update(2.0) == 0            # s_0 = 1: 2 * 1 <= 448
+    assert h.scale[0] == np.float32(224.0)
+    for _ in range(5):
+        assert h.update(2.0) == 0
+        assert h.scale[0] == np.float32(224.0)
+    assert h.update(16.0) == 1           # spike: 16 * 224 > 448 -> saturation flag
+    assert h.scale[0] == np.float32(28.0)
+    for i in range(15):
+        h.update(2.0)
+        assert h.scale[0] == np.float32(28.0), i      # spike still in the window
+    h.update(2.0)
+    assert h.scale[0] == np.float32(224.0)            # 16 steps later it has left
+    assert h.scale_inv[0] == np.float32(1.0) / np.float32(224.0)
+    assert h.pos[0] == (6 + 1 + 16) % 16
+
+
+def test_history_checkpoint_resume(orc):
+    """The state is (history, pos, scale): save at step 8 and resume."""
+    amaxes = np.random.default_rng(1).uniform(0.1, 5, 24).astype(np.float32)
+    a = orc.AmaxHistory(16, 1)
+    for v in amaxes:
+        a.update(v)
+    b = orc.AmaxHistory(16, 1)
+    for v in amaxes[:8]:
+        b.update(v)
+    saved = (b.history.copy(), b.pos.copy(), b.scale.copy(), b.scale_inv.copy())
+    c = orc.AmaxHistory(16, 1)
+    c.history[:], c.pos[:], c.scale[:], c.scale_inv[:] = saved
+    for v in amaxes[8:]:
+        c.update(v)
+    assert np.array_equal(a.history, c.history) and a.pos[0] == c.pos[0]
+    assert a.scale[0] == c.scale[0] and a.scale_inv[0] == c.scale_inv[0]
+    assert a.scale[0] == np.float32(57344.0) / np.float32(amaxes[-16:].max())
+
+
+# ---------------------------------------------------------------- KV cache --
+
+def test_kv_round_trip(orc):
+    """Per-(b, h) scales; the round trip stays within half an E4M3 step plus
+    the bf16 rounding; K8 memory halves (1 byte per element)."""
+    x = inputs.normal_bf16((2, 3, 64, 128), 1.0, seed=10)
+    bits = _bits(x)
+    q, sinv = orc.kv_quant(bits)
+    assert q.dtype == np.uint8 and q.nbytes * 2 == bits.nbytes
+    xf = x.float().numpy().reshape(6, -1)
+    for i in range(6):
+        assert sinv[i] == np.float32(1.0) / (np.float32(448.0) / np.float32(np.abs(xf[i]).max()))
+        qi, si, *_ = orc.quantize_tensorwise(bits.reshape(6, -1)[i], 0)
+        assert np.array_equal(q.reshape(6, -1)[i], qi.ravel()) and si == sinv[i]
+    back = orc.kv_dequant(q, sinv)
+    bf = torch.from_numpy(back.view(np.int16)).view(torch.bfloat16).float().numpy().reshape(6, -1)
+    tiny = 2.0 ** -9 * sinv[:, None]
+    assert np.all(np.abs(bf - xf) <= (2.0 ** -4 + 2.0 ** -8) * np.abs(xf) + tiny)
+    # dequant equals bf16(decoded * d) computed by torch's own bf16 cast
+    t = orc.decode_table(0).astype(np.float32)
+    y = (t[q.reshape(6, -1)] * sinv[:, None]).astype(np.float32)
+    lib = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(back.reshape(6, -1), lib)
