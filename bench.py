@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 scaled-quantization hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One "step" is one pass of the whole hot path over one batch of synthetic
+input already resident in HBM.  Default workload ``rowwise``: per-row
+power-of-two E4M3 quantization of activations A [4096, 4096] (N(0,1) with 0.1 %
+x100 outliers) and weights B [4096, 4096] (N(0, 0.02)), then the rowwise-scaled
+FP8 GEMM D = A8 x B8^T (fp32 accumulate, bf16 out).  Other workloads:
+``tensor`` (per-tensor E4M3, 256^3), ``blockmlp`` (1x128 / 128x128 block
+scales, X[8192, 4096] -> W_up[11008, 4096] -> W_down[4096, 11008]),
+``dgrad`` (E5M2 gradients [8192, 4096] x E4M3 W^T [4096, 4096] with delayed
+scaling over a 16-step history) and ``kv`` (FP8 KV cache K, V [32, 32, 8192,
+128] quantize + dequantize, GB/s).
+
+Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then K steps
+bracketed by a barrier and a device synchronize; each step's kernels are
+timed with CUDA events on the launching stream, L2 is flushed (a 256 MiB write)
+before every step outside the events; multi-GPU takes the max over ranks.
+``--impl reference`` times the CPU oracle (the only reference this project
+has) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FP8 scaled GEMM TFLOP/s (% dense FP8 peak); quantize/KV GB/s (% HBM)"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0     # nominal dense ratio: 4.5 PFLOP/s fp8 / 2.25 PFLOP/s bf16
+DEFAULT_STEPS = {"rowwise": 2000, "tensor": 2000, "blockmlp": 100, "dgrad": 400, "kv": 40}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------- workloads --
+
+class Workload:
+    """Inputs resident on the device and the step as a list of library calls."""
+
+    def __init__(self, name: str, device, seed: int):
+        from fp8_scaled_quantization_amax_b200 import fp8q, inputs
+        self.f, self.inp = fp8q, inputs
+        self.name = name
+        self.dev = device
+        self.seed = seed
+        getattr(self, "_setup_" + name)()
+
+    # per-row pow2 E4M3, M = N = K = 4096
+    def _setup_rowwise(self):
+        f, inp, d, s = self.f, self.inp, self.dev, self.seed
+        M = N = K = 4096
+        self.A = inp.outlier_activations_bf16((M, K), seed=s, device=d)
+        self.B = inp.normal_bf16((N, K), 0.02, seed=s + 1, device=d)
+        self.qa = torch.empty((M, K), dtype=torch.uint8, device=d)
+        self.qb = torch.empty((N, K), dtype=torch.uint8, device=d)
+        self.sa = torch.empty(M, dtype=torch.float32, device=d)
+        self.sb = torch.empty(N, dtype=torch.float32, device=d)
+        self.D = torch.empty((M, N), dtype=torch.bfloat16, device=d)
+        self.flops = 2.0 * M * N * K
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.launches = 3
+        self.config = {"workload": "rowwise pow2 E4M3 GEMM", "M": M, "N": N, "K": K,
+                       "A": "N(0,1) bf16, 0.1% entries x100", "B": "N(0,0.02) bf16",
+                       "scales": "per-row A, per-row B (= per output column), powers of two"}
+        self.host_inputs = [("A", self.A), ("B", self.B)]
+        self.host_output = self.D
+
+    def _step_rowwise(self, ev=None):
+        f = self.f
+        M, K = self.A.shape
+        N = self.B.shape[0]
+        f.fp8_quantize_rowwise(self.A, M, K, K, f.E4M3, True, self.qa, self.sa)
+        f.fp8_quantize_rowwise(self.B, N, K, K, f.E4M3, True, self.qb, self.sb)
+        if ev:
+            ev[0].record()
+        f.fp8_gemm_scaled(self.qa, f.E4M3, self.qb, f.E4M3, M, N, K, f.SCALE_ROW, self.sa, self.sb, self.D, N)
+        if ev:
+            ev[1].record()
+
+    # per-tensor E4M3, 256^3
+    def _setup_tensor(self):
+        f, inp, d, s = self.f, self.inp, self.dev, self.seed
+        M = N = K = 256
+        self.A = inp.normal_bf16((M, K), 1.0, seed=s, device=d)
+        self.B = inp.normal_bf16((N, K), 1.0, seed=s + 1, device=d)
+        self.qa = torch.empty((M, K), dtype=torch.uint8, device=d)
+        self.qb = torch.empty((N, K), dtype=torch.uint8, device=d)
+        self.sa, self.sb = (torch.empty(1, dtype=torch.float32, device=d) for _ in range(2))
+        self.ama, self.amb = (torch.empty(1, dtype=torch.float32, device=d) for _ in range(2))
+        self.D = torch.empty((M, N), dtype=torch.bfloat16, device=d)
+        self.flops = 2.0 * M * N * K
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.launches = 5
+        self.config = {"workload": "per-tensor E4M3 GEMM", "M": M, "N": N, "K": K,
+                       "A": "N(0,1) bf16", "B": "N(0,1) bf16", "scales": "s = 448/amax per tensor"}
+        self.host_inputs = [("A", self.A), ("B", self.B)]
+        self.host_output = self.D
+
+    def _step_tensor(self, ev=None):
+        f = self.f
+        M, K = self.A.shape
+        N = self.B.shape[0]
+        f.fp8_quantize_tensorwise(self.A, M, K, f.E4M3, None, self.qa, 0, self.sa, self.ama)
+        f.fp8_quantize_tensorwise(self.B, N, K, f.E4M3, None, self.qb, 0, self.sb, self.amb)
+        if ev:
+            ev[0].record()
+        f.fp8_gemm_scaled(self.qa, f.E4M3, self.qb, f.E4M3, M, N, K, f.SCALE_TENSOR, self.sa, self.sb, self.D, N)
+        if ev:
+            ev[1].record()
+
+    # block-scaled MLP: X -> up -> H -> down
+    def _setup_blockmlp(self):
+        f, inp, d, s = self.f, self.inp, self.dev, self.seed
+        M, Dm, F = 8192, 4096, 11008
+        self.X = inp.normal_bf16((M, Dm), 1.0, seed=s, device=d)
+        self.Wu = inp.normal_bf16((F, Dm), 0.02, seed=s + 1, device=d)
+        self.Wd = inp.normal_bf16((Dm, F), 0.02, seed=s + 2, device=d)
+        self.qx = torch.empty((M, Dm), dtype=torch.uint8, device=d)
+        self.sx = torch.empty(((Dm + 127) // 128, M), dtype=torch.float32, device=d)
+        self.qwu = torch.empty((F, Dm), dtype=torch.uint8, device=d)
+        self.swu = torch.empty(((F + 127) // 128, (Dm + 127) // 128), dtype=torch.float32, device=d)
+        self.H = torch.empty((M, F), dtype=torch.bfloat16, device=d)
+        self.qh = torch.empty((M, F), dtype=torch.uint8, device=d)
+        self.sh = torch.empty(((F + 127) // 128, M), dtype=torch.float32, device=d)
+        self.qwd = torch.empty((Dm, F), dtype=torch.uint8, device=d)
+        self.swd = torch.empty(((Dm + 127) // 128, (F + 127) // 128), dtype=torch.float32, device=d)
+        self.Y = torch.empty((M, Dm), dtype=torch.bfloat16, device=d)
+        self.dims = (M, Dm, F)
+        self.flops = 2 * 2.0 * M * Dm * F
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.launches = 6
+        self.config = {"workload": "block-scaled E4M3 MLP (up then down)", "M": M, "D": Dm, "F": F,
+                       "X": "N(0,1) bf16", "W": "N(0,0.02) bf16",
+                       "scales": "1x128 activation blocks, 128x128 weight blocks, fp32",
+                       "chain": "H = up(X) in bf16 is requantized 1x128 for the down GEMM"}
+        self.host_inputs = [("X", self.X), ("W_up", self.Wu), ("W_down", self.Wd)]
+        self.host_output = self.Y
+
+    def _step_blockmlp(self, ev=None):
+        f = self.f
+        M, Dm, F = self.dims
+        f.fp8_quantize_blockwise(self.X, M, Dm, Dm, f.E4M3, 1, self.qx, self.sx)
+        f.fp8_quantize_blockwise(self.Wu, F, Dm, Dm, f.E4M3, 128, self.qwu, self.swu)
+        if ev:
+            ev[0].record()
+        f.fp8_gemm_scaled(self.qx, f.E4M3, self.qwu, f.E4M3, M, F, Dm, f.SCALE_BLOCK, self.sx, self.swu, self.H, F)
+        if ev:
+            ev[1].record()
+        f.fp8_quantize_blockwise(self.H, M, F, F, f.E4M3, 1, self.qh, self.sh)
+        f.fp8_quantize_blockwise(self.Wd, Dm, F, F, f.E4M3, 128, self.qwd, self.swd)
+        f.fp8_gemm_scaled(self.qh, f.E4M3, self.qwd, f.E4M3, M, Dm, F, f.SCALE_BLOCK, self.sh, self.swd, self.Y, Dm)
+
+    # dgrad with delayed scaling
+    def _setup_dgrad(self):
+        f, inp, d, s = self.f, self.inp, self.dev, self.seed
+        M, N_out, K_in, T = 8192, 4096, 4096, 16
+        self.G = [inp.lognormal_grads_bf16((M, N_out), seed=s + 100 + t, device=d) for t in range(T)]
+        W = inp.normal_bf16((N_out, K_in), 0.02, seed=s + 1, device=d)
+        self.wq, self.wsinv, _ = f.quantize_tensorwise(W, f.E4M3, transpose=True)   # W^T [K_in, N_out]
+        del W
+        self.hist = f.AmaxHistory(16, f.E5M2, device=d)
+        self.qg = torch.empty((M, N_out), dtype=torch.uint8, device=d)
+        self.sg = torch.empty(1, dtype=torch.float32, device=d)
+        self.am = torch.empty(1, dtype=torch.float32, device=d)
+        self.DX = torch.empty((M, K_in), dtype=torch.bfloat16, device=d)
+        self.t = 0
+        self.dims = (M, N_out, K_in)
+        self.flops = 2.0 * M * N_out * K_in
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.launches = 3
+        self.config = {"workload": "dgrad E5M2 x E4M3, delayed scaling", "M": M, "N_out": N_out, "K_in": K_in,
+                       "dY": "|g| = 10^u, u ~ N(-2, (4/3)^2) clipped to [-6, 2], random sign, 16 seeded steps",
+                       "W": "N(0,0.02) bf16, E4M3 per-tensor, transposed once", "history": 16}
+        self.host_inputs = [("dY_t", self.G[0])]
+        self.host_output = self.DX
+
+    def _step_dgrad(self, ev=None):
+        f = self.f
+        M, N_out, K_in = self.dims
+        g = self.G[self.t % len(self.G)]
+        self.t += 1
+        f.fp8_quantize_tensorwise(g, M, N_out, f.E5M2, self.hist.scale, self.qg, 0, self.sg, self.am)
+        if ev:
+            ev[0].record()
+        f.fp8_gemm_scaled(self.qg, f.E5M2, self.wq, f.E4M3, M, K_in, N_out, f.SCALE_TENSOR, self.sg, self.wsinv,
+                          self.DX, K_in)
+        if ev:
+            ev[1].record()
+        self.hist.update(self.am)
+
+    # FP8 KV cache round trip
+    def _setup_kv(self):
+        f, inp, d, s = self.f, self.inp, self.dev, self.seed
+        B, H, S, Dh = 32, 32, 8192, 128
+        self.K = inp.normal_bf16((B, H, S, Dh), 1.0, seed=s, device=d)
+        self.V = inp.normal_bf16((B, H, S, Dh), 1.0, seed=s + 1, device=d)
+        self.qk = torch.empty(self.K.shape, dtype=torch.uint8, device=d)
+        self.qv = torch.empty(self.V.shape, dtype=torch.uint8, device=d)
+        self.sk = torch.empty(B * H, dtype=torch.float32, device=d)
+        self.sv = torch.empty(B * H, dtype=torch.float32, device=d)
+        self.Kd = torch.empty_like(self.K)
+        self.Vd = torch.empty_like(self.V)
+        self.dims = (B, H, S, Dh)
+        n = B * H * S * Dh
+        self.bytes = 2 * (3.0 * n + 4 * B * H) * 2    # K and V: quantize (2 B in, 1 B out) + dequantize (1 B in, 2 B out)
+        self.kernel_bytes = 3.0 * n + 4 * B * H       # one kv_quant launch
+        self.unit, self.bound = "GB/s", "hbm"
+        self.launches = 4
+        self.config = {"workload": "FP8 KV cache quantize + dequantize", "B": B, "H": H, "S": S, "Dh": Dh,
+                       "K,V": "N(0,1) bf16", "scale": "per (b, h): 448/amax, E4M3"}
+        self.host_inputs = [("K", self.K), ("V", self.V)]
+        self.host_output = self.Kd
+
+    def _step_kv(self, ev=None):
+        f = self.f
+        B, H, S, Dh = self.dims
+        if ev:
+            ev[0].record()
+        f.fp8_kv_quant(self.K, B, H, S, Dh, f.E4M3, self.qk, self.sk)
+        if ev:
+            ev[1].record()
+        f.fp8_kv_quant(self.V, B, H, S, Dh, f.E4M3, self.qv, self.sv)
+        f.fp8_kv_dequant(self.qk, self.sk, B, H, S, Dh, f.E4M3, self.Kd)
+        f.fp8_kv_dequant(self.qv, self.sv, B, H, S, Dh, f.E4M3, self.Vd)
+
+    def step(self, ev=None):
+        getattr(self, "_step_" + self.name)(ev)
+
+    def work(self):
+        return self.flops / 1e12 if self.unit == "TFLOP/s" else self.bytes / 1e9
+
+    def kernel_work(self):
+        """Work of one launch of the dominant kernel (events ev[0]..ev[1])."""
+        if self.unit == "TFLOP/s":
+            if self.name == "blockmlp":
+                M, Dm, F = self.dims
+                return 2.0 * M * Dm * F / 1e12
+            return self.flops / 1e12
+        return self.kernel_bytes / 1e9
+
+
+# --------------------------------------------------------- CPU (oracle) arm --
+
+def cpu_sample(name: str, seed: int = 0):
+    """Time the CPU oracle, as it stands, on a bounded sample of the workload;
+    returns (value in the workload's unit for a full step, sample description)."""
+    import numpy as np
+    from fp8_scaled_quantization_amax_b200 import inputs
+    from oracle import oracle as orc
+    orc.lib()
+    if name in ("rowwise", "tensor", "blockmlp", "dgrad"):
+        if name == "rowwise":
+            M = N = K = 4096
+            r = 8
+            a = inputs.bf16_bits(inputs.outlier_activations_bf16((r, K), seed=seed))
+            b = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, seed=seed + 1))
+            t0 = time.perf_counter()
+            qb, sb = orc.quantize_rowwise(b, 0, True)
+            tb = time.perf_counter() - t0
+            t0 = time.perf_counter()
+            qa, sa = orc.quantize_rowwise(a, 0, True)
+            im = np.repeat(np.arange(r), N)
+            inn = np.tile(np.arange(N), r)
+            orc.gemm_scaled_sampled(qa, 0, qb, 0, 1, sa, sb, im, inn)
+            tr = time.perf_counter() - t0
+            full = tb + tr * (M / r)
+            return 2.0 * M * N * K / full / 1e12, (
+                f"rowwise-quantize all of B [4096,4096] + {r} rows of A, then those {r}x4096 outputs "
+                f"(fp64 sums); full step extrapolated as t_B + (4096/{r}) x t_rows")
+        if name == "tensor":
+            M = N = K = 256
+            a = inputs.bf16_bits(inputs.normal_bf16((M, K), 1.0, seed=seed))
+            b = inputs.bf16_bits(inputs.normal_bf16((N, K), 1.0, seed=seed + 1))
+            t0 = time.perf_counter()
+            qa, sa, _, _ = orc.quantize_tensorwise(a, 0)
+            qb, sb, _, _ = orc.quantize_tensorwise(b, 0)
+            orc.gemm_scaled(qa, 0, qb, 0, 0, np.float32([sa]), np.float32([sb]))
+            t = time.perf_counter() - t0
+            return 2.0 * M * N * K / t / 1e12, "the whole 256^3 per-tensor step"
+        if name == "blockmlp":
+            M, Dm, F = 8192, 4096, 11008
+            r = 4
+            x = inputs.bf16_bits(inputs.normal_bf16((r, Dm), 1.0, seed=seed))
+            w = inputs.bf16_bits(inputs.normal_bf16((256, Dm), 0.02, seed=seed + 1))
+            t0 = time.perf_counter()
+            qw, sw = orc.quantize_blockwise(w, 0, 128)
+            tw = (time.perf_counter() - t0) * (F / 256) * 2
+            t0 = time.perf_counter()
+            qx, sx = orc.quantize_blockwise(x, 0, 1)
+            im = np.repeat(np.arange(r), 256)
+            inn = np.tile(np.arange(256), r)
+            orc.gemm_scaled_sampled(qx, 0, qw, 0, 2, sx, sw, im, inn)
+            tr = (time.perf_counter() - t0) * (M / r) * (F / 256) * 2
+            return 4.0 * M * Dm * F / (tw + tr) / 1e12, (
+                f"blockwise-quantize 256 W rows and {r} X rows, then {r}x256 outputs at K=4096; "
+                "scaled to both MLP GEMMs")
+        if name == "dgrad":
+            M, N_out, K_in = 8192, 4096, 4096
+            r = 16
+            g = inputs.bf16_bits(inputs.lognormal_grads_bf16((r, N_out), seed=seed))
+            w = inputs.bf16_bits(inputs.normal_bf16((256, N_out), 0.02, seed=seed + 1))
+            t0 = time.perf_counter()
+            qw, sw, _, _ = orc.quantize_tensorwise(w, 0)
+            qg, sg, _, _ = orc.quantize_tensorwise(g, 1, scale_in=1.0)
+            im = np.repeat(np.arange(r), 256)
+            inn = np.tile(np.arange(256), r)
+            orc.gemm_scaled_sampled(qg, 1, qw, 0, 0, np.float32([sg]), np.float32([sw]), im, inn)
+            t = (time.perf_counter() - t0) * (M / r) * (K_in / 256)
+            return 2.0 * M * N_out * K_in / t / 1e12, (
+                f"quantize {r} gradient rows (E5M2) + 256 weight rows, then {r}x256 outputs; scaled to the step")
+    # kv
+    B, H, S, Dh = 32, 32, 8192, 128
+    k = inputs.bf16_bits(inputs.normal_bf16((1, 2, S, Dh), 1.0, seed=seed))
+    t0 = time.perf_counter()
+    q, s = orc.kv_quant(k, 0)
+    orc.kv_dequant(q, s, 0)
+    t = time.perf_counter() - t0
+    per_slice = t / 2
+    n = B * H * S * Dh
+    full = per_slice * B * H * 2
+    return 2 * (3.0 * n) * 2 / full / 1e9, "2 of the 2048 (b,h) slices of K/V quantized and dequantized; scaled"
+
+
+# -------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="rowwise", choices=list(DEFAULT_STEPS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    steps = args.steps if args.steps is not None else DEFAULT_STEPS[args.workload]
+    warmup = max(3, args.warmup)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    unit = "GB/s" if args.workload == "kv" else "TFLOP/s"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        desc = ""
+        for _ in range(warmup):
+            cpu_sample(args.workload)
+        for i in range(steps if args.steps is not None else 3):
+            v, desc = cpu_sample(args.workload, seed=i)
+            vals.append(v)
+        v = statistics.mean(vals)
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
+                "steps": len(vals), "warmup": warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64 sums / fp32 scales (CPU oracle)", "data": "synthetic",
+                "config": {"workload": args.workload},
+                "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle", "sample": desc},
+                "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    from fp8_scaled_quantization_amax_b200 import fp8q
+    fp8q.lib()
+    wl = Workload(args.workload, dev, seed=1000 * rank)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(warmup):
+        flush.zero_()
+        wl.step()
+    torch.cuda.synchronize(dev)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        t_wall0 = time.perf_counter()
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            wl.step(kev[i])
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall0
+        barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kern_ms = [a.elapsed_time(b) for a, b in kev]
+    total_ms = max_over_ranks(sum(step_ms))
+    ms_per_step = total_ms / steps
+    value = world * wl.work() * steps / (total_ms * 1e-3)
+    kern_avg_ms = max_over_ranks(statistics.mean(kern_ms))
+
+    # end to end through the public API: pinned host inputs -> device, the
+    # step, the result back to pinned host memory, every step
+    e2e_steps = min(steps, 10 if wl.unit == "TFLOP/s" and args.workload != "blockmlp" else 3)
+    host_in = [(name, t.detach().cpu().pin_memory()) for name, t in wl.host_inputs]
+    host_out = torch.empty(wl.host_output.shape, dtype=wl.host_output.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for _, t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(e2e_steps):
+        flush.zero_()
+        e_s[i].record(stream)
+        for (name, h), (_, d) in zip(host_in, wl.host_inputs):
+            d.copy_(h, non_blocking=True)
+        wl.step()
+        host_out.copy_(wl.host_output, non_blocking=True)
+        e_e[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)) / e2e_steps)
+    e2e_value = world * wl.work() / (e2e_ms * 1e-3)
+    assert fp8q.fp8_device_error(clear=True) == 0, "a kernel gave up a bounded wait"
+
+    hbm, bf16, src = peaks()
+    if wl.bound == "tensor":
+        peak = bf16 * FP8_OVER_BF16
+        peak_src = (f"FP8 dense peak = {src} bf16 burst {bf16} TFLOP/s x nominal fp8/bf16 ratio 2 "
+                    "(MEASURED_PEAKS.json)" if src == "measured" else f"fallback bf16 {bf16} x 2")
+    else:
+        peak = hbm
+        peak_src = f"{src} HBM copy bandwidth {hbm} GB/s"
+    achieved = wl.kernel_work() / (kern_avg_ms * 1e-3)
+
+    if rank != 0:
+        return
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        v, desc = cpu_sample(args.workload)
+        cpu = {"value": v, "unit": wl.unit, "cores": 1, "kind": "oracle", "sample": desc}
+    dtype = {"rowwise": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate -> bf16",
+             "tensor": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate -> bf16",
+             "blockmlp": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate (per-128-K promotion) -> bf16",
+             "dgrad": "fp8_e5m2 x fp8_e4m3 -> f32 accumulate -> bf16",
+             "kv": "bf16 <-> fp8_e4m3 (f32 scale)"}[args.workload]
+    cfg = dict(wl.config)
+    cfg["l2"] = "flushed before every step (256 MiB write, outside the step's events)"
+    line = {
+        "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype, "data": "synthetic (seeded, per rank)", "config": cfg,
+        "roofline": {"bound": wl.bound, "achieved": achieved, "peak": peak, "unit": wl.unit,
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "fp8_gemm_scaled" if wl.bound == "tensor" else "fp8_kv_quant",
+                     "kernel_ms": kern_avg_ms, "peak_source": peak_src},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": wl.launches * steps,
+        "clocks": clk.summary(),
+        "wall_s_timed_region": t_wall,
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    try:
+        main()
+    finally:
+        if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()

@@ -1,0 +1,192 @@
+// common.cuh -- device helpers shared by the FP8 quantization kernels and the
+// host-side validation used by every entry point.
+//
+// Numerics (bit-exact contract of the quantizers):
+//   * amax is max |x| over the finite bf16 elements: exact, order independent.
+//   * s = fmax / amax is one IEEE round-to-nearest fp32 division (__fdiv_rn);
+//     amax == 0 gives 1, an overflowing quotient is clamped to FLT_MAX.
+//   * the power-of-two scale keeps only the exponent of that quotient (the
+//     largest 2^k not above it, clamped to [2^-126, 2^127]).
+//   * the cast is y = x * s with one rounded fp32 multiply (__fmul_rn, never
+//     contracted into an FMA), then the hardware's saturating
+//     round-to-nearest-even convert (cvt.rn.satfinite.{e4m3,e5m2}x2.f32).
+//   * no flush-to-zero anywhere (the library is built without fast math).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fp8q.h"
+
+namespace fp8q {
+
+// Largest finite magnitude of each format: E4M3 448, E5M2 57344.
+template <int FMT>
+__host__ __device__ constexpr float fmax_of() { return FMT == FP8_E4M3 ? 448.0f : 57344.0f; }
+
+__device__ __forceinline__ float scale_from_amax(float amax, float fm) {
+    if (!(amax > 0.0f)) return 1.0f;
+    float s = __fdiv_rn(fm, amax);
+    if (isinf(s)) s = 3.402823466e38f;
+    return s;
+}
+
+__device__ __forceinline__ float pow2_scale_from_amax(float amax, float fm) {
+    if (!(amax > 0.0f)) return 1.0f;
+    uint32_t e = __float_as_uint(__fdiv_rn(fm, amax)) & 0x7F800000u;
+    if (e == 0x7F800000u) e = 0x7F000000u;   // 2^127
+    if (e == 0u) e = 0x00800000u;            // 2^-126
+    return __uint_as_float(e);
+}
+
+// Two bf16 in a 32-bit word -> two fp32 (exact).
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Saturating RNE cast of two fp32 values to two FP8 codes; a lands in the low byte.
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt2(float a, float b) {
+    uint16_t r;
+    if (FMT == FP8_E4M3)
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+    else
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+    return r;
+}
+
+// Cast one 32-bit word (two bf16) scaled by s to two FP8 codes (16 bits).
+template <int FMT>
+__device__ __forceinline__ uint32_t cast_word(uint32_t w, float s) {
+    return cvt2<FMT>(__fmul_rn(bf_lo(w), s), __fmul_rn(bf_hi(w), s));
+}
+
+// Eight bf16 (uint4) -> eight FP8 codes (uint2).
+template <int FMT>
+__device__ __forceinline__ uint2 cast8(uint4 v, float s) {
+    uint2 o;
+    o.x = cast_word<FMT>(v.x, s) | (cast_word<FMT>(v.y, s) << 16);
+    o.y = cast_word<FMT>(v.z, s) | (cast_word<FMT>(v.w, s) << 16);
+    return o;
+}
+
+// Two FP8 codes (low 16 bits of c) -> two fp32 (exact, via f16x2).
+template <int FMT>
+__device__ __forceinline__ float2 fp8x2_to_float2(uint16_t c) {
+    uint32_t h;
+    if (FMT == FP8_E4M3)
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(c));
+    else
+        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(c));
+    __half2 hh = *reinterpret_cast<__half2 *>(&h);
+    return __half22float2(hh);
+}
+
+// fp32 pair -> packed bf16x2 (RNE), a in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
+}
+
+// ---------------------------------------------------------------- amax ----
+// Fast running max over packed bf16 pairs: |x| via the sign mask, then a
+// NaN-propagating bf16x2 max.  If the result is non-finite (some element was
+// NaN or Inf) the caller redoes its elements with amax_exact_word(), which
+// skips non-finite values and counts them.
+__device__ __forceinline__ uint32_t amax_fast_word(uint32_t m, uint32_t w) {
+    uint32_t a = w & 0x7FFF7FFFu;
+    uint32_t r;
+    asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(m), "r"(a));
+    return r;
+}
+__device__ __forceinline__ uint32_t amax_fast8(uint32_t m, uint4 v) {
+    m = amax_fast_word(m, v.x);
+    m = amax_fast_word(m, v.y);
+    m = amax_fast_word(m, v.z);
+    return amax_fast_word(m, v.w);
+}
+// Packed running max -> the max magnitude bits (of one bf16, as uint32), or
+// 0xFFFFFFFF if a non-finite value was seen.
+__device__ __forceinline__ uint32_t amax_fast_final(uint32_t m) {
+    uint32_t lo = m & 0xFFFFu, hi = m >> 16;
+    if (lo >= 0x7F80u || hi >= 0x7F80u) return 0xFFFFFFFFu;
+    return lo > hi ? lo : hi;
+}
+// Exact: max over finite magnitudes (bf16 bits), counting non-finite ones.
+__device__ __forceinline__ uint32_t amax_exact_word(uint32_t m, uint32_t w, uint32_t &bad) {
+    uint32_t lo = w & 0x7FFFu, hi = (w >> 16) & 0x7FFFu;
+    if (lo < 0x7F80u) { m = lo > m ? lo : m; } else { ++bad; }
+    if (hi < 0x7F80u) { m = hi > m ? hi : m; } else { ++bad; }
+    return m;
+}
+__device__ __forceinline__ uint32_t amax_exact8(uint32_t m, uint4 v, uint32_t &bad) {
+    m = amax_exact_word(m, v.x, bad);
+    m = amax_exact_word(m, v.y, bad);
+    m = amax_exact_word(m, v.z, bad);
+    return amax_exact_word(m, v.w, bad);
+}
+// bf16 magnitude bits -> fp32 value.
+__device__ __forceinline__ float bf16bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Number of elements among 8 (uint4 of bf16) whose scaled magnitude exceeds fm.
+__device__ __forceinline__ uint32_t count_sat8(uint4 v, float s, float fm) {
+    uint32_t c = 0;
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float a = __fmul_rn(bf_lo(w[i]), s), b = __fmul_rn(bf_hi(w[i]), s);
+        c += (fabsf(a) > fm) ? 1u : 0u;
+        c += (fabsf(b) > fm) ? 1u : 0u;
+    }
+    return c;
+}
+
+// Streaming 16-byte load that does not allocate in L1.
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Block-wide max of a uint32 (all threads get the result).  smem >= 32 words.
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *smem) {
+    v = __reduce_max_sync(0xFFFFFFFFu, v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (blockDim.x + 31) >> 5;
+    __syncthreads();
+    if (lane == 0) smem[warp] = v;
+    __syncthreads();
+    uint32_t r = lane < nwarps ? smem[lane] : 0u;
+    r = __reduce_max_sync(0xFFFFFFFFu, r);
+    return r;
+}
+__device__ __forceinline__ uint32_t block_sum_u32(uint32_t v, uint32_t *smem) {
+    v = __reduce_add_sync(0xFFFFFFFFu, v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (blockDim.x + 31) >> 5;
+    __syncthreads();
+    if (lane == 0) smem[warp] = v;
+    __syncthreads();
+    uint32_t r = lane < nwarps ? smem[lane] : 0u;
+    r = __reduce_add_sync(0xFFFFFFFFu, r);
+    return r;
+}
+
+}  // namespace fp8q
+
+// ------------------------------------------------------------- host side --
+namespace fp8q_host {
+
+// Current device must be compute capability 10.0 (B200, sm_100a); cached
+// per device ordinal.  Also returns the SM count.
+fp8_status check_device(int *sm_count);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace fp8q_host

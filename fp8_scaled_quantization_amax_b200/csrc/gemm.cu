@@ -1,0 +1,511 @@
+// gemm.cu -- FP8 scaled GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Sources: "H100 FP8加速实测：新一代计算架构的飞跃" (the multiply-accumulate runs
+// directly on 8-bit floating-point operands on the tensor cores);
+// "FP8训练与QAT量化感知训练：…用Soup把大模型微调提速2倍", section
+// "FP8 三种缩放配方怎么选" (tensorwise and rowwise scaled matmuls);
+// "DeepL押注FP8：大模型训练与推理统一精度实战解析" §2.3 (per-block scales),
+// §2.1 (E5M2 gradients against E4M3 weights), §5.3 (FP8 GEMM results depend
+// on the tiling; this kernel uses one fixed K order and no split-K, so it is
+// deterministic run to run).
+//
+//   D[m, n] = bf16( epilogue( sum_k A[m, k] * B[n, k] ) )
+//   A [M, K], B [N, K]: FP8 codes, K contiguous; fp32 accumulation in TMEM.
+//
+// Design (one CTA per SM, persistent over 128x256 output tiles):
+//   warp 0      TMA producer: 128x128 A and 256x128 B tiles (128-byte
+//               swizzle) into a 4-stage shared-memory ring, one mbarrier per
+//               stage carrying the transaction byte count.
+//   warp 1      TMEM allocator and MMA issuer: per 128-wide K chunk, four
+//               tcgen05.mma.kind::f8f6f4 of 128x256x32 from shared-memory
+//               descriptors; tcgen05.commit frees the stage when the tensor
+//               core has read it.
+//   warps 2-9   epilogue: tcgen05.ld of the fp32 accumulator (warp w reads
+//               TMEM lanes 32*(w%4)..+31 = tile rows, columns split in two
+//               128-wide halves), scales applied in fp32, RNE to bf16, 16-byte
+//               stores.
+//   TENSOR/ROW: the accumulator is double-buffered in TMEM (2 x 256 columns),
+//               so the epilogue of tile i overlaps the mainloop of tile i+1.
+//   BLOCK:      per-block scales vary along K, so each 128-wide K chunk is
+//               accumulated alone into one of two TMEM partial buffers
+//               (ping-pong); the epilogue warps read it, multiply by
+//               sa[kb, m] * sb[n/128, kb] and add it into an fp32 register
+//               accumulator ("promotion"); the MMA of chunk c+1 runs while
+//               chunk c is promoted.
+// Every wait on an mbarrier is bounded (about one second); on expiry the
+// kernel records a bit in the library's device error word, stops issuing,
+// waits (bounded) for its own copies and MMAs in flight, frees TMEM and
+// returns.  No trap, no unbounded spin.
+#include <cuda.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+
+using namespace fp8q;
+
+namespace {
+
+constexpr int BM = 128;                 // tile rows (TMEM lanes)
+constexpr int BN = 256;                 // tile columns (TMEM columns per accumulator)
+constexpr int BK = 128;                 // K chunk: one 128-byte swizzle row of FP8
+constexpr int STAGES = 4;
+constexpr int A_TILE = BM * BK;         // 16 KiB
+constexpr int B_TILE = BN * BK;         // 32 KiB
+constexpr int STAGE_BYTES = A_TILE + B_TILE;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, acc_full[2], acc_empty[2], drain
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_BARS * 8 + 16;
+constexpr uint64_t kTimeoutNs = 1000000000ull;
+
+enum { kModeTensor = 0, kModeRow = 1, kModeBlock = 2 };
+enum : uint32_t { kErrProducer = 1u, kErrMma = 2u, kErrEpilogue = 4u, kErrDrain = 8u };
+
+__device__ unsigned int g_gemm_error;
+
+// ------------------------------------------------------------- PTX glue --
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase of `bar` with the given parity.  Gives up when
+// the CTA's abort flag is raised or after kTimeoutNs (then it raises the flag
+// and records `code` in the device error word).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag,
+                                      uint32_t code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > kTimeoutNs) {
+                atomicOr(&g_gemm_error, code);
+                *abort_flag = 1u;
+                return false;
+            }
+        }
+    }
+}
+// Bounded wait that ignores the abort flag (used to drain work in flight).
+__device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > kTimeoutNs) {
+            atomicOr(&g_gemm_error, kErrDrain);
+            return false;
+        }
+    }
+    return true;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// 32 lanes x 32 consecutive fp32 columns: thread i gets lane (base + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart (the layout TMA writes with
+// CU_TENSOR_MAP_SWIZZLE_128B and a 128-byte inner box).
+__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);    // start address (16-byte units)
+    d |= (uint64_t)1u << 16;                    // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024u >> 4) << 32;          // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1u << 46;                    // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                    // layout: SWIZZLE_128B
+    return d;
+}
+
+// ------------------------------------------------------------- kernel ----
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+           int K, uint32_t idesc, const float *__restrict__ sa, const float *__restrict__ sb,
+           __nv_bfloat16 *__restrict__ D, int64_t ldd) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)STAGES * STAGE_BYTES);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int nk = (K + BK - 1) / BK;
+
+    auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+    auto empty_bar = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+    auto accf_bar = [&](int b) { return smem_u32(&bars[2 * STAGES + b]); };
+    auto acce_bar = [&](int b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
+    const uint32_t drain_bar = smem_u32(&bars[2 * STAGES + 4]);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf_bar(b), 1);
+            mbar_init(acce_bar(b), EPI_WARPS);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            int last_round[STAGES];
+            for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int m_blk = tile % num_m, n_blk = tile / num_m;
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const int stage = it % STAGES;
+                    const uint32_t round = it / STAGES;
+                    if (!wait_bar(empty_bar(stage), (round & 1u) ^ 1u, abort_flag, kErrProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_u32(smem + (size_t)stage * STAGE_BYTES);
+                    mbar_expect_tx(full_bar(stage), STAGE_BYTES);
+                    tma_load_2d(a_dst, &tmA, full_bar(stage), kc * BK, m_blk * BM);
+                    tma_load_2d(a_dst + A_TILE, &tmB, full_bar(stage), kc * BK, n_blk * BN);
+                    last_round[stage] = (int)round;
+                }
+            }
+            if (!ok || *abort_flag) {   // copies in flight must land before the CTA exits
+                for (int s = 0; s < STAGES; ++s)
+                    if (last_round[s] >= 0) wait_bar_drain(full_bar(s), (uint32_t)last_round[s] & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer ----
+        if (lane == 0) {
+            uint32_t it = 0, lt = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++lt) {
+                uint32_t d_tmem = tmem;
+                if (MODE != kModeBlock) {
+                    const uint32_t ab = lt & 1u, use = lt >> 1;
+                    if (!wait_bar(acce_bar(ab), (use & 1u) ^ 1u, abort_flag, kErrMma)) break;
+                    tc_fence_after();
+                    d_tmem = tmem + ab * BN;
+                }
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const int stage = it % STAGES;
+                    const uint32_t round = it / STAGES;
+                    if (MODE == kModeBlock) {
+                        const uint32_t pb = it & 1u, use = it >> 1;
+                        if (!wait_bar(acce_bar(pb), (use & 1u) ^ 1u, abort_flag, kErrMma)) { ok = false; break; }
+                        d_tmem = tmem + pb * BN;
+                    }
+                    if (!wait_bar(full_bar(stage), round & 1u, abort_flag, kErrMma)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + (size_t)stage * STAGE_BYTES);
+                    const uint64_t adesc = sdesc_k_sw128(a_addr);
+                    const uint64_t bdesc = sdesc_k_sw128(a_addr + A_TILE);
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k) {
+                        // +32 bytes along K inside the swizzled 128-byte row = +2 in the address field
+                        const uint32_t acc = (MODE == kModeBlock) ? (k > 0) : (kc > 0 || k > 0);
+                        tc_mma(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, acc);
+                    }
+                    tc_commit(empty_bar(stage));
+                    if (MODE == kModeBlock) tc_commit(accf_bar(it & 1u));
+                }
+                if (ok && MODE != kModeBlock) tc_commit(accf_bar(lt & 1u));
+            }
+            // all MMAs issued by this thread complete before TMEM is freed
+            tc_commit(drain_bar);
+            wait_bar_drain(drain_bar, 0u);
+        }
+        __syncwarp();
+    } else {
+        // --------------------------------------------------- epilogue ----
+        const int sp = warp & 3;                 // TMEM lane quarter this warp may access
+        const int ch = (warp - 2) >> 2;          // column half of the tile
+        const int row_in_tile = sp * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+        uint32_t it = 0, lt = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++lt) {
+            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            const int m = m_blk * BM + row_in_tile;
+            const int n_base = n_blk * BN + ch * 128;
+            __nv_bfloat16 *drow = D + (int64_t)m * ldd;
+            if (MODE != kModeBlock) {
+                const uint32_t ab = lt & 1u, use = lt >> 1;
+                float rs;
+                if (MODE == kModeRow) rs = (m < M) ? sa[m] : 0.0f;
+                else rs = __fmul_rn(sa[0], sb[0]);
+                bool w = true;
+                if (lane == 0) w = wait_bar(accf_bar(ab), use & 1u, abort_flag, kErrEpilogue);
+                w = __shfl_sync(0xFFFFFFFFu, w, 0);
+                if (!w) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + ab * BN + ch * 128 + c * 32, v);
+                    const int col0 = n_base + c * 32;
+                    if (MODE == kModeRow) {
+                        const float cb = (col0 + lane < N) ? sb[col0 + lane] : 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = v[j] * (rs * __shfl_sync(0xFFFFFFFFu, cb, j));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
+                    }
+                    if (m < M) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (col0 + g * 8 < N) {
+                                uint4 o;
+                                o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+                                o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+                                o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+                                o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+                                *reinterpret_cast<uint4 *>(drow + col0 + g * 8) = o;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acce_bar(ab));
+            } else {
+                float acc[128];
+#pragma unroll
+                for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+                const int nkb_b = nk;                     // K blocks per row of sb
+                const int nb = n_base / 128;              // this half's 128-row block of B
+                const bool nb_ok = n_base < N;
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const uint32_t pb = it & 1u, use = it >> 1;
+                    const float a_s = (m < M) ? sa[(int64_t)kc * M + m] : 0.0f;
+                    const float b_s = nb_ok ? sb[(int64_t)nb * nkb_b + kc] : 0.0f;
+                    const float sc = __fmul_rn(a_s, b_s);
+                    bool w = true;
+                    if (lane == 0) w = wait_bar(accf_bar(pb), use & 1u, abort_flag, kErrEpilogue);
+                    w = __shfl_sync(0xFFFFFFFFu, w, 0);
+                    if (!w) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float v[32];
+                        tmem_ld32(tmem + lane_base + pb * BN + ch * 128 + c * 32, v);
+                        if (c == 3) {   // the partial buffer is free once the last slice is in registers
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(acce_bar(pb));
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(v[j], sc, acc[c * 32 + j]);
+                    }
+                }
+                if (!ok) break;
+                if (m < M) {
+#pragma unroll
+                    for (int g = 0; g < 16; ++g) {
+                        const int col = n_base + g * 8;
+                        if (col < N) {
+                            uint4 o;
+                            o.x = pack_bf16x2(acc[g * 8 + 0], acc[g * 8 + 1]);
+                            o.y = pack_bf16x2(acc[g * 8 + 2], acc[g * 8 + 3]);
+                            o.z = pack_bf16x2(acc[g * 8 + 4], acc[g * 8 + 5]);
+                            o.w = pack_bf16x2(acc[g * 8 + 6], acc[g * 8 + 7]);
+                            *reinterpret_cast<uint4 *>(drow + col) = o;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- host ----
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D map over a [rows, K] FP8 matrix (row pitch K bytes), box 128 x box_rows,
+// 128-byte swizzle; out-of-range boxes read zeros.
+bool make_map(CUtensorMap *map, const void *base, int64_t K, int64_t rows, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_gemm(cudaStream_t st, int sms, const CUtensorMap &ta, const CUtensorMap &tb, int M, int N, int K,
+                        uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(k_gemm_fp8<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = std::max(1, std::min(tiles, sms));
+    k_gemm_fp8<MODE><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, M, N, K, idesc, sa, sb,
+                                                        static_cast<__nv_bfloat16 *>(D), ldd);
+    return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+using namespace fp8q_host;
+
+extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int64_t M,
+                                      int64_t N, int64_t K, fp8_scale_mode mode, const float *a_scale_inv,
+                                      const float *b_scale_inv, void *D_bf16, int64_t ldd, void *stream) {
+    if ((fa != FP8_E4M3 && fa != FP8_E5M2) || (fb != FP8_E4M3 && fb != FP8_E5M2)) return FP8_ERR_INVALID_ARG;
+    if (mode != FP8_SCALE_TENSOR && mode != FP8_SCALE_ROW && mode != FP8_SCALE_BLOCK) return FP8_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0 || ldd < N) return FP8_ERR_SHAPE;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP8_ERR_SHAPE;
+    if (K % 16) return FP8_ERR_SHAPE;
+    if (N % 8 || ldd % 8) return FP8_ERR_ALIGNMENT;
+    if (M == 0 || N == 0) {
+        int sms;
+        return check_device(&sms);
+    }
+    if (!D_bf16) return FP8_ERR_INVALID_ARG;
+    if (K > 0 && (!A || !B || !a_scale_inv || !b_scale_inv)) return FP8_ERR_INVALID_ARG;
+    if (!aligned16(D_bf16) || (A && !aligned16(A)) || (B && !aligned16(B))) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    cudaStream_t s = as_stream(stream);
+    if (K == 0) {
+        return cudaMemset2DAsync(D_bf16, (size_t)ldd * 2, 0, (size_t)N * 2, (size_t)M, s) == cudaSuccess ? FP8_OK
+                                                                                                       : FP8_ERR_CUDA;
+    }
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A, K, M, BM) || !make_map(&tb, B, K, N, BN)) return FP8_ERR_CUDA;
+    // instruction descriptor: fp32 accumulator, A/B formats, K-major A and B, N>>3, M>>4
+    const uint32_t idesc = (1u << 4) | ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(BN >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+    cudaError_t e;
+    if (mode == FP8_SCALE_TENSOR)
+        e = launch_gemm<kModeTensor>(s, sms, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd);
+    else if (mode == FP8_SCALE_ROW)
+        e = launch_gemm<kModeRow>(s, sms, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd);
+    else
+        e = launch_gemm<kModeBlock>(s, sms, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd);
+    return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+extern "C" fp8_status fp8_device_error(uint32_t *host_out, int clear) {
+    if (!host_out) return FP8_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return FP8_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_gemm_error, sizeof(v)) != cudaSuccess) return FP8_ERR_CUDA;
+    *host_out = v;
+    if (clear) {
+        const unsigned int z = 0;
+        if (cudaMemcpyToSymbol(g_gemm_error, &z, sizeof(z)) != cudaSuccess) return FP8_ERR_CUDA;
+    }
+    return FP8_OK;
+}

@@ -1,0 +1,195 @@
+// kv.cu -- FP8 KV cache: per-(batch, head) quantize and dequantize.
+//
+// Source: "DeepL押注FP8：大模型训练与推理统一精度实战解析" §3.1 (K and V kept
+// in FP8 halve the cache; each is dequantized when attention reads it).
+//
+// Quantize: a (b, h) slice (S*Dh elements, 2 MiB of bf16 at S=8192, Dh=128)
+// needs its own amax before any element can be cast.  One 8-CTA thread-block
+// cluster owns one slice at a time: every CTA streams its eighth of the slice
+// from HBM for the amax, the eight partial maxima meet through distributed
+// shared memory behind a cluster barrier, and the cast pass re-reads the same
+// eighth while it is still in L2 (18 clusters x 2 MiB in flight stays far
+// below the 126 MB L2).  HBM traffic is the algorithmic 2 B in + 1 B out per
+// element, in one launch, with no scratch memory and no grid-wide wait.
+//
+// Dequantize: a plain stream, 16 FP8 codes in (one 16-byte load), 16 bf16 out
+// (two 16-byte stores), one scale per (b, h) from the grid's y index.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace cg = cooperative_groups;
+using namespace fp8q;
+
+namespace {
+
+constexpr int kClusterCtas = 8;
+constexpr int kKvThreads = 1024;
+
+template <int FMT>
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kKvThreads, 1)
+k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64_t nunit,
+           float *__restrict__ scale_inv) {
+    __shared__ uint32_t red[32];
+    __shared__ uint32_t slot[2];        // this CTA's partial amax, double-buffered by slice parity
+    __shared__ uint32_t slice_amax;
+    constexpr float fm = fmax_of<FMT>();
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned rank = cluster.block_rank();
+    const int64_t cid = blockIdx.x / kClusterCtas, ncl = gridDim.x / kClusterCtas;
+    const int64_t per = (nunit + kClusterCtas - 1) / kClusterCtas;
+    const int64_t u0 = min((int64_t)rank * per, nunit);
+    const int64_t u1 = min(u0 + per, nunit);
+    int it = 0;
+    for (int64_t sl = cid; sl < BH; sl += ncl, ++it) {
+        const uint4 *xs = x + 2 * sl * nunit;   // a unit is 16 elements = two uint4 of bf16
+        uint4 *qs = q + sl * nunit;             // and one uint4 of FP8
+        // pass 1: amax of this CTA's part of the slice
+        uint32_t m2 = 0;
+        int64_t u = u0 + threadIdx.x;
+        for (; u + kKvThreads < u1; u += 2 * kKvThreads) {
+            uint4 a0 = ld_stream(xs + 2 * u), a1 = ld_stream(xs + 2 * u + 1);
+            uint4 b0 = ld_stream(xs + 2 * (u + kKvThreads)), b1 = ld_stream(xs + 2 * (u + kKvThreads) + 1);
+            m2 = amax_fast8(amax_fast8(amax_fast8(amax_fast8(m2, a0), a1), b0), b1);
+        }
+        for (; u < u1; u += kKvThreads) m2 = amax_fast8(amax_fast8(m2, ld_stream(xs + 2 * u)), ld_stream(xs + 2 * u + 1));
+        uint32_t m = amax_fast_final(m2);
+        if (m == 0xFFFFFFFFu) {
+            uint32_t bad = 0;
+            m = 0;
+            for (int64_t j = u0 + threadIdx.x; j < u1; j += kKvThreads)
+                m = amax_exact8(amax_exact8(m, xs[2 * j], bad), xs[2 * j + 1], bad);
+        }
+        m = block_max_u32(m, red);
+        if (threadIdx.x == 0) slot[it & 1] = m;
+        cluster.sync();   // every CTA's partial is published
+        if (threadIdx.x < 32) {
+            uint32_t v = 0;
+            if (threadIdx.x < kClusterCtas) v = *cluster.map_shared_rank(&slot[it & 1], threadIdx.x);
+            v = __reduce_max_sync(0xFFFFFFFFu, v);
+            if (threadIdx.x == 0) slice_amax = v;
+        }
+        __syncthreads();
+        const float s = scale_from_amax(bf16bits_to_float(slice_amax), fm);
+        if (rank == 0 && threadIdx.x == 0) scale_inv[sl] = __fdiv_rn(1.0f, s);
+        // pass 2: cast (the re-read hits L2)
+        for (int64_t j = u0 + threadIdx.x; j < u1; j += kKvThreads) {
+            uint4 a0 = xs[2 * j], a1 = xs[2 * j + 1];
+            uint2 c0 = cast8<FMT>(a0, s), c1 = cast8<FMT>(a1, s);
+            qs[j] = make_uint4(c0.x, c0.y, c1.x, c1.y);
+        }
+    }
+    cluster.sync();   // no CTA leaves while a peer may still read its slots
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256)
+k_kv_dequant(const uint4 *__restrict__ q, const float *__restrict__ scale_inv, int64_t nunit,
+             uint4 *__restrict__ out) {
+    const int64_t sl = blockIdx.y;
+    const float d = scale_inv[sl];
+    const uint4 *qs = q + sl * nunit;
+    uint4 *os = out + 2 * sl * nunit;
+    for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < nunit;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        uint4 c = ld_stream(qs + u);
+        uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 lo = fp8x2_to_float2<FMT>((uint16_t)(w[i] & 0xFFFFu));
+            float2 hi = fp8x2_to_float2<FMT>((uint16_t)(w[i] >> 16));
+            o[2 * i] = pack_bf16x2(__fmul_rn(lo.x, d), __fmul_rn(lo.y, d));
+            o[2 * i + 1] = pack_bf16x2(__fmul_rn(hi.x, d), __fmul_rn(hi.y, d));
+        }
+        os[2 * u] = make_uint4(o[0], o[1], o[2], o[3]);
+        os[2 * u + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+}  // namespace
+
+using namespace fp8q_host;
+
+// Clusters of the quantize kernel that fit on the device at once (GPCs hold a
+// whole number of 8-SM clusters, so this is below sm_count / 8); cached per
+// device.  The grid never exceeds it, so no cluster waits for another to
+// finish before it can start.
+template <int FMT>
+static int max_active_clusters() {
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cache[dev] > 0) return cache[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kClusterCtas * 64);
+    cfg.blockDim = dim3(kKvThreads);
+    cfg.dynamicSmemBytes = 0;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = kClusterCtas;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_kv_quant<FMT>, &cfg) != cudaSuccess) return 0;
+    cache[dev] = n;
+    return n;
+}
+
+static fp8_status kv_check(int64_t B, int64_t H, int64_t S, int64_t Dh) {
+    if (B < 0 || H < 0 || S < 0 || Dh < 0) return FP8_ERR_SHAPE;
+    if ((S * Dh) % 16) return FP8_ERR_SHAPE;
+    if (B * H > 65535 && S * Dh > 0) return FP8_ERR_SHAPE;   // one grid row per (b, h) slice
+    return FP8_OK;
+}
+
+extern "C" fp8_status fp8_kv_quant(const void *kv_bf16, int64_t B, int64_t H, int64_t S, int64_t Dh,
+                                   fp8_format fmt, uint8_t *q, float *scale_inv, void *stream) {
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    fp8_status c = kv_check(B, H, S, Dh);
+    if (c != FP8_OK) return c;
+    const int64_t BH = B * H, nunit = S * Dh / 16;
+    if (BH > 0 && (!scale_inv || (nunit > 0 && (!kv_bf16 || !q)))) return FP8_ERR_INVALID_ARG;
+    if ((kv_bf16 && !aligned16(kv_bf16)) || (q && !aligned16(q))) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (BH == 0) return FP8_OK;
+    cudaStream_t s = as_stream(stream);
+    const int active = fmt == FP8_E4M3 ? max_active_clusters<FP8_E4M3>() : max_active_clusters<FP8_E5M2>();
+    if (active <= 0) return FP8_ERR_CUDA;
+    const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(BH, active));
+    const dim3 grid(clusters * kClusterCtas);
+    if (fmt == FP8_E4M3)
+        k_kv_quant<FP8_E4M3><<<grid, kKvThreads, 0, s>>>(static_cast<const uint4 *>(kv_bf16), reinterpret_cast<uint4 *>(q), BH, nunit, scale_inv);
+    else
+        k_kv_quant<FP8_E5M2><<<grid, kKvThreads, 0, s>>>(static_cast<const uint4 *>(kv_bf16), reinterpret_cast<uint4 *>(q), BH, nunit, scale_inv);
+    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+extern "C" fp8_status fp8_kv_dequant(const uint8_t *q, const float *scale_inv, int64_t B, int64_t H,
+                                     int64_t S, int64_t Dh, fp8_format fmt, void *out_bf16, void *stream) {
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    fp8_status c = kv_check(B, H, S, Dh);
+    if (c != FP8_OK) return c;
+    const int64_t BH = B * H, nunit = S * Dh / 16;
+    if (BH > 0 && nunit > 0 && (!q || !scale_inv || !out_bf16)) return FP8_ERR_INVALID_ARG;
+    if ((q && !aligned16(q)) || (out_bf16 && !aligned16(out_bf16))) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (BH == 0 || nunit == 0) return FP8_OK;
+    cudaStream_t s = as_stream(stream);
+    // about 8 CTAs of 256 threads per SM in total, at least one per slice
+    const int64_t per_slice = std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * 8 / BH, (nunit + 255) / 256));
+    const dim3 grid((unsigned)per_slice, (unsigned)BH);
+    if (fmt == FP8_E4M3)
+        k_kv_dequant<FP8_E4M3><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(q), scale_inv, nunit, static_cast<uint4 *>(out_bf16));
+    else
+        k_kv_dequant<FP8_E5M2><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(q), scale_inv, nunit, static_cast<uint4 *>(out_bf16));
+    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}

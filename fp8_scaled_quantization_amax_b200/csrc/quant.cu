@@ -1,0 +1,495 @@
+// quant.cu -- amax and the three quantizers (per-tensor, per-row, per-block).
+//
+// Sources: "DeepL押注FP8：大模型训练与推理统一精度实战解析" §2.3 (per-tensor,
+// per-row and per-block scaling; delayed scaling), §4.2 (max-absolute-value
+// statistics); "FP8训练与QAT量化感知训练：…用Soup把大模型微调提速2倍", section
+// "FP8 三种缩放配方怎么选" (tensorwise; rowwise with power-of-two e4m3 scales).
+//
+// All kernels are HBM-bound streams: 16-byte coalesced loads of bf16, 8- or
+// 16-byte stores of FP8, the amax folded into the same pass wherever the scale
+// does not depend on it (per-row and per-block data stays in registers between
+// the amax and the cast, so each element is read from HBM exactly once).
+#include <algorithm>
+
+#include "common.cuh"
+
+using namespace fp8q;
+
+namespace {
+
+constexpr int kStreamThreads = 512;
+
+// ------------------------------------------------------------------ amax --
+// Grid-stride max over 8-element vectors; one atomicMax per CTA on the fp32
+// bit pattern of the non-negative result (monotone as an unsigned integer).
+__global__ void __launch_bounds__(kStreamThreads) k_amax(const uint4 *__restrict__ xv, int64_t nvec,
+                                                         const uint16_t *__restrict__ xs, int64_t n,
+                                                         uint32_t *__restrict__ amax_bits,
+                                                         uint32_t *__restrict__ counts) {
+    __shared__ uint32_t red[32];
+    const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    uint32_t m2 = 0;
+    int64_t i = tid;
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        uint4 a = ld_stream(xv + i), b = ld_stream(xv + i + stride);
+        uint4 c = ld_stream(xv + i + 2 * stride), d = ld_stream(xv + i + 3 * stride);
+        m2 = amax_fast8(amax_fast8(amax_fast8(amax_fast8(m2, a), b), c), d);
+    }
+    for (; i < nvec; i += stride) m2 = amax_fast8(m2, ld_stream(xv + i));
+    uint32_t m = amax_fast_final(m2), bad = 0;
+    if (m == 0xFFFFFFFFu) {   // a NaN or Inf among this thread's elements: exact pass
+        m = 0;
+        for (int64_t j = tid; j < nvec; j += stride) m = amax_exact8(m, ld_stream(xv + j), bad);
+    }
+    for (int64_t j = nvec * 8 + tid; j < n; j += stride) {   // tail (< 8 elements)
+        uint32_t h = xs[j] & 0x7FFFu;
+        if (h < 0x7F80u) m = h > m ? h : m; else ++bad;
+    }
+    m = block_max_u32(m, red);
+    if (counts) bad = block_sum_u32(bad, red);
+    if (threadIdx.x == 0) {
+        atomicMax(amax_bits, m << 16);
+        if (counts && bad) atomicAdd(counts, bad);
+    }
+}
+
+// -------------------------------------------------- tensorwise cast pass --
+// q = cast(x * s) over 16-element units (two 16-byte loads, one 16-byte
+// store).  s comes from *scale_in (delayed scaling) or from *amax_in
+// (current scaling, written by k_amax earlier on the same stream).
+// AMAX: also reduce this tensor's amax into amax_bits (delayed scaling feeds
+// it to the history).  COUNT: count non-finite and saturated elements.
+template <int FMT, bool AMAX, bool COUNT>
+__global__ void __launch_bounds__(kStreamThreads)
+k_cast_tensor(const uint4 *__restrict__ xv, uint4 *__restrict__ qv, int64_t nunit,
+              const uint16_t *__restrict__ xs, uint8_t *__restrict__ qs, int64_t n,
+              const float *__restrict__ scale_in, const float *__restrict__ amax_in,
+              float *__restrict__ scale_inv_out, uint32_t *__restrict__ amax_bits,
+              uint32_t *__restrict__ nf_ctr, uint32_t *__restrict__ sat_ctr) {
+    __shared__ uint32_t red[32];
+    constexpr float fm = fmax_of<FMT>();
+    const float s = scale_in ? *scale_in : scale_from_amax(*amax_in, fm);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *scale_inv_out = __fdiv_rn(1.0f, s);
+    const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    uint32_t m2 = 0;
+    int64_t i = tid;
+    for (; i + stride < nunit; i += 2 * stride) {
+        uint4 a0 = ld_stream(xv + 2 * i), a1 = ld_stream(xv + 2 * i + 1);
+        uint4 b0 = ld_stream(xv + 2 * (i + stride)), b1 = ld_stream(xv + 2 * (i + stride) + 1);
+        if (AMAX || COUNT) m2 = amax_fast8(amax_fast8(amax_fast8(amax_fast8(m2, a0), a1), b0), b1);
+        uint2 qa0 = cast8<FMT>(a0, s), qa1 = cast8<FMT>(a1, s);
+        uint2 qb0 = cast8<FMT>(b0, s), qb1 = cast8<FMT>(b1, s);
+        qv[i] = make_uint4(qa0.x, qa0.y, qa1.x, qa1.y);
+        qv[i + stride] = make_uint4(qb0.x, qb0.y, qb1.x, qb1.y);
+    }
+    for (; i < nunit; i += stride) {
+        uint4 a0 = ld_stream(xv + 2 * i), a1 = ld_stream(xv + 2 * i + 1);
+        if (AMAX || COUNT) m2 = amax_fast8(amax_fast8(m2, a0), a1);
+        uint2 qa0 = cast8<FMT>(a0, s), qa1 = cast8<FMT>(a1, s);
+        qv[i] = make_uint4(qa0.x, qa0.y, qa1.x, qa1.y);
+    }
+    // tail (< 16 elements), exact and scalar
+    uint32_t mt = 0, badt = 0, satt = 0;
+    for (int64_t j = nunit * 16 + tid; j < n; j += stride) {
+        uint32_t h = xs[j];
+        float y = __fmul_rn(__uint_as_float(h << 16), s);
+        qs[j] = (uint8_t)(cvt2<FMT>(y, 0.0f) & 0xFFu);
+        uint32_t a = h & 0x7FFFu;
+        if (a < 0x7F80u) mt = a > mt ? a : mt; else ++badt;
+        if (fabsf(y) > fm) ++satt;
+    }
+    if (AMAX || COUNT) {
+        uint32_t m = amax_fast_final(m2), bad = 0, sat = 0;
+        const bool nonfinite = (m == 0xFFFFFFFFu);
+        const bool maybe_sat = COUNT && !nonfinite && __fmul_rn(bf16bits_to_float(m), s) > fm;
+        if (nonfinite || maybe_sat) {   // rare: redo this thread's units exactly
+            m = 0;
+            for (int64_t j = tid; j < nunit; j += stride) {
+                uint4 a0 = ld_stream(xv + 2 * j), a1 = ld_stream(xv + 2 * j + 1);
+                m = amax_exact8(amax_exact8(m, a0, bad), a1, bad);
+                if (COUNT) sat += count_sat8(a0, s, fm) + count_sat8(a1, s, fm);
+            }
+        }
+        m = mt > m ? mt : m;
+        bad += badt;
+        sat += satt;
+        m = block_max_u32(m, red);
+        if (COUNT) {
+            bad = block_sum_u32(bad, red);
+            sat = block_sum_u32(sat, red);
+        }
+        if (threadIdx.x == 0) {
+            if (AMAX) atomicMax(amax_bits, m << 16);
+            if (COUNT && nf_ctr && bad) atomicAdd(nf_ctr, bad);
+            if (COUNT && sat_ctr && sat) atomicAdd(sat_ctr, sat);
+        }
+    }
+}
+
+// ---------------------------------------- tensorwise cast with transpose --
+// 64x64 tiles: coalesced 16-byte bf16 loads, the FP8 codes written transposed
+// into shared memory, then coalesced 16-byte stores of the [cols, rows] output.
+template <int FMT, bool AMAX, bool COUNT>
+__global__ void __launch_bounds__(256)
+k_cast_transpose(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t rows, int64_t cols,
+                 const float *__restrict__ scale_in, const float *__restrict__ amax_in,
+                 float *__restrict__ scale_inv_out, uint32_t *__restrict__ amax_bits,
+                 uint32_t *__restrict__ nf_ctr, uint32_t *__restrict__ sat_ctr) {
+    __shared__ __align__(16) uint8_t tile[64][64 + 16];
+    __shared__ uint32_t red[32];
+    constexpr float fm = fmax_of<FMT>();
+    const float s = scale_in ? *scale_in : scale_from_amax(*amax_in, fm);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *scale_inv_out = __fdiv_rn(1.0f, s);
+    const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+    uint32_t m = 0, bad = 0, sat = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int u = threadIdx.x + h * 256;
+        const int row = u >> 3, cv = u & 7;
+        const int64_t gr = r0 + row, gc = c0 + cv * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (gr < rows && gc < cols) v = ld_stream(reinterpret_cast<const uint4 *>(x + gr * cols + gc));
+        if (AMAX || COUNT) {
+            m = amax_exact8(m, v, bad);
+            if (COUNT) sat += count_sat8(v, s, fm);
+        }
+        uint2 c = cast8<FMT>(v, s);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tile[cv * 8 + j][row] = (uint8_t)(c.x >> (8 * j));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tile[cv * 8 + 4 + j][row] = (uint8_t)(c.y >> (8 * j));
+    }
+    __syncthreads();
+    {
+        const int oc = threadIdx.x >> 2, part = threadIdx.x & 3;
+        const int64_t go = c0 + oc, gi = r0 + part * 16;
+        if (go < cols && gi < rows)
+            *reinterpret_cast<uint4 *>(qt + go * rows + gi) = *reinterpret_cast<const uint4 *>(&tile[oc][part * 16]);
+    }
+    if (AMAX || COUNT) {
+        m = block_max_u32(m, red);
+        if (COUNT) {
+            bad = block_sum_u32(bad, red);
+            sat = block_sum_u32(sat, red);
+        }
+        if (threadIdx.x == 0) {
+            if (AMAX) atomicMax(amax_bits, m << 16);
+            if (COUNT && nf_ctr && bad) atomicAdd(nf_ctr, bad);
+            if (COUNT && sat_ctr && sat) atomicAdd(sat_ctr, sat);
+        }
+    }
+}
+
+// --------------------------------------------------------------- rowwise --
+// One CTA (256 threads) per row, the row held in registers (V vectors of 8
+// per thread) between the amax and the cast: one HBM read per element.
+// V == 0: rows too long for registers, two passes (the second from L2).
+template <int FMT, bool POW2, int V>
+__global__ void __launch_bounds__(256)
+k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+          uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
+    __shared__ uint32_t red[32];
+    constexpr float fm = fmax_of<FMT>();
+    const int64_t ncv = cols / 8;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + r * ld);
+        uint2 *qr = reinterpret_cast<uint2 *>(q + r * cols);
+        uint32_t m;
+        if constexpr (V > 0) {
+            uint4 v[V];
+            uint32_t m2 = 0;
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                const int64_t cv = threadIdx.x + j * 256;
+                v[j] = cv < ncv ? ld_stream(xr + cv) : make_uint4(0, 0, 0, 0);
+                m2 = amax_fast8(m2, v[j]);
+            }
+            m = amax_fast_final(m2);
+            if (m == 0xFFFFFFFFu) {
+                uint32_t bad = 0;
+                m = 0;
+#pragma unroll
+                for (int j = 0; j < V; ++j) m = amax_exact8(m, v[j], bad);
+            }
+            m = block_max_u32(m, red);
+            const float a = bf16bits_to_float(m);
+            const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                const int64_t cv = threadIdx.x + j * 256;
+                if (cv < ncv) qr[cv] = cast8<FMT>(v[j], s);
+            }
+            if (threadIdx.x == 0) scale_inv[r] = __fdiv_rn(1.0f, s);
+        } else {
+            uint32_t bad = 0;
+            m = 0;
+            for (int64_t cv = threadIdx.x; cv < ncv; cv += 256) m = amax_exact8(m, ld_stream(xr + cv), bad);
+            m = block_max_u32(m, red);
+            const float a = bf16bits_to_float(m);
+            const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
+            for (int64_t cv = threadIdx.x; cv < ncv; cv += 256) qr[cv] = cast8<FMT>(xr[cv], s);
+            if (threadIdx.x == 0) scale_inv[r] = __fdiv_rn(1.0f, s);
+        }
+    }
+}
+
+// ---------------------------------------------------------- block 1x128 --
+// A half-warp per 1x128 block (16 lanes x 8 elements); each warp takes U
+// pairs of blocks per iteration so U 16-byte loads per lane are in flight.
+// Blocks are numbered row-major (row, kb); scale_inv is stored [kb][row].
+template <int FMT, int U>
+__global__ void __launch_bounds__(256)
+k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+             uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
+    constexpr float fm = fmax_of<FMT>();
+    const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
+    const int64_t nkb = (cols + 127) / 128;
+    const int64_t nblocks = rows * nkb;
+    const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t wb = warp * 2 * U; wb < nblocks; wb += nwarps * 2 * U) {
+        uint4 v[U];
+        int64_t row[U], cidx[U];
+        bool valid[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t b = wb + 2 * u + half;
+            row[u] = b / nkb;
+            const int64_t kb = b - row[u] * nkb;
+            cidx[u] = kb * 128 + l16 * 8;
+            valid[u] = (b < nblocks) && (cidx[u] < cols);
+            v[u] = valid[u] ? ld_stream(reinterpret_cast<const uint4 *>(x + row[u] * ld + cidx[u]))
+                            : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            uint32_t m = amax_fast_final(amax_fast8(0u, v[u]));
+            if (m == 0xFFFFFFFFu) {
+                uint32_t bad = 0;
+                m = amax_exact8(0u, v[u], bad);
+            }
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1) {
+                const uint32_t t = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+                m = t > m ? t : m;
+            }
+            const float s = scale_from_amax(bf16bits_to_float(m), fm);
+            if (valid[u]) *reinterpret_cast<uint2 *>(q + row[u] * cols + cidx[u]) = cast8<FMT>(v[u], s);
+            const int64_t b = wb + 2 * u + half;
+            if (l16 == 0 && b < nblocks) {
+                const int64_t kb = b - row[u] * nkb;
+                scale_inv[kb * rows + row[u]] = __fdiv_rn(1.0f, s);
+            }
+        }
+    }
+}
+
+// -------------------------------------------------------- block 128x128 --
+// One CTA (256 threads) per 128x128 tile, the tile held in registers (8
+// vectors of 8 per thread: 16 threads across a 128-wide row, 16 rows per
+// pass, 8 passes).
+template <int FMT>
+__global__ void __launch_bounds__(256)
+k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+           uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
+    __shared__ uint32_t red[32];
+    constexpr float fm = fmax_of<FMT>();
+    const int64_t nkb = (cols + 127) / 128, nrb = (rows + 127) / 128;
+    const int rsub = threadIdx.x >> 4, cv = threadIdx.x & 15;
+    for (int64_t t = blockIdx.x; t < nrb * nkb; t += gridDim.x) {
+        const int64_t rb = t / nkb, kb = t - rb * nkb;
+        const int64_t c = kb * 128 + cv * 8;
+        uint4 v[8];
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int64_t r = rb * 128 + p * 16 + rsub;
+            v[p] = (r < rows && c < cols) ? ld_stream(reinterpret_cast<const uint4 *>(x + r * ld + c))
+                                          : make_uint4(0, 0, 0, 0);
+            m2 = amax_fast8(m2, v[p]);
+        }
+        uint32_t m = amax_fast_final(m2);
+        if (m == 0xFFFFFFFFu) {
+            uint32_t bad = 0;
+            m = 0;
+#pragma unroll
+            for (int p = 0; p < 8; ++p) m = amax_exact8(m, v[p], bad);
+        }
+        m = block_max_u32(m, red);
+        const float s = scale_from_amax(bf16bits_to_float(m), fm);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int64_t r = rb * 128 + p * 16 + rsub;
+            if (r < rows && c < cols) *reinterpret_cast<uint2 *>(q + r * cols + c) = cast8<FMT>(v[p], s);
+        }
+        if (threadIdx.x == 0) scale_inv[rb * nkb + kb] = __fdiv_rn(1.0f, s);
+    }
+}
+
+int stream_grid(int sms, int64_t work_units, int threads) {
+    int64_t want = (work_units + threads - 1) / threads;
+    int64_t cap = (int64_t)sms * (2048 / threads);
+    return (int)std::max<int64_t>(1, std::min(want, cap));
+}
+
+template <int FMT>
+void launch_cast(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, const float *scale_in,
+                 const float *amax_in, uint8_t *q, int transpose_out, float *scale_inv,
+                 uint32_t *amax_bits, uint32_t *nf_ctr, uint32_t *sat_ctr) {
+    const bool amax = amax_bits != nullptr, count = nf_ctr != nullptr || sat_ctr != nullptr;
+    const uint16_t *xs = static_cast<const uint16_t *>(x);
+    if (transpose_out) {
+        dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+        if (amax && count) k_cast_transpose<FMT, true, true><<<grid, 256, 0, st>>>(xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+        else if (amax) k_cast_transpose<FMT, true, false><<<grid, 256, 0, st>>>(xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+        else if (count) k_cast_transpose<FMT, false, true><<<grid, 256, 0, st>>>(xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+        else k_cast_transpose<FMT, false, false><<<grid, 256, 0, st>>>(xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+        return;
+    }
+    const int64_t n = rows * cols, nunit = n / 16;
+    const int grid = stream_grid(sms, std::max<int64_t>(nunit / 2, 1), kStreamThreads);
+    const uint4 *xv = static_cast<const uint4 *>(x);
+    uint4 *qv = reinterpret_cast<uint4 *>(q);
+    if (amax && count) k_cast_tensor<FMT, true, true><<<grid, kStreamThreads, 0, st>>>(xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+    else if (amax) k_cast_tensor<FMT, true, false><<<grid, kStreamThreads, 0, st>>>(xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+    else if (count) k_cast_tensor<FMT, false, true><<<grid, kStreamThreads, 0, st>>>(xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+    else k_cast_tensor<FMT, false, false><<<grid, kStreamThreads, 0, st>>>(xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+}
+
+template <int FMT, bool POW2>
+void launch_rowwise(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, int64_t ld,
+                    uint8_t *q, float *scale_inv) {
+    const uint16_t *xs = static_cast<const uint16_t *>(x);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(rows, (int64_t)sms * 8));
+    const int64_t ncv = cols / 8;
+    if (ncv <= 256) k_rowwise<FMT, POW2, 1><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 512) k_rowwise<FMT, POW2, 2><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 1024) k_rowwise<FMT, POW2, 4><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 2048) k_rowwise<FMT, POW2, 8><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else k_rowwise<FMT, POW2, 0><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+}
+
+template <int FMT>
+void launch_block(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, int64_t ld,
+                  int block_rows, uint8_t *q, float *scale_inv) {
+    const uint16_t *xs = static_cast<const uint16_t *>(x);
+    const int64_t nkb = (cols + 127) / 128;
+    if (block_rows == 1) {
+        constexpr int U = 4;
+        const int64_t warps = (rows * nkb + 2 * U - 1) / (2 * U);
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sms * 8));
+        k_block1x128<FMT, U><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    } else {
+        const int64_t tiles = ((rows + 127) / 128) * nkb;
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)sms * 8));
+        k_block128<FMT><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    }
+}
+
+}  // namespace
+
+using namespace fp8q_host;
+
+extern "C" fp8_status fp8_amax(const void *x_bf16, int64_t n, float *amax, uint32_t *counts, void *stream) {
+    if (!amax || (n > 0 && !x_bf16)) return FP8_ERR_INVALID_ARG;
+    if (n < 0) return FP8_ERR_SHAPE;
+    if ((n > 0 && !aligned16(x_bf16)) || (reinterpret_cast<uintptr_t>(amax) & 3u) ||
+        (counts && (reinterpret_cast<uintptr_t>(counts) & 3u)))
+        return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemsetAsync(amax, 0, sizeof(float), s) != cudaSuccess) return FP8_ERR_CUDA;
+    const int64_t nvec = n / 8;
+    const int grid = stream_grid(sms, std::max<int64_t>(nvec / 4, 1), kStreamThreads);
+    k_amax<<<grid, kStreamThreads, 0, s>>>(static_cast<const uint4 *>(x_bf16), nvec,
+                                            static_cast<const uint16_t *>(x_bf16), n,
+                                            reinterpret_cast<uint32_t *>(amax), counts);
+    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+extern "C" fp8_status fp8_quantize_tensorwise(const void *x_bf16, int64_t rows, int64_t cols, fp8_format fmt,
+                                              const float *scale_in, uint8_t *q, int transpose_out,
+                                              float *scale_inv_out, float *amax_out, uint32_t *counts,
+                                              void *stream) {
+    if (rows < 0 || cols < 0) return FP8_ERR_SHAPE;
+    const int64_t n = rows * cols;
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (!scale_inv_out || (n > 0 && (!x_bf16 || !q))) return FP8_ERR_INVALID_ARG;
+    if (!scale_in && !amax_out) return FP8_ERR_INVALID_ARG;   // current scaling needs the amax buffer
+    if (transpose_out && ((rows % 16) || (cols % 16))) return FP8_ERR_SHAPE;
+    if (n > 0 && (!aligned16(x_bf16) || !aligned16(q))) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    cudaStream_t s = as_stream(stream);
+    uint32_t *amax_bits = reinterpret_cast<uint32_t *>(amax_out);
+    const float *amax_in = nullptr;
+    uint32_t *nf_ctr = counts, *sat_ctr = counts ? counts + 1 : nullptr;
+    if (!scale_in) {
+        // Current scaling: an amax pass first (fills amax_out and counts the
+        // non-finite inputs), then the cast pass reads the amax back.
+        fp8_status a = fp8_amax(x_bf16, n, amax_out, counts, stream);
+        if (a != FP8_OK) return a;
+        amax_in = amax_out;
+        amax_bits = nullptr;
+        nf_ctr = nullptr;
+    } else if (amax_bits) {
+        if (cudaMemsetAsync(amax_bits, 0, sizeof(float), s) != cudaSuccess) return FP8_ERR_CUDA;
+    }
+    if (fmt == FP8_E4M3)
+        launch_cast<FP8_E4M3>(s, sms, x_bf16, rows, cols, scale_in, amax_in, q, transpose_out, scale_inv_out, amax_bits, nf_ctr, sat_ctr);
+    else
+        launch_cast<FP8_E5M2>(s, sms, x_bf16, rows, cols, scale_in, amax_in, q, transpose_out, scale_inv_out, amax_bits, nf_ctr, sat_ctr);
+    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+extern "C" fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                           fp8_format fmt, int pow2, uint8_t *q, float *scale_inv,
+                                           void *stream) {
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return FP8_ERR_SHAPE;
+    if (cols % 16) return FP8_ERR_SHAPE;
+    if (rows == 0 || cols == 0) {
+        if (rows > 0 && !scale_inv) return FP8_ERR_INVALID_ARG;
+    } else if (!x_bf16 || !q || !scale_inv) {
+        return FP8_ERR_INVALID_ARG;
+    }
+    if (ld % 8) return FP8_ERR_ALIGNMENT;
+    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q))) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (rows == 0) return FP8_OK;
+    cudaStream_t s = as_stream(stream);
+    if (fmt == FP8_E4M3) {
+        if (pow2) launch_rowwise<FP8_E4M3, true>(s, sms, x_bf16, rows, cols, ld, q, scale_inv);
+        else launch_rowwise<FP8_E4M3, false>(s, sms, x_bf16, rows, cols, ld, q, scale_inv);
+    } else {
+        if (pow2) launch_rowwise<FP8_E5M2, true>(s, sms, x_bf16, rows, cols, ld, q, scale_inv);
+        else launch_rowwise<FP8_E5M2, false>(s, sms, x_bf16, rows, cols, ld, q, scale_inv);
+    }
+    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+extern "C" fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                             fp8_format fmt, int block_rows, uint8_t *q, float *scale_inv,
+                                             void *stream) {
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (block_rows != 1 && block_rows != 128) return FP8_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols || (cols % 16)) return FP8_ERR_SHAPE;
+    if (rows > 0 && cols > 0 && (!x_bf16 || !q || !scale_inv)) return FP8_ERR_INVALID_ARG;
+    if (ld % 8) return FP8_ERR_ALIGNMENT;
+    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q))) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (rows == 0 || cols == 0) return FP8_OK;
+    cudaStream_t s = as_stream(stream);
+    if (fmt == FP8_E4M3) launch_block<FP8_E4M3>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv);
+    else launch_block<FP8_E5M2>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv);
+    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}

@@ -1,0 +1,249 @@
+"""Python binding of the C ABI in ``include/fp8q.h`` (``libfp8q.so``).
+
+Argument marshalling only: every function here checks tensor dtypes, devices
+and contiguity, passes raw device pointers and the current CUDA stream to the
+library function of the same name, and raises :class:`Fp8Error` on a non-OK
+status.  All arithmetic runs in the library's CUDA kernels; there is no CPU or
+PyTorch fallback -- if the library is missing the first call raises.
+
+The ``quantize_*`` / ``gemm`` / ``kv_*`` helpers at the bottom only allocate
+the outputs with torch (device memory) and call the raw entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8q.so")
+
+E4M3 = 0
+E5M2 = 1
+SCALE_TENSOR = 0
+SCALE_ROW = 1
+SCALE_BLOCK = 2
+FMAX = {E4M3: 448.0, E5M2: 57344.0}
+
+# every symbol the header declares, with (restype, argtypes)
+_P, _I64, _I, _F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+_S = ctypes.c_int
+SIGNATURES = {
+    "fp8_status_string": (ctypes.c_char_p, [_S]),
+    "fp8_amax": (_S, [_P, _I64, _P, _P, _P]),
+    "fp8_quantize_tensorwise": (_S, [_P, _I64, _I64, _I, _P, _P, _I, _P, _P, _P, _P]),
+    "fp8_quantize_rowwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
+    "fp8_quantize_blockwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
+    "fp8_gemm_scaled": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
+    "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
+    "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
+    "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
+    "fp8_device_error": (_S, [_P, _I]),
+}
+
+
+class Fp8Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = lib().fp8_status_string(status)
+        super().__init__(f"{fn} failed: {msg.decode() if msg else status}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libfp8q.so`` (built in-tree by ``build.py``); raise if absent."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(
+                        f"{LIB_PATH} is missing: build it with "
+                        "`python -m fp8_scaled_quantization_amax_b200.build` (no fallback exists)")
+                L = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in SIGNATURES.items():
+                    f = getattr(L, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = L
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(name, status):
+    if status != 0:
+        raise Fp8Error(name, status)
+
+
+def _dev(t, dtype, what):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{what}: must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{what}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: must be contiguous")
+
+
+# ------------------------------------------------------- raw entry points --
+
+def fp8_amax(x, amax, counts=None, stream=None):
+    _dev(x, torch.bfloat16, "x"); _dev(amax, torch.float32, "amax"); _dev(counts, torch.int32, "counts")
+    _check("fp8_amax", lib().fp8_amax(_ptr(x), x.numel(), _ptr(amax), _ptr(counts), _stream(stream)))
+
+
+def fp8_quantize_tensorwise(x, rows, cols, fmt, scale_in, q, transpose_out, scale_inv_out,
+                            amax_out=None, counts=None, stream=None):
+    _dev(x, torch.bfloat16, "x"); _dev(q, torch.uint8, "q")
+    _dev(scale_in, torch.float32, "scale_in"); _dev(scale_inv_out, torch.float32, "scale_inv_out")
+    _dev(amax_out, torch.float32, "amax_out"); _dev(counts, torch.int32, "counts")
+    _check("fp8_quantize_tensorwise", lib().fp8_quantize_tensorwise(
+        _ptr(x), rows, cols, fmt, _ptr(scale_in), _ptr(q), int(transpose_out), _ptr(scale_inv_out),
+        _ptr(amax_out), _ptr(counts), _stream(stream)))
+
+
+def fp8_quantize_rowwise(x, rows, cols, ld, fmt, pow2, q, scale_inv, stream=None):
+    _dev(x, torch.bfloat16, "x"); _dev(q, torch.uint8, "q"); _dev(scale_inv, torch.float32, "scale_inv")
+    _check("fp8_quantize_rowwise", lib().fp8_quantize_rowwise(
+        _ptr(x), rows, cols, ld, fmt, int(pow2), _ptr(q), _ptr(scale_inv), _stream(stream)))
+
+
+def fp8_quantize_blockwise(x, rows, cols, ld, fmt, block_rows, q, scale_inv, stream=None):
+    _dev(x, torch.bfloat16, "x"); _dev(q, torch.uint8, "q"); _dev(scale_inv, torch.float32, "scale_inv")
+    _check("fp8_quantize_blockwise", lib().fp8_quantize_blockwise(
+        _ptr(x), rows, cols, ld, fmt, block_rows, _ptr(q), _ptr(scale_inv), _stream(stream)))
+
+
+def fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, ldd, stream=None):
+    _dev(A, torch.uint8, "A"); _dev(B, torch.uint8, "B"); _dev(D, torch.bfloat16, "D")
+    _dev(a_scale_inv, torch.float32, "a_scale_inv"); _dev(b_scale_inv, torch.float32, "b_scale_inv")
+    _check("fp8_gemm_scaled", lib().fp8_gemm_scaled(
+        _ptr(A), fa, _ptr(B), fb, M, N, K, mode, _ptr(a_scale_inv), _ptr(b_scale_inv), _ptr(D), ldd,
+        _stream(stream)))
+
+
+def fp8_amax_history_update(history, pos, amax_cur, fmt, scale, scale_inv, saturated, stream=None):
+    _dev(history, torch.float32, "history"); _dev(pos, torch.int32, "pos")
+    _dev(amax_cur, torch.float32, "amax_cur"); _dev(scale, torch.float32, "scale")
+    _dev(scale_inv, torch.float32, "scale_inv"); _dev(saturated, torch.int32, "saturated")
+    _check("fp8_amax_history_update", lib().fp8_amax_history_update(
+        _ptr(history), _ptr(pos), history.numel(), _ptr(amax_cur), fmt, _ptr(scale), _ptr(scale_inv),
+        _ptr(saturated), _stream(stream)))
+
+
+def fp8_kv_quant(kv, B, H, S, Dh, fmt, q, scale_inv, stream=None):
+    _dev(kv, torch.bfloat16, "kv"); _dev(q, torch.uint8, "q"); _dev(scale_inv, torch.float32, "scale_inv")
+    _check("fp8_kv_quant", lib().fp8_kv_quant(_ptr(kv), B, H, S, Dh, fmt, _ptr(q), _ptr(scale_inv),
+                                              _stream(stream)))
+
+
+def fp8_kv_dequant(q, scale_inv, B, H, S, Dh, fmt, out, stream=None):
+    _dev(q, torch.uint8, "q"); _dev(scale_inv, torch.float32, "scale_inv"); _dev(out, torch.bfloat16, "out")
+    _check("fp8_kv_dequant", lib().fp8_kv_dequant(_ptr(q), _ptr(scale_inv), B, H, S, Dh, fmt, _ptr(out),
+                                                  _stream(stream)))
+
+
+def fp8_device_error(clear: bool = False) -> int:
+    v = ctypes.c_uint32(0)
+    _check("fp8_device_error", lib().fp8_device_error(ctypes.byref(v), int(clear)))
+    return int(v.value)
+
+
+# ------------------------------------------------ allocating conveniences --
+
+def amax(x, counts=None):
+    out = torch.empty(1, dtype=torch.float32, device=x.device)
+    fp8_amax(x, out, counts)
+    return out
+
+
+def quantize_tensorwise(x, fmt=E4M3, scale_in=None, transpose=False, counts=None, want_amax=True):
+    """Returns (q, scale_inv[1], amax[1] or None).  x is 2-D [rows, cols] or 1-D."""
+    rows, cols = (1, x.numel()) if x.dim() == 1 else tuple(x.shape)
+    q = torch.empty((cols, rows) if transpose else (rows, cols), dtype=torch.uint8, device=x.device)
+    if x.dim() == 1 and not transpose:
+        q = q.view(-1)
+    sinv = torch.empty(1, dtype=torch.float32, device=x.device)
+    am = torch.empty(1, dtype=torch.float32, device=x.device) if (want_amax or scale_in is None) else None
+    fp8_quantize_tensorwise(x, rows, cols, fmt, scale_in, q, transpose, sinv, am, counts)
+    return q, sinv, am
+
+
+def quantize_rowwise(x, fmt=E4M3, pow2=True):
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    sinv = torch.empty(rows, dtype=torch.float32, device=x.device)
+    fp8_quantize_rowwise(x, rows, cols, x.stride(0), fmt, pow2, q, sinv)
+    return q, sinv
+
+
+def quantize_blockwise(x, fmt=E4M3, block_rows=1):
+    rows, cols = x.shape
+    nkb = (cols + 127) // 128
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if block_rows == 1:
+        sinv = torch.empty((nkb, rows), dtype=torch.float32, device=x.device)
+    else:
+        sinv = torch.empty(((rows + block_rows - 1) // block_rows, nkb), dtype=torch.float32, device=x.device)
+    fp8_quantize_blockwise(x, rows, cols, x.stride(0), fmt, block_rows, q, sinv)
+    return q, sinv
+
+
+def gemm(A, fa, B, fb, mode, a_scale_inv, b_scale_inv, out=None):
+    M, K = A.shape
+    N = B.shape[0]
+    D = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, D.stride(0))
+    return D
+
+
+def kv_quant(kv, fmt=E4M3):
+    B, H, S, Dh = kv.shape
+    q = torch.empty(kv.shape, dtype=torch.uint8, device=kv.device)
+    sinv = torch.empty(B * H, dtype=torch.float32, device=kv.device)
+    fp8_kv_quant(kv, B, H, S, Dh, fmt, q, sinv)
+    return q, sinv
+
+
+def kv_dequant(q, scale_inv, fmt=E4M3):
+    B, H, S, Dh = q.shape
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    fp8_kv_dequant(q, scale_inv, B, H, S, Dh, fmt, out)
+    return out
+
+
+class AmaxHistory:
+    """Device-resident delayed-scaling state (history ring, position, scale)."""
+
+    def __init__(self, length: int, fmt: int, device="cuda"):
+        self.fmt = fmt
+        self.history = torch.zeros(length, dtype=torch.float32, device=device)
+        self.pos = torch.zeros(1, dtype=torch.int32, device=device)
+        self.scale = torch.ones(1, dtype=torch.float32, device=device)
+        self.scale_inv = torch.ones(1, dtype=torch.float32, device=device)
+        self.saturated = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def update(self, amax_cur):
+        fp8_amax_history_update(self.history, self.pos, amax_cur, self.fmt, self.scale, self.scale_inv,
+                                self.saturated)

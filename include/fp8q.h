@@ -1,0 +1,204 @@
+/*
+ * fp8q.h -- C ABI of the FP8 scaled-quantization library for NVIDIA B200
+ * (sm_100a): amax -> scale -> saturating RNE cast to E4M3 / E5M2 -> FP8
+ * scaled GEMM with fp32 accumulation and a bf16 epilogue, plus the
+ * delayed-scaling amax-history update and the FP8 KV-cache quantize /
+ * dequantize.
+ *
+ * Sources (web pages on FP8 scaled quantization):
+ *   [DeepL]  "DeepL押注FP8：大模型训练与推理统一精度实战解析"
+ *   [H100]   "H100 FP8加速实测：新一代计算架构的飞跃"
+ *   [Soup]   "FP8训练与QAT量化感知训练：如何在Hopper GPU上用Soup把大模型微调提速2倍"
+ *   Format bit semantics not fixed by the pages follow the OCP 8-bit
+ *   floating point specification (E4M3: max 448, no Inf; E5M2: max 57344).
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is DEVICE memory owned by the caller (allocate it
+ *     with cudaMalloc, torch, ...).  The library allocates nothing on the
+ *     device, keeps no per-call state and never synchronises the host.
+ *   - bf16 tensors are raw 16-bit bfloat16 words; FP8 tensors are one byte per
+ *     element (the format's code); scales are IEEE fp32.
+ *   - "scale" s multiplies before the cast (q = cast(x * s)); "scale_inv"
+ *     d = 1 / s is what the GEMM and the dequantizer multiply by.
+ *   - Layouts are row-major.  Data pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously; the return value covers argument validation
+ *     and the launch only.  Data-dependent events (non-finite inputs,
+ *     saturation) are reported through the optional device counters.
+ *   - Errors: FP8_ERR_INVALID_ARG (null pointer, bad enum), FP8_ERR_SHAPE
+ *     (negative or unsupported extents), FP8_ERR_ALIGNMENT (pointer or
+ *     leading dimension not aligned as stated), FP8_ERR_UNSUPPORTED_DEVICE
+ *     (the current device is not compute capability 10.0), FP8_ERR_CUDA (a
+ *     CUDA runtime call failed; the CUDA error is left for the caller).
+ *     Nothing is enqueued when a call returns an error.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8Q_API __attribute__((visibility("default")))
+#else
+#define FP8Q_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8_OK = 0,
+    FP8_ERR_INVALID_ARG = 1,
+    FP8_ERR_SHAPE = 2,
+    FP8_ERR_ALIGNMENT = 3,
+    FP8_ERR_UNSUPPORTED_DEVICE = 4,
+    FP8_ERR_CUDA = 5
+} fp8_status;
+
+/* [DeepL] §2.1: E4M3 (1-4-3 bits) for forward weights and activations, E5M2
+ * (1-5-2 bits, range +-57344 per [H100]) for gradients. */
+typedef enum { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_format;
+
+/* [DeepL] §2.3 scaling granularity; [Soup] "FP8 三种缩放配方怎么选". */
+typedef enum { FP8_SCALE_TENSOR = 0, FP8_SCALE_ROW = 1, FP8_SCALE_BLOCK = 2 } fp8_scale_mode;
+
+/* Human-readable name of a status code (static string). */
+FP8Q_API const char *fp8_status_string(fp8_status s);
+
+/*
+ * amax = max |x| over the finite elements of a bf16 tensor ([DeepL] §4.2:
+ * the maximum absolute value per tensor).  NaN and +-Inf are excluded and
+ * counted.
+ *   x_bf16  [n] bf16, 16-byte aligned;  n >= 0 (n == 0 gives amax 0).
+ *   amax    [1] fp32, overwritten.
+ *   counts  [2] uint32 or NULL: counts[0] += number of non-finite elements.
+ */
+FP8Q_API fp8_status fp8_amax(const void *x_bf16, int64_t n, float *amax, uint32_t *counts, void *stream);
+
+/*
+ * Per-tensor quantization ([DeepL] §2.3 per-tensor scaling; [Soup] tensorwise
+ * recipe) of a [rows, cols] bf16 tensor.
+ *   scale_in == NULL : current scaling.  amax_out receives amax(x) and
+ *                      s = fmax / amax (amax == 0 gives 1; overflow clamps
+ *                      to FLT_MAX).  amax_out is REQUIRED in this mode.
+ *   scale_in != NULL : delayed scaling ([DeepL] §2.3): s = *scale_in (from
+ *                      the amax history); amax_out (may be NULL) receives this
+ *                      tensor's amax for the next history update.
+ *   q             [rows, cols] FP8, or [cols, rows] when transpose_out != 0
+ *                 (the transposed copy feeds the GEMM's B operand when the
+ *                 weight is needed as W^T, e.g. a data-gradient GEMM).
+ *   scale_inv_out [1] fp32: d = 1 / s.
+ *   counts        [2] uint32 or NULL: [0] += non-finite inputs,
+ *                 [1] += elements with |x * s| > fmax (saturated).
+ *   Cast: q = RNE(fp32(x) * s) with saturation to +-fmax; NaN stays NaN.
+ *   Shapes: rows, cols >= 0.  transpose_out requires rows % 16 == 0 and
+ *   cols % 16 == 0.
+ */
+FP8Q_API fp8_status fp8_quantize_tensorwise(const void *x_bf16, int64_t rows, int64_t cols, fp8_format fmt,
+                                   const float *scale_in, uint8_t *q, int transpose_out,
+                                   float *scale_inv_out, float *amax_out, uint32_t *counts,
+                                   void *stream);
+
+/*
+ * Per-row quantization ([DeepL] §2.3 per-row scaling; [Soup] rowwise recipe
+ * with e4m3 and power-of-two scales) of x [rows, cols] with leading
+ * dimension ld (elements).  pow2 != 0: s_r = the largest power of two with
+ * amax_r * s_r <= fmax; pow2 == 0: s_r = fmax / amax_r.
+ *   q          [rows, cols] FP8, dense.
+ *   scale_inv  [rows] fp32, d_r = 1 / s_r.
+ *   Shapes: cols % 16 == 0, ld % 8 == 0, ld >= cols.
+ */
+FP8Q_API fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                fp8_format fmt, int pow2, uint8_t *q, float *scale_inv,
+                                void *stream);
+
+/*
+ * Per-block quantization ([DeepL] §2.3: the tensor is cut into small blocks
+ * with one scale each) of x [rows, cols] (leading dimension ld).  Blocks are
+ * block_rows x 128: block_rows = 1 for activations (1x128), 128 for weights
+ * (128x128).  Edge blocks use their valid elements.  s = fmax / amax_block.
+ *   q          [rows, cols] FP8, dense.
+ *   scale_inv  block_rows == 1  : [ceil(cols/128), rows]  (row index fastest,
+ *                                  the layout the GEMM reads per K block);
+ *              block_rows == 128: [ceil(rows/128), ceil(cols/128)].
+ *   Shapes: cols % 16 == 0, ld % 8 == 0, ld >= cols.
+ */
+FP8Q_API fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                  fp8_format fmt, int block_rows, uint8_t *q, float *scale_inv,
+                                  void *stream);
+
+/*
+ * FP8 scaled GEMM ([H100]: the multiply-accumulate runs on FP8 operands on
+ * the tensor cores; [Soup] tensorwise / rowwise scaled matmuls; per-block
+ * scales per [DeepL] §2.3):
+ *   D[m, n] = bf16( scales * sum_k A[m, k] * B[n, k] ), fp32 accumulation.
+ *   A  [M, K] FP8 (format fa), K contiguous.   B [N, K] FP8 (format fb), K
+ *   contiguous (an nn.Linear weight [out, in]).  fa and fb may differ
+ *   (E5M2 gradient x E4M3 weight).
+ *   mode TENSOR: a_scale_inv [1], b_scale_inv [1]:  D = da*db*acc.
+ *   mode ROW   : a_scale_inv [M], b_scale_inv [N]:  D = da[m]*db[n]*acc.
+ *   mode BLOCK : a_scale_inv [ceil(K/128), M] (1x128 blocks of A),
+ *                b_scale_inv [ceil(N/128), ceil(K/128)] (128x128 blocks of B):
+ *                D = sum_kb da[kb, m] * db[n/128, kb] * acc_kb  (each 128-wide
+ *                K block accumulated on the tensor cores, then promoted into
+ *                an fp32 register accumulator with its two scales).
+ *   D  [M, N] bf16 with leading dimension ldd (elements).
+ *   The result is deterministic (fixed K order, no split-K).
+ *   Shapes: M, N, K >= 0; K % 16 == 0; N % 8 == 0; ldd % 8 == 0, ldd >= N.
+ *   K == 0 writes zeros.
+ */
+FP8Q_API fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
+                           int64_t M, int64_t N, int64_t K, fp8_scale_mode mode,
+                           const float *a_scale_inv, const float *b_scale_inv, void *D_bf16,
+                           int64_t ldd, void *stream);
+
+/*
+ * Delayed-scaling update ([DeepL] §2.3: the scale of a step is predicted
+ * from the statistics of previous steps; a deviation above a threshold
+ * forces recomputation).  In order:
+ *   *saturated = (amax_cur * scale_t > fmax)   [the scale in use could not
+ *                                               represent this step's amax]
+ *   history[*pos] = amax_cur;  *pos = (*pos + 1) % len;
+ *   *scale = fmax / max(history) (1 if the max is 0);  *scale_inv = 1 / *scale.
+ *   history [len] fp32, pos [1] int32, amax_cur [1] fp32, scale / scale_inv
+ *   [1] fp32 (scale is read as scale_t, then overwritten), saturated [1]
+ *   uint32.  1 <= len <= 1024.  The state (history, pos, scale) is the whole
+ *   checkpoint.
+ */
+FP8Q_API fp8_status fp8_amax_history_update(float *history, int32_t *pos, int len, const float *amax_cur,
+                                   fp8_format fmt, float *scale, float *scale_inv,
+                                   uint32_t *saturated, void *stream);
+
+/*
+ * FP8 KV-cache quantization ([DeepL] §3.1: K and V stored in FP8 halve the
+ * cache).  kv [B, H, S, Dh] bf16; each (b, h) slice of S*Dh elements gets a
+ * per-tensor scale s = fmax / amax(slice).
+ *   q          [B, H, S, Dh] FP8.   scale_inv [B*H] fp32.
+ *   Shapes: (S*Dh) % 16 == 0, B*H <= 65535.
+ */
+FP8Q_API fp8_status fp8_kv_quant(const void *kv_bf16, int64_t B, int64_t H, int64_t S, int64_t Dh,
+                        fp8_format fmt, uint8_t *q, float *scale_inv, void *stream);
+
+/*
+ * FP8 KV-cache dequantization when the cache is read ([DeepL] §3.1):
+ *   out = bf16_RNE(fp32(q) * scale_inv[b*H + h]).
+ *   q [B, H, S, Dh] FP8, scale_inv [B*H], out [B, H, S, Dh] bf16.
+ *   Shapes: (S*Dh) % 16 == 0, B*H <= 65535.
+ */
+FP8Q_API fp8_status fp8_kv_dequant(const uint8_t *q, const float *scale_inv, int64_t B, int64_t H,
+                          int64_t S, int64_t Dh, fp8_format fmt, void *out_bf16, void *stream);
+
+/*
+ * Device error word of the library on the current device: a bit is set when
+ * a kernel gave up a bounded wait (a pipeline barrier that did not complete
+ * within about one second) and returned early instead of hanging.  0 means
+ * no such event.  Synchronises the current device.  clear != 0 resets it.
+ */
+FP8Q_API fp8_status fp8_device_error(uint32_t *host_out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol ``include/fp8q.h`` declares, and rejects bad arguments before
+touching the device; with no device a valid call fails loudly (no fallback)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from fp8_scaled_quantization_amax_b200 import fp8q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8q.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUPPORTED, CUDA = range(6)
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return re.findall(r"^FP8Q_API\s+[^;(]*?\b(fp8_\w+)\s*\(", txt, flags=re.M)
+
+
+def test_header_declares_the_abi():
+    names = declared_symbols()
+    assert len(names) == len(set(names)) >= 10
+    assert set(names) == set(fp8q.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol():
+    L = fp8q.lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    L = fp8q.lib()
+    for s in range(6):
+        assert L.fp8_status_string(s)
+    assert b"sm_100a" in L.fp8_status_string(UNSUPPORTED)
+    assert L.fp8_status_string(99) == b"FP8_ERR_UNKNOWN"
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)          # a 16-byte aligned non-null address never dereferenced
+FAKE_ODD = P(0x10002)
+
+
+def test_validation_before_device_access():
+    L = fp8q.lib()
+    n = P(0)
+    # GEMM: bad format, bad mode, K % 16, N % 8, null D, misaligned A
+    assert L.fp8_gemm_scaled(FAKE, 3, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 64, n) == INVALID
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 5, FAKE, FAKE, FAKE, 64, n) == INVALID
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 40, 0, FAKE, FAKE, FAKE, 64, n) == SHAPE
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 60, 64, 0, FAKE, FAKE, FAKE, 64, n) == ALIGN
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, None, 64, n) == INVALID
+    assert L.fp8_gemm_scaled(FAKE_ODD, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 64, n) == ALIGN
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, -1, 64, 64, 0, FAKE, FAKE, FAKE, 64, n) == SHAPE
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 32, n) == SHAPE  # ldd < N
+    # quantizers
+    assert L.fp8_quantize_rowwise(FAKE, 4, 24, 32, 0, 1, FAKE, FAKE, n) == SHAPE
+    assert L.fp8_quantize_rowwise(FAKE, 4, 16, 20, 0, 1, FAKE, FAKE, n) == ALIGN
+    assert L.fp8_quantize_rowwise(FAKE, 4, 16, 16, 2, 1, FAKE, FAKE, n) == INVALID
+    assert L.fp8_quantize_blockwise(FAKE, 4, 32, 32, 0, 64, FAKE, FAKE, n) == INVALID
+    assert L.fp8_quantize_tensorwise(FAKE, 4, 32, 0, None, FAKE, 0, FAKE, None, None, n) == INVALID
+    assert L.fp8_quantize_tensorwise(FAKE, 4, 40, 0, FAKE, FAKE, 1, FAKE, None, None, n) == SHAPE
+    assert L.fp8_amax(FAKE_ODD, 100, FAKE, None, n) == ALIGN
+    assert L.fp8_amax(FAKE, -1, FAKE, None, n) == SHAPE
+    assert L.fp8_amax(FAKE, 10, None, None, n) == INVALID
+    # KV cache and history
+    assert L.fp8_kv_quant(FAKE, 2, 2, 3, 5, 0, FAKE, FAKE, n) == SHAPE
+    assert L.fp8_kv_dequant(FAKE, FAKE, 2, 2, 16, 8, 7, FAKE, n) == INVALID
+    assert L.fp8_amax_history_update(FAKE, FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
+    assert L.fp8_amax_history_update(FAKE, FAKE, 2000, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
+    assert L.fp8_amax_history_update(None, FAKE, 16, FAKE, 0, FAKE, FAKE, FAKE, n) == INVALID
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_fails_loudly():
+    L = fp8q.lib()
+    st = L.fp8_amax(FAKE, 64, FAKE, None, P(0))
+    assert st in (UNSUPPORTED, CUDA)
+    with pytest.raises((fp8q.Fp8Error, RuntimeError, ValueError)):
+        fp8q.amax(torch.zeros(64, dtype=torch.bfloat16))

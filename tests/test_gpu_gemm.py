@@ -1,0 +1,179 @@
+"""GPU parity of the FP8 scaled GEMM (tcgen05 kernel) against the CPU oracle.
+
+The FP8 operands and scales fed to BOTH sides come from the oracle's own
+quantizer applied to seeded bf16 inputs (never from the CUDA path).  The
+oracle sums exact products in fp64; the tolerance per element is
+1e-2 x sum_k |a_k b_k| (scaled) plus the bf16 rounding of the output.
+
+Sources: "H100 FP8加速实测：新一代计算架构的飞跃" (FP8 multiply-accumulate on
+tensor cores); "FP8训练与QAT量化感知训练：…用Soup把大模型微调提速2倍", section
+"FP8 三种缩放配方怎么选" (tensorwise / rowwise scaled matmul);
+"DeepL押注FP8：大模型训练与推理统一精度实战解析" §2.1 (E5M2 gradients x E4M3
+weights), §2.3 (per-block scales), §5.3 (determinism).
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_scaled_quantization_amax_b200 import fp8q, inputs
+from tests.gpu_util import assert_gemm_close, bf16_to_f64, need_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    need_gpu()
+    yield
+    assert fp8q.fp8_device_error(clear=True) == 0
+
+
+def _cuda(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda")
+
+
+def _operands(orc, mode, M, N, K, fa=0, fb=0, seed=0, wstd=0.02):
+    """Oracle-quantized operands: A from N(0,1) activations, B from N(0,wstd) weights."""
+    a_bits = inputs.bf16_bits(inputs.normal_bf16((M, K), 1.0, seed=seed))
+    b_bits = inputs.bf16_bits(inputs.normal_bf16((N, K), wstd, seed=seed + 1))
+    if mode == orc.SCALE_TENSOR:
+        A, da, _, _ = orc.quantize_tensorwise(a_bits, fa)
+        B, db, _, _ = orc.quantize_tensorwise(b_bits, fb)
+        da, db = np.float32([da]), np.float32([db])
+    elif mode == orc.SCALE_ROW:
+        A, da = orc.quantize_rowwise(a_bits, fa, True)
+        B, db = orc.quantize_rowwise(b_bits, fb, True)
+    else:
+        A, da = orc.quantize_blockwise(a_bits, fa, 1)
+        B, db = orc.quantize_blockwise(b_bits, fb, 128)
+    return A, da, B, db
+
+
+def _run(A, fa, B, fb, mode, da, db):
+    return fp8q.gemm(_cuda(A), fa, _cuda(B), fb, mode, _cuda(da), _cuda(db))
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("shape", [(256, 256, 256), (300, 272, 400), (128, 512, 1024), (1, 8, 16),
+                                   (129, 264, 144), (520, 776, 640)])
+def test_gemm_full_compare(orc, mode, shape):
+    M, N, K = shape
+    A, da, B, db = _operands(orc, mode, M, N, K, seed=M + N + K)
+    D = _run(A, 0, B, 0, mode, da, db)
+    ref, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
+    assert_gemm_close(bf16_to_f64(D), ref, mag)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_gemm_e5m2_grad_times_e4m3_weight(orc, mode):
+    M, N, K = 264, 320, 512
+    g = inputs.bf16_bits(inputs.lognormal_grads_bf16((M, K), seed=7))
+    w = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, seed=8))
+    if mode == 0:
+        A, da, _, _ = orc.quantize_tensorwise(g, 1)
+        B, db, _, _ = orc.quantize_tensorwise(w, 0)
+        da, db = np.float32([da]), np.float32([db])
+    elif mode == 1:
+        A, da = orc.quantize_rowwise(g, 1, True)
+        B, db = orc.quantize_rowwise(w, 0, True)
+    else:
+        A, da = orc.quantize_blockwise(g, 1, 1)
+        B, db = orc.quantize_blockwise(w, 0, 128)
+    D = _run(A, 1, B, 0, mode, da, db)
+    ref, mag = orc.gemm_scaled(A, 1, B, 0, mode, da, db)
+    assert_gemm_close(bf16_to_f64(D), ref, mag)
+
+
+def test_gemm_integer_values_exact(orc):
+    """Codes of small integers with unit scales: every partial sum is an
+    integer below 2^24, so the GPU result is exact (up to bf16 output)."""
+    rng = np.random.default_rng(3)
+    M, N, K = 192, 264, 384
+    enc = {v: orc.encode(float(v), 0) for v in range(-16, 17)}
+    va = rng.integers(-16, 17, (M, K))
+    vb = rng.integers(-16, 17, (N, K))
+    A = np.vectorize(enc.get)(va).astype(np.uint8)
+    B = np.vectorize(enc.get)(vb).astype(np.uint8)
+    one = np.ones(1, np.float32)
+    D = _run(A, 0, B, 0, 0, one, one)
+    exact = (va @ vb.T).astype(np.float32)
+    bf = torch.from_numpy(exact).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(D.float().cpu().numpy(), bf)
+
+
+def test_gemm_identity_weight(orc):
+    K = 256
+    A, da, _, _ = orc.quantize_tensorwise(inputs.bf16_bits(inputs.normal_bf16((200, K), 1.0, seed=9)), 0)
+    B = np.zeros((K, K), np.uint8)
+    B[np.arange(K), np.arange(K)] = 0x38      # 1.0
+    D = _run(A, 0, B, 0, 0, np.float32([da]), np.float32([1.0]))
+    t = orc.decode_table(0)
+    ref = torch.from_numpy((t[A] * np.float64(np.float32(da))).astype(np.float32)).to(torch.bfloat16)
+    assert torch.equal(D.cpu(), ref)
+
+
+def test_gemm_deterministic_and_zero_k(orc):
+    A, da, B, db = _operands(orc, 1, 384, 512, 1024, seed=4)
+    D1 = _run(A, 0, B, 0, 1, da, db)
+    D2 = _run(A, 0, B, 0, 1, da, db)
+    assert torch.equal(D1, D2)
+    D0 = torch.full((5, 16), 7.0, dtype=torch.bfloat16, device="cuda")
+    z = torch.empty((5, 0), dtype=torch.uint8, device="cuda")
+    fp8q.fp8_gemm_scaled(z, 0, torch.empty((16, 0), dtype=torch.uint8, device="cuda"), 0, 5, 16, 0, 0,
+                         torch.ones(1, device="cuda"), torch.ones(1, device="cuda"), D0, 16)
+    assert torch.count_nonzero(D0).item() == 0
+
+
+def test_gemm_invalid_shapes_rejected():
+    A = torch.zeros((64, 40), dtype=torch.uint8, device="cuda")
+    s = torch.ones(64, device="cuda")
+    D = torch.empty((64, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fp8q.Fp8Error, match="SHAPE"):
+        fp8q.fp8_gemm_scaled(A, 0, A, 0, 64, 64, 40, 1, s, s, D, 64)      # K % 16
+    with pytest.raises(fp8q.Fp8Error, match="ALIGNMENT"):
+        fp8q.fp8_gemm_scaled(A, 0, A, 0, 64, 60, 32, 1, s, s, D, 64)      # N % 8
+    with pytest.raises(fp8q.Fp8Error, match="INVALID_ARG"):
+        fp8q.fp8_gemm_scaled(A, 0, A, 0, 64, 64, 32, 7, s, s, D, 64)      # mode
+
+
+# ---------------------------------------------------- full-size, sampled --
+
+def _sampled_check(orc, D, A, fa, B, fb, mode, da, db, n=4096, seed=0):
+    rng = np.random.default_rng(seed)
+    M, N = D.shape
+    im = rng.integers(0, M, n)
+    inn = rng.integers(0, N, n)
+    # always include the corners of the last (ragged) tiles
+    im[:4] = [0, M - 1, M - 1, 0]
+    inn[:4] = [0, N - 1, 0, N - 1]
+    ref, mag = orc.gemm_scaled_sampled(A, fa, B, fb, mode, da, db, im, inn)
+    got = D.float().cpu().numpy().astype(np.float64)[im, inn]
+    return assert_gemm_close(got, ref, mag)
+
+
+def test_gemm_rowwise_4096_cube_sampled(orc):
+    """Rowwise pow2 E4M3 GEMM at M = N = K = 4096 (activations with 0.1 %
+    x100 outliers, N(0, 0.02) weights)."""
+    a = inputs.bf16_bits(inputs.outlier_activations_bf16((4096, 4096), seed=1, device="cuda"))
+    b = inputs.bf16_bits(inputs.normal_bf16((4096, 4096), 0.02, seed=2, device="cuda"))
+    A, da = orc.quantize_rowwise(a, 0, True)
+    B, db = orc.quantize_rowwise(b, 0, True)
+    D = _run(A, 0, B, 0, 1, da, db)
+    _sampled_check(orc, D, A, 0, B, 0, 1, da, db)
+
+
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_gemm_blockwise_mlp_sampled(orc, which):
+    """Block-scaled MLP GEMMs: [8192, 4096] x W_up[11008, 4096]^T and
+    [8192, 11008] x W_down[4096, 11008]^T (the second GEMM's input is a seeded
+    bf16 tensor of the same shape, so no oracle input comes from the GPU)."""
+    if which == "up":
+        M, N, K = 8192, 11008, 4096
+    else:
+        M, N, K = 8192, 4096, 11008
+    x = inputs.bf16_bits(inputs.normal_bf16((M, K), 1.0, seed=5, device="cuda"))
+    w = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, seed=6, device="cuda"))
+    A, da = orc.quantize_blockwise(x, 0, 1)
+    B, db = orc.quantize_blockwise(w, 0, 128)
+    D = _run(A, 0, B, 0, 2, da, db)
+    _sampled_check(orc, D, A, 0, B, 0, 2, da, db, n=2048)
