@@ -16,7 +16,8 @@ scaling over a 16-step history) and ``kv`` (FP8 KV cache K, V [32, 32, 8192,
 
 Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then K steps
 bracketed by a barrier and a device synchronize; each step's kernels are
-timed with CUDA events on the launching stream, L2 is flushed (a 256 MiB write)
+timed with CUDA events on the launching stream, L2 is flushed (a 256 MiB write
+and a 256 MiB read)
 before every step outside the events; multi-GPU takes the max over ranks.
 ``--impl reference`` times the CPU oracle (the only reference this project
 has) on a bounded sample of the same workload.
@@ -41,7 +42,7 @@ METRIC = "FP8 scaled GEMM TFLOP/s (% dense FP8 peak); quantize/KV GB/s (% HBM)"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_OVER_BF16 = 2.0     # nominal dense ratio: 4.5 PFLOP/s fp8 / 2.25 PFLOP/s bf16
-DEFAULT_STEPS = {"rowwise": 2000, "tensor": 2000, "blockmlp": 100, "dgrad": 400, "kv": 40}
+DEFAULT_STEPS = {"rowwise": 6000, "tensor": 6000, "blockmlp": 300, "dgrad": 1500, "kv": 60}
 
 
 def peaks():
@@ -69,7 +70,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.dev)],
+                 "-lms", "100", "-i", str(self.dev)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -457,7 +458,18 @@ def main():
     from fp8_scaled_quantization_amax_b200 import fp8q
     fp8q.lib()
     wl = Workload(args.workload, dev, seed=1000 * rank)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    # L2 flush before every step: write 256 MiB, then read another 256 MiB so
+    # the flush's own dirty lines are written back before the step starts
+    flush_w = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    class _Flush:
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            flush_r.sum()
+
+    flush = _Flush()
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(warmup):
@@ -534,7 +546,7 @@ def main():
              "dgrad": "fp8_e5m2 x fp8_e4m3 -> f32 accumulate -> bf16",
              "kv": "bf16 <-> fp8_e4m3 (f32 scale)"}[args.workload]
     cfg = dict(wl.config)
-    cfg["l2"] = "flushed before every step (256 MiB write, outside the step's events)"
+    cfg["l2"] = "flushed before every step (256 MiB write + 256 MiB read, outside the step's events)"
     line = {
         "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": world, "steps": steps, "warmup": warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

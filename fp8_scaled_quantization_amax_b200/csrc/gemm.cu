@@ -81,8 +81,10 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
+// Local arrive used to release a TMEM buffer (relaxed for the same reason as
+// mbar_arrive_cluster below: the guarded TMEM loads have completed).
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -161,6 +163,37 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// 32 lanes x 32 columns, issued without waiting: the registers are only
+// valid after tmem_wait64() on the array that contains them.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+// One wait for all loads in flight; the 64 registers are named read-write so
+// no use of them can move above the wait.
+__device__ __forceinline__ void tmem_wait64(uint32_t (&r)[64]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31]), "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]),
+                   "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]), "+r"(r[40]), "+r"(r[41]), "+r"(r[42]),
+                   "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]), "+r"(r[48]), "+r"(r[49]),
+                   "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]), "+r"(r[56]),
+                   "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
+                 :
+                 : "memory");
 }
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
@@ -356,11 +389,11 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 const int nkb_b = nk;                     // K blocks per row of sb
                 const int nb = n_base / 128;              // this half's 128-row block of B
                 const bool nb_ok = n_base < N;
+                float a_next = (m < M) ? sa[m] : 0.0f;
+                float b_next = nb_ok ? sb[(int64_t)nb * nkb_b] : 0.0f;
                 for (int kc = 0; kc < nk; ++kc, ++it) {
                     const uint32_t pb = it & 1u, use = it >> 1;
-                    const float a_s = (m < M) ? sa[(int64_t)kc * M + m] : 0.0f;
-                    const float b_s = nb_ok ? sb[(int64_t)nb * nkb_b + kc] : 0.0f;
-                    const float sc = __fmul_rn(a_s, b_s);
+                    const float sc = __fmul_rn(a_next, b_next);
                     bool w = true;
                     if (lane == 0) w = wait_bar(accf_bar(pb), use & 1u, abort_flag, kErrEpilogue);
                     w = __shfl_sync(0xFFFFFFFFu, w, 0);
@@ -374,6 +407,10 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(acce_bar(pb));
+                            if (kc + 1 < nk) {   // next block's scales, after the release (see the pair kernel)
+                                a_next = (m < M) ? sa[(int64_t)(kc + 1) * M + m] : 0.0f;
+                                b_next = nb_ok ? sb[(int64_t)nb * nkb_b + kc + 1] : 0.0f;
+                            }
                         }
 #pragma unroll
                         for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(v[j], sc, acc[c * 32 + j]);
@@ -403,6 +440,346 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ------------------------------------------------------ 2-SM variant ----
+// A CTA pair (cluster of 2) computes a 256 x BN tile with
+// tcgen05.mma.cta_group::2 (M = 256): each CTA TMA-loads its own 128 rows of
+// A and its own BN/2 rows of B (no multicast), the even CTA ("leader")
+// issues the MMAs, which read both CTAs' shared memory and write each CTA's
+// 128 accumulator rows into its own TMEM.  Per CTA and K chunk this moves
+// 16 KiB + BN/2 x 128 B instead of 16 KiB + 32 KiB, so 6 (BN = 256) or 8
+// (BN = 128) stages fit in shared memory and hide more TMA latency.
+//   * The leader's full barrier counts both CTAs' bytes (the peer's TMA
+//     signals it through its cluster address);
+//   * tcgen05.commit multicasts to the same barrier in both CTAs (stage
+//     free, accumulator / partial ready);
+//   * both CTAs' epilogue warps release a TMEM buffer by arriving on the
+//     leader's barrier (count 2 x 8 warps).
+// BLOCK mode uses BN = 128 and four 128-column TMEM partial buffers, so the
+// MMA can run three K chunks ahead of the promotion.
+namespace sm2 {
+constexpr int EPI = 8;                 // epilogue warps 4..11 (warpgroups 1 and 2)
+constexpr int THREADS = 12 * 32;       // warpgroup 0: producer (warp 0), MMA (warp 1), two idle warps
+// BLOCK mode moves registers from warpgroup 0 to the epilogue warpgroups,
+// which hold a 128-wide fp32 accumulator row per thread.  The split must
+// not exceed the launch pool: 128 * 56 + 256 * 224 = 64512 = 384 * 168,
+// so the kernel must launch at exactly 168 registers per thread (checked on
+// the host before the first launch).
+constexpr int REGS_LAUNCH = 168, REGS_LOW = 56, REGS_HIGH = 224;
+static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * REGS_LAUNCH, "register split exceeds the launch pool");
+template <int BN>
+struct Cfg {
+    static constexpr int B_HALF = (BN / 2) * BK;
+    static constexpr int STAGE = A_TILE + B_HALF;
+    static constexpr int STAGES = (BN == 256) ? 6 : 8;
+    static constexpr int NBUF = 512 / BN;
+    static constexpr int NBARS = 2 * STAGES + 2 * NBUF + 1;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + NBARS * 8 + 16;
+};
+}  // namespace sm2
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Release of a TMEM buffer to the leader's MMA thread.  Relaxed: the TMEM
+// loads it guards have already completed (tcgen05.wait::ld) and are ordered
+// by tcgen05.fence::before_thread_sync; a release fence here would also wait
+// for unrelated global loads and stores in flight (measured as the dominant
+// "membar" stall of the block-scaled epilogue).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, uint32_t bar_cluster, int x,
+                                                 int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// arrive on the barrier at this shared offset in both CTAs of the pair
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)0x3)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair_self(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+template <int MODE, int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
+k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+               int K, uint32_t idesc, const float *__restrict__ sa, const float *__restrict__ sb,
+               __nv_bfloat16 *__restrict__ D, int64_t ldd) {
+    using C = sm2::Cfg<BN>;
+    constexpr int STG = C::STAGES, NBUF = C::NBUF;
+    constexpr int HALF = BN / 2;             // columns per epilogue warp
+    static_assert(BN == 256, "the pair kernel runs 256 x 256 tiles");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)STG * C::STAGE);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBARS);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = (rank == 0);
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int num_m = (M + 255) / 256, num_n = (N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int nk = (K + BK - 1) / BK;
+
+    auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+    auto empty_bar = [&](int s) { return smem_u32(&bars[STG + s]); };
+    auto accf_bar = [&](int b) { return smem_u32(&bars[2 * STG + b]); };
+    auto acce_bar = [&](int b) { return smem_u32(&bars[2 * STG + NBUF + b]); };
+    const uint32_t drain_bar = smem_u32(&bars[2 * STG + 2 * NBUF]);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STG; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(accf_bar(b), 1);
+            mbar_init(acce_bar(b), 2 * sm2::EPI);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();   // both CTAs' barriers are initialised before any remote signal
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // BLOCK mode: each role branch resizes its own warpgroup's registers, so
+    // the epilogue code is only reachable after the increase.
+    if (warp == 0) {
+        if constexpr (MODE == kModeBlock) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            int last_round[STG];
+            for (int s = 0; s < STG; ++s) last_round[s] = -1;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+                const int m_blk = tile % num_m, n_blk = tile / num_m;
+                const int a_row = m_blk * 256 + (int)rank * 128;
+                const int b_row = n_blk * BN + (int)rank * HALF;
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const int stage = it % STG;
+                    const uint32_t round = it / STG;
+                    if (!wait_bar(empty_bar(stage), (round & 1u) ^ 1u, abort_flag, kErrProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_leader = mapa_shared(full_bar(stage), 0);
+                    if (leader) mbar_expect_tx(full_bar(stage), 2 * C::STAGE);
+                    const uint32_t a_dst = smem_u32(smem + (size_t)stage * C::STAGE);
+                    tma_load_2d_pair(a_dst, &tmA, full_leader, kc * BK, a_row);
+                    tma_load_2d_pair(a_dst + A_TILE, &tmB, full_leader, kc * BK, b_row);
+                    last_round[stage] = (int)round;
+                }
+            }
+            if (leader && (!ok || *abort_flag)) {
+                for (int s = 0; s < STG; ++s)
+                    if (last_round[s] >= 0) wait_bar_drain(full_bar(s), (uint32_t)last_round[s] & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if constexpr (MODE == kModeBlock) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
+        // ------------------------------------- MMA issuer (leader only) --
+        if (leader && lane == 0) {
+            uint32_t it = 0, lt = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < num_tiles; tile += npairs, ++lt) {
+                uint32_t d_tmem = tmem;
+                if (MODE != kModeBlock) {
+                    const uint32_t ab = lt % NBUF, use = lt / NBUF;
+                    if (!wait_bar(acce_bar(ab), (use & 1u) ^ 1u, abort_flag, kErrMma)) break;
+                    tc_fence_after();
+                    d_tmem = tmem + ab * BN;
+                }
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const int stage = it % STG;
+                    const uint32_t round = it / STG;
+                    if (MODE == kModeBlock) {
+                        const uint32_t pb = it % NBUF, use = it / NBUF;
+                        if (!wait_bar(acce_bar(pb), (use & 1u) ^ 1u, abort_flag, kErrMma)) { ok = false; break; }
+                        d_tmem = tmem + pb * BN;
+                    }
+                    if (!wait_bar(full_bar(stage), round & 1u, abort_flag, kErrMma)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + (size_t)stage * C::STAGE);
+                    const uint64_t adesc = sdesc_k_sw128(a_addr);
+                    const uint64_t bdesc = sdesc_k_sw128(a_addr + A_TILE);
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k) {
+                        const uint32_t acc = (MODE == kModeBlock) ? (k > 0) : (kc > 0 || k > 0);
+                        tc_mma_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, acc);
+                    }
+                    tc_commit_pair_both(empty_bar(stage));
+                    if (MODE == kModeBlock) tc_commit_pair_both(accf_bar(it % NBUF));
+                }
+                if (ok && MODE != kModeBlock) tc_commit_pair_both(accf_bar(lt % NBUF));
+            }
+            tc_commit_pair_self(drain_bar);
+            wait_bar_drain(drain_bar, 0u);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        if constexpr (MODE == kModeBlock) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
+    } else {
+        if constexpr (MODE == kModeBlock) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(sm2::REGS_HIGH));
+        // --------------------------------------------------- epilogue ----
+        const int sp = warp & 3;
+        const int ch = (warp - 4) >> 2;
+        const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+        uint32_t it = 0, lt = 0;
+        bool ok = true;
+        for (int tile = pair; ok && tile < num_tiles; tile += npairs, ++lt) {
+            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            const int m = m_blk * 256 + (int)rank * 128 + sp * 32 + lane;
+            const int n_base = n_blk * BN + ch * HALF;
+            __nv_bfloat16 *drow = D + (int64_t)m * ldd;
+            if (MODE != kModeBlock) {
+                const uint32_t ab = lt % NBUF, use = lt / NBUF;
+                float rs;
+                if (MODE == kModeRow) rs = (m < M) ? sa[m] : 0.0f;
+                else rs = __fmul_rn(sa[0], sb[0]);
+                bool w = true;
+                if (lane == 0) w = wait_bar(accf_bar(ab), use & 1u, abort_flag, kErrEpilogue);
+                w = __shfl_sync(0xFFFFFFFFu, w, 0);
+                if (!w) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < HALF / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + ab * BN + ch * HALF + c * 32, v);
+                    const int col0 = n_base + c * 32;
+                    if (MODE == kModeRow) {
+                        const float cb = (col0 + lane < N) ? sb[col0 + lane] : 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = v[j] * (rs * __shfl_sync(0xFFFFFFFFu, cb, j));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
+                    }
+                    if (m < M) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (col0 + g * 8 < N) {
+                                uint4 o;
+                                o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+                                o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+                                o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+                                o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+                                *reinterpret_cast<uint4 *>(drow + col0 + g * 8) = o;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(ab), 0));
+            } else {
+                float acc[HALF];
+#pragma unroll
+                for (int j = 0; j < HALF; ++j) acc[j] = 0.0f;
+                const int nb = n_base / 128;
+                const bool nb_ok = n_base < N;
+                // The scales of K block kc + 1 are fetched right after block kc's
+                // buffer is released (the release arrive would otherwise wait
+                // for those loads), one block ahead of their use.
+                float a_next = (m < M) ? sa[m] : 0.0f;
+                float b_next = nb_ok ? sb[(int64_t)nb * nk] : 0.0f;
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const uint32_t pb = it % NBUF, use = it / NBUF;
+                    const float sc = __fmul_rn(a_next, b_next);
+                    bool w = true;
+                    if (lane == 0) w = wait_bar(accf_bar(pb), use & 1u, abort_flag, kErrEpilogue);
+                    w = __shfl_sync(0xFFFFFFFFu, w, 0);
+                    if (!w) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t src = tmem + lane_base + pb * BN + ch * HALF;
+                    // two 64-column halves, one TMEM round trip each
+                    uint32_t r[64];
+                    tmem_ld32_async(src, r);
+                    tmem_ld32_async(src + 32, r + 32);
+                    tmem_wait64(r);
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) acc[j] = fmaf(__uint_as_float(r[j]), sc, acc[j]);
+                    tmem_ld32_async(src + 64, r);
+                    tmem_ld32_async(src + 96, r + 32);
+                    tmem_wait64(r);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(pb), 0));
+                    if (kc + 1 < nk) {   // next block's scales, after the release
+                        a_next = (m < M) ? sa[(int64_t)(kc + 1) * M + m] : 0.0f;
+                        b_next = nb_ok ? sb[(int64_t)nb * nk + kc + 1] : 0.0f;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) acc[64 + j] = fmaf(__uint_as_float(r[j]), sc, acc[64 + j]);
+                }
+                if (!ok) break;
+                if (m < M) {
+#pragma unroll
+                    for (int g = 0; g < HALF / 8; ++g) {
+                        const int col = n_base + g * 8;
+                        if (col < N) {
+                            uint4 o;
+                            o.x = pack_bf16x2(acc[g * 8 + 0], acc[g * 8 + 1]);
+                            o.y = pack_bf16x2(acc[g * 8 + 2], acc[g * 8 + 3]);
+                            o.z = pack_bf16x2(acc[g * 8 + 4], acc[g * 8 + 5]);
+                            o.w = pack_bf16x2(acc[g * 8 + 6], acc[g * 8 + 7]);
+                            *reinterpret_cast<uint4 *>(drow + col) = o;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();   // every TMEM read and MMA of both CTAs is done
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
     }
 }
 
@@ -454,6 +831,56 @@ cudaError_t launch_gemm(cudaStream_t st, int sms, const CUtensorMap &ta, const C
     return cudaPeekAtLastError();
 }
 
+// Pairs of the 2-SM kernel that fit on the device at once (cached per device).
+template <int MODE, int BN>
+int pair_capacity() {
+    static int cache[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev] > 0) return cache[dev];
+    if (cudaFuncSetAttribute(k_gemm_fp8_2sm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm2::Cfg<BN>::SMEM) != cudaSuccess)
+        return 0;
+    if (MODE == kModeBlock) {   // the setmaxnreg split assumes this launch register count
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, k_gemm_fp8_2sm<MODE, BN>) != cudaSuccess || fa.numRegs != sm2::REGS_LAUNCH)
+            return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 64);
+    cfg.blockDim = dim3(sm2::THREADS);
+    cfg.dynamicSmemBytes = sm2::Cfg<BN>::SMEM;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_fp8_2sm<MODE, BN>, &cfg) != cudaSuccess) return 0;
+    cache[dev] = n;
+    return n;
+}
+
+template <int MODE, int BN>
+cudaError_t launch_gemm_2sm(cudaStream_t st, const CUtensorMap &ta, const CUtensorMap &tb, int M, int N, int K,
+                            uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd, int pairs_cap) {
+    const int tiles = ((M + 255) / 256) * ((N + BN - 1) / BN);
+    const int pairs = std::max(1, std::min(tiles, pairs_cap));
+    k_gemm_fp8_2sm<MODE, BN><<<2 * pairs, sm2::THREADS, sm2::Cfg<BN>::SMEM, st>>>(
+        ta, tb, M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd);
+    return cudaPeekAtLastError();
+}
+
+uint32_t make_idesc(fp8_format fa, fp8_format fb, int mma_m, int mma_n) {
+    // fp32 accumulator, A/B formats, K-major A and B, N >> 3, M >> 4
+    return (1u << 4) | ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(mma_n >> 3) << 17) |
+           ((uint32_t)(mma_m >> 4) << 24);
+}
+
 }  // namespace
 
 using namespace fp8q_host;
@@ -482,11 +909,28 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
         return cudaMemset2DAsync(D_bf16, (size_t)ldd * 2, 0, (size_t)N * 2, (size_t)M, s) == cudaSuccess ? FP8_OK
                                                                                                        : FP8_ERR_CUDA;
     }
+    // M > 128: a CTA pair per 256-row tile (2-SM MMA); otherwise one CTA per 128-row tile.
+    if (M > BM) {
+        CUtensorMap ta, tb;
+        if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
+        const uint32_t idesc = make_idesc(fa, fb, 256, 256);
+        cudaError_t e = cudaErrorUnknown;
+        int cap;
+        if (mode == FP8_SCALE_TENSOR) {
+            if ((cap = pair_capacity<kModeTensor, 256>()) > 0)
+                e = launch_gemm_2sm<kModeTensor, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap);
+        } else if (mode == FP8_SCALE_ROW) {
+            if ((cap = pair_capacity<kModeRow, 256>()) > 0)
+                e = launch_gemm_2sm<kModeRow, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap);
+        } else {
+            if ((cap = pair_capacity<kModeBlock, 256>()) > 0)
+                e = launch_gemm_2sm<kModeBlock, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap);
+        }
+        return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    }
     CUtensorMap ta, tb;
     if (!make_map(&ta, A, K, M, BM) || !make_map(&tb, B, K, N, BN)) return FP8_ERR_CUDA;
-    // instruction descriptor: fp32 accumulator, A/B formats, K-major A and B, N>>3, M>>4
-    const uint32_t idesc = (1u << 4) | ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(BN >> 3) << 17) |
-                           ((uint32_t)(BM >> 4) << 24);
+    const uint32_t idesc = make_idesc(fa, fb, BM, BN);
     cudaError_t e;
     if (mode == FP8_SCALE_TENSOR)
         e = launch_gemm<kModeTensor>(s, sms, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd);

@@ -4,16 +4,21 @@
 // in FP8 halve the cache; each is dequantized when attention reads it).
 //
 // Quantize: a (b, h) slice (S*Dh elements, 2 MiB of bf16 at S=8192, Dh=128)
-// needs its own amax before any element can be cast.  One 8-CTA thread-block
-// cluster owns one slice at a time: every CTA streams its eighth of the slice
-// from HBM for the amax, the eight partial maxima meet through distributed
-// shared memory behind a cluster barrier, and the cast pass re-reads the same
-// eighth while it is still in L2 (18 clusters x 2 MiB in flight stays far
-// below the 126 MB L2).  HBM traffic is the algorithmic 2 B in + 1 B out per
-// element, in one launch, with no scratch memory and no grid-wide wait.
+// needs its own amax before any element can be cast.  One 4-CTA thread-block
+// cluster owns one slice at a time: every CTA streams its quarter of the
+// slice from HBM for the amax (loads marked L2 evict-last), the four partial
+// maxima meet through distributed shared memory behind a cluster barrier, and
+// the cast pass re-reads the same quarter from L2 (loads and FP8 stores
+// marked evict-first, so the slices still waiting for their second pass stay
+// resident; about 37 clusters x 2 MiB are in flight against the 126 MB L2).
+// HBM traffic is the algorithmic 2 B in + 1 B out per element, in one
+// launch, with no scratch memory and no grid-wide wait.
 //
-// Dequantize: a plain stream, 16 FP8 codes in (one 16-byte load), 16 bf16 out
-// (two 16-byte stores), one scale per (b, h) from the grid's y index.
+// Dequantize: each CTA streams a contiguous 256 KiB of FP8 codes (16 codes
+// in per 16-byte load, 16 bf16 out as two 16-byte stores); contiguous
+// per-CTA chunks keep the write-heavy stream at DRAM-page locality (a
+// grid-stride layout measured ~20 % slower).  One scale per (b, h) from the
+// grid's y index.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -25,7 +30,7 @@ using namespace fp8q;
 
 namespace {
 
-constexpr int kClusterCtas = 8;
+constexpr int kClusterCtas = 4;
 constexpr int kKvThreads = 1024;
 
 template <int FMT>
@@ -42,6 +47,7 @@ k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64
     const int64_t per = (nunit + kClusterCtas - 1) / kClusterCtas;
     const int64_t u0 = min((int64_t)rank * per, nunit);
     const int64_t u1 = min(u0 + per, nunit);
+    const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
     int it = 0;
     for (int64_t sl = cid; sl < BH; sl += ncl, ++it) {
         const uint4 *xs = x + 2 * sl * nunit;   // a unit is 16 elements = two uint4 of bf16
@@ -49,12 +55,18 @@ k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64
         // pass 1: amax of this CTA's part of the slice
         uint32_t m2 = 0;
         int64_t u = u0 + threadIdx.x;
-        for (; u + kKvThreads < u1; u += 2 * kKvThreads) {
-            uint4 a0 = ld_stream(xs + 2 * u), a1 = ld_stream(xs + 2 * u + 1);
-            uint4 b0 = ld_stream(xs + 2 * (u + kKvThreads)), b1 = ld_stream(xs + 2 * (u + kKvThreads) + 1);
-            m2 = amax_fast8(amax_fast8(amax_fast8(amax_fast8(m2, a0), a1), b0), b1);
+        for (; u + 3 * kKvThreads < u1; u += 4 * kKvThreads) {
+            uint4 v[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                v[2 * k] = ld_hint(xs + 2 * (u + k * kKvThreads), keep);
+                v[2 * k + 1] = ld_hint(xs + 2 * (u + k * kKvThreads) + 1, keep);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m2 = amax_fast8(m2, v[k]);
         }
-        for (; u < u1; u += kKvThreads) m2 = amax_fast8(amax_fast8(m2, ld_stream(xs + 2 * u)), ld_stream(xs + 2 * u + 1));
+        for (; u < u1; u += kKvThreads)
+            m2 = amax_fast8(amax_fast8(m2, ld_hint(xs + 2 * u, keep)), ld_hint(xs + 2 * u + 1, keep));
         uint32_t m = amax_fast_final(m2);
         if (m == 0xFFFFFFFFu) {
             uint32_t bad = 0;
@@ -75,15 +87,48 @@ k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64
         const float s = scale_from_amax(bf16bits_to_float(slice_amax), fm);
         if (rank == 0 && threadIdx.x == 0) scale_inv[sl] = __fdiv_rn(1.0f, s);
         // pass 2: cast (the re-read hits L2)
-        for (int64_t j = u0 + threadIdx.x; j < u1; j += kKvThreads) {
-            uint4 a0 = xs[2 * j], a1 = xs[2 * j + 1];
+        int64_t j = u0 + threadIdx.x;
+        for (; j + 3 * kKvThreads < u1; j += 4 * kKvThreads) {
+            uint4 v[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                v[2 * k] = ld_hint(xs + 2 * (j + k * kKvThreads), drop);
+                v[2 * k + 1] = ld_hint(xs + 2 * (j + k * kKvThreads) + 1, drop);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                uint2 c0 = cast8<FMT>(v[2 * k], s), c1 = cast8<FMT>(v[2 * k + 1], s);
+                st_hint(qs + j + k * kKvThreads, make_uint4(c0.x, c0.y, c1.x, c1.y), drop);
+            }
+        }
+        for (; j < u1; j += kKvThreads) {
+            uint4 a0 = ld_hint(xs + 2 * j, drop), a1 = ld_hint(xs + 2 * j + 1, drop);
             uint2 c0 = cast8<FMT>(a0, s), c1 = cast8<FMT>(a1, s);
-            qs[j] = make_uint4(c0.x, c0.y, c1.x, c1.y);
+            st_hint(qs + j, make_uint4(c0.x, c0.y, c1.x, c1.y), drop);
         }
     }
     cluster.sync();   // no CTA leaves while a peer may still read its slots
 }
 
+template <int FMT>
+__device__ __forceinline__ void dequant16(uint4 c, float d, uint4 &o0, uint4 &o1) {
+    uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 lo = fp8x2_to_float2<FMT>((uint16_t)(w[i] & 0xFFFFu));
+        float2 hi = fp8x2_to_float2<FMT>((uint16_t)(w[i] >> 16));
+        o[2 * i] = pack_bf16x2(__fmul_rn(lo.x, d), __fmul_rn(lo.y, d));
+        o[2 * i + 1] = pack_bf16x2(__fmul_rn(hi.x, d), __fmul_rn(hi.y, d));
+    }
+    o0 = make_uint4(o[0], o[1], o[2], o[3]);
+    o1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// A CTA dequantizes the contiguous units [blockIdx.x * per, +per) of slice
+// blockIdx.y: four 16-byte loads in flight per thread, then eight 16-byte
+// stores.
+constexpr int64_t kDequantUnitsPerCta = 16384;   // 256 KiB of FP8 codes
 template <int FMT>
 __global__ void __launch_bounds__(256)
 k_kv_dequant(const uint4 *__restrict__ q, const float *__restrict__ scale_inv, int64_t nunit,
@@ -92,20 +137,26 @@ k_kv_dequant(const uint4 *__restrict__ q, const float *__restrict__ scale_inv, i
     const float d = scale_inv[sl];
     const uint4 *qs = q + sl * nunit;
     uint4 *os = out + 2 * sl * nunit;
-    for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < nunit;
-         u += (int64_t)gridDim.x * blockDim.x) {
-        uint4 c = ld_stream(qs + u);
-        uint32_t w[4] = {c.x, c.y, c.z, c.w};
-        uint32_t o[8];
+    const int64_t u0 = blockIdx.x * kDequantUnitsPerCta;
+    const int64_t u1 = min(u0 + kDequantUnitsPerCta, nunit);
+    int64_t u = u0 + threadIdx.x;
+    for (; u + 3 * 256 < u1; u += 4 * 256) {
+        uint4 c[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float2 lo = fp8x2_to_float2<FMT>((uint16_t)(w[i] & 0xFFFFu));
-            float2 hi = fp8x2_to_float2<FMT>((uint16_t)(w[i] >> 16));
-            o[2 * i] = pack_bf16x2(__fmul_rn(lo.x, d), __fmul_rn(lo.y, d));
-            o[2 * i + 1] = pack_bf16x2(__fmul_rn(hi.x, d), __fmul_rn(hi.y, d));
+        for (int k = 0; k < 4; ++k) c[k] = ld_stream(qs + u + k * 256);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint4 o0, o1;
+            dequant16<FMT>(c[k], d, o0, o1);
+            os[2 * (u + k * 256)] = o0;
+            os[2 * (u + k * 256) + 1] = o1;
         }
-        os[2 * u] = make_uint4(o[0], o[1], o[2], o[3]);
-        os[2 * u + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    for (; u < u1; u += 256) {
+        uint4 o0, o1;
+        dequant16<FMT>(ld_stream(qs + u), d, o0, o1);
+        os[2 * u] = o0;
+        os[2 * u + 1] = o1;
     }
 }
 
@@ -184,8 +235,8 @@ extern "C" fp8_status fp8_kv_dequant(const uint8_t *q, const float *scale_inv, i
     if (st != FP8_OK) return st;
     if (BH == 0 || nunit == 0) return FP8_OK;
     cudaStream_t s = as_stream(stream);
-    // about 8 CTAs of 256 threads per SM in total, at least one per slice
-    const int64_t per_slice = std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * 8 / BH, (nunit + 255) / 256));
+    const int64_t per_slice = (nunit + kDequantUnitsPerCta - 1) / kDequantUnitsPerCta;
+    if (per_slice > 2147483647LL) return FP8_ERR_SHAPE;
     const dim3 grid((unsigned)per_slice, (unsigned)BH);
     if (fmt == FP8_E4M3)
         k_kv_dequant<FP8_E4M3><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(q), scale_inv, nunit, static_cast<uint4 *>(out_bf16));

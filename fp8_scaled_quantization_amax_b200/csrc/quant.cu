@@ -183,11 +183,12 @@ k_cast_transpose(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64
 }
 
 // --------------------------------------------------------------- rowwise --
-// One CTA (256 threads) per row, the row held in registers (V vectors of 8
+// One CTA (128 threads) per row, the row held in registers (V vectors of 8
 // per thread) between the amax and the cast: one HBM read per element.
 // V == 0: rows too long for registers, two passes (the second from L2).
+constexpr int kRowThreads = 128;
 template <int FMT, bool POW2, int V>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kRowThreads)
 k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
           uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
     __shared__ uint32_t red[32];
@@ -202,7 +203,7 @@ k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
             uint32_t m2 = 0;
 #pragma unroll
             for (int j = 0; j < V; ++j) {
-                const int64_t cv = threadIdx.x + j * 256;
+                const int64_t cv = threadIdx.x + j * kRowThreads;
                 v[j] = cv < ncv ? ld_stream(xr + cv) : make_uint4(0, 0, 0, 0);
                 m2 = amax_fast8(m2, v[j]);
             }
@@ -218,18 +219,18 @@ k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
             const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
 #pragma unroll
             for (int j = 0; j < V; ++j) {
-                const int64_t cv = threadIdx.x + j * 256;
+                const int64_t cv = threadIdx.x + j * kRowThreads;
                 if (cv < ncv) qr[cv] = cast8<FMT>(v[j], s);
             }
             if (threadIdx.x == 0) scale_inv[r] = __fdiv_rn(1.0f, s);
         } else {
             uint32_t bad = 0;
             m = 0;
-            for (int64_t cv = threadIdx.x; cv < ncv; cv += 256) m = amax_exact8(m, ld_stream(xr + cv), bad);
+            for (int64_t cv = threadIdx.x; cv < ncv; cv += kRowThreads) m = amax_exact8(m, ld_stream(xr + cv), bad);
             m = block_max_u32(m, red);
             const float a = bf16bits_to_float(m);
             const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
-            for (int64_t cv = threadIdx.x; cv < ncv; cv += 256) qr[cv] = cast8<FMT>(xr[cv], s);
+            for (int64_t cv = threadIdx.x; cv < ncv; cv += kRowThreads) qr[cv] = cast8<FMT>(xr[cv], s);
             if (threadIdx.x == 0) scale_inv[r] = __fdiv_rn(1.0f, s);
         }
     }
@@ -362,13 +363,15 @@ template <int FMT, bool POW2>
 void launch_rowwise(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, int64_t ld,
                     uint8_t *q, float *scale_inv) {
     const uint16_t *xs = static_cast<const uint16_t *>(x);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(rows, (int64_t)sms * 8));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(rows, (int64_t)sms * 16));
     const int64_t ncv = cols / 8;
-    if (ncv <= 256) k_rowwise<FMT, POW2, 1><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 512) k_rowwise<FMT, POW2, 2><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 1024) k_rowwise<FMT, POW2, 4><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 2048) k_rowwise<FMT, POW2, 8><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else k_rowwise<FMT, POW2, 0><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    const int T = kRowThreads;
+    if (ncv <= T) k_rowwise<FMT, POW2, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 2 * T) k_rowwise<FMT, POW2, 2><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 4 * T) k_rowwise<FMT, POW2, 4><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 8 * T) k_rowwise<FMT, POW2, 8><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 16 * T) k_rowwise<FMT, POW2, 16><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else k_rowwise<FMT, POW2, 0><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
 }
 
 template <int FMT>
