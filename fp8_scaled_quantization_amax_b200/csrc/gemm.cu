@@ -721,14 +721,18 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 for (int j = 0; j < HALF; ++j) acc[j] = 0.0f;
                 const int nb = n_base / 128;
                 const bool nb_ok = n_base < N;
-                // The scales of K block kc + 1 are fetched right after block kc's
-                // buffer is released (the release arrive would otherwise wait
-                // for those loads), one block ahead of their use.
-                float a_next = (m < M) ? sa[m] : 0.0f;
-                float b_next = nb_ok ? sb[(int64_t)nb * nk] : 0.0f;
+                // Scales run two K blocks ahead in registers: block kc + 2's are
+                // fetched right after block kc's partial is released, so a
+                // global load is never waited on inside the promotion.
+                float a0 = (m < M) ? sa[m] : 0.0f;
+                float b0 = nb_ok ? sb[(int64_t)nb * nk] : 0.0f;
+                float a1 = (nk > 1 && m < M) ? sa[(int64_t)M + m] : 0.0f;
+                float b1 = (nk > 1 && nb_ok) ? sb[(int64_t)nb * nk + 1] : 0.0f;
                 for (int kc = 0; kc < nk; ++kc, ++it) {
                     const uint32_t pb = it % NBUF, use = it / NBUF;
-                    const float sc = __fmul_rn(a_next, b_next);
+                    const float sc = __fmul_rn(a0, b0);
+                    a0 = a1;
+                    b0 = b1;
                     bool w = true;
                     if (lane == 0) w = wait_bar(accf_bar(pb), use & 1u, abort_flag, kErrEpilogue);
                     w = __shfl_sync(0xFFFFFFFFu, w, 0);
@@ -748,9 +752,9 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(pb), 0));
-                    if (kc + 1 < nk) {   // next block's scales, after the release
-                        a_next = (m < M) ? sa[(int64_t)(kc + 1) * M + m] : 0.0f;
-                        b_next = nb_ok ? sb[(int64_t)nb * nk + kc + 1] : 0.0f;
+                    if (kc + 2 < nk) {   // block kc + 2's scales, after the release
+                        a1 = (m < M) ? sa[(int64_t)(kc + 2) * M + m] : 0.0f;
+                        b1 = nb_ok ? sb[(int64_t)nb * nk + kc + 2] : 0.0f;
                     }
 #pragma unroll
                     for (int j = 0; j < 64; ++j) acc[64 + j] = fmaf(__uint_as_float(r[j]), sc, acc[64 + j]);

@@ -231,3 +231,16 @@ def test_invalid_arguments_rejected_before_launch():
         fp8q.fp8_quantize_tensorwise(x, 4, 32, 0, None, q, 0, s[:1], None)   # current scaling needs amax_out
     with pytest.raises(fp8q.Fp8Error, match="ALIGNMENT"):
         fp8q.fp8_amax(x.view(-1)[1:], s[:1])                             # 2-byte offset pointer
+
+
+def test_quantize_tensorwise_global_single_rank(orc):
+    """Global-scale per-tensor path with one rank: library amax -> (no-op
+    exchange) -> scale from the history kernel -> cast; equals the oracle's
+    current scaling bit for bit."""
+    from fp8_scaled_quantization_amax_b200 import dist as fdist
+    x = inputs.normal_bf16((300, 512), 2.0, seed=77)
+    q, sinv, am = fdist.quantize_tensorwise_global(x.to("cuda"), 0)
+    rq, rsinv, ramax, _ = orc.quantize_tensorwise(inputs.bf16_bits(x), 0)
+    assert_codes_equal(to_np(q), rq, 0)
+    assert_f32_equal(to_np(sinv), np.float32([rsinv]))
+    assert_f32_equal(to_np(am), np.float32([ramax]))
