@@ -196,6 +196,19 @@ __device__ __forceinline__ void tmem_wait64(uint32_t (&r)[64]) {
                  : "memory");
 }
 
+// Packed fp32 pair arithmetic (sm_100): two IEEE round-to-nearest FMAs per
+// instruction, which halves the issue cost of the block-scale promotion.
+__device__ __forceinline__ uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row groups 1024 bytes apart (the layout TMA writes with
 // CU_TENSOR_MAP_SWIZZLE_128B and a 128-byte inner box).
@@ -716,27 +729,32 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(ab), 0));
             } else {
-                float acc[HALF];
+                // fp32 accumulator of this thread's row, 128 columns as 64 packed pairs
+                uint64_t acc[HALF / 2];
 #pragma unroll
-                for (int j = 0; j < HALF; ++j) acc[j] = 0.0f;
+                for (int j = 0; j < HALF / 2; ++j) acc[j] = 0ull;
                 const int nb = n_base / 128;
                 const bool nb_ok = n_base < N;
-                // Scales run two K blocks ahead in registers: block kc + 2's are
-                // fetched right after block kc's partial is released, so a
-                // global load is never waited on inside the promotion.
-                float a0 = (m < M) ? sa[m] : 0.0f;
-                float b0 = nb_ok ? sb[(int64_t)nb * nk] : 0.0f;
-                float a1 = (nk > 1 && m < M) ? sa[(int64_t)M + m] : 0.0f;
-                float b1 = (nk > 1 && nb_ok) ? sb[(int64_t)nb * nk + 1] : 0.0f;
-                for (int kc = 0; kc < nk; ++kc, ++it) {
+                // Scales run PF K blocks ahead in PF register sets (the K loop
+                // unrolled by PF so no register copy waits on a load): block
+                // kc + PF's pair is fetched right after block kc's partial is
+                // released, well before its use.
+                constexpr int PF = 2;   // scale prefetch distance in K blocks (= unroll)
+                float as_[PF], bs_[PF];
+#pragma unroll
+                for (int i = 0; i < PF; ++i) {
+                    as_[i] = (i < nk && m < M) ? sa[(int64_t)i * M + m] : 0.0f;
+                    bs_[i] = (i < nk && nb_ok) ? sb[(int64_t)nb * nk + i] : 0.0f;
+                }
+                // one K block: wait for its partial, promote it, release it
+                auto promote = [&](int kc, float &as, float &bs) -> bool {
                     const uint32_t pb = it % NBUF, use = it / NBUF;
-                    const float sc = __fmul_rn(a0, b0);
-                    a0 = a1;
-                    b0 = b1;
+                    const float sc = __fmul_rn(as, bs);
+                    const uint64_t sc2 = pack_f32x2(__float_as_uint(sc), __float_as_uint(sc));
                     bool w = true;
                     if (lane == 0) w = wait_bar(accf_bar(pb), use & 1u, abort_flag, kErrEpilogue);
                     w = __shfl_sync(0xFFFFFFFFu, w, 0);
-                    if (!w) { ok = false; break; }
+                    if (!w) return false;
                     tc_fence_after();
                     const uint32_t src = tmem + lane_base + pb * BN + ch * HALF;
                     // two 64-column halves, one TMEM round trip each
@@ -745,19 +763,27 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     tmem_ld32_async(src + 32, r + 32);
                     tmem_wait64(r);
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) acc[j] = fmaf(__uint_as_float(r[j]), sc, acc[j]);
+                    for (int j = 0; j < 32; ++j) acc[j] = fma_f32x2(pack_f32x2(r[2 * j], r[2 * j + 1]), sc2, acc[j]);
                     tmem_ld32_async(src + 64, r);
                     tmem_ld32_async(src + 96, r + 32);
                     tmem_wait64(r);
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(pb), 0));
-                    if (kc + 2 < nk) {   // block kc + 2's scales, after the release
-                        a1 = (m < M) ? sa[(int64_t)(kc + 2) * M + m] : 0.0f;
-                        b1 = nb_ok ? sb[(int64_t)nb * nk + kc + 2] : 0.0f;
+                    if (kc + PF < nk) {   // block kc + PF's scales, after the release
+                        as = (m < M) ? sa[(int64_t)(kc + PF) * M + m] : 0.0f;
+                        bs = nb_ok ? sb[(int64_t)nb * nk + kc + PF] : 0.0f;
                     }
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) acc[64 + j] = fmaf(__uint_as_float(r[j]), sc, acc[64 + j]);
+                    for (int j = 0; j < 32; ++j)
+                        acc[32 + j] = fma_f32x2(pack_f32x2(r[2 * j], r[2 * j + 1]), sc2, acc[32 + j]);
+                    ++it;
+                    return true;
+                };
+                for (int kc = 0; ok && kc < nk; kc += PF) {
+#pragma unroll
+                    for (int i = 0; i < PF; ++i)
+                        if (ok && kc + i < nk && !promote(kc + i, as_[i], bs_[i])) ok = false;
                 }
                 if (!ok) break;
                 if (m < M) {
@@ -766,10 +792,10 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         const int col = n_base + g * 8;
                         if (col < N) {
                             uint4 o;
-                            o.x = pack_bf16x2(acc[g * 8 + 0], acc[g * 8 + 1]);
-                            o.y = pack_bf16x2(acc[g * 8 + 2], acc[g * 8 + 3]);
-                            o.z = pack_bf16x2(acc[g * 8 + 4], acc[g * 8 + 5]);
-                            o.w = pack_bf16x2(acc[g * 8 + 6], acc[g * 8 + 7]);
+                            o.x = pack_bf16x2(__uint_as_float((uint32_t)acc[g * 4 + 0]), __uint_as_float((uint32_t)(acc[g * 4 + 0] >> 32)));
+                            o.y = pack_bf16x2(__uint_as_float((uint32_t)acc[g * 4 + 1]), __uint_as_float((uint32_t)(acc[g * 4 + 1] >> 32)));
+                            o.z = pack_bf16x2(__uint_as_float((uint32_t)acc[g * 4 + 2]), __uint_as_float((uint32_t)(acc[g * 4 + 2] >> 32)));
+                            o.w = pack_bf16x2(__uint_as_float((uint32_t)acc[g * 4 + 3]), __uint_as_float((uint32_t)(acc[g * 4 + 3] >> 32)));
                             *reinterpret_cast<uint4 *>(drow + col) = o;
                         }
                     }
