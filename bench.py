@@ -153,6 +153,7 @@ class Workload:
         self.sa = torch.empty(M, dtype=torch.float32, device=d)
         self.sb = torch.empty(N, dtype=torch.float32, device=d)
         self.D = torch.empty((M, N), dtype=torch.bfloat16, device=d)
+        self.ws = f.gemm_workspace(M, N, K, f.SCALE_ROW, device=d)   # split-K tail of the last wave
         self.flops = 2.0 * M * N * K
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.launches = 3
@@ -170,7 +171,7 @@ class Workload:
         f.fp8_quantize_rowwise(self.B, N, K, K, f.E4M3, True, self.qb, self.sb)
         if ev:
             ev[0].record()
-        f.fp8_gemm_scaled(self.qa, f.E4M3, self.qb, f.E4M3, M, N, K, f.SCALE_ROW, self.sa, self.sb, self.D, N)
+        f.fp8_gemm_scaled(self.qa, f.E4M3, self.qb, f.E4M3, M, N, K, f.SCALE_ROW, self.sa, self.sb, self.D, N, self.ws)
         if ev:
             ev[1].record()
 
@@ -260,6 +261,7 @@ class Workload:
         self.sg = torch.empty(1, dtype=torch.float32, device=d)
         self.am = torch.empty(1, dtype=torch.float32, device=d)
         self.DX = torch.empty((M, K_in), dtype=torch.bfloat16, device=d)
+        self.ws = f.gemm_workspace(M, K_in, N_out, f.SCALE_TENSOR, device=d)
         self.t = 0
         self.dims = (M, N_out, K_in)
         self.flops = 2.0 * M * N_out * K_in
@@ -280,7 +282,7 @@ class Workload:
         if ev:
             ev[0].record()
         f.fp8_gemm_scaled(self.qg, f.E5M2, self.wq, f.E4M3, M, K_in, N_out, f.SCALE_TENSOR, self.sg, self.wsinv,
-                          self.DX, K_in)
+                          self.DX, K_in, self.ws)
         if ev:
             ev[1].record()
         self.hist.update(self.am)

@@ -39,6 +39,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -62,7 +63,7 @@ constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_BARS * 8
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 
 enum { kModeTensor = 0, kModeRow = 1, kModeBlock = 2 };
-enum : uint32_t { kErrProducer = 1u, kErrMma = 2u, kErrEpilogue = 4u, kErrDrain = 8u };
+enum : uint32_t { kErrProducer = 1u, kErrMma = 2u, kErrEpilogue = 4u, kErrDrain = 8u, kErrSplit = 16u };
 
 __device__ unsigned int g_gemm_error;
 
@@ -126,6 +127,32 @@ __device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity) {
         }
     }
     return true;
+}
+// Split-K hand-off flag: the first-half pair publishes its partial with a
+// release store of the launch's epoch; the second-half pair polls with
+// acquire loads (bounded, like every wait in this file).
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u32(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool wait_flag(const uint32_t *p, uint32_t epoch, volatile uint32_t *abort_flag) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (ld_acquire_u32(p) == epoch) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > kTimeoutNs) {
+                atomicOr(&g_gemm_error, kErrSplit);
+                *abort_flag = 1u;
+                return false;
+            }
+        }
+        __nanosleep(32);
+    }
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
     asm volatile(
@@ -488,9 +515,13 @@ struct Cfg {
     static constexpr int STAGE = A_TILE + B_HALF;
     static constexpr int STAGES = (BN == 256) ? 6 : 8;
     static constexpr int NBUF = 512 / BN;
-    static constexpr int NBARS = 2 * STAGES + 2 * NBUF + 1;
+    static constexpr int NBARS = 2 * STAGES + 2 * NBUF + 2;   // + drain, + split partial written
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + NBARS * 8 + 16;
 };
+// Split-K tail workspace: per split tile, per CTA of the pair, a 128 x 256
+// fp32 partial stored column-major (row index fastest, so a warp's lanes write
+// consecutive words), then one flag word per (tile, CTA).
+constexpr size_t kSplitPartialFloats = 128 * 256;
 }  // namespace sm2
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -546,7 +577,8 @@ template <int MODE, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
 k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                int K, uint32_t idesc, const float *__restrict__ sa, const float *__restrict__ sb,
-               __nv_bfloat16 *__restrict__ D, int64_t ldd) {
+               __nv_bfloat16 *__restrict__ D, int64_t ldd, int full_tiles, int split_units,
+               float *__restrict__ ws, uint32_t *__restrict__ flags, uint32_t epoch) {
     using C = sm2::Cfg<BN>;
     constexpr int STG = C::STAGES, NBUF = C::NBUF;
     constexpr int HALF = BN / 2;             // columns per epilogue warp
@@ -561,15 +593,27 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const uint32_t rank = cluster_rank();
     const bool leader = (rank == 0);
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int num_m = (M + 255) / 256, num_n = (N + BN - 1) / BN;
-    const int num_tiles = num_m * num_n;
+    const int num_m = (M + 255) / 256;
     const int nk = (K + BK - 1) / BK;
+    // Work items of this pair: whole tiles pair, pair + npairs, ... below
+    // full_tiles, then (pair < split_units) one half of a split tail tile:
+    // tile full_tiles + pair / 2, K blocks [0, nk/2) for the even pair and
+    // [nk/2, nk) for the odd one.  With no split, full_tiles = every tile.
+    const int n_full = (pair < full_tiles) ? (full_tiles - 1 - pair) / npairs + 1 : 0;
+    const int n_items = n_full + (pair < split_units ? 1 : 0);
+    struct Item { int tile, k0, k1, half; };
+    auto item = [&](int i) -> Item {
+        if (i < n_full) return Item{pair + i * npairs, 0, nk, -1};
+        const int h = pair & 1, kh = nk / 2;
+        return Item{full_tiles + pair / 2, h ? kh : 0, h ? nk : kh, h};
+    };
 
     auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
     auto empty_bar = [&](int s) { return smem_u32(&bars[STG + s]); };
     auto accf_bar = [&](int b) { return smem_u32(&bars[2 * STG + b]); };
     auto acce_bar = [&](int b) { return smem_u32(&bars[2 * STG + NBUF + b]); };
     const uint32_t drain_bar = smem_u32(&bars[2 * STG + 2 * NBUF]);
+    const uint32_t part_bar = smem_u32(&bars[2 * STG + 2 * NBUF + 1]);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STG; ++s) {
@@ -581,6 +625,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             mbar_init(acce_bar(b), 2 * sm2::EPI);
         }
         mbar_init(drain_bar, 1);
+        mbar_init(part_bar, sm2::EPI);
         *abort_flag = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
@@ -607,11 +652,12 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int s = 0; s < STG; ++s) last_round[s] = -1;
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
-                const int m_blk = tile % num_m, n_blk = tile / num_m;
+            for (int i = 0; ok && i < n_items; ++i) {
+                const Item w = item(i);
+                const int m_blk = w.tile % num_m, n_blk = w.tile / num_m;
                 const int a_row = m_blk * 256 + (int)rank * 128;
                 const int b_row = n_blk * BN + (int)rank * HALF;
-                for (int kc = 0; kc < nk; ++kc, ++it) {
+                for (int kc = w.k0; kc < w.k1; ++kc, ++it) {
                     const int stage = it % STG;
                     const uint32_t round = it / STG;
                     if (!wait_bar(empty_bar(stage), (round & 1u) ^ 1u, abort_flag, kErrProducer)) {
@@ -638,7 +684,8 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (leader && lane == 0) {
             uint32_t it = 0, lt = 0;
             bool ok = true;
-            for (int tile = pair; ok && tile < num_tiles; tile += npairs, ++lt) {
+            for (int i = 0; ok && i < n_items; ++i, ++lt) {
+                const Item w = item(i);
                 uint32_t d_tmem = tmem;
                 if (MODE != kModeBlock) {
                     const uint32_t ab = lt % NBUF, use = lt / NBUF;
@@ -646,7 +693,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     tc_fence_after();
                     d_tmem = tmem + ab * BN;
                 }
-                for (int kc = 0; kc < nk; ++kc, ++it) {
+                for (int kc = w.k0; kc < w.k1; ++kc, ++it) {
                     const int stage = it % STG;
                     const uint32_t round = it / STG;
                     if (MODE == kModeBlock) {
@@ -661,7 +708,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     const uint64_t bdesc = sdesc_k_sw128(a_addr + A_TILE);
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) {
-                        const uint32_t acc = (MODE == kModeBlock) ? (k > 0) : (kc > 0 || k > 0);
+                        const uint32_t acc = (MODE == kModeBlock) ? (k > 0) : (kc > w.k0 || k > 0);
                         tc_mma_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, acc);
                     }
                     tc_commit_pair_both(empty_bar(stage));
@@ -683,8 +730,9 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
         uint32_t it = 0, lt = 0;
         bool ok = true;
-        for (int tile = pair; ok && tile < num_tiles; tile += npairs, ++lt) {
-            const int m_blk = tile % num_m, n_blk = tile / num_m;
+        for (int i = 0; ok && i < n_items; ++i, ++lt) {
+            const Item wi = item(i);
+            const int m_blk = wi.tile % num_m, n_blk = wi.tile / num_m;
             const int m = m_blk * 256 + (int)rank * 128 + sp * 32 + lane;
             const int n_base = n_blk * BN + ch * HALF;
             __nv_bfloat16 *drow = D + (int64_t)m * ldd;
@@ -698,11 +746,37 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 w = __shfl_sync(0xFFFFFFFFu, w, 0);
                 if (!w) break;
                 tc_fence_after();
+                // split tail tile: this CTA's 128 x 256 partial in the workspace
+                float *part = nullptr;
+                uint32_t *flag = nullptr;
+                if (wi.half >= 0) {
+                    const int slot = wi.tile - full_tiles;
+                    part = ws + ((size_t)slot * 2 + rank) * sm2::kSplitPartialFloats + (sp * 32 + lane);
+                    flag = flags + slot * 2 + rank;
+                    if (wi.half == 1) {   // wait for the first half's partial
+                        bool f = true;
+                        if (lane == 0) f = wait_flag(flag, epoch, abort_flag);
+                        f = __shfl_sync(0xFFFFFFFFu, f, 0);
+                        if (!f) break;
+                        (void)ld_acquire_u32(flag);   // acquire on every lane
+                    }
+                }
 #pragma unroll 1
                 for (int c = 0; c < HALF / 32; ++c) {
                     float v[32];
                     tmem_ld32(tmem + lane_base + ab * BN + ch * HALF + c * 32, v);
                     const int col0 = n_base + c * 32;
+                    if (wi.half == 0) {   // first half: store the raw fp32 partial, no output
+                        float *pc = part + (size_t)(ch * HALF + c * 32) * 128;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) pc[(size_t)j * 128] = v[j];
+                        continue;
+                    }
+                    if (wi.half == 1) {   // second half: add the first half's partial (fixed order)
+                        const float *pc = part + (size_t)(ch * HALF + c * 32) * 128;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = v[j] + pc[(size_t)j * 128];
+                    }
                     if (MODE == kModeRow) {
                         const float cb = (col0 + lane < N) ? sb[col0 + lane] : 0.0f;
 #pragma unroll
@@ -728,6 +802,14 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(ab), 0));
+                if (wi.half == 0) {   // publish: every epilogue warp's stores, then the flag
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(part_bar);
+                    if (warp == 4 && lane == 0) {
+                        if (wait_bar(part_bar, 0u, abort_flag, kErrSplit)) st_release_u32(flag, epoch);
+                    }
+                }
             } else {
                 // fp32 accumulator of this thread's row, 128 columns as 64 packed pairs
                 uint64_t acc[HALF / 2];
@@ -895,13 +977,38 @@ int pair_capacity() {
     return n;
 }
 
+// Split-K plan for a grid of `cap` CTA pairs.  When all tiles fit in half
+// the pairs, each tile is computed as two K halves on two pairs (twice the
+// tensor cores on the problem).  The kernel also supports splitting only the
+// last wave of a multi-wave grid (full_tiles > 0), but measured at 4096^3 the
+// half-empty last wave already runs uncontended and faster than a full one,
+// so the fp32 hand-off did not pay (63.5 vs 61.4 us): the plan splits only
+// single-wave problems.
+struct SplitPlan { int full_tiles, units; size_t bytes; };
+SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int cap) {
+    const int tiles = (int)(((M + 255) / 256) * ((N + 255) / 256));
+    const int nk = (int)((K + BK - 1) / BK);
+    const int r = tiles % cap;
+    if (cap <= 0 || nk < 2 || r == 0 || tiles >= cap || 2 * r > cap) return SplitPlan{tiles, 0, 0};
+    const size_t flags_off = (size_t)r * 2 * sm2::kSplitPartialFloats * sizeof(float);
+    return SplitPlan{tiles - r, 2 * r, flags_off + (((size_t)r * 2 * sizeof(uint32_t) + 255) & ~(size_t)255)};
+}
+
 template <int MODE, int BN>
 cudaError_t launch_gemm_2sm(cudaStream_t st, const CUtensorMap &ta, const CUtensorMap &tb, int M, int N, int K,
-                            uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd, int pairs_cap) {
+                            uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd, int pairs_cap,
+                            const SplitPlan &plan, void *ws, uint32_t epoch) {
     const int tiles = ((M + 255) / 256) * ((N + BN - 1) / BN);
-    const int pairs = std::max(1, std::min(tiles, pairs_cap));
+    // with a split, full_tiles is a whole number of waves of pairs_cap pairs
+    // (or zero, when the split halves are all the work)
+    const int pairs = plan.units ? (plan.full_tiles > 0 ? pairs_cap : plan.units) : std::max(1, std::min(tiles, pairs_cap));
+    float *part = static_cast<float *>(ws);
+    uint32_t *flags = plan.units ? reinterpret_cast<uint32_t *>(static_cast<char *>(ws) +
+                                                                (size_t)(plan.units / 2) * 2 * sm2::kSplitPartialFloats * sizeof(float))
+                                 : nullptr;
     k_gemm_fp8_2sm<MODE, BN><<<2 * pairs, sm2::THREADS, sm2::Cfg<BN>::SMEM, st>>>(
-        ta, tb, M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd);
+        ta, tb, M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd,
+        plan.units ? plan.full_tiles : tiles, plan.units, part, flags, epoch);
     return cudaPeekAtLastError();
 }
 
@@ -915,9 +1022,29 @@ uint32_t make_idesc(fp8_format fa, fp8_format fb, int mma_m, int mma_n) {
 
 using namespace fp8q_host;
 
+namespace {
+std::atomic<uint32_t> g_split_epoch[64];   // per device; a split launch publishes with a fresh value
+}
+
+extern "C" fp8_status fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8_scale_mode mode, size_t *bytes) {
+    if (!bytes) return FP8_ERR_INVALID_ARG;
+    if (mode != FP8_SCALE_TENSOR && mode != FP8_SCALE_ROW && mode != FP8_SCALE_BLOCK) return FP8_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0) return FP8_ERR_SHAPE;
+    *bytes = 0;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (mode == FP8_SCALE_BLOCK || M <= BM || N == 0 || K == 0) return FP8_OK;
+    const int cap = (mode == FP8_SCALE_TENSOR) ? pair_capacity<kModeTensor, 256>() : pair_capacity<kModeRow, 256>();
+    if (cap <= 0) return FP8_ERR_CUDA;
+    *bytes = split_plan(M, N, K, cap).bytes;
+    return FP8_OK;
+}
+
 extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int64_t M,
                                       int64_t N, int64_t K, fp8_scale_mode mode, const float *a_scale_inv,
-                                      const float *b_scale_inv, void *D_bf16, int64_t ldd, void *stream) {
+                                      const float *b_scale_inv, void *D_bf16, int64_t ldd, void *workspace,
+                                      size_t workspace_bytes, void *stream) {
     if ((fa != FP8_E4M3 && fa != FP8_E5M2) || (fb != FP8_E4M3 && fb != FP8_E5M2)) return FP8_ERR_INVALID_ARG;
     if (mode != FP8_SCALE_TENSOR && mode != FP8_SCALE_ROW && mode != FP8_SCALE_BLOCK) return FP8_ERR_INVALID_ARG;
     if (M < 0 || N < 0 || K < 0 || ldd < N) return FP8_ERR_SHAPE;
@@ -931,6 +1058,7 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
     if (!D_bf16) return FP8_ERR_INVALID_ARG;
     if (K > 0 && (!A || !B || !a_scale_inv || !b_scale_inv)) return FP8_ERR_INVALID_ARG;
     if (!aligned16(D_bf16) || (A && !aligned16(A)) || (B && !aligned16(B))) return FP8_ERR_ALIGNMENT;
+    if (workspace && !aligned16(workspace)) return FP8_ERR_ALIGNMENT;
     int sms;
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
@@ -946,15 +1074,30 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
         const uint32_t idesc = make_idesc(fa, fb, 256, 256);
         cudaError_t e = cudaErrorUnknown;
         int cap;
+        const int dev_cap = (mode == FP8_SCALE_TENSOR) ? pair_capacity<kModeTensor, 256>()
+                            : (mode == FP8_SCALE_ROW) ? pair_capacity<kModeRow, 256>() : pair_capacity<kModeBlock, 256>();
+        if (dev_cap <= 0) return FP8_ERR_CUDA;
+        SplitPlan plan{(int)(((M + 255) / 256) * ((N + 255) / 256)), 0, 0};
+        uint32_t epoch = 0;
+        if (mode != FP8_SCALE_BLOCK && workspace) {
+            const SplitPlan sp = split_plan(M, N, K, dev_cap);
+            if (sp.units > 0 && workspace_bytes >= sp.bytes) {
+                int dev = 0;
+                if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
+                plan = sp;
+                epoch = ++g_split_epoch[dev];
+                if (epoch == 0) epoch = ++g_split_epoch[dev];   // 0 is what a fresh workspace holds
+            }
+        }
         if (mode == FP8_SCALE_TENSOR) {
             if ((cap = pair_capacity<kModeTensor, 256>()) > 0)
-                e = launch_gemm_2sm<kModeTensor, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap);
+                e = launch_gemm_2sm<kModeTensor, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap, plan, workspace, epoch);
         } else if (mode == FP8_SCALE_ROW) {
             if ((cap = pair_capacity<kModeRow, 256>()) > 0)
-                e = launch_gemm_2sm<kModeRow, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap);
+                e = launch_gemm_2sm<kModeRow, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap, plan, workspace, epoch);
         } else {
             if ((cap = pair_capacity<kModeBlock, 256>()) > 0)
-                e = launch_gemm_2sm<kModeBlock, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap);
+                e = launch_gemm_2sm<kModeBlock, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap, plan, workspace, epoch);
         }
         return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
     }

@@ -36,7 +36,8 @@ SIGNATURES = {
     "fp8_quantize_tensorwise": (_S, [_P, _I64, _I64, _I, _P, _P, _I, _P, _P, _P, _P]),
     "fp8_quantize_rowwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
     "fp8_quantize_blockwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
-    "fp8_gemm_scaled": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
+    "fp8_gemm_scaled": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P, ctypes.c_size_t, _P]),
+    "fp8_gemm_workspace_size": (_S, [_I64, _I64, _I64, _I, _P]),
     "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
     "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
@@ -135,12 +136,20 @@ def fp8_quantize_blockwise(x, rows, cols, ld, fmt, block_rows, q, scale_inv, str
         _ptr(x), rows, cols, ld, fmt, block_rows, _ptr(q), _ptr(scale_inv), _stream(stream)))
 
 
-def fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, ldd, stream=None):
+def fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, ldd, workspace=None,
+                    stream=None):
     _dev(A, torch.uint8, "A"); _dev(B, torch.uint8, "B"); _dev(D, torch.bfloat16, "D")
     _dev(a_scale_inv, torch.float32, "a_scale_inv"); _dev(b_scale_inv, torch.float32, "b_scale_inv")
+    _dev(workspace, torch.uint8, "workspace")
     _check("fp8_gemm_scaled", lib().fp8_gemm_scaled(
         _ptr(A), fa, _ptr(B), fb, M, N, K, mode, _ptr(a_scale_inv), _ptr(b_scale_inv), _ptr(D), ldd,
-        _stream(stream)))
+        _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+def fp8_gemm_workspace_size(M, N, K, mode) -> int:
+    b = ctypes.c_size_t(0)
+    _check("fp8_gemm_workspace_size", lib().fp8_gemm_workspace_size(M, N, K, mode, ctypes.byref(b)))
+    return int(b.value)
 
 
 def fp8_amax_history_update(history, pos, amax_cur, fmt, scale, scale_inv, saturated, stream=None):
@@ -210,11 +219,17 @@ def quantize_blockwise(x, fmt=E4M3, block_rows=1):
     return q, sinv
 
 
-def gemm(A, fa, B, fb, mode, a_scale_inv, b_scale_inv, out=None):
+def gemm_workspace(M, N, K, mode, device="cuda"):
+    """Zero-filled workspace of the size fp8_gemm_scaled can use (None if 0)."""
+    n = fp8_gemm_workspace_size(M, N, K, mode)
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
+
+
+def gemm(A, fa, B, fb, mode, a_scale_inv, b_scale_inv, out=None, workspace=None):
     M, K = A.shape
     N = B.shape[0]
     D = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
-    fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, D.stride(0))
+    fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, D.stride(0), workspace)
     return D
 
 

@@ -35,6 +35,7 @@
 #ifndef FP8Q_H
 #define FP8Q_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -144,14 +145,32 @@ FP8Q_API fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int
  *                K block accumulated on the tensor cores, then promoted into
  *                an fp32 register accumulator with its two scales).
  *   D  [M, N] bf16 with leading dimension ldd (elements).
- *   The result is deterministic (fixed K order, no split-K).
+ *   workspace / workspace_bytes: optional device scratch (NULL, 0 = none).
+ *       With at least fp8_gemm_workspace_size() bytes, a problem whose
+ *       256 x 256 tiles fill at most half of the GPU's CTA pairs (few tiles,
+ *       long K) has each tile computed as two K halves on two CTA pairs, the
+ *       first half handing its fp32 partial to the second through the
+ *       workspace (TENSOR and ROW modes, M > 128).  The
+ *       workspace must be zero-filled when first allocated; later calls leave
+ *       it in a state the next call accepts.  Calls that share a workspace
+ *       must not overlap on the device.  A workspace belongs to one device.
+ *   The result is deterministic: a fixed K order per tile and a fixed
+ *   summation order for split tiles (second half + first half), so repeated
+ *   calls with the same shapes and workspace setting are bit-identical.
  *   Shapes: M, N, K >= 0; K % 16 == 0; N % 8 == 0; ldd % 8 == 0, ldd >= N.
- *   K == 0 writes zeros.
+ *   K == 0 writes zeros.  workspace 16-byte aligned.
  */
 FP8Q_API fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
                            int64_t M, int64_t N, int64_t K, fp8_scale_mode mode,
                            const float *a_scale_inv, const float *b_scale_inv, void *D_bf16,
-                           int64_t ldd, void *stream);
+                           int64_t ldd, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of workspace fp8_gemm_scaled can use for this shape on the current
+ * device (0: the shape fills whole waves, or the mode takes none).
+ */
+FP8Q_API fp8_status fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8_scale_mode mode,
+                                            size_t *bytes);
 
 /*
  * Delayed-scaling update ([DeepL] §2.3: the scale of a step is predicted

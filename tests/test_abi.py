@@ -50,14 +50,14 @@ def test_validation_before_device_access():
     L = fp8q.lib()
     n = P(0)
     # GEMM: bad format, bad mode, K % 16, N % 8, null D, misaligned A
-    assert L.fp8_gemm_scaled(FAKE, 3, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 64, n) == INVALID
-    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 5, FAKE, FAKE, FAKE, 64, n) == INVALID
-    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 40, 0, FAKE, FAKE, FAKE, 64, n) == SHAPE
-    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 60, 64, 0, FAKE, FAKE, FAKE, 64, n) == ALIGN
-    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, None, 64, n) == INVALID
-    assert L.fp8_gemm_scaled(FAKE_ODD, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 64, n) == ALIGN
-    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, -1, 64, 64, 0, FAKE, FAKE, FAKE, 64, n) == SHAPE
-    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 32, n) == SHAPE  # ldd < N
+    assert L.fp8_gemm_scaled(FAKE, 3, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 64, None, 0, n) == INVALID
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 5, FAKE, FAKE, FAKE, 64, None, 0, n) == INVALID
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 40, 0, FAKE, FAKE, FAKE, 64, None, 0, n) == SHAPE
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 60, 64, 0, FAKE, FAKE, FAKE, 64, None, 0, n) == ALIGN
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, None, 64, None, 0, n) == INVALID
+    assert L.fp8_gemm_scaled(FAKE_ODD, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 64, None, 0, n) == ALIGN
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, -1, 64, 64, 0, FAKE, FAKE, FAKE, 64, None, 0, n) == SHAPE
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 32, None, 0, n) == SHAPE  # ldd < N
     # quantizers
     assert L.fp8_quantize_rowwise(FAKE, 4, 24, 32, 0, 1, FAKE, FAKE, n) == SHAPE
     assert L.fp8_quantize_rowwise(FAKE, 4, 16, 20, 0, 1, FAKE, FAKE, n) == ALIGN
@@ -65,6 +65,10 @@ def test_validation_before_device_access():
     assert L.fp8_quantize_blockwise(FAKE, 4, 32, 32, 0, 64, FAKE, FAKE, n) == INVALID
     assert L.fp8_quantize_tensorwise(FAKE, 4, 32, 0, None, FAKE, 0, FAKE, None, None, n) == INVALID
     assert L.fp8_quantize_tensorwise(FAKE, 4, 40, 0, FAKE, FAKE, 1, FAKE, None, None, n) == SHAPE
+    assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 256, 256, 256, 0, FAKE, FAKE, FAKE, 256, FAKE_ODD, 1024, n) == ALIGN
+    assert L.fp8_gemm_workspace_size(64, 64, 64, 9, ctypes.byref(ctypes.c_size_t())) == INVALID
+    assert L.fp8_gemm_workspace_size(-1, 64, 64, 0, ctypes.byref(ctypes.c_size_t())) == SHAPE
+    assert L.fp8_gemm_workspace_size(64, 64, 64, 0, None) == INVALID
     assert L.fp8_amax(FAKE_ODD, 100, FAKE, None, n) == ALIGN
     assert L.fp8_amax(FAKE, -1, FAKE, None, n) == SHAPE
     assert L.fp8_amax(FAKE, 10, None, None, n) == INVALID

@@ -177,3 +177,43 @@ def test_gemm_blockwise_mlp_sampled(orc, which):
     B, db = orc.quantize_blockwise(w, 0, 128)
     D = _run(A, 0, B, 0, 2, da, db)
     _sampled_check(orc, D, A, 0, B, 0, 2, da, db, n=2048)
+
+
+# ---------------------------------------------------- split-K tail (workspace) --
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("shape", [(512, 512, 512), (300, 272, 400), (768, 520, 384)])
+def test_gemm_split_tail_full_compare_and_repeatable(orc, mode, shape):
+    """With a workspace, the tiles of a partly filled last wave are computed
+    as two K halves on two CTA pairs; the result stays within tolerance of the
+    oracle and is bit-identical over repeated calls (the hand-off flag is a
+    fresh epoch per call, so a reused workspace is safe)."""
+    M, N, K = shape
+    A, da, B, db = _operands(orc, mode, M, N, K, seed=M + 3 * N + K)
+    ws = fp8q.gemm_workspace(M, N, K, mode)
+    assert ws is not None and ws.numel() > 0
+    A_, B_, da_, db_ = _cuda(A), _cuda(B), _cuda(da), _cuda(db)
+    D1 = fp8q.gemm(A_, 0, B_, 0, mode, da_, db_, workspace=ws)
+    ref, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
+    assert_gemm_close(bf16_to_f64(D1), ref, mag)
+    for _ in range(3):
+        assert torch.equal(fp8q.gemm(A_, 0, B_, 0, mode, da_, db_, workspace=ws), D1)
+    # too small a workspace: the unsplit schedule, still correct
+    small = torch.zeros(ws.numel() - 256, dtype=torch.uint8, device="cuda")
+    D0 = fp8q.gemm(A_, 0, B_, 0, mode, da_, db_, workspace=small)
+    assert_gemm_close(bf16_to_f64(D0), ref, mag)
+
+
+def test_gemm_split_k_long_k_sampled(orc):
+    """A skinny, long-K GEMM (1024 x 1024 x 16384: 16 tiles for ~74 CTA
+    pairs) runs as 32 K halves with a workspace; sampled against the oracle."""
+    M, N, K = 1024, 1024, 16384
+    a = inputs.bf16_bits(inputs.outlier_activations_bf16((M, K), seed=11, device="cuda"))
+    b = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, seed=12, device="cuda"))
+    A, da = orc.quantize_rowwise(a, 0, True)
+    B, db = orc.quantize_rowwise(b, 0, True)
+    ws = fp8q.gemm_workspace(M, N, K, 1)
+    assert ws is not None
+    D = fp8q.gemm(_cuda(A), 0, _cuda(B), 0, 1, _cuda(da), _cuda(db), workspace=ws)
+    _sampled_check(orc, D, A, 0, B, 0, 1, da, db, n=1024, seed=4)
+    assert fp8q.fp8_gemm_workspace_size(4096, 4096, 4096, 1) == 0   # multi-wave: no split
