@@ -1126,3 +1126,52 @@ extern "C" fp8_status fp8_device_error(uint32_t *host_out, int clear) {
     }
     return FP8_OK;
 }
+
+// ---------------------------------------------- entry point without allocation --
+// Some callers cannot allocate device memory at the point where they run the
+// GEMM: code inside a framework that owns every device byte through its own
+// caching allocator, or latency-critical paths where cudaMalloc's implicit
+// device synchronisation is not acceptable.  fp8_gemm_scaled_noalloc gives
+// them the split-K schedule without a caller workspace: the scratch lives in
+// this file-scope array, which every GPU that loads the library holds until
+// the process exits.
+constexpr size_t kNoAllocScratchBytes = (size_t)10 << 20;   // 10 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64];   // device address of g_noalloc_scratch, per device
+}
+
+// One-time set-up per device (with that device current): look up the
+// array's device address and clear it on the caller's stream.
+static fp8_status noalloc_scratch(cudaStream_t stream, void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return FP8_ERR_CUDA;
+    if (dev >= 64) return FP8_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress((void **)&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return FP8_ERR_CUDA;
+        if (cudaMemsetAsync(ptr, 0, kNoAllocScratchBytes, stream) != cudaSuccess) return FP8_ERR_CUDA;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return FP8_OK;
+}
+
+extern "C" fp8_status fp8_gemm_scaled_noalloc(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
+                                              int64_t M, int64_t N, int64_t K, fp8_scale_mode mode,
+                                              const float *a_scale_inv, const float *b_scale_inv, void *D_bf16,
+                                              int64_t ldd, void *stream) {
+    size_t need = 0;
+    fp8_status st = fp8_gemm_workspace_size(M, N, K, mode, &need);
+    if (st != FP8_OK) return st;
+    if (need > kNoAllocScratchBytes) return FP8_ERR_SHAPE;   // the split needs more than the built-in scratch
+    void *scratch = nullptr;
+    if (need > 0) {
+        st = noalloc_scratch(as_stream(stream), &scratch);
+        if (st != FP8_OK) return st;
+    }
+    return fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D_bf16, ldd, scratch, need, stream);
+}

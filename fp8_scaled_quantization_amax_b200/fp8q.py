@@ -38,6 +38,7 @@ SIGNATURES = {
     "fp8_quantize_blockwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
     "fp8_gemm_scaled": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P, ctypes.c_size_t, _P]),
     "fp8_gemm_workspace_size": (_S, [_I64, _I64, _I64, _I, _P]),
+    "fp8_gemm_scaled_noalloc": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
     "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
     "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
@@ -144,6 +145,16 @@ def fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, ld
     _check("fp8_gemm_scaled", lib().fp8_gemm_scaled(
         _ptr(A), fa, _ptr(B), fb, M, N, K, mode, _ptr(a_scale_inv), _ptr(b_scale_inv), _ptr(D), ldd,
         _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+def fp8_gemm_scaled_noalloc(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, ldd, stream=None):
+    """fp8_gemm_scaled with the split-K scratch built into the library (for
+    callers that cannot allocate device memory; see include/fp8q.h)."""
+    _dev(A, torch.uint8, "A"); _dev(B, torch.uint8, "B"); _dev(D, torch.bfloat16, "D")
+    _dev(a_scale_inv, torch.float32, "a_scale_inv"); _dev(b_scale_inv, torch.float32, "b_scale_inv")
+    _check("fp8_gemm_scaled_noalloc", lib().fp8_gemm_scaled_noalloc(
+        _ptr(A), fa, _ptr(B), fb, M, N, K, mode, _ptr(a_scale_inv), _ptr(b_scale_inv), _ptr(D), ldd,
+        _stream(stream)))
 
 
 def fp8_gemm_workspace_size(M, N, K, mode) -> int:

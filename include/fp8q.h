@@ -173,6 +173,31 @@ FP8Q_API fp8_status fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8
                                             size_t *bytes);
 
 /*
+ * fp8_gemm_scaled for callers that cannot allocate device memory where they
+ * run the GEMM (for example code inside a framework whose own caching
+ * allocator owns every device byte, or latency-critical paths that cannot
+ * afford cudaMalloc's implicit device synchronisation).  The source pages
+ * have no counterpart to this entry point; it is a service of this library.
+ *   Same arguments and result as fp8_gemm_scaled without the workspace: the
+ *   split-K scratch comes from a 10 MiB array built into the library, which
+ *   every GPU that loads the library holds until the process exits.  The
+ *   caller still passes A, B, the scales and D.
+ *   Returns FP8_ERR_SHAPE when the shape's split needs more scratch than the
+ *   10 MiB (fp8_gemm_workspace_size() > 10 MiB); nothing is enqueued then.
+ *   The first call on a device that needs the scratch does a one-time
+ *   set-up (looks up the array's device address, clears it on `stream`);
+ *   make that first call before any stream capture.
+ *   Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents; calls that overlap on the GPU (other streams, other threads)
+ *   race on it.
+ */
+FP8Q_API fp8_status fp8_gemm_scaled_noalloc(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
+                                            int64_t M, int64_t N, int64_t K, fp8_scale_mode mode,
+                                            const float *a_scale_inv, const float *b_scale_inv, void *D_bf16,
+                                            int64_t ldd, void *stream);
+
+/*
  * Delayed-scaling update ([DeepL] §2.3: the scale of a step is predicted
  * from the statistics of previous steps; a deviation above a threshold
  * forces recomputation).  In order:
