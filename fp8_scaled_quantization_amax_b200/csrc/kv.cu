@@ -4,13 +4,14 @@
 // in FP8 halve the cache; each is dequantized when attention reads it).
 //
 // Quantize: a (b, h) slice (S*Dh elements, 2 MiB of bf16 at S=8192, Dh=128)
-// needs its own amax before any element can be cast.  One 4-CTA thread-block
-// cluster owns one slice at a time: every CTA streams its quarter of the
-// slice from HBM for the amax (loads marked L2 evict-last), the four partial
-// maxima meet through distributed shared memory behind a cluster barrier, and
-// the cast pass re-reads the same quarter from L2 (loads and FP8 stores
-// marked evict-first, so the slices still waiting for their second pass stay
-// resident; about 37 clusters x 2 MiB are in flight against the 126 MB L2).
+// needs its own amax before any element can be cast.  One 8-CTA thread-block
+// cluster (two 512-thread CTAs per SM) owns one slice at a time: every CTA
+// streams its eighth of the slice from HBM for the amax (loads marked L2
+// evict-last), the eight partial maxima meet through distributed shared
+// memory behind a cluster barrier, and the cast pass re-reads the same eighth
+// from L2 (loads and FP8 stores marked evict-first, so the slices still
+// waiting for their second pass stay resident; about 37 clusters x 2 MiB are
+// in flight against the 126 MB L2).
 // HBM traffic is the algorithmic 2 B in + 1 B out per element, in one
 // launch, with no scratch memory and no grid-wide wait.
 //
@@ -30,11 +31,11 @@ using namespace fp8q;
 
 namespace {
 
-constexpr int kClusterCtas = 4;
-constexpr int kKvThreads = 1024;
+constexpr int kClusterCtas = 8;
+constexpr int kKvThreads = 512;
 
 template <int FMT>
-__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kKvThreads, 1)
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kKvThreads, 2)
 k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64_t nunit,
            float *__restrict__ scale_inv) {
     __shared__ uint32_t red[32];

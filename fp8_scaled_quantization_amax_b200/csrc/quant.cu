@@ -183,63 +183,90 @@ k_cast_transpose(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64
 }
 
 // --------------------------------------------------------------- rowwise --
-// One CTA (128 threads) per row, the row held in registers (V vectors of 8
-// per thread) between the amax and the cast: one HBM read per element.
+// A CTA (128 threads) quantizes R rows at a time, every row held in registers
+// (V vectors of 8 per thread) between its amax and its cast: one HBM read per
+// element, and all R rows' loads are issued before the first reduction.
 // V == 0: rows too long for registers, two passes (the second from L2).
 constexpr int kRowThreads = 128;
-template <int FMT, bool POW2, int V>
+template <int FMT, bool POW2, int V, int R>
 __global__ void __launch_bounds__(kRowThreads)
 k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
           uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
-    __shared__ uint32_t red[32];
+    __shared__ uint32_t red[R][32];
     constexpr float fm = fmax_of<FMT>();
     const int64_t ncv = cols / 8;
-    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-        const uint4 *xr = reinterpret_cast<const uint4 *>(x + r * ld);
-        uint2 *qr = reinterpret_cast<uint2 *>(q + r * cols);
-        uint32_t m;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int64_t r0 = (int64_t)blockIdx.x * R; r0 < rows; r0 += (int64_t)gridDim.x * R) {
         if constexpr (V > 0) {
-            uint4 v[V];
-            uint32_t m2 = 0;
+            uint4 v[R][V];
+            uint32_t m[R];
 #pragma unroll
-            for (int j = 0; j < V; ++j) {
-                const int64_t cv = threadIdx.x + j * kRowThreads;
-                v[j] = cv < ncv ? ld_stream(xr + cv) : make_uint4(0, 0, 0, 0);
-                m2 = amax_fast8(m2, v[j]);
-            }
-            m = amax_fast_final(m2);
-            if (m == 0xFFFFFFFFu) {
-                uint32_t bad = 0;
-                m = 0;
+            for (int rr = 0; rr < R; ++rr) {
+                const uint4 *xr = reinterpret_cast<const uint4 *>(x + (r0 + rr) * ld);
+                const bool row_ok = r0 + rr < rows;
 #pragma unroll
-                for (int j = 0; j < V; ++j) m = amax_exact8(m, v[j], bad);
+                for (int j = 0; j < V; ++j) {
+                    const int64_t cv = threadIdx.x + j * kRowThreads;
+                    v[rr][j] = (row_ok && cv < ncv) ? ld_stream(xr + cv) : make_uint4(0, 0, 0, 0);
+                }
             }
-            m = block_max_u32(m, red);
-            const float a = bf16bits_to_float(m);
-            const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
 #pragma unroll
-            for (int j = 0; j < V; ++j) {
-                const int64_t cv = threadIdx.x + j * kRowThreads;
-                if (cv < ncv) qr[cv] = cast8<FMT>(v[j], s);
+            for (int rr = 0; rr < R; ++rr) {
+                uint32_t m2 = 0;
+#pragma unroll
+                for (int j = 0; j < V; ++j) m2 = amax_fast8(m2, v[rr][j]);
+                m[rr] = amax_fast_final(m2);
+                if (m[rr] == 0xFFFFFFFFu) {
+                    uint32_t bad = 0;
+                    m[rr] = 0;
+#pragma unroll
+                    for (int j = 0; j < V; ++j) m[rr] = amax_exact8(m[rr], v[rr][j], bad);
+                }
+                m[rr] = __reduce_max_sync(0xFFFFFFFFu, m[rr]);
+                if (lane == 0) red[rr][warp] = m[rr];
             }
-            if (threadIdx.x == 0) scale_inv[r] = __fdiv_rn(1.0f, s);
+            __syncthreads();
+#pragma unroll
+            for (int rr = 0; rr < R; ++rr) {
+                uint32_t mm = lane < kRowThreads / 32 ? red[rr][lane] : 0u;
+                mm = __reduce_max_sync(0xFFFFFFFFu, mm);
+                const float a = bf16bits_to_float(mm);
+                const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
+                if (r0 + rr < rows) {
+                    uint2 *qr = reinterpret_cast<uint2 *>(q + (r0 + rr) * cols);
+#pragma unroll
+                    for (int j = 0; j < V; ++j) {
+                        const int64_t cv = threadIdx.x + j * kRowThreads;
+                        if (cv < ncv) qr[cv] = cast8<FMT>(v[rr][j], s);
+                    }
+                    if (threadIdx.x == 0) scale_inv[r0 + rr] = __fdiv_rn(1.0f, s);
+                }
+            }
+            __syncthreads();   // red[] is reused by the next rows
         } else {
-            uint32_t bad = 0;
-            m = 0;
-            for (int64_t cv = threadIdx.x; cv < ncv; cv += kRowThreads) m = amax_exact8(m, ld_stream(xr + cv), bad);
-            m = block_max_u32(m, red);
-            const float a = bf16bits_to_float(m);
-            const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
-            for (int64_t cv = threadIdx.x; cv < ncv; cv += kRowThreads) qr[cv] = cast8<FMT>(xr[cv], s);
-            if (threadIdx.x == 0) scale_inv[r] = __fdiv_rn(1.0f, s);
+            for (int rr = 0; rr < R && r0 + rr < rows; ++rr) {
+                const int64_t r = r0 + rr;
+                const uint4 *xr = reinterpret_cast<const uint4 *>(x + r * ld);
+                uint2 *qr = reinterpret_cast<uint2 *>(q + r * cols);
+                uint32_t bad = 0, mm = 0;
+                for (int64_t cv = threadIdx.x; cv < ncv; cv += kRowThreads) mm = amax_exact8(mm, ld_stream(xr + cv), bad);
+                mm = block_max_u32(mm, red[0]);
+                const float a = bf16bits_to_float(mm);
+                const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
+                for (int64_t cv = threadIdx.x; cv < ncv; cv += kRowThreads) qr[cv] = cast8<FMT>(xr[cv], s);
+                if (threadIdx.x == 0) scale_inv[r] = __fdiv_rn(1.0f, s);
+                __syncthreads();
+            }
         }
     }
 }
 
 // ---------------------------------------------------------- block 1x128 --
-// A half-warp per 1x128 block (16 lanes x 8 elements); each warp takes U
-// pairs of blocks per iteration so U 16-byte loads per lane are in flight.
-// Blocks are numbered row-major (row, kb); scale_inv is stored [kb][row].
+// A half-warp per 1x128 block (16 lanes x 8 elements).  A warp walks rows
+// (warp, warp + nwarps, ...) and, inside a row, U pairs of blocks per
+// iteration (the two half-warps take neighbouring blocks), so U 16-byte loads
+// per lane are in flight and no index division is needed.  scale_inv is
+// stored [kb][row].
 template <int FMT, int U>
 __global__ void __launch_bounds__(256)
 k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
@@ -247,41 +274,38 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
     constexpr float fm = fmax_of<FMT>();
     const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
     const int64_t nkb = (cols + 127) / 128;
-    const int64_t nblocks = rows * nkb;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t wb = warp * 2 * U; wb < nblocks; wb += nwarps * 2 * U) {
-        uint4 v[U];
-        int64_t row[U], cidx[U];
-        bool valid[U];
+    for (int64_t row = warp; row < rows; row += nwarps) {
+        const uint16_t *xr = x + row * ld;
+        uint8_t *qr = q + row * cols;
+        for (int64_t kb0 = 0; kb0 < nkb; kb0 += 2 * U) {
+            uint4 v[U];
+            int64_t cidx[U];
+            bool valid[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t b = wb + 2 * u + half;
-            row[u] = b / nkb;
-            const int64_t kb = b - row[u] * nkb;
-            cidx[u] = kb * 128 + l16 * 8;
-            valid[u] = (b < nblocks) && (cidx[u] < cols);
-            v[u] = valid[u] ? ld_stream(reinterpret_cast<const uint4 *>(x + row[u] * ld + cidx[u]))
-                            : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            uint32_t m = amax_fast_final(amax_fast8(0u, v[u]));
-            if (m == 0xFFFFFFFFu) {
-                uint32_t bad = 0;
-                m = amax_exact8(0u, v[u], bad);
+            for (int u = 0; u < U; ++u) {
+                const int64_t kb = kb0 + 2 * u + half;
+                cidx[u] = kb * 128 + l16 * 8;
+                valid[u] = (kb < nkb) && (cidx[u] < cols);
+                v[u] = valid[u] ? ld_stream(reinterpret_cast<const uint4 *>(xr + cidx[u])) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int o = 8; o >= 1; o >>= 1) {
-                const uint32_t t = __shfl_xor_sync(0xFFFFFFFFu, m, o);
-                m = t > m ? t : m;
-            }
-            const float s = scale_from_amax(bf16bits_to_float(m), fm);
-            if (valid[u]) *reinterpret_cast<uint2 *>(q + row[u] * cols + cidx[u]) = cast8<FMT>(v[u], s);
-            const int64_t b = wb + 2 * u + half;
-            if (l16 == 0 && b < nblocks) {
-                const int64_t kb = b - row[u] * nkb;
-                scale_inv[kb * rows + row[u]] = __fdiv_rn(1.0f, s);
+            for (int u = 0; u < U; ++u) {
+                uint32_t m = amax_fast_final(amax_fast8(0u, v[u]));
+                if (m == 0xFFFFFFFFu) {
+                    uint32_t bad = 0;
+                    m = amax_exact8(0u, v[u], bad);
+                }
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1) {
+                    const uint32_t t = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+                    m = t > m ? t : m;
+                }
+                const float s = scale_from_amax(bf16bits_to_float(m), fm);
+                if (valid[u]) *reinterpret_cast<uint2 *>(qr + cidx[u]) = cast8<FMT>(v[u], s);
+                const int64_t kb = kb0 + 2 * u + half;
+                if (l16 == 0 && kb < nkb) scale_inv[kb * rows + row] = __fdiv_rn(1.0f, s);
             }
         }
     }
@@ -363,15 +387,25 @@ template <int FMT, bool POW2>
 void launch_rowwise(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, int64_t ld,
                     uint8_t *q, float *scale_inv) {
     const uint16_t *xs = static_cast<const uint16_t *>(x);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(rows, (int64_t)sms * 16));
+    const int64_t slots = (int64_t)sms * 16;   // resident 128-thread CTAs
     const int64_t ncv = cols / 8;
     const int T = kRowThreads;
-    if (ncv <= T) k_rowwise<FMT, POW2, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 2 * T) k_rowwise<FMT, POW2, 2><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 4 * T) k_rowwise<FMT, POW2, 4><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 8 * T) k_rowwise<FMT, POW2, 8><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 16 * T) k_rowwise<FMT, POW2, 16><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else k_rowwise<FMT, POW2, 0><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    // two rows per CTA when that lets one wave of CTAs cover every row
+    const bool two = rows > slots && ncv <= 4 * T;
+    const int R = two ? 2 : 1;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + R - 1) / R, slots));
+    if (two) {
+        if (ncv <= T) k_rowwise<FMT, POW2, 1, 2><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+        else if (ncv <= 2 * T) k_rowwise<FMT, POW2, 2, 2><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+        else k_rowwise<FMT, POW2, 4, 2><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+        return;
+    }
+    if (ncv <= T) k_rowwise<FMT, POW2, 1, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 2 * T) k_rowwise<FMT, POW2, 2, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 4 * T) k_rowwise<FMT, POW2, 4, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 8 * T) k_rowwise<FMT, POW2, 8, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 16 * T) k_rowwise<FMT, POW2, 16, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    else k_rowwise<FMT, POW2, 0, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
 }
 
 template <int FMT>
@@ -381,8 +415,7 @@ void launch_block(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t
     const int64_t nkb = (cols + 127) / 128;
     if (block_rows == 1) {
         constexpr int U = 4;
-        const int64_t warps = (rows * nkb + 2 * U - 1) / (2 * U);
-        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sms * 8));
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + 7) / 8, (int64_t)sms * 8));
         k_block1x128<FMT, U><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
     } else {
         const int64_t tiles = ((rows + 127) / 128) * nkb;
