@@ -573,12 +573,13 @@ __device__ __forceinline__ void tc_commit_pair_self(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool GROUPED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
 k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                int K, uint32_t idesc, const float *__restrict__ sa, const float *__restrict__ sb,
                __nv_bfloat16 *__restrict__ D, int64_t ldd, int full_tiles, int split_units,
-               float *__restrict__ ws, uint32_t *__restrict__ flags, uint32_t epoch) {
+               float *__restrict__ ws, uint32_t *__restrict__ flags, uint32_t epoch,
+               const int64_t *__restrict__ goff, int G) {
     using C = sm2::Cfg<BN>;
     constexpr int STG = C::STAGES, NBUF = C::NBUF;
     constexpr int HALF = BN / 2;             // columns per epilogue warp
@@ -599,13 +600,42 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // full_tiles, then (pair < split_units) one half of a split tail tile:
     // tile full_tiles + pair / 2, K blocks [0, nk/2) for the even pair and
     // [nk/2, nk) for the odd one.  With no split, full_tiles = every tile.
-    const int n_full = (pair < full_tiles) ? (full_tiles - 1 - pair) / npairs + 1 : 0;
+    // Grouped GEMM (MoE experts): group e owns rows [goff[e], goff[e+1]) of A
+    // and D and rows [e*N, (e+1)*N) of B; its tiles follow group e-1's, m
+    // fastest.  The tile count comes from one scan of the offsets.
+    const int num_n = (N + BN - 1) / BN;
+    int total_tiles = full_tiles;
+    if constexpr (GROUPED) {
+        total_tiles = 0;
+        for (int e = 0; e < G; ++e) total_tiles += (int)((goff[e + 1] - goff[e] + 255) / 256) * num_n;
+    }
+    const int n_full = (pair < total_tiles) ? (total_tiles - 1 - pair) / npairs + 1 : 0;
     const int n_items = n_full + (pair < split_units ? 1 : 0);
-    struct Item { int tile, k0, k1, half; };
+    struct Item {
+        int tile, k0, k1, half, m_blk, n_blk, e;
+        int64_t row0, row_end;   // rows of A / D this item's tile may write
+    };
     auto item = [&](int i) -> Item {
-        if (i < n_full) return Item{pair + i * npairs, 0, nk, -1};
-        const int h = pair & 1, kh = nk / 2;
-        return Item{full_tiles + pair / 2, h ? kh : 0, h ? nk : kh, h};
+        if constexpr (GROUPED) {
+            int t = pair + i * npairs, e = 0;
+            int64_t r0 = goff[0], r1 = goff[1];
+            int mt = (int)((r1 - r0 + 255) / 256);
+            while (t >= mt * num_n) {   // empty groups own no tiles and are skipped
+                t -= mt * num_n;
+                ++e;
+                r0 = r1;
+                r1 = goff[e + 1];
+                mt = (int)((r1 - r0 + 255) / 256);
+            }
+            return Item{pair + i * npairs, 0, nk, -1, t % mt, t / mt, e, r0, r1};
+        } else {
+            if (i < n_full) {
+                const int t = pair + i * npairs;
+                return Item{t, 0, nk, -1, t % num_m, t / num_m, 0, 0, (int64_t)M};
+            }
+            const int h = pair & 1, kh = nk / 2, t = full_tiles + pair / 2;
+            return Item{t, h ? kh : 0, h ? nk : kh, h, t % num_m, t / num_m, 0, 0, (int64_t)M};
+        }
     };
 
     auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
@@ -654,9 +684,8 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             bool ok = true;
             for (int i = 0; ok && i < n_items; ++i) {
                 const Item w = item(i);
-                const int m_blk = w.tile % num_m, n_blk = w.tile / num_m;
-                const int a_row = m_blk * 256 + (int)rank * 128;
-                const int b_row = n_blk * BN + (int)rank * HALF;
+                const int a_row = (int)(w.row0 + w.m_blk * 256 + (int)rank * 128);
+                const int b_row = w.e * N + w.n_blk * BN + (int)rank * HALF;
                 for (int kc = w.k0; kc < w.k1; ++kc, ++it) {
                     const int stage = it % STG;
                     const uint32_t round = it / STG;
@@ -732,15 +761,17 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         bool ok = true;
         for (int i = 0; ok && i < n_items; ++i, ++lt) {
             const Item wi = item(i);
-            const int m_blk = wi.tile % num_m, n_blk = wi.tile / num_m;
-            const int m = m_blk * 256 + (int)rank * 128 + sp * 32 + lane;
+            const int n_blk = wi.n_blk;
+            const int64_t m = wi.row0 + wi.m_blk * 256 + (int)rank * 128 + sp * 32 + lane;
+            const bool m_ok = m < wi.row_end;
             const int n_base = n_blk * BN + ch * HALF;
-            __nv_bfloat16 *drow = D + (int64_t)m * ldd;
+            __nv_bfloat16 *drow = D + m * ldd;
+            const float *sbe = sb + (int64_t)wi.e * N;   // group e's column scales (ROW)
             if (MODE != kModeBlock) {
                 const uint32_t ab = lt % NBUF, use = lt / NBUF;
                 float rs;
-                if (MODE == kModeRow) rs = (m < M) ? sa[m] : 0.0f;
-                else rs = __fmul_rn(sa[0], sb[0]);
+                if (MODE == kModeRow) rs = m_ok ? sa[m] : 0.0f;
+                else rs = __fmul_rn(sa[wi.e], sb[wi.e]);
                 bool w = true;
                 if (lane == 0) w = wait_bar(accf_bar(ab), use & 1u, abort_flag, kErrEpilogue);
                 w = __shfl_sync(0xFFFFFFFFu, w, 0);
@@ -778,14 +809,14 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         for (int j = 0; j < 32; ++j) v[j] = v[j] + pc[(size_t)j * 128];
                     }
                     if (MODE == kModeRow) {
-                        const float cb = (col0 + lane < N) ? sb[col0 + lane] : 0.0f;
+                        const float cb = (col0 + lane < N) ? sbe[col0 + lane] : 0.0f;
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = v[j] * (rs * __shfl_sync(0xFFFFFFFFu, cb, j));
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
                     }
-                    if (m < M) {
+                    if (m_ok) {
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
                             if (col0 + g * 8 < N) {
@@ -825,7 +856,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 float as_[PF], bs_[PF];
 #pragma unroll
                 for (int i = 0; i < PF; ++i) {
-                    as_[i] = (i < nk && m < M) ? sa[(int64_t)i * M + m] : 0.0f;
+                    as_[i] = (i < nk && m_ok) ? sa[(int64_t)i * M + m] : 0.0f;
                     bs_[i] = (i < nk && nb_ok) ? sb[(int64_t)nb * nk + i] : 0.0f;
                 }
                 // one K block: wait for its partial, promote it, release it
@@ -853,7 +884,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(pb), 0));
                     if (kc + PF < nk) {   // block kc + PF's scales, after the release
-                        as = (m < M) ? sa[(int64_t)(kc + PF) * M + m] : 0.0f;
+                        as = m_ok ? sa[(int64_t)(kc + PF) * M + m] : 0.0f;
                         bs = nb_ok ? sb[(int64_t)nb * nk + kc + PF] : 0.0f;
                     }
 #pragma unroll
@@ -868,7 +899,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         if (ok && kc + i < nk && !promote(kc + i, as_[i], bs_[i])) ok = false;
                 }
                 if (!ok) break;
-                if (m < M) {
+                if (m_ok) {
 #pragma unroll
                     for (int g = 0; g < HALF / 8; ++g) {
                         const int col = n_base + g * 8;
@@ -944,7 +975,7 @@ cudaError_t launch_gemm(cudaStream_t st, int sms, const CUtensorMap &ta, const C
 }
 
 // Pairs of the 2-SM kernel that fit on the device at once (cached per device).
-template <int MODE, int BN>
+template <int MODE, int BN, bool GROUPED = false>
 int pair_capacity() {
     static int cache[64];
     static std::mutex mu;
@@ -952,12 +983,12 @@ int pair_capacity() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     std::lock_guard<std::mutex> lk(mu);
     if (cache[dev] > 0) return cache[dev];
-    if (cudaFuncSetAttribute(k_gemm_fp8_2sm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(k_gemm_fp8_2sm<MODE, BN, GROUPED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm2::Cfg<BN>::SMEM) != cudaSuccess)
         return 0;
     if (MODE == kModeBlock) {   // the setmaxnreg split assumes this launch register count
         cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, k_gemm_fp8_2sm<MODE, BN>) != cudaSuccess || fa.numRegs != sm2::REGS_LAUNCH)
+        if (cudaFuncGetAttributes(&fa, k_gemm_fp8_2sm<MODE, BN, GROUPED>) != cudaSuccess || fa.numRegs != sm2::REGS_LAUNCH)
             return 0;
     }
     cudaLaunchConfig_t cfg = {};
@@ -972,7 +1003,7 @@ int pair_capacity() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_fp8_2sm<MODE, BN>, &cfg) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_fp8_2sm<MODE, BN, GROUPED>, &cfg) != cudaSuccess) return 0;
     cache[dev] = n;
     return n;
 }
@@ -1006,9 +1037,21 @@ cudaError_t launch_gemm_2sm(cudaStream_t st, const CUtensorMap &ta, const CUtens
     uint32_t *flags = plan.units ? reinterpret_cast<uint32_t *>(static_cast<char *>(ws) +
                                                                 (size_t)(plan.units / 2) * 2 * sm2::kSplitPartialFloats * sizeof(float))
                                  : nullptr;
-    k_gemm_fp8_2sm<MODE, BN><<<2 * pairs, sm2::THREADS, sm2::Cfg<BN>::SMEM, st>>>(
+    k_gemm_fp8_2sm<MODE, BN, false><<<2 * pairs, sm2::THREADS, sm2::Cfg<BN>::SMEM, st>>>(
         ta, tb, M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd,
-        plan.units ? plan.full_tiles : tiles, plan.units, part, flags, epoch);
+        plan.units ? plan.full_tiles : tiles, plan.units, part, flags, epoch, nullptr, 0);
+    return cudaPeekAtLastError();
+}
+
+// Grouped launch: a persistent grid of every pair that fits; each pair
+// derives its tiles from the group offsets on the device.
+template <int MODE>
+cudaError_t launch_gemm_grouped(cudaStream_t st, const CUtensorMap &ta, const CUtensorMap &tb, int64_t total_M,
+                                int N, int K, uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd,
+                                const int64_t *goff, int G, int pairs_cap) {
+    k_gemm_fp8_2sm<MODE, 256, true><<<2 * pairs_cap, sm2::THREADS, sm2::Cfg<256>::SMEM, st>>>(
+        ta, tb, (int)total_M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd, 0, 0, nullptr, nullptr, 0,
+        goff, G);
     return cudaPeekAtLastError();
 }
 
@@ -1125,6 +1168,44 @@ extern "C" fp8_status fp8_device_error(uint32_t *host_out, int clear) {
         if (cudaMemcpyToSymbol(g_gemm_error, &z, sizeof(z)) != cudaSuccess) return FP8_ERR_CUDA;
     }
     return FP8_OK;
+}
+
+// ------------------------------------------------------------- grouped GEMM --
+extern "C" fp8_status fp8_gemm_grouped(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int G,
+                                       const int64_t *group_offsets, int64_t total_M, int64_t N, int64_t K,
+                                       fp8_scale_mode mode, const float *a_scale_inv, const float *b_scale_inv,
+                                       void *D_bf16, int64_t ldd, void *stream) {
+    if ((fa != FP8_E4M3 && fa != FP8_E5M2) || (fb != FP8_E4M3 && fb != FP8_E5M2)) return FP8_ERR_INVALID_ARG;
+    if (mode != FP8_SCALE_TENSOR && mode != FP8_SCALE_ROW) return FP8_ERR_INVALID_ARG;
+    if (G < 0 || total_M < 0 || N < 0 || K < 0 || ldd < N) return FP8_ERR_SHAPE;
+    if (total_M >= (1 << 30) || (int64_t)G * N >= (1 << 30) || K > (1 << 30)) return FP8_ERR_SHAPE;
+    if (K % 16) return FP8_ERR_SHAPE;
+    if (N % 8 || ldd % 8) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (G == 0 || total_M == 0 || N == 0) return FP8_OK;
+    if (!group_offsets || !D_bf16) return FP8_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(group_offsets) & 7u) return FP8_ERR_ALIGNMENT;
+    cudaStream_t s = as_stream(stream);
+    if (K == 0)
+        return cudaMemset2DAsync(D_bf16, (size_t)ldd * 2, 0, (size_t)N * 2, (size_t)total_M, s) == cudaSuccess
+                   ? FP8_OK : FP8_ERR_CUDA;
+    if (!A || !B || !a_scale_inv || !b_scale_inv) return FP8_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D_bf16)) return FP8_ERR_ALIGNMENT;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A, K, total_M, 128) || !make_map(&tb, B, K, (int64_t)G * N, 128)) return FP8_ERR_CUDA;
+    const uint32_t idesc = make_idesc(fa, fb, 256, 256);
+    cudaError_t e = cudaErrorUnknown;
+    int cap;
+    if (mode == FP8_SCALE_TENSOR) {
+        if ((cap = pair_capacity<kModeTensor, 256, true>()) > 0)
+            e = launch_gemm_grouped<kModeTensor>(s, ta, tb, total_M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, group_offsets, G, cap);
+    } else {
+        if ((cap = pair_capacity<kModeRow, 256, true>()) > 0)
+            e = launch_gemm_grouped<kModeRow>(s, ta, tb, total_M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, group_offsets, G, cap);
+    }
+    return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 // ---------------------------------------------- entry point without allocation --

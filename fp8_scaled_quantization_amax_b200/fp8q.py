@@ -38,6 +38,7 @@ SIGNATURES = {
     "fp8_quantize_blockwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
     "fp8_gemm_scaled": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P, ctypes.c_size_t, _P]),
     "fp8_gemm_workspace_size": (_S, [_I64, _I64, _I64, _I, _P]),
+    "fp8_gemm_grouped": (_S, [_P, _I, _P, _I, _I, _P, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
     "fp8_gemm_scaled_noalloc": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
     "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
     "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
@@ -157,6 +158,16 @@ def fp8_gemm_scaled_noalloc(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_in
         _stream(stream)))
 
 
+def fp8_gemm_grouped(A, fa, B, fb, G, group_offsets, total_M, N, K, mode, a_scale_inv, b_scale_inv, D, ldd,
+                     stream=None):
+    _dev(A, torch.uint8, "A"); _dev(B, torch.uint8, "B"); _dev(D, torch.bfloat16, "D")
+    _dev(group_offsets, torch.int64, "group_offsets")
+    _dev(a_scale_inv, torch.float32, "a_scale_inv"); _dev(b_scale_inv, torch.float32, "b_scale_inv")
+    _check("fp8_gemm_grouped", lib().fp8_gemm_grouped(
+        _ptr(A), fa, _ptr(B), fb, G, _ptr(group_offsets), total_M, N, K, mode, _ptr(a_scale_inv),
+        _ptr(b_scale_inv), _ptr(D), ldd, _stream(stream)))
+
+
 def fp8_gemm_workspace_size(M, N, K, mode) -> int:
     b = ctypes.c_size_t(0)
     _check("fp8_gemm_workspace_size", lib().fp8_gemm_workspace_size(M, N, K, mode, ctypes.byref(b)))
@@ -241,6 +252,16 @@ def gemm(A, fa, B, fb, mode, a_scale_inv, b_scale_inv, out=None, workspace=None)
     N = B.shape[0]
     D = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, D.stride(0), workspace)
+    return D
+
+
+def gemm_grouped(A, fa, B, fb, group_offsets, mode, a_scale_inv, b_scale_inv, out=None):
+    """A [total_M, K], B [G, N, K], group_offsets int64 [G+1] on the device."""
+    total_M, K = A.shape
+    G, N, _ = B.shape
+    D = out if out is not None else torch.empty((total_M, N), dtype=torch.bfloat16, device=A.device)
+    fp8_gemm_grouped(A, fa, B.reshape(G * N, K), fb, G, group_offsets, total_M, N, K, mode, a_scale_inv,
+                     b_scale_inv, D, D.stride(0))
     return D
 
 

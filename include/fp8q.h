@@ -166,6 +166,29 @@ FP8Q_API fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8
                            int64_t ldd, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Grouped FP8 GEMM for mixture-of-experts layers ("DeepL押注FP8：…" §3.2: the
+ * tokens routed to each expert form a group, and one grouped GEMM multiplies
+ * every group by its own expert weight):
+ *   for every group e:  D[r, :] = scales * A[r, :] x B_e^T  for the rows
+ *   r in [group_offsets[e], group_offsets[e+1]).
+ *   A  [total_M, K] FP8, the groups' rows stacked in order (K contiguous).
+ *   B  [G, N, K] FP8, expert e's weight [N, K] at B + e*N*K.
+ *   group_offsets  DEVICE int64 [G+1], group_offsets[0] = 0, nondecreasing,
+ *                  group_offsets[G] = total_M (a group may be empty).
+ *   mode TENSOR: a_scale_inv [G] (one per group's activations),
+ *                b_scale_inv [G] (one per expert weight).
+ *   mode ROW   : a_scale_inv [total_M], b_scale_inv [G*N].
+ *   (BLOCK is not supported here: FP8_ERR_INVALID_ARG.)
+ *   D  [total_M, N] bf16, leading dimension ldd.
+ *   Same arithmetic, determinism and alignment rules as fp8_gemm_scaled;
+ *   total_M < 2^30, G*N < 2^30.
+ */
+FP8Q_API fp8_status fp8_gemm_grouped(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int G,
+                                     const int64_t *group_offsets, int64_t total_M, int64_t N, int64_t K,
+                                     fp8_scale_mode mode, const float *a_scale_inv, const float *b_scale_inv,
+                                     void *D_bf16, int64_t ldd, void *stream);
+
+/*
  * Bytes of workspace fp8_gemm_scaled can use for this shape on the current
  * device (0: the shape fills whole waves, or the mode takes none).
  */

@@ -221,6 +221,28 @@ def gemm_scaled_sampled(A: np.ndarray, fa: int, B: np.ndarray, fb: int, mode: in
     return val, mag
 
 
+def gemm_grouped(A: np.ndarray, fa: int, B: np.ndarray, fb: int, offsets, mode: int,
+                 da: np.ndarray, db: np.ndarray):
+    """Grouped (mixture-of-experts) GEMM: rows [offsets[e], offsets[e+1]) of A
+    times expert e's weight B[e] ([G, N, K]); tensor mode takes da[e], db[e],
+    row mode da[row], db[e, col].  Each group is the plain scaled GEMM above
+    ("DeepL押注FP8：…" §3.2: one GEMM per expert's token group)."""
+    G, N, K = B.shape
+    M = A.shape[0]
+    D = np.zeros((M, N), np.float64)
+    mag = np.zeros((M, N), np.float64)
+    for e in range(G):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r1 == r0:
+            continue
+        if mode == SCALE_TENSOR:
+            sa, sb = np.float32([da[e]]), np.float32([db[e]])
+        else:
+            sa, sb = np.ascontiguousarray(da[r0:r1]), np.ascontiguousarray(np.asarray(db).reshape(G, N)[e])
+        D[r0:r1], mag[r0:r1] = gemm_scaled(A[r0:r1], fa, B[e], fb, mode, sa, sb)
+    return D, mag
+
+
 # --------------------------------------------------------- delayed scaling --
 
 class AmaxHistory:

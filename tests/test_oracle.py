@@ -441,3 +441,30 @@ def test_kv_round_trip(orc):
     y = (t[q.reshape(6, -1)] * sinv[:, None]).astype(np.float32)
     lib = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(back.reshape(6, -1), lib)
+
+
+def test_grouped_gemm_is_the_per_group_gemm(orc):
+    """The grouped oracle equals numpy's per-group products (empty groups and
+    ragged sizes included) -- catches a swapped expert index or row offset."""
+    rng = np.random.default_rng(21)
+    sizes = [0, 5, 3, 0, 7]
+    off = np.concatenate([[0], np.cumsum(sizes)])
+    G, N, K = len(sizes), 6, 40
+    t = orc.decode_table(0)
+    fin = np.where(np.isfinite(t))[0]
+    A = rng.choice(fin, (off[-1], K)).astype(np.uint8)
+    B = rng.choice(fin, (G, N, K)).astype(np.uint8)
+    da = rng.uniform(0.5, 2, G).astype(np.float32)
+    db = rng.uniform(0.5, 2, G).astype(np.float32)
+    D, _ = orc.gemm_grouped(A, 0, B, 0, off, orc.SCALE_TENSOR, da, db)
+    for e in range(G):
+        r0, r1 = off[e], off[e + 1]
+        ref = (t[A[r0:r1]] @ t[B[e]].T) * np.float64(da[e]) * np.float64(db[e])
+        assert np.allclose(D[r0:r1], ref, rtol=1e-12, atol=1e-12)
+    dra = rng.uniform(0.5, 2, off[-1]).astype(np.float32)
+    drb = rng.uniform(0.5, 2, G * N).astype(np.float32)
+    D2, _ = orc.gemm_grouped(A, 0, B, 0, off, orc.SCALE_ROW, dra, drb)
+    for e in range(G):
+        r0, r1 = off[e], off[e + 1]
+        ref = (t[A[r0:r1]] @ t[B[e]].T) * dra[r0:r1, None] * drb.reshape(G, N)[e][None, :]
+        assert np.allclose(D2[r0:r1], ref, rtol=1e-12, atol=1e-12)
