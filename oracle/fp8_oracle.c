@@ -430,3 +430,94 @@ void orc_kv_dequant(const uint8_t *q, const float *scale_inv, int64_t BH, int64_
             out[i * SD + j] = orc_f32_to_bf16(y);
         }
 }
+
+/* ------------------------------------------------------ scale health check -- */
+
+/* Health check of a set of scale factors ([DeepL] §6.2: periodically report
+ * the min / max / mean of every layer's scales and watch for step changes,
+ * the early sign of outliers or a distribution shift).
+ *   valid entries: finite and > 0; stats = {min, max, mean} over them (mean =
+ *   fp64 sum / count, rounded to fp32), all 0 when none is valid;
+ *   counts[0] = entries whose ratio to prev (both valid) exceeds jump_ratio
+ *   in either direction (fp32 divisions), 0 without prev;
+ *   counts[1] = invalid entries. */
+void orc_scale_stats(const float *s, const float *prev, int64_t n, float jump_ratio, float *stats,
+                     uint32_t *counts)
+{
+    double sum = 0.0;
+    float mn = 0.0f, mx = 0.0f;
+    int64_t nv = 0;
+    uint32_t jumps = 0, invalid = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        float v = s[i];
+        if (!(isfinite(v) && v > 0.0f)) { ++invalid; continue; }
+        if (nv == 0 || v < mn) mn = v;
+        if (nv == 0 || v > mx) mx = v;
+        sum += (double)v;
+        ++nv;
+        if (prev) {
+            float p = prev[i];
+            if (isfinite(p) && p > 0.0f && (v / p > jump_ratio || p / v > jump_ratio)) ++jumps;
+        }
+    }
+    stats[0] = mn;
+    stats[1] = mx;
+    stats[2] = nv ? (float)(sum / (double)nv) : 0.0f;
+    counts[0] = jumps;
+    counts[1] = invalid;
+}
+
+/* ------------------------------------------------------- paged KV cache -- */
+
+/* Paged FP8 KV cache.  The cache is split into fixed-size blocks handed out on
+ * demand ("FP8量化首次支持！ms-swift引领大模型低精度计算新浪潮", vLLM's block
+ * KV cache) and stores K / V in FP8 ([DeepL] §3.1).  Tokens arrive a few at a
+ * time, so a scale over a whole (sequence, head) slice is not known when a
+ * token is written: each (token, head) row of Dh elements gets its own scale.
+ *   x     [T, H, Dh] bf16, the new tokens' K (or V);
+ *   slot  [T] int64, slot = block * block_size + offset; entries outside
+ *         [0, nslots) are padding and write nothing;
+ *   cache [nslots, H, Dh] FP8  (= [num_blocks, block_size, H, Dh]);
+ *   scale_cache [nslots, H] fp32, 1/s of each written row. */
+void orc_paged_kv_write(const uint16_t *x, const int64_t *slot, int64_t T, int64_t H, int64_t Dh,
+                        int64_t nslots, int fmt, uint8_t *cache, float *scale_cache)
+{
+    float fm = (float)orc_fmax(fmt);
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t sl = slot[t];
+        if (sl < 0 || sl >= nslots) continue;
+        for (int64_t h = 0; h < H; ++h) {
+            const uint16_t *row = x + (t * H + h) * Dh;
+            float s = orc_scale_from_amax(orc_amax_bf16(row, Dh, NULL), fmt);
+            for (int64_t j = 0; j < Dh; ++j) cache[(sl * H + h) * Dh + j] = cast_one(row[j], s, fmt, fm, NULL);
+            scale_cache[sl * H + h] = orc_inverse(s);
+        }
+    }
+}
+
+/* Read a sequence's tokens back through its block table, dequantized:
+ *   token t of sequence b lives in block block_table[b][t / block_size] at
+ *   offset t % block_size; out[b][t][h][:] = bf16(fp32(dec(q)) * scale_inv).
+ *   out [B, S_out, H, Dh] bf16; positions t >= seq_lens[b], past the table's
+ *   max_blocks * block_size, or in a block id outside [0, num_blocks) are 0. */
+void orc_paged_kv_gather(const uint8_t *cache, const float *scale_cache, const int32_t *block_table,
+                         const int32_t *seq_lens, int64_t B, int64_t max_blocks, int64_t H, int64_t Dh,
+                         int64_t block_size, int64_t num_blocks, int64_t S_out, int fmt, uint16_t *out)
+{
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t t = 0; t < S_out; ++t) {
+            uint16_t *dst = out + (b * S_out + t) * H * Dh;
+            int64_t blk = -1;
+            if (t < seq_lens[b] && t / block_size < max_blocks) blk = block_table[b * max_blocks + t / block_size];
+            if (blk < 0 || blk >= num_blocks) {
+                memset(dst, 0, (size_t)(H * Dh) * sizeof(uint16_t));
+                continue;
+            }
+            int64_t sl = blk * block_size + t % block_size;
+            for (int64_t h = 0; h < H; ++h)
+                for (int64_t j = 0; j < Dh; ++j) {
+                    float v = (float)orc_decode(cache[(sl * H + h) * Dh + j], fmt);
+                    dst[h * Dh + j] = orc_f32_to_bf16(v * scale_cache[sl * H + h]);
+                }
+        }
+}

@@ -81,6 +81,12 @@ def lib():
         L.orc_kv_quant.argtypes = [P, I64, I64, I, P, P]
         L.orc_kv_dequant.restype = None
         L.orc_kv_dequant.argtypes = [P, P, I64, I64, I, P]
+        L.orc_paged_kv_write.restype = None
+        L.orc_paged_kv_write.argtypes = [P, P, I64, I64, I64, I64, I, P, P]
+        L.orc_paged_kv_gather.restype = None
+        L.orc_paged_kv_gather.argtypes = [P, P, P, P, I64, I64, I64, I64, I64, I64, I64, I, P]
+        L.orc_scale_stats.restype = None
+        L.orc_scale_stats.argtypes = [P, P, I64, F, P, P]
         _lib = L
     return _lib
 
@@ -282,3 +288,46 @@ def kv_dequant(q: np.ndarray, scale_inv: np.ndarray, fmt: int = E4M3) -> np.ndar
     out = np.empty(q.shape, np.uint16)
     lib().orc_kv_dequant(_p(q), _p(sinv), B * H, S * Dh, fmt, _p(out))
     return out
+
+
+# --------------------------------------------------------- paged KV cache --
+
+def paged_kv_write(x_bits: np.ndarray, slot: np.ndarray, cache: np.ndarray, scale_cache: np.ndarray,
+                   fmt: int = E4M3):
+    """x [T, H, Dh] bf16 bits written into copies of cache [num_blocks,
+    block_size, H, Dh] / scale_cache [num_blocks, block_size, H]; returns them."""
+    x = _u16(x_bits)
+    T, H, Dh = x.shape
+    sl = np.ascontiguousarray(slot, np.int64)
+    c = np.array(cache, np.uint8, copy=True, order="C")
+    sc = np.array(scale_cache, np.float32, copy=True, order="C")
+    nslots = c.shape[0] * c.shape[1]
+    assert c.shape[2:] == (H, Dh) and sc.shape == c.shape[:3] and sl.shape == (T,)
+    lib().orc_paged_kv_write(_p(x), _p(sl), T, H, Dh, nslots, fmt, _p(c), _p(sc))
+    return c, sc
+
+
+def paged_kv_gather(cache: np.ndarray, scale_cache: np.ndarray, block_table: np.ndarray,
+                    seq_lens: np.ndarray, S_out: int, fmt: int = E4M3) -> np.ndarray:
+    """Dequantized [B, S_out, H, Dh] bf16 bits of each sequence's tokens."""
+    c = np.ascontiguousarray(cache, np.uint8)
+    sc = np.ascontiguousarray(scale_cache, np.float32)
+    bt = np.ascontiguousarray(block_table, np.int32)
+    sl = np.ascontiguousarray(seq_lens, np.int32)
+    NB, bs, H, Dh = c.shape
+    B, mb = bt.shape
+    out = np.empty((B, S_out, H, Dh), np.uint16)
+    lib().orc_paged_kv_gather(_p(c), _p(sc), _p(bt), _p(sl), B, mb, H, Dh, bs, NB, S_out, fmt, _p(out))
+    return out
+
+
+# ------------------------------------------------------- scale health check --
+
+def scale_stats(scales: np.ndarray, prev: np.ndarray | None = None, jump_ratio: float = 4.0):
+    """(min, max, mean) over the finite positive scales, (jumps, invalid)."""
+    s = np.ascontiguousarray(scales, np.float32)
+    p = None if prev is None else np.ascontiguousarray(prev, np.float32)
+    st = np.zeros(3, np.float32)
+    c = np.zeros(2, np.uint32)
+    lib().orc_scale_stats(_p(s), None if p is None else _p(p), s.size, float(jump_ratio), _p(st), _p(c))
+    return st, c

@@ -468,3 +468,82 @@ def test_grouped_gemm_is_the_per_group_gemm(orc):
         r0, r1 = off[e], off[e + 1]
         ref = (t[A[r0:r1]] @ t[B[e]].T) * dra[r0:r1, None] * drb.reshape(G, N)[e][None, :]
         assert np.allclose(D2[r0:r1], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_scale_stats_closed_forms(orc):
+    """Health check of scale factors (DeepL page §6.2): min / max / mean over
+    the valid scales, step changes against a previous snapshot, invalid ones."""
+    s = np.array([1.0, 4.0, 2.0, 0.5, np.nan, -1.0, 0.0, np.inf, 8.0], np.float32)
+    st, c = orc.scale_stats(s)
+    assert list(st) == [0.5, 8.0, np.float32(15.5 / 5)] and list(c) == [0, 4]
+    prev = np.array([1.0, 1.0, 2.0, 0.25, 1.0, 1.0, 1.0, 1.0, 64.0], np.float32)
+    st, c = orc.scale_stats(s, prev, 3.0)
+    assert list(c) == [2, 4]        # 4/1 > 3 and 64/8 > 3; 0.5/0.25 = 2 is not
+    st, c = orc.scale_stats(np.zeros(0, np.float32))
+    assert list(st) == [0, 0, 0] and list(c) == [0, 0]
+    rng = np.random.default_rng(0)
+    v = (10.0 ** rng.uniform(-3, 3, 10000)).astype(np.float32)
+    st, c = orc.scale_stats(v)
+    assert st[0] == v.min() and st[1] == v.max() and np.isclose(st[2], v.astype(np.float64).mean(), rtol=1e-7)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_paged_kv_write_and_gather(orc, fmt):
+    """Paged FP8 KV cache (block KV cache of the ms-swift page; FP8 KV of the
+    DeepL page §3.1), against torch built independently: per (token, head) the
+    amax by torch, s = fmax / amax as one fp32 division, the cast by torch's
+    float8 conversion of the clamped product, the read-back by torch's bf16
+    cast.  Pages are scattered through a shuffled block table; padding slots
+    (-1) write nothing; positions past a sequence's length read as 0."""
+    rng = np.random.default_rng(40 + fmt)
+    H, Dh, bs, NB = 3, 32, 16, 12
+    fm = np.float32(orc.fmax(fmt))
+    lens = np.array([37, 5, 0, 16], np.int32)
+    B, mb = len(lens), 4
+    table = np.full((B, mb), -1, np.int32)
+    perm = rng.permutation(NB).astype(np.int32)
+    k = 0
+    for b in range(B):
+        for j in range((lens[b] + bs - 1) // bs):
+            table[b, j] = perm[k]
+            k += 1
+    # token list: every position of every sequence plus two padding tokens
+    seq_of = np.concatenate([np.full(n, b) for b, n in enumerate(lens)] + [[0, 0]]).astype(np.int64)
+    pos_of = np.concatenate([np.arange(n) for n in lens] + [[0, 0]]).astype(np.int64)
+    T = len(seq_of)
+    slot = table[seq_of, pos_of // bs].astype(np.int64) * bs + pos_of % bs
+    slot[-2:] = -1
+    x = inputs.normal_bf16((T, H, Dh), 3.0, seed=50 + fmt)
+    x.view(-1)[7] = 0.0
+    x[1, 1] = 0.0                                   # an all-zero row: scale 1
+    c0 = rng.integers(0, 256, (NB, bs, H, Dh)).astype(np.uint8)   # stale pages
+    s0 = np.full((NB, bs, H), 7.0, np.float32)
+    cache, sc = orc.paged_kv_write(_bits(x), slot, c0, s0, fmt)
+
+    xf = x.float()
+    amax = xf.abs().amax(dim=-1)                    # [T, H]
+    s = torch.where(amax > 0, torch.tensor(float(fm)) / amax, torch.tensor(1.0))
+    y = (xf * s[..., None]).clamp(-float(fm), float(fm))
+    qref = y.to(TORCH_FP8[fmt]).view(torch.uint8).numpy()
+    sinv = (1.0 / s).numpy().astype(np.float32)
+    written = np.zeros(NB * bs, bool)
+    for t in range(T):
+        if slot[t] < 0:
+            continue
+        written[slot[t]] = True
+        assert np.array_equal(cache.reshape(NB * bs, H, Dh)[slot[t]], qref[t]), t
+        assert np.array_equal(sc.reshape(NB * bs, H)[slot[t]], sinv[t]), t
+    assert np.array_equal(cache.reshape(NB * bs, H, Dh)[~written], c0.reshape(NB * bs, H, Dh)[~written])
+    assert np.all(sc.reshape(NB * bs, H)[~written] == 7.0)
+
+    S_out = 40
+    out = orc.paged_kv_gather(cache, sc, table, lens, S_out, fmt)
+    deq = torch.from_numpy(qref).view(TORCH_FP8[fmt]).float()
+    ref = (deq * torch.from_numpy(sinv)[..., None]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    for b in range(B):
+        for t in range(S_out):
+            if t < lens[b]:
+                i = int(np.flatnonzero((seq_of[:-2] == b) & (pos_of[:-2] == t))[0])
+                assert np.array_equal(out[b, t], ref[i]), (b, t)
+            else:
+                assert not out[b, t].any(), (b, t)
