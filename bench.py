@@ -42,7 +42,7 @@ METRIC = "FP8 scaled GEMM TFLOP/s (% dense FP8 peak); quantize/KV GB/s (% HBM)"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_OVER_BF16 = 2.0     # nominal dense ratio: 4.5 PFLOP/s fp8 / 2.25 PFLOP/s bf16
-DEFAULT_STEPS = {"rowwise": 6000, "tensor": 6000, "blockmlp": 1500, "dgrad": 6000, "kv": 600}
+DEFAULT_STEPS = {"rowwise": 6000, "tensor": 6000, "blockmlp": 1500, "dgrad": 6000, "kv": 600, "paged": 600, "health": 6000}
 
 
 def peaks():
@@ -322,6 +322,83 @@ class Workload:
         f.fp8_kv_dequant(self.qk, self.sk, B, H, S, Dh, f.E4M3, self.Kd)
         f.fp8_kv_dequant(self.qv, self.sv, B, H, S, Dh, f.E4M3, self.Vd)
 
+    # paged FP8 KV cache: prefill write of K and V into shuffled 16-token pages,
+    # then both read back through the block table
+    def _setup_paged(self):
+        inp, d, s = self.inp, self.dev, self.seed
+        P = inp.PAGED_KV
+        B, S, H, Dh, bs = P["B"], P["S"], P["H"], P["Dh"], P["block_size"]
+        if self.profile:
+            B = 8
+        NB = B * S // bs
+        table, slots = inp.paged_layout([S] * B, bs, NB, seed=s + 3)
+        self.table, self.slots = table.to(d), slots.to(d)
+        self.lens = torch.full((B,), S, dtype=torch.int32, device=d)
+        self.K = inp.normal_bf16((B * S, H, Dh), 1.0, seed=s, device=d)
+        self.V = inp.normal_bf16((B * S, H, Dh), 1.0, seed=s + 1, device=d)
+        self.kc = self.f.PagedKVCache(NB, bs, H, Dh, self.f.E4M3, device=d)
+        self.vc = self.f.PagedKVCache(NB, bs, H, Dh, self.f.E4M3, device=d)
+        self.Kd = torch.empty((B, S, H, Dh), dtype=torch.bfloat16, device=d)
+        self.Vd = torch.empty_like(self.Kd)
+        self.dims = (B, S, H, Dh, bs, NB)
+        T = B * S
+        wbytes = 3.0 * T * H * Dh + 4.0 * T * H + 8.0 * T            # bf16 in, FP8 + 1/s out, slot ids
+        gbytes = 3.0 * T * H * Dh + 4.0 * T * H + 4.0 * table.numel() + 4.0 * B
+        self.bytes = 2 * (wbytes + gbytes)
+        self.kernel_bytes = wbytes                                    # one fp8_paged_kv_write launch
+        self.unit, self.bound = "GB/s", "hbm"
+        self.launches = 4
+        self.config = {"workload": "paged FP8 KV cache write + gather", "sequences": B, "tokens_per_seq": S,
+                       "H": H, "Dh": Dh, "block_size": bs, "num_blocks": NB, "pages": "shuffled pool",
+                       "K,V": "N(0,1) bf16", "scale": "per (token, head): 448/amax, E4M3"}
+        self.host_inputs = [("K", self.K), ("V", self.V)]
+        self.host_output = self.Kd
+
+    def _step_paged(self, ev=None):
+        f = self.f
+        B, S, H, Dh, bs, NB = self.dims
+        if ev:
+            ev[0].record()
+        f.fp8_paged_kv_write(self.K, self.slots, B * S, H, Dh, NB * bs, f.E4M3, self.kc.cache, self.kc.scale_inv)
+        if ev:
+            ev[1].record()
+        f.fp8_paged_kv_write(self.V, self.slots, B * S, H, Dh, NB * bs, f.E4M3, self.vc.cache, self.vc.scale_inv)
+        mb = self.table.shape[1]
+        f.fp8_paged_kv_gather(self.kc.cache, self.kc.scale_inv, self.table, self.lens, B, mb, H, Dh, bs, NB, S,
+                              f.E4M3, self.Kd)
+        f.fp8_paged_kv_gather(self.vc.cache, self.vc.scale_inv, self.table, self.lens, B, mb, H, Dh, bs, NB, S,
+                              f.E4M3, self.Vd)
+
+    # scale health check over every layer's rowwise scales
+    def _setup_health(self):
+        inp, d = self.inp, self.dev
+        L, n = inp.SCALE_HEALTH["layers"], inp.SCALE_HEALTH["per_layer"]
+        if self.profile:
+            L *= 8     # inputs above L2 size for the DRAM counters
+        prev, cur = inp.scale_snapshots_f32(L * n, seed=self.seed + 7)
+        self.prev, self.cur = prev.to(d), cur.to(d)
+        self.offs = (torch.arange(L + 1, dtype=torch.int64) * n).to(d)
+        self.stats = torch.empty((L, 3), dtype=torch.float32, device=d)
+        self.counts = torch.empty((L, 2), dtype=torch.int32, device=d)
+        self.dims = (L, n)
+        self.bytes = 2 * 4.0 * L * n + 8 * (L + 1) + 20 * L
+        self.kernel_bytes = self.bytes
+        self.unit, self.bound = "GB/s", "hbm"
+        self.launches = 1
+        self.config = {"workload": "scale health check (min/max/mean + step changes)", "segments": L,
+                       "scales_per_segment": n, "scales": "log10 s ~ N(1, 0.25); next snapshot drifted, "
+                       "0.1 % stepped x16 or /16", "jump_ratio": 4.0}
+        self.host_inputs = [("cur", self.cur)]
+        self.host_output = self.stats
+
+    def _step_health(self, ev=None):
+        L, n = self.dims
+        if ev:
+            ev[0].record()
+        self.f.fp8_scale_stats(self.cur, self.prev, L * n, self.offs, L, 4.0, self.stats, self.counts)
+        if ev:
+            ev[1].record()
+
     def step(self, ev=None):
         getattr(self, "_step_" + self.name)(ev)
 
@@ -407,6 +484,29 @@ def cpu_sample(name: str, seed: int = 0):
             t = (time.perf_counter() - t0) * (M / r) * (K_in / 256)
             return 2.0 * M * N_out * K_in / t / 1e12, (
                 f"quantize {r} gradient rows (E5M2) + 256 weight rows, then {r}x256 outputs; scaled to the step")
+    if name == "paged":
+        P = inputs.PAGED_KV
+        B, S, H, Dh, bs = P["B"], P["S"], P["H"], P["Dh"], P["block_size"]
+        r = 2048
+        x = inputs.bf16_bits(inputs.normal_bf16((r, H, Dh), 1.0, seed=seed))
+        table, slots = inputs.paged_layout([r], bs, r // bs, seed=seed + 3)
+        t0 = time.perf_counter()
+        c, sc = orc.paged_kv_write(x, slots.numpy(), np.zeros((r // bs, bs, H, Dh), np.uint8),
+                                   np.zeros((r // bs, bs, H), np.float32), 0)
+        orc.paged_kv_gather(c, sc, table.numpy(), np.array([r], np.int32), r, 0)
+        t = (time.perf_counter() - t0) * (B * S / r) * 2
+        T = B * S
+        full = 2 * (2 * (3.0 * T * H * Dh + 4.0 * T * H) + 8.0 * T + 4.0 * T / bs + 4.0 * B)
+        return full / t / 1e9, f"{r} tokens of K written and gathered; scaled to K and V of all {B}x{S} tokens"
+    if name == "health":
+        L, n = inputs.SCALE_HEALTH["layers"], inputs.SCALE_HEALTH["per_layer"]
+        prev, cur = inputs.scale_snapshots_f32(L * n, seed=seed + 7)
+        p, c = prev.numpy(), cur.numpy()
+        t0 = time.perf_counter()
+        for g in range(L):
+            orc.scale_stats(c[g * n:(g + 1) * n], p[g * n:(g + 1) * n], 4.0)
+        t = time.perf_counter() - t0
+        return (2 * 4.0 * L * n + 8 * (L + 1) + 20 * L) / t / 1e9, "the whole step (all 224 segments)"
     # kv
     B, H, S, Dh = 32, 32, 8192, 128
     k = inputs.bf16_bits(inputs.normal_bf16((1, 2, S, Dh), 1.0, seed=seed))
@@ -438,7 +538,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    unit = "GB/s" if args.workload == "kv" else "TFLOP/s"
+    unit = "GB/s" if args.workload in ("kv", "paged", "health") else "TFLOP/s"
 
     if args.impl == "reference":
         if rank != 0:
@@ -574,7 +674,9 @@ def main():
              "tensor": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate -> bf16",
              "blockmlp": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate (per-128-K promotion) -> bf16",
              "dgrad": "fp8_e5m2 x fp8_e4m3 -> f32 accumulate -> bf16",
-             "kv": "bf16 <-> fp8_e4m3 (f32 scale)"}[args.workload]
+             "kv": "bf16 <-> fp8_e4m3 (f32 scale)",
+             "paged": "bf16 <-> fp8_e4m3 (f32 scale per token and head)",
+             "health": "f32 scales, f64 sums"}[args.workload]
     cfg = dict(wl.config)
     cfg["l2"] = "flushed before every step (256 MiB write + 256 MiB read, outside the step's events)"
     line = {
@@ -584,7 +686,8 @@ def main():
         "roofline": {"bound": wl.bound, "achieved": achieved, "peak": peak, "unit": wl.unit,
                      "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-                     "kernel": "fp8_gemm_scaled" if wl.bound == "tensor" else "fp8_kv_quant",
+                     "kernel": {"kv": "fp8_kv_quant", "paged": "fp8_paged_kv_write",
+                                "health": "fp8_scale_stats"}.get(args.workload, "fp8_gemm_scaled"),
                      "kernel_ms": kern_avg_ms, "peak_source": peak_src},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

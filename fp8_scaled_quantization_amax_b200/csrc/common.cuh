@@ -153,6 +153,12 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
 }
 
 // L2 eviction-priority policies and loads / stores carrying them.
+__device__ __forceinline__ uint2 ld_stream_u2(const uint2 *p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+
 __device__ __forceinline__ uint64_t policy_evict_last() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));

@@ -43,6 +43,9 @@ SIGNATURES = {
     "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
     "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
+    "fp8_paged_kv_write": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
+    "fp8_paged_kv_gather": (_S, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P]),
+    "fp8_scale_stats": (_S, [_P, _P, _I64, _P, _I64, _F, _P, _P, _P]),
     "fp8_device_error": (_S, [_P, _I]),
 }
 
@@ -195,6 +198,32 @@ def fp8_kv_dequant(q, scale_inv, B, H, S, Dh, fmt, out, stream=None):
                                                   _stream(stream)))
 
 
+def fp8_paged_kv_write(kv, slot_mapping, T, H, Dh, num_slots, fmt, cache, scale_cache, stream=None):
+    _dev(kv, torch.bfloat16, "kv"); _dev(slot_mapping, torch.int64, "slot_mapping")
+    _dev(cache, torch.uint8, "cache"); _dev(scale_cache, torch.float32, "scale_cache")
+    _check("fp8_paged_kv_write", lib().fp8_paged_kv_write(
+        _ptr(kv), _ptr(slot_mapping), T, H, Dh, num_slots, fmt, _ptr(cache), _ptr(scale_cache), _stream(stream)))
+
+
+def fp8_paged_kv_gather(cache, scale_cache, block_table, seq_lens, B, max_blocks, H, Dh, block_size, num_blocks,
+                        S_out, fmt, out, stream=None):
+    _dev(cache, torch.uint8, "cache"); _dev(scale_cache, torch.float32, "scale_cache")
+    _dev(block_table, torch.int32, "block_table"); _dev(seq_lens, torch.int32, "seq_lens")
+    _dev(out, torch.bfloat16, "out")
+    _check("fp8_paged_kv_gather", lib().fp8_paged_kv_gather(
+        _ptr(cache), _ptr(scale_cache), _ptr(block_table), _ptr(seq_lens), B, max_blocks, H, Dh, block_size,
+        num_blocks, S_out, fmt, _ptr(out), _stream(stream)))
+
+
+def fp8_scale_stats(scales, prev, n, seg_offsets, num_segments, jump_ratio, stats, counts, stream=None):
+    _dev(scales, torch.float32, "scales"); _dev(prev, torch.float32, "prev")
+    _dev(seg_offsets, torch.int64, "seg_offsets")
+    _dev(stats, torch.float32, "stats"); _dev(counts, torch.int32, "counts")
+    _check("fp8_scale_stats", lib().fp8_scale_stats(
+        _ptr(scales), _ptr(prev), n, _ptr(seg_offsets), num_segments, jump_ratio, _ptr(stats), _ptr(counts),
+        _stream(stream)))
+
+
 def fp8_device_error(clear: bool = False) -> int:
     v = ctypes.c_uint32(0)
     _check("fp8_device_error", lib().fp8_device_error(ctypes.byref(v), int(clear)))
@@ -278,6 +307,46 @@ def kv_dequant(q, scale_inv, fmt=E4M3):
     out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     fp8_kv_dequant(q, scale_inv, B, H, S, Dh, fmt, out)
     return out
+
+
+class PagedKVCache:
+    """Device-resident paged FP8 cache of one tensor (K or V of one layer):
+    codes [num_blocks, block_size, H, Dh] and 1/s per (slot, head)."""
+
+    def __init__(self, num_blocks: int, block_size: int, H: int, Dh: int, fmt: int = E4M3, device="cuda"):
+        self.fmt, self.block_size, self.H, self.Dh = fmt, block_size, H, Dh
+        self.num_blocks = num_blocks
+        self.cache = torch.zeros((num_blocks, block_size, H, Dh), dtype=torch.uint8, device=device)
+        self.scale_inv = torch.zeros((num_blocks, block_size, H), dtype=torch.float32, device=device)
+
+    def write(self, kv, slot_mapping):
+        """kv [T, H, Dh] bf16 into the slots slot_mapping [T] (int64; < 0 = padding)."""
+        T = kv.shape[0]
+        fp8_paged_kv_write(kv, slot_mapping, T, self.H, self.Dh, self.num_blocks * self.block_size, self.fmt,
+                           self.cache, self.scale_inv)
+
+    def gather(self, block_table, seq_lens, S_out: int):
+        """[B, S_out, H, Dh] bf16 of every sequence (0 past its length)."""
+        B, mb = block_table.shape
+        out = torch.empty((B, S_out, self.H, self.Dh), dtype=torch.bfloat16, device=self.cache.device)
+        fp8_paged_kv_gather(self.cache, self.scale_inv, block_table, seq_lens, B, mb, self.H, self.Dh,
+                            self.block_size, self.num_blocks, S_out, self.fmt, out)
+        return out
+
+
+def scale_stats(scales, seg_offsets=None, prev=None, jump_ratio=4.0):
+    """Health check of scale factors: per segment {min, max, mean} (fp32 [G, 3])
+    and {step changes against prev, invalid entries} (int32 [G, 2], read as
+    unsigned).  seg_offsets: device int64 [G + 1] or None for one segment."""
+    s = scales.reshape(-1)
+    p = None if prev is None else prev.reshape(-1)
+    if p is not None and p.numel() != s.numel():
+        raise ValueError("prev must have as many entries as scales")
+    G = 1 if seg_offsets is None else seg_offsets.numel() - 1
+    stats = torch.empty((G, 3), dtype=torch.float32, device=s.device)
+    counts = torch.empty((G, 2), dtype=torch.int32, device=s.device)
+    fp8_scale_stats(s, p, s.numel(), seg_offsets, G, jump_ratio, stats, counts)
+    return stats, counts
 
 
 class AmaxHistory:

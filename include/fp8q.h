@@ -257,6 +257,72 @@ FP8Q_API fp8_status fp8_kv_dequant(const uint8_t *q, const float *scale_inv, int
                           int64_t S, int64_t Dh, fp8_format fmt, void *out_bf16, void *stream);
 
 /*
+ * Paged FP8 KV cache, write side ("FP8量化首次支持！ms-swift引领大模型低精度计算
+ * 新浪潮": the KV cache is cut into fixed-size blocks allocated on demand;
+ * [DeepL] §3.1: K and V stored in FP8).  Each (token, head) row of Dh
+ * elements is quantized with its own scale s = fmax / amax(row) (tokens
+ * arrive a few at a time, so a per-sequence amax is not known yet).
+ *   kv_bf16       [T, H, Dh] bf16, device, 16-byte aligned.
+ *   slot_mapping  [T] int64, device: slot = block * block_size + offset of
+ *                 each token; a slot outside [0, num_slots) marks padding and
+ *                 writes nothing.  Slots must be distinct (otherwise which
+ *                 token lands in a shared slot is unspecified).
+ *   cache         [num_slots, H, Dh] FP8 (= [num_blocks, block_size, H, Dh]),
+ *                 device, 16-byte aligned; only the mapped slots are written.
+ *   scale_cache   [num_slots, H] fp32, device: 1/s of each written row.
+ *   Shapes: Dh % 8 == 0, H * Dh <= 8192.
+ *   Errors: FP8_ERR_SHAPE, FP8_ERR_INVALID_ARG (NULL pointer, format),
+ *   FP8_ERR_ALIGNMENT.
+ */
+FP8Q_API fp8_status fp8_paged_kv_write(const void *kv_bf16, const int64_t *slot_mapping, int64_t T,
+                              int64_t H, int64_t Dh, int64_t num_slots, fp8_format fmt, uint8_t *cache,
+                              float *scale_cache, void *stream);
+
+/*
+ * Paged FP8 KV cache, read side: every sequence's tokens read back through
+ * its block table, dequantized ([DeepL] §3.1):
+ *   out[b][t][h][:] = bf16_RNE(fp32(q) * scale_cache[slot][h]),
+ *   slot = block_table[b][t / block_size] * block_size + t % block_size.
+ *   block_table [B, max_blocks] int32, seq_lens [B] int32, device.
+ *   out         [B, S_out, H, Dh] bf16, device, 16-byte aligned; a position
+ *               t >= seq_lens[b], past max_blocks * block_size, or whose
+ *               block id is outside [0, num_blocks) is written as 0.
+ *   Shapes: Dh % 8 == 0, H * Dh <= 8192, B <= 65535, block_size >= 1.
+ *   Errors: as fp8_paged_kv_write.
+ */
+FP8Q_API fp8_status fp8_paged_kv_gather(const uint8_t *cache, const float *scale_cache,
+                               const int32_t *block_table, const int32_t *seq_lens, int64_t B,
+                               int64_t max_blocks, int64_t H, int64_t Dh, int64_t block_size,
+                               int64_t num_blocks, int64_t S_out, fp8_format fmt, void *out_bf16,
+                               void *stream);
+
+/*
+ * Health check of scale factors ([DeepL] §6.2: report the min / max / mean of
+ * each layer's scales at intervals; a step change in a scale signals an
+ * outlier or a drift of the data distribution).
+ *   scales      [n] fp32, device.  Segment g covers
+ *               scales[seg_offsets[g] .. seg_offsets[g+1]) (device int64
+ *               [num_segments + 1], non-decreasing, clamped to [0, n] on the
+ *               device); seg_offsets == NULL means one segment, the whole
+ *               array (num_segments must then be 1).
+ *   prev        [n] fp32, device, the previous snapshot of the same scales, or
+ *               NULL (no step-change check).
+ *   jump_ratio  >= 1: an entry is a step change when it and its previous value
+ *               are both valid and either ratio (fp32 division) exceeds it.
+ *   stats       [num_segments][3] fp32, device: {min, max, mean} over the
+ *               valid entries (finite and > 0); mean = fp64 sum / count,
+ *               rounded to fp32; all three 0 when a segment has none.
+ *   counts      [num_segments][2] uint32, device: {step changes, invalid
+ *               entries (NaN, +-Inf, <= 0)}.
+ *   Deterministic: a fixed reduction order per segment.  n < 2^32.
+ *   Errors: FP8_ERR_INVALID_ARG (NULL output, jump_ratio < 1 or not finite),
+ *   FP8_ERR_SHAPE (segment count).
+ */
+FP8Q_API fp8_status fp8_scale_stats(const float *scales, const float *prev, int64_t n,
+                           const int64_t *seg_offsets, int64_t num_segments, float jump_ratio,
+                           float *stats, uint32_t *counts, void *stream);
+
+/*
  * Device error word of the library on the current device: a bit is set when
  * a kernel gave up a bounded wait (a pipeline barrier that did not complete
  * within about one second) and returned early instead of hanging.  0 means

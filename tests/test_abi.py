@@ -78,6 +78,22 @@ def test_validation_before_device_access():
     assert L.fp8_amax_history_update(FAKE, FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
     assert L.fp8_amax_history_update(FAKE, FAKE, 2000, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
     assert L.fp8_amax_history_update(None, FAKE, 16, FAKE, 0, FAKE, FAKE, FAKE, n) == INVALID
+    # paged KV cache
+    assert L.fp8_paged_kv_write(FAKE, FAKE, 4, 2, 12, 64, 0, FAKE, FAKE, n) == SHAPE        # Dh % 8
+    assert L.fp8_paged_kv_write(FAKE, FAKE, 4, 128, 128, 64, 0, FAKE, FAKE, n) == SHAPE     # H*Dh > 8192
+    assert L.fp8_paged_kv_write(FAKE, FAKE, 4, 2, 64, 64, 3, FAKE, FAKE, n) == INVALID
+    assert L.fp8_paged_kv_write(FAKE_ODD, FAKE, 4, 2, 64, 64, 0, FAKE, FAKE, n) == ALIGN
+    assert L.fp8_paged_kv_write(FAKE, None, 4, 2, 64, 64, 0, FAKE, FAKE, n) == INVALID
+    assert L.fp8_paged_kv_gather(FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 64, 0, 8, 16, 0, FAKE, n) == SHAPE
+    assert L.fp8_paged_kv_gather(FAKE, FAKE, FAKE, FAKE, 70000, 4, 2, 64, 16, 8, 16, 0, FAKE, n) == SHAPE
+    assert L.fp8_paged_kv_gather(FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 64, 16, 8, 16, 0, FAKE_ODD, n) == ALIGN
+    assert L.fp8_paged_kv_gather(FAKE, FAKE, FAKE, None, 2, 4, 2, 64, 16, 8, 16, 0, FAKE, n) == INVALID
+    # scale health check
+    assert L.fp8_scale_stats(FAKE, None, 16, None, 1, 0.5, FAKE, FAKE, n) == INVALID   # ratio < 1
+    assert L.fp8_scale_stats(FAKE, None, 16, None, 1, float("nan"), FAKE, FAKE, n) == INVALID
+    assert L.fp8_scale_stats(FAKE, None, 16, None, 1, 4.0, None, FAKE, n) == INVALID
+    assert L.fp8_scale_stats(FAKE, None, 16, None, 2, 4.0, FAKE, FAKE, n) == SHAPE   # no table, 2 segments
+    assert L.fp8_scale_stats(FAKE, None, 16, FAKE, 0, 4.0, FAKE, FAKE, n) == SHAPE
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
