@@ -267,17 +267,38 @@ k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
 // iteration (the two half-warps take neighbouring blocks), so U 16-byte loads
 // per lane are in flight and no index division is needed.  scale_inv is
 // stored [kb][row].
-template <int FMT, int U>
+// E8M0 scale image (the operand layout of the hardware block-scaled MMA):
+// for K block kb and row r, the four bytes at
+//   ((kb * ceil(rows / 128) + r / 128) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4)
+// hold the biased exponent e of the dequantization factor 2^(e - 127), once
+// per 32-wide quarter of the 128-wide block (all four equal here).  For a
+// power-of-two scale s = 2^k the factor is 2^-k, so e = 127 - k
+// = 254 - (biased exponent of s).
+__device__ __forceinline__ uint32_t e8m0_word_of_scale(float s) {
+    const uint32_t e = 254u - ((__float_as_uint(s) >> 23) & 0xFFu);
+    return e * 0x01010101u;
+}
+__device__ __forceinline__ int64_t e8m0_offset(int64_t kb, int64_t rt, int64_t r) {
+    return (kb * rt + (r >> 7)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+}
+
+// SF = false: fp32 scale_inv[kb * rows + row], s = fmax / amax.
+// SF = true:  E8M0 image (sf_image), s the pow2 rule; the image's padding rows
+//             (up to a multiple of 128) get e = 127 (factor 1).
+template <int FMT, int U, bool SF>
 __global__ void __launch_bounds__(256)
 k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-             uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
+             uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image) {
     constexpr float fm = fmax_of<FMT>();
     const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
     const int64_t nkb = (cols + 127) / 128;
+    const int64_t rt = (rows + 127) / 128;
+    const int64_t row_end = SF ? rt * 128 : rows;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t row = warp; row < rows; row += nwarps) {
-        const uint16_t *xr = x + row * ld;
+    for (int64_t row = warp; row < row_end; row += nwarps) {
+        const bool live = row < rows;
+        const uint16_t *xr = x + (live ? row : 0) * ld;
         uint8_t *qr = q + row * cols;
         for (int64_t kb0 = 0; kb0 < nkb; kb0 += 2 * U) {
             uint4 v[U];
@@ -287,7 +308,7 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
             for (int u = 0; u < U; ++u) {
                 const int64_t kb = kb0 + 2 * u + half;
                 cidx[u] = kb * 128 + l16 * 8;
-                valid[u] = (kb < nkb) && (cidx[u] < cols);
+                valid[u] = live && (kb < nkb) && (cidx[u] < cols);
                 v[u] = valid[u] ? ld_stream(reinterpret_cast<const uint4 *>(xr + cidx[u])) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
@@ -302,10 +323,14 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
                     const uint32_t t = __shfl_xor_sync(0xFFFFFFFFu, m, o);
                     m = t > m ? t : m;
                 }
-                const float s = scale_from_amax(bf16bits_to_float(m), fm);
+                const float s = SF ? pow2_scale_from_amax(bf16bits_to_float(m), fm)
+                                   : scale_from_amax(bf16bits_to_float(m), fm);
                 if (valid[u]) *reinterpret_cast<uint2 *>(qr + cidx[u]) = cast8<FMT>(v[u], s);
                 const int64_t kb = kb0 + 2 * u + half;
-                if (l16 == 0 && kb < nkb) scale_inv[kb * rows + row] = __fdiv_rn(1.0f, s);
+                if (l16 == 0 && kb < nkb) {
+                    if (SF) *reinterpret_cast<uint32_t *>(sf_image + e8m0_offset(kb, rt, row)) = e8m0_word_of_scale(s);
+                    else scale_inv[kb * rows + row] = __fdiv_rn(1.0f, s);
+                }
             }
         }
     }
@@ -315,10 +340,12 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
 // One CTA (256 threads) per 128x128 tile, the tile held in registers (8
 // vectors of 8 per thread: 16 threads across a 128-wide row, 16 rows per
 // pass, 8 passes).
-template <int FMT>
+// SF = true: pow2 scale, the tile's 512-byte E8M0 image entry written by the
+// first 32 threads (every byte the tile's exponent).
+template <int FMT, bool SF>
 __global__ void __launch_bounds__(256)
 k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-           uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
+           uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image) {
     __shared__ uint32_t red[32];
     constexpr float fm = fmax_of<FMT>();
     const int64_t nkb = (cols + 127) / 128, nrb = (rows + 127) / 128;
@@ -343,13 +370,20 @@ k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t l
             for (int p = 0; p < 8; ++p) m = amax_exact8(m, v[p], bad);
         }
         m = block_max_u32(m, red);
-        const float s = scale_from_amax(bf16bits_to_float(m), fm);
+        const float s = SF ? pow2_scale_from_amax(bf16bits_to_float(m), fm) : scale_from_amax(bf16bits_to_float(m), fm);
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
             const int64_t r = rb * 128 + p * 16 + rsub;
             if (r < rows && c < cols) *reinterpret_cast<uint2 *>(q + r * cols + c) = cast8<FMT>(v[p], s);
         }
-        if (threadIdx.x == 0) scale_inv[rb * nkb + kb] = __fdiv_rn(1.0f, s);
+        if (SF) {
+            if (threadIdx.x < 32) {
+                const uint32_t w = e8m0_word_of_scale(s);
+                reinterpret_cast<uint4 *>(sf_image + (kb * nrb + rb) * 512)[threadIdx.x] = make_uint4(w, w, w, w);
+            }
+        } else if (threadIdx.x == 0) {
+            scale_inv[rb * nkb + kb] = __fdiv_rn(1.0f, s);
+        }
     }
 }
 
@@ -408,19 +442,20 @@ void launch_rowwise(cudaStream_t st, int sms, const void *x, int64_t rows, int64
     else k_rowwise<FMT, POW2, 0, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
 }
 
-template <int FMT>
+template <int FMT, bool SF>
 void launch_block(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, int64_t ld,
-                  int block_rows, uint8_t *q, float *scale_inv) {
+                  int block_rows, uint8_t *q, float *scale_inv, uint8_t *sf_image) {
     const uint16_t *xs = static_cast<const uint16_t *>(x);
     const int64_t nkb = (cols + 127) / 128;
     if (block_rows == 1) {
         constexpr int U = 4;
-        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + 7) / 8, (int64_t)sms * 8));
-        k_block1x128<FMT, U><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+        const int64_t r = SF ? (rows + 127) / 128 * 128 : rows;
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((r + 7) / 8, (int64_t)sms * 8));
+        k_block1x128<FMT, U, SF><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv, sf_image);
     } else {
         const int64_t tiles = ((rows + 127) / 128) * nkb;
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)sms * 8));
-        k_block128<FMT><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+        k_block128<FMT, SF><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv, sf_image);
     }
 }
 
@@ -525,7 +560,27 @@ extern "C" fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, i
     if (st != FP8_OK) return st;
     if (rows == 0 || cols == 0) return FP8_OK;
     cudaStream_t s = as_stream(stream);
-    if (fmt == FP8_E4M3) launch_block<FP8_E4M3>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv);
-    else launch_block<FP8_E5M2>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv);
+    if (fmt == FP8_E4M3) launch_block<FP8_E4M3, false>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv, nullptr);
+    else launch_block<FP8_E5M2, false>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv, nullptr);
+    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+extern "C" fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                                  fp8_format fmt, int block_rows, uint8_t *q, uint8_t *sf_image,
+                                                  void *stream) {
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (block_rows != 1 && block_rows != 128) return FP8_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols || (cols % 16)) return FP8_ERR_SHAPE;
+    if (rows > 0 && cols > 0 && (!x_bf16 || !q || !sf_image)) return FP8_ERR_INVALID_ARG;
+    if (ld % 8) return FP8_ERR_ALIGNMENT;
+    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q)) || (sf_image && !aligned16(sf_image)))
+        return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (rows == 0 || cols == 0) return FP8_OK;
+    cudaStream_t s = as_stream(stream);
+    if (fmt == FP8_E4M3) launch_block<FP8_E4M3, true>(s, sms, x_bf16, rows, cols, ld, block_rows, q, nullptr, sf_image);
+    else launch_block<FP8_E5M2, true>(s, sms, x_bf16, rows, cols, ld, block_rows, q, nullptr, sf_image);
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }

@@ -43,6 +43,8 @@ SIGNATURES = {
     "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
     "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
+    "fp8_quantize_blockwise_e8m0": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
+    "fp8_gemm_block_e8m0": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _P, _P, _P, _I64, _P]),
     "fp8_paged_kv_write": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_paged_kv_gather": (_S, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P]),
     "fp8_scale_stats": (_S, [_P, _P, _I64, _P, _I64, _F, _P, _P, _P]),
@@ -196,6 +198,40 @@ def fp8_kv_dequant(q, scale_inv, B, H, S, Dh, fmt, out, stream=None):
     _dev(q, torch.uint8, "q"); _dev(scale_inv, torch.float32, "scale_inv"); _dev(out, torch.bfloat16, "out")
     _check("fp8_kv_dequant", lib().fp8_kv_dequant(_ptr(q), _ptr(scale_inv), B, H, S, Dh, fmt, _ptr(out),
                                                   _stream(stream)))
+
+
+def fp8_quantize_blockwise_e8m0(x, rows, cols, ld, fmt, block_rows, q, sf_image, stream=None):
+    _dev(x, torch.bfloat16, "x"); _dev(q, torch.uint8, "q"); _dev(sf_image, torch.uint8, "sf_image")
+    _check("fp8_quantize_blockwise_e8m0", lib().fp8_quantize_blockwise_e8m0(
+        _ptr(x), rows, cols, ld, fmt, block_rows, _ptr(q), _ptr(sf_image), _stream(stream)))
+
+
+def fp8_gemm_block_e8m0(A, fa, B, fb, M, N, K, a_sf, b_sf, D, ldd, stream=None):
+    _dev(A, torch.uint8, "A"); _dev(B, torch.uint8, "B"); _dev(D, torch.bfloat16, "D")
+    _dev(a_sf, torch.uint8, "a_sf"); _dev(b_sf, torch.uint8, "b_sf")
+    _check("fp8_gemm_block_e8m0", lib().fp8_gemm_block_e8m0(
+        _ptr(A), fa, _ptr(B), fb, M, N, K, _ptr(a_sf), _ptr(b_sf), _ptr(D), ldd, _stream(stream)))
+
+
+def e8m0_image_bytes(rows: int, cols: int) -> int:
+    return ((cols + 127) // 128) * ((rows + 127) // 128) * 512
+
+
+def quantize_blockwise_e8m0(x, fmt, block_rows):
+    """(q, sf_image) of x [rows, cols] with power-of-two block scales."""
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    img = torch.empty(e8m0_image_bytes(rows, cols), dtype=torch.uint8, device=x.device)
+    fp8_quantize_blockwise_e8m0(x, rows, cols, x.stride(0), fmt, block_rows, q, img)
+    return q, img
+
+
+def gemm_block_e8m0(A, fa, B, fb, a_sf, b_sf, out=None):
+    M, K = A.shape
+    N = B.shape[0]
+    D = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    fp8_gemm_block_e8m0(A, fa, B, fb, M, N, K, a_sf, b_sf, D, D.stride(0))
+    return D
 
 
 def fp8_paged_kv_write(kv, slot_mapping, T, H, Dh, num_slots, fmt, cache, scale_cache, stream=None):

@@ -130,6 +130,27 @@ FP8Q_API fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int
                                   void *stream);
 
 /*
+ * Per-block quantization with power-of-two scales written as an E8M0 scale
+ * image, the operand format of the hardware block-scaled MMA
+ * (fp8_gemm_block_e8m0).  Blocks as in fp8_quantize_blockwise ([DeepL] §2.3
+ * per-block scaling; power-of-two scales as in [Soup]'s rowwise recipe):
+ * s = the largest power of two with amax_block * s <= fmax (2^-126 ..
+ * 2^127; amax 0 gives 1), q = sat_RNE(fp32(x) * s).
+ *   q         [rows, cols] FP8, dense.
+ *   sf_image  ceil(cols/128) * ceil(rows/128) * 512 bytes, 16-byte aligned.
+ *             The dequantization factor of row r in K block kb is
+ *             2^(e - 127) with e = sf_image[(kb * ceil(rows/128) + r/128) * 512
+ *             + (r % 32) * 16 + ((r % 128) / 32) * 4 + j] for each of the
+ *             four 32-wide slices j of the block (all four equal here).
+ *             Rows past `rows` in the last 128-row group: e = 127 when
+ *             block_rows == 1, the block's e when block_rows == 128.
+ *   Shapes and errors: as fp8_quantize_blockwise.
+ */
+FP8Q_API fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                       fp8_format fmt, int block_rows, uint8_t *q, uint8_t *sf_image,
+                                       void *stream);
+
+/*
  * FP8 scaled GEMM ([H100]: the multiply-accumulate runs on FP8 operands on
  * the tensor cores; [Soup] tensorwise / rowwise scaled matmuls; per-block
  * scales per [DeepL] §2.3):
@@ -164,6 +185,25 @@ FP8Q_API fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8
                            int64_t M, int64_t N, int64_t K, fp8_scale_mode mode,
                            const float *a_scale_inv, const float *b_scale_inv, void *D_bf16,
                            int64_t ldd, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * FP8 GEMM with power-of-two block scales applied by the tensor core
+ * (tcgen05.mma.kind::mxf8f6f4.block_scale; [DeepL] §2.3 per-block scales):
+ *   D[m, n] = bf16( sum_kb 2^(ea[m,kb] - 127) * 2^(eb[n,kb] - 127)
+ *                   * sum_{k in kb} A[m, k] * B[n, k] ),  fp32 accumulation,
+ *   exactly the BLOCK mode of fp8_gemm_scaled when its scales are powers of
+ *   two, without the per-block promotion in the epilogue.
+ *   A [M, K], B [N, K] FP8, K contiguous (formats fa, fb).
+ *   a_sf, b_sf: E8M0 scale images of A and B in the layout
+ *   fp8_quantize_blockwise_e8m0 writes (a per-row or per-128-row-block
+ *   exponent for every 128-wide K block), 16-byte aligned, device.
+ *   D [M, N] bf16, leading dimension ldd.  Deterministic (one fixed K order).
+ *   Shapes: K % 16 == 0, N % 8 == 0, ldd % 8 == 0, ldd >= N; K == 0 writes
+ *   zeros.  Errors as fp8_gemm_scaled.
+ */
+FP8Q_API fp8_status fp8_gemm_block_e8m0(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
+                               int64_t M, int64_t N, int64_t K, const uint8_t *a_sf, const uint8_t *b_sf,
+                               void *D_bf16, int64_t ldd, void *stream);
 
 /*
  * Grouped FP8 GEMM for mixture-of-experts layers ("DeepL押注FP8：…" §3.2: the

@@ -78,6 +78,14 @@ def test_validation_before_device_access():
     assert L.fp8_amax_history_update(FAKE, FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
     assert L.fp8_amax_history_update(FAKE, FAKE, 2000, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
     assert L.fp8_amax_history_update(None, FAKE, 16, FAKE, 0, FAKE, FAKE, FAKE, n) == INVALID
+    # E8M0 block scales
+    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 32, 32, 0, 64, FAKE, FAKE, n) == INVALID    # block_rows
+    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 24, 32, 0, 1, FAKE, FAKE, n) == SHAPE       # cols % 16
+    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 32, 32, 0, 1, FAKE, FAKE_ODD, n) == ALIGN
+    assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 40, FAKE, FAKE, FAKE, 64, n) == SHAPE   # K % 16
+    assert L.fp8_gemm_block_e8m0(FAKE, 2, FAKE, 0, 64, 64, 64, FAKE, FAKE, FAKE, 64, n) == INVALID
+    assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 64, None, FAKE, FAKE, 64, n) == INVALID
+    assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 64, FAKE_ODD, FAKE, FAKE, 64, n) == ALIGN
     # paged KV cache
     assert L.fp8_paged_kv_write(FAKE, FAKE, 4, 2, 12, 64, 0, FAKE, FAKE, n) == SHAPE        # Dh % 8
     assert L.fp8_paged_kv_write(FAKE, FAKE, 4, 128, 128, 64, 0, FAKE, FAKE, n) == SHAPE     # H*Dh > 8192
