@@ -42,7 +42,7 @@ METRIC = "FP8 scaled GEMM TFLOP/s (% dense FP8 peak); quantize/KV GB/s (% HBM)"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_OVER_BF16 = 2.0     # nominal dense ratio: 4.5 PFLOP/s fp8 / 2.25 PFLOP/s bf16
-DEFAULT_STEPS = {"rowwise": 6000, "tensor": 6000, "blockmlp": 1500, "dgrad": 6000, "kv": 600, "paged": 600, "health": 6000}
+DEFAULT_STEPS = {"rowwise": 6000, "tensor": 6000, "blockmlp": 1500, "blockmlp_e8m0": 1500, "dgrad": 6000, "kv": 600, "paged": 600, "health": 6000}
 
 
 def peaks():
@@ -248,6 +248,45 @@ class Workload:
         f.fp8_quantize_blockwise(self.Wd, Dm, F, F, f.E4M3, 128, self.qwd, self.swd)
         f.fp8_gemm_scaled(self.qh, f.E4M3, self.qwd, f.E4M3, M, Dm, F, f.SCALE_BLOCK, self.sh, self.swd, self.Y, Dm)
 
+    # the same MLP with power-of-two block scales applied by the tensor core
+    def _setup_blockmlp_e8m0(self):
+        f, inp, d, s = self.f, self.inp, self.dev, self.seed
+        M, Dm, F = (2048 if self.profile else 8192), 4096, 11008
+        img = lambda r, c: torch.empty(f.e8m0_image_bytes(r, c), dtype=torch.uint8, device=d)
+        self.X = inp.normal_bf16((M, Dm), 1.0, seed=s, device=d)
+        self.Wu = inp.normal_bf16((F, Dm), 0.02, seed=s + 1, device=d)
+        self.Wd = inp.normal_bf16((Dm, F), 0.02, seed=s + 2, device=d)
+        self.qx, self.sx = torch.empty((M, Dm), dtype=torch.uint8, device=d), img(M, Dm)
+        self.qwu, self.swu = torch.empty((F, Dm), dtype=torch.uint8, device=d), img(F, Dm)
+        self.H = torch.empty((M, F), dtype=torch.bfloat16, device=d)
+        self.qh, self.sh = torch.empty((M, F), dtype=torch.uint8, device=d), img(M, F)
+        self.qwd, self.swd = torch.empty((Dm, F), dtype=torch.uint8, device=d), img(Dm, F)
+        self.Y = torch.empty((M, Dm), dtype=torch.bfloat16, device=d)
+        self.dims = (M, Dm, F)
+        self.flops = 2 * 2.0 * M * Dm * F
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.launches = 6
+        self.config = {"workload": "block-scaled E4M3 MLP (up then down), E8M0 scales in the MMA", "M": M,
+                       "D": Dm, "F": F, "X": "N(0,1) bf16", "W": "N(0,0.02) bf16",
+                       "scales": "1x128 activation blocks, 128x128 weight blocks, powers of two (E8M0)",
+                       "chain": "H = up(X) in bf16 is requantized 1x128 for the down GEMM"}
+        self.host_inputs = [("X", self.X), ("W_up", self.Wu), ("W_down", self.Wd)]
+        self.host_output = self.Y
+
+    def _step_blockmlp_e8m0(self, ev=None):
+        f = self.f
+        M, Dm, F = self.dims
+        f.fp8_quantize_blockwise_e8m0(self.X, M, Dm, Dm, f.E4M3, 1, self.qx, self.sx)
+        f.fp8_quantize_blockwise_e8m0(self.Wu, F, Dm, Dm, f.E4M3, 128, self.qwu, self.swu)
+        if ev:
+            ev[0].record()
+        f.fp8_gemm_block_e8m0(self.qx, f.E4M3, self.qwu, f.E4M3, M, F, Dm, self.sx, self.swu, self.H, F)
+        if ev:
+            ev[1].record()
+        f.fp8_quantize_blockwise_e8m0(self.H, M, F, F, f.E4M3, 1, self.qh, self.sh)
+        f.fp8_quantize_blockwise_e8m0(self.Wd, Dm, F, F, f.E4M3, 128, self.qwd, self.swd)
+        f.fp8_gemm_block_e8m0(self.qh, f.E4M3, self.qwd, f.E4M3, M, Dm, F, self.sh, self.swd, self.Y, Dm)
+
     # dgrad with delayed scaling
     def _setup_dgrad(self):
         f, inp, d, s = self.f, self.inp, self.dev, self.seed
@@ -408,7 +447,7 @@ class Workload:
     def kernel_work(self):
         """Work of one launch of the dominant kernel (events ev[0]..ev[1])."""
         if self.unit == "TFLOP/s":
-            if self.name == "blockmlp":
+            if self.name in ("blockmlp", "blockmlp_e8m0"):
                 M, Dm, F = self.dims
                 return 2.0 * M * Dm * F / 1e12
             return self.flops / 1e12
@@ -424,6 +463,8 @@ def cpu_sample(name: str, seed: int = 0):
     from fp8_scaled_quantization_amax_b200 import inputs
     from oracle import oracle as orc
     orc.lib()
+    if name == "blockmlp_e8m0":
+        name = "blockmlp"   # the same per-block GEMM in the oracle (its cost does not depend on the scale rule)
     if name in ("rowwise", "tensor", "blockmlp", "dgrad"):
         if name == "rowwise":
             M = N = K = 4096
@@ -631,7 +672,7 @@ def main():
 
     # end to end through the public API: pinned host inputs -> device, the
     # step, the result back to pinned host memory, every step
-    e2e_steps = min(steps, 10 if wl.unit == "TFLOP/s" and args.workload != "blockmlp" else 3)
+    e2e_steps = min(steps, 10 if wl.unit == "TFLOP/s" and args.workload not in ("blockmlp", "blockmlp_e8m0") else 3)
     host_in = [(name, t.detach().cpu().pin_memory()) for name, t in wl.host_inputs]
     host_out = torch.empty(wl.host_output.shape, dtype=wl.host_output.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for _, t in host_in)
@@ -673,6 +714,7 @@ def main():
     dtype = {"rowwise": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate -> bf16",
              "tensor": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate -> bf16",
              "blockmlp": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate (per-128-K promotion) -> bf16",
+             "blockmlp_e8m0": "fp8_e4m3 x fp8_e4m3, e8m0 block scales in the MMA -> f32 accumulate -> bf16",
              "dgrad": "fp8_e5m2 x fp8_e4m3 -> f32 accumulate -> bf16",
              "kv": "bf16 <-> fp8_e4m3 (f32 scale)",
              "paged": "bf16 <-> fp8_e4m3 (f32 scale per token and head)",
@@ -687,7 +729,8 @@ def main():
                      "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "kernel": {"kv": "fp8_kv_quant", "paged": "fp8_paged_kv_write",
-                                "health": "fp8_scale_stats"}.get(args.workload, "fp8_gemm_scaled"),
+                                "health": "fp8_scale_stats",
+                                "blockmlp_e8m0": "fp8_gemm_block_e8m0"}.get(args.workload, "fp8_gemm_scaled"),
                      "kernel_ms": kern_avg_ms, "peak_source": peak_src},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

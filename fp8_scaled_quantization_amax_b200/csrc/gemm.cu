@@ -36,218 +36,26 @@
 // kernel records a bit in the library's device error word, stops issuing,
 // waits (bounded) for its own copies and MMAs in flight, frees TMEM and
 // returns.  No trap, no unbounded spin.
-#include <cuda.h>
-
 #include <algorithm>
 #include <atomic>
 #include <mutex>
 
-#include "common.cuh"
+#include "tc.cuh"
 
 using namespace fp8q;
 
 namespace {
 
-constexpr int BM = 128;                 // tile rows (TMEM lanes)
 constexpr int BN = 256;                 // tile columns (TMEM columns per accumulator)
-constexpr int BK = 128;                 // K chunk: one 128-byte swizzle row of FP8
 constexpr int STAGES = 4;
-constexpr int A_TILE = BM * BK;         // 16 KiB
 constexpr int B_TILE = BN * BK;         // 32 KiB
 constexpr int STAGE_BYTES = A_TILE + B_TILE;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
-constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, acc_full[2], acc_empty[2], drain
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_BARS * 8 + 16;
-constexpr uint64_t kTimeoutNs = 1000000000ull;
 
 enum { kModeTensor = 0, kModeRow = 1, kModeBlock = 2 };
-enum : uint32_t { kErrProducer = 1u, kErrMma = 2u, kErrEpilogue = 4u, kErrDrain = 8u, kErrSplit = 16u };
-
-__device__ unsigned int g_gemm_error;
-
-// ------------------------------------------------------------- PTX glue --
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-// Local arrive used to release a TMEM buffer (relaxed for the same reason as
-// mbar_arrive_cluster below: the guarded TMEM loads have completed).
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait for the phase of `bar` with the given parity.  Gives up when
-// the CTA's abort flag is raised or after kTimeoutNs (then it raises the flag
-// and records `code` in the device error word).
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag,
-                                      uint32_t code) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (globaltimer() - t0 > kTimeoutNs) {
-                atomicOr(&g_gemm_error, code);
-                *abort_flag = 1u;
-                return false;
-            }
-        }
-    }
-}
-// Bounded wait that ignores the abort flag (used to drain work in flight).
-__device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer() - t0 > kTimeoutNs) {
-            atomicOr(&g_gemm_error, kErrDrain);
-            return false;
-        }
-    }
-    return true;
-}
-// Split-K hand-off flag: the first-half pair publishes its partial with a
-// release store of the launch's epoch; the second-half pair polls with
-// acquire loads (bounded, like every wait in this file).
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_u32(uint32_t *p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ bool wait_flag(const uint32_t *p, uint32_t epoch, volatile uint32_t *abort_flag) {
-    const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (ld_acquire_u32(p) == epoch) return true;
-        if ((it & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (globaltimer() - t0 > kTimeoutNs) {
-                atomicOr(&g_gemm_error, kErrSplit);
-                *abort_flag = 1u;
-                return false;
-            }
-        }
-        __nanosleep(32);
-    }
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-        : "memory");
-}
-// 32 lanes x 32 consecutive fp32 columns: thread i gets lane (base + i).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-// 32 lanes x 32 columns, issued without waiting: the registers are only
-// valid after tmem_wait64() on the array that contains them.
-__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t *r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-// One wait for all loads in flight; the 64 registers are named read-write so
-// no use of them can move above the wait.
-__device__ __forceinline__ void tmem_wait64(uint32_t (&r)[64]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
-                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
-                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31]), "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]),
-                   "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]), "+r"(r[40]), "+r"(r[41]), "+r"(r[42]),
-                   "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]), "+r"(r[48]), "+r"(r[49]),
-                   "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]), "+r"(r[56]),
-                   "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
-                 :
-                 : "memory");
-}
-
-// Packed fp32 pair arithmetic (sm_100): two IEEE round-to-nearest FMAs per
-// instruction, which halves the issue cost of the block-scale promotion.
-__device__ __forceinline__ uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
-    uint64_t d;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
-    return d;
-}
-__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
-// 128 bytes, 8-row groups 1024 bytes apart (the layout TMA writes with
-// CU_TENSOR_MAP_SWIZZLE_128B and a 128-byte inner box).
-__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t addr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFFu);    // start address (16-byte units)
-    d |= (uint64_t)1u << 16;                    // leading byte offset (unused for swizzled K-major)
-    d |= (uint64_t)(1024u >> 4) << 32;          // stride byte offset: 8 rows x 128 B
-    d |= (uint64_t)1u << 46;                    // descriptor version for sm_100
-    d |= (uint64_t)2u << 61;                    // layout: SWIZZLE_128B
-    return d;
-}
 
 // ------------------------------------------------------------- kernel ----
 template <int MODE>
@@ -499,80 +307,6 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 //     leader's barrier (count 2 x 8 warps).
 // BLOCK mode uses BN = 128 and four 128-column TMEM partial buffers, so the
 // MMA can run three K chunks ahead of the promotion.
-namespace sm2 {
-constexpr int EPI = 8;                 // epilogue warps 4..11 (warpgroups 1 and 2)
-constexpr int THREADS = 12 * 32;       // warpgroup 0: producer (warp 0), MMA (warp 1), two idle warps
-// BLOCK mode moves registers from warpgroup 0 to the epilogue warpgroups,
-// which hold a 128-wide fp32 accumulator row per thread.  The split must
-// not exceed the launch pool: 128 * 56 + 256 * 224 = 64512 = 384 * 168,
-// so the kernel must launch at exactly 168 registers per thread (checked on
-// the host before the first launch).
-constexpr int REGS_LAUNCH = 168, REGS_LOW = 56, REGS_HIGH = 224;
-static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * REGS_LAUNCH, "register split exceeds the launch pool");
-template <int BN>
-struct Cfg {
-    static constexpr int B_HALF = (BN / 2) * BK;
-    static constexpr int STAGE = A_TILE + B_HALF;
-    static constexpr int STAGES = (BN == 256) ? 6 : 8;
-    static constexpr int NBUF = 512 / BN;
-    static constexpr int NBARS = 2 * STAGES + 2 * NBUF + 2;   // + drain, + split partial written
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + NBARS * 8 + 16;
-};
-// Split-K tail workspace: per split tile, per CTA of the pair, a 128 x 256
-// fp32 partial stored column-major (row index fastest, so a warp's lanes write
-// consecutive words), then one flag word per (tile, CTA).
-constexpr size_t kSplitPartialFloats = 128 * 256;
-}  // namespace sm2
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Release of a TMEM buffer to the leader's MMA thread.  Relaxed: the TMEM
-// loads it guards have already completed (tcgen05.wait::ld) and are ordered
-// by tcgen05.fence::before_thread_sync; a release fence here would also wait
-// for unrelated global loads and stores in flight (measured as the dominant
-// "membar" stall of the block-scaled epilogue).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, uint32_t bar_cluster, int x,
-                                                 int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
-        : "memory");
-}
-__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-        : "memory");
-}
-// arrive on the barrier at this shared offset in both CTAs of the pair
-__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-        "h"((uint16_t)0x3)
-        : "memory");
-}
-__device__ __forceinline__ void tc_commit_pair_self(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
 template <int MODE, int BN, bool GROUPED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
 k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
@@ -926,276 +660,6 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
-// ----------------------------------------- hardware block scales (E8M0) ----
-// Power-of-two block scales applied inside the tensor core:
-// tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale multiplies every
-// 32-wide K slice of A's row m by 2^(sfa - 127) and of B's row n by
-// 2^(sfb - 127) before accumulating, so the fp32 accumulator already holds
-// sum_kb dA[m, kb] * dB[n, kb] * sum_{k in kb} A[m, k] B[n, k] and the
-// epilogue only rounds to bf16 -- no per-128-K promotion.
-//
-// The E8M0 factors come as images in the MMA's scale-factor layout (see the
-// quantizer): per 128-wide K block, 512 bytes per 128 rows.  Every stage, each
-// CTA of the pair TMA-loads its own 128 rows' SFA entry (512 B) and the SFB
-// entries of all 256 tile columns (1 KiB; both CTAs need all columns, since
-// each CTA's accumulator rows span the whole tile width) next to its A and B
-// tiles; the leader copies them into TMEM with
-// tcgen05.cp.cta_group::2.32x128b.warpx4 (32 lanes x 16 bytes broadcast to
-// the four lane quarters: TMEM lane m % 32 (+ 32 q), column m / 32 holds row
-// m's four bytes) ahead of the stage's four MMAs, which run in issue order
-// behind the copies.  The SF columns sit after a single 256-column
-// accumulator (TMEM has 512 columns), so the epilogue drains the whole
-// accumulator into registers and releases it before converting and storing,
-// to get the MMA going on the next tile as early as possible.
-namespace mx {
-constexpr int SFA_BYTES = 512;                    // 128 rows x 4 bytes
-constexpr int SFB_BYTES = 1024;                   // 256 columns x 4 bytes
-constexpr int AB_STAGE = A_TILE + 128 * BK;       // this CTA's 128 rows of A and of B
-constexpr int SF_STAGE = SFA_BYTES + SFB_BYTES;
-constexpr int STAGES = 6;
-constexpr int NBARS = 2 * STAGES + 3;             // full, empty, acc full, acc empty, drain
-constexpr size_t SMEM = 1024 + (size_t)STAGES * (AB_STAGE + SF_STAGE) + NBARS * 8 + 16;
-constexpr uint32_t SFA_COL = 256, SFB_COL = 260;  // TMEM columns after the accumulator
-static_assert(SMEM <= 232448, "shared memory per block");
-}  // namespace mx
-
-// Shared-memory descriptor of a 32-row x 16-byte block without swizzle
-// (8-row core matrices 128 bytes apart): the source of a 32x128b tcgen05.cp.
-__device__ __forceinline__ uint64_t sdesc_sf(uint32_t addr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFFu);    // start address (16-byte units)
-    d |= (uint64_t)(128u >> 4) << 32;           // stride byte offset: 8 rows x 16 B
-    d |= (uint64_t)1u << 46;                    // descriptor version for sm_100
-    return d;                                   // layout type 0: no swizzle
-}
-__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-__device__ __forceinline__ void tc_mma_pair_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                               uint32_t sfa, uint32_t sfb, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
-        : "memory");
-}
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
-k_gemm_mx_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, int M, int N,
-              int K, uint32_t idesc, __nv_bfloat16 *__restrict__ D, int64_t ldd) {
-    constexpr int STG = mx::STAGES;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sf_smem = smem + (size_t)STG * mx::AB_STAGE;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sf_smem + (size_t)STG * mx::SF_STAGE);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + mx::NBARS);
-    volatile uint32_t *abort_flag = tmem_slot + 1;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_rank();
-    const bool leader = (rank == 0);
-    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int num_m = (M + 255) / 256, num_n = (N + 255) / 256;
-    const int tiles = num_m * num_n;
-    const int mt = (M + 127) / 128, nt = (N + 127) / 128;   // 128-row entries per K block of each image
-    const int nk = (K + BK - 1) / BK;
-    const int n_items = (pair < tiles) ? (tiles - 1 - pair) / npairs + 1 : 0;
-
-    auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
-    auto empty_bar = [&](int s) { return smem_u32(&bars[STG + s]); };
-    const uint32_t accf_bar = smem_u32(&bars[2 * STG]);
-    const uint32_t acce_bar = smem_u32(&bars[2 * STG + 1]);
-    const uint32_t drain_bar = smem_u32(&bars[2 * STG + 2]);
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STG; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
-        }
-        mbar_init(accf_bar, 1);
-        mbar_init(acce_bar, 2 * sm2::EPI);
-        mbar_init(drain_bar, 1);
-        *abort_flag = 0u;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmSA)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmSB)) : "memory");
-    }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();   // both CTAs' barriers are initialised before any remote signal
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer --
-        if (lane == 0) {
-            int last_round[STG];
-            for (int s = 0; s < STG; ++s) last_round[s] = -1;
-            uint32_t it = 0;
-            bool ok = true;
-            for (int i = 0; ok && i < n_items; ++i) {
-                const int t = pair + i * npairs;
-                const int m_blk = t % num_m, n_blk = t / num_m;
-                const int a_row = m_blk * 256 + (int)rank * 128;
-                const int b_row = n_blk * 256 + (int)rank * 128;
-                const int sa_ent = m_blk * 2 + (int)rank, sb_ent = n_blk * 2;
-                for (int kc = 0; kc < nk; ++kc, ++it) {
-                    const int stage = it % STG;
-                    const uint32_t round = it / STG;
-                    if (!wait_bar(empty_bar(stage), (round & 1u) ^ 1u, abort_flag, kErrProducer)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t full_leader = mapa_shared(full_bar(stage), 0);
-                    if (leader) mbar_expect_tx(full_bar(stage), 2 * (mx::AB_STAGE + mx::SF_STAGE));
-                    const uint32_t a_dst = smem_u32(smem + (size_t)stage * mx::AB_STAGE);
-                    const uint32_t sf_dst = smem_u32(sf_smem + (size_t)stage * mx::SF_STAGE);
-                    tma_load_2d_pair(a_dst, &tmA, full_leader, kc * BK, a_row);
-                    tma_load_2d_pair(a_dst + A_TILE, &tmB, full_leader, kc * BK, b_row);
-                    // image rows of 16 bytes: 32 per 128-row entry
-                    tma_load_2d_pair(sf_dst, &tmSA, full_leader, 0, (kc * mt + sa_ent) * 32);
-                    tma_load_2d_pair(sf_dst + mx::SFA_BYTES, &tmSB, full_leader, 0, (kc * nt + sb_ent) * 32);
-                    last_round[stage] = (int)round;
-                }
-            }
-            if (leader && (!ok || *abort_flag)) {
-                for (int s = 0; s < STG; ++s)
-                    if (last_round[s] >= 0) wait_bar_drain(full_bar(s), (uint32_t)last_round[s] & 1u);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------- MMA issuer (leader only) --
-        if (leader && lane == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            const uint32_t sfa_t = tmem + mx::SFA_COL, sfb_t = tmem + mx::SFB_COL;
-            for (int i = 0; ok && i < n_items; ++i) {
-                if (!wait_bar(acce_bar, ((uint32_t)i & 1u) ^ 1u, abort_flag, kErrMma)) break;
-                tc_fence_after();
-                for (int kc = 0; kc < nk; ++kc, ++it) {
-                    const int stage = it % STG;
-                    const uint32_t round = it / STG;
-                    if (!wait_bar(full_bar(stage), round & 1u, abort_flag, kErrMma)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t a_addr = smem_u32(smem + (size_t)stage * mx::AB_STAGE);
-                    const uint32_t sf_addr = smem_u32(sf_smem + (size_t)stage * mx::SF_STAGE);
-                    tc_cp_sf_pair(sfa_t, sdesc_sf(sf_addr));
-                    tc_cp_sf_pair(sfb_t, sdesc_sf(sf_addr + mx::SFA_BYTES));
-                    tc_cp_sf_pair(sfb_t + 4, sdesc_sf(sf_addr + mx::SFA_BYTES + 512));
-                    const uint64_t adesc = sdesc_k_sw128(a_addr);
-                    const uint64_t bdesc = sdesc_k_sw128(a_addr + A_TILE);
-#pragma unroll
-                    for (int k = 0; k < BK / 32; ++k) {
-                        // scale-factor byte k of each 32-bit TMEM word: the k-th 32-wide slice
-                        const uint32_t id = idesc | ((uint32_t)k << 4) | ((uint32_t)k << 29);
-                        tc_mma_pair_mx(tmem, adesc + 2u * k, bdesc + 2u * k, id, sfa_t, sfb_t,
-                                       (kc > 0 || k > 0) ? 1u : 0u);
-                    }
-                    tc_commit_pair_both(empty_bar(stage));
-                }
-                if (ok) tc_commit_pair_both(accf_bar);
-            }
-            tc_commit_pair_self(drain_bar);
-            wait_bar_drain(drain_bar, 0u);
-        }
-        __syncwarp();
-    } else if (warp >= 4) {
-        // --------------------------------------------------- epilogue ----
-        const int sp = warp & 3;
-        const int ch = (warp - 4) >> 2;
-        const uint32_t src = tmem + ((uint32_t)(sp * 32) << 16) + ch * 128;
-        for (int i = 0; i < n_items; ++i) {
-            const int t = pair + i * npairs;
-            const int m_blk = t % num_m, n_blk = t / num_m;
-            const int64_t m = (int64_t)m_blk * 256 + (int)rank * 128 + sp * 32 + lane;
-            const int n_base = n_blk * 256 + ch * 128;
-            bool w = true;
-            if (lane == 0) w = wait_bar(accf_bar, (uint32_t)i & 1u, abort_flag, kErrEpilogue);
-            w = __shfl_sync(0xFFFFFFFFu, w, 0);
-            if (!w) break;
-            tc_fence_after();
-            // the whole 128-column slice of this warp, then hand TMEM back
-            uint32_t r0[64], r1[64];
-            tmem_ld32_async(src, r0);
-            tmem_ld32_async(src + 32, r0 + 32);
-            tmem_ld32_async(src + 64, r1);
-            tmem_ld32_async(src + 96, r1 + 32);
-            tmem_wait64(r0);
-            tmem_wait64(r1);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar, 0));
-            if (m < M) {
-                __nv_bfloat16 *drow = D + m * ldd;
-#pragma unroll
-                for (int g = 0; g < 16; ++g) {
-                    const int col = n_base + g * 8;
-                    const uint32_t *r = (g < 8) ? (r0 + g * 8) : (r1 + (g - 8) * 8);
-                    if (col < N) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                        o.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                        o.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                        o.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                        *reinterpret_cast<uint4 *>(drow + col) = o;
-                    }
-                }
-            }
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();   // every TMEM read and MMA of both CTAs is done
-    if (warp == 1) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
-    }
-}
-
-// ---------------------------------------------------------------- host ----
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// 2-D map over a [rows, K] FP8 matrix (row pitch K bytes), box 128 x box_rows,
-// 128-byte swizzle; out-of-range boxes read zeros.
-bool make_map(CUtensorMap *map, const void *base, int64_t K, int64_t rows, uint32_t box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K};
-    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int MODE>
 cudaError_t launch_gemm(cudaStream_t st, int sms, const CUtensorMap &ta, const CUtensorMap &tb, int M, int N, int K,
                         uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd) {
@@ -1291,56 +755,6 @@ cudaError_t launch_gemm_grouped(cudaStream_t st, const CUtensorMap &ta, const CU
         ta, tb, (int)total_M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd, 0, 0, nullptr, nullptr, 0,
         goff, G);
     return cudaPeekAtLastError();
-}
-
-// 2-D map over an E8M0 scale image viewed as rows of 16 bytes, box 16 x
-// box_rows, no swizzle (the 32x128b tcgen05.cp source layout).
-bool make_sf_map(CUtensorMap *map, const void *base, int64_t rows16, uint32_t box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {16, (cuuint64_t)rows16};
-    cuuint64_t strides[1] = {16};
-    cuuint32_t box[2] = {16, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// Pairs of the E8M0 kernel that fit on the device at once (cached per device).
-int mx_pair_capacity() {
-    static int cache[64];
-    static std::mutex mu;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    std::lock_guard<std::mutex> lk(mu);
-    if (cache[dev] > 0) return cache[dev];
-    if (cudaFuncSetAttribute(k_gemm_mx_2sm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mx::SMEM) !=
-        cudaSuccess)
-        return 0;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * 64);
-    cfg.blockDim = dim3(sm2::THREADS);
-    cfg.dynamicSmemBytes = mx::SMEM;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_mx_2sm, &cfg) != cudaSuccess) return 0;
-    cache[dev] = n;
-    return n;
-}
-
-// Instruction descriptor of kind::mxf8f6f4 with E8M0 scale factors: A/B
-// formats, K-major A and B, N >> 3, scale type E8M0 (bit 23), M >> 4; the
-// scale-factor byte selectors (bits 4-5 for B, 29-30 for A) are set per MMA.
-uint32_t make_idesc_mx(fp8_format fa, fp8_format fb, int mma_m, int mma_n) {
-    return ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(mma_n >> 3) << 17) | (1u << 23) |
-           ((uint32_t)(mma_m >> 4) << 24);
 }
 
 uint32_t make_idesc(fp8_format fa, fp8_format fb, int mma_m, int mma_n) {
@@ -1445,51 +859,18 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
     return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-extern "C" fp8_status fp8_gemm_block_e8m0(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
-                                          int64_t M, int64_t N, int64_t K, const uint8_t *a_sf, const uint8_t *b_sf,
-                                          void *D_bf16, int64_t ldd, void *stream) {
-    if ((fa != FP8_E4M3 && fa != FP8_E5M2) || (fb != FP8_E4M3 && fb != FP8_E5M2)) return FP8_ERR_INVALID_ARG;
-    if (M < 0 || N < 0 || K < 0 || ldd < N) return FP8_ERR_SHAPE;
-    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP8_ERR_SHAPE;
-    if (K % 16) return FP8_ERR_SHAPE;
-    if (N % 8 || ldd % 8) return FP8_ERR_ALIGNMENT;
-    const int64_t nk = (K + BK - 1) / BK;
-    // image rows of 16 bytes must stay addressable by a 32-bit TMA coordinate
-    if (nk * ((M + 127) / 128) * 32 >= (1ll << 31) || nk * ((N + 127) / 128) * 32 >= (1ll << 31)) return FP8_ERR_SHAPE;
-    int sms;
-    if (M == 0 || N == 0) return check_device(&sms);
-    if (!D_bf16) return FP8_ERR_INVALID_ARG;
-    if (K > 0 && (!A || !B || !a_sf || !b_sf)) return FP8_ERR_INVALID_ARG;
-    if (!aligned16(D_bf16) || (A && !aligned16(A)) || (B && !aligned16(B)) || (a_sf && !aligned16(a_sf)) ||
-        (b_sf && !aligned16(b_sf)))
-        return FP8_ERR_ALIGNMENT;
-    fp8_status st = check_device(&sms);
-    if (st != FP8_OK) return st;
-    cudaStream_t s = as_stream(stream);
-    if (K == 0)
-        return cudaMemset2DAsync(D_bf16, (size_t)ldd * 2, 0, (size_t)N * 2, (size_t)M, s) == cudaSuccess ? FP8_OK
-                                                                                                       : FP8_ERR_CUDA;
-    CUtensorMap ta, tb, tsa, tsb;
-    if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
-    if (!make_sf_map(&tsa, a_sf, nk * ((M + 127) / 128) * 32, 32) ||
-        !make_sf_map(&tsb, b_sf, nk * ((N + 127) / 128) * 32, 64))
-        return FP8_ERR_CUDA;
-    const int cap = mx_pair_capacity();
-    if (cap <= 0) return FP8_ERR_CUDA;
-    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
-    k_gemm_mx_2sm<<<2 * pairs, sm2::THREADS, mx::SMEM, s>>>(ta, tb, tsa, tsb, (int)M, (int)N, (int)K,
-                                                          make_idesc_mx(fa, fb, 256, 256),
-                                                          static_cast<__nv_bfloat16 *>(D_bf16), ldd);
-    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
-}
+// The E8M0 GEMM's translation unit keeps its own error word (gemm_mx.cu).
+fp8_status fp8q_mx_device_error(uint32_t *out, int clear);
 
 extern "C" fp8_status fp8_device_error(uint32_t *host_out, int clear) {
     if (!host_out) return FP8_ERR_INVALID_ARG;
     if (cudaDeviceSynchronize() != cudaSuccess) return FP8_ERR_CUDA;
     unsigned int v = 0;
     if (cudaMemcpyFromSymbol(&v, g_gemm_error, sizeof(v)) != cudaSuccess) return FP8_ERR_CUDA;
-    *host_out = v;
+    uint32_t w = 0;
+    const fp8_status st = fp8q_mx_device_error(&w, clear);
+    if (st != FP8_OK) return st;
+    *host_out = v | w;
     if (clear) {
         const unsigned int z = 0;
         if (cudaMemcpyToSymbol(g_gemm_error, &z, sizeof(z)) != cudaSuccess) return FP8_ERR_CUDA;

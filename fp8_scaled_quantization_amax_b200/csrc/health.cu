@@ -7,9 +7,11 @@
 // when finite and > 0; a step change is a ratio to the previous snapshot's
 // scale above a caller threshold, in either direction.
 //
-// One cluster of kCluster CTAs per segment (a layer's scales): each CTA
-// reduces a contiguous quarter of the segment with all of a thread's loads in
-// flight together, then the leading CTA combines the four partials through
+// One CTA of 512 threads per segment (a layer's scales), two CTAs per SM, a
+// thread's loads of both snapshots for a batch of 10 in flight together (a
+// larger batch spills at the 64 registers two CTAs per SM allow).
+// Segments averaging more than 32768 scales get a cluster of 8 CTAs each,
+// every CTA reducing a contiguous eighth, combined by the leading CTA through
 // distributed shared memory in rank order.  The sum is kept in fp64 and every
 // reduction runs in a fixed order, so a result never depends on timing.
 #include <cooperative_groups.h>
@@ -23,9 +25,10 @@ using namespace fp8q;
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kUnroll = 8;
-constexpr int kCluster = 4;
+constexpr int kThreads = 512;
+constexpr int kUnroll = 10;
+constexpr int kBigCluster = 8;
+constexpr int64_t kBigSegment = 32768;   // average segment length above which clusters are used
 
 struct Acc {
     uint32_t mn, mx;   // bit patterns of positive finite floats (ordered as integers)
@@ -62,18 +65,18 @@ __device__ __forceinline__ void warp_reduce(Acc &a) {
     }
 }
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads)
+template <int CL>
+__global__ void __launch_bounds__(kThreads, 2)
 k_scale_stats(const float *__restrict__ s, const float *__restrict__ prev, int64_t n,
               const int64_t *__restrict__ offsets, float r, float *__restrict__ stats,
               uint32_t *__restrict__ counts) {
-    cg::cluster_group cluster = cg::this_cluster();
-    const unsigned rank = cluster.block_rank();
-    const int g = blockIdx.x / kCluster;
+    const unsigned rank = (CL > 1) ? cg::this_cluster().block_rank() : 0u;
+    const int g = blockIdx.x / CL;
     int64_t lo = offsets ? offsets[g] : 0;
     int64_t hi = offsets ? offsets[g + 1] : n;
     lo = lo < 0 ? 0 : (lo > n ? n : lo);   // a corrupted table reads nothing out of range
     hi = hi < lo ? lo : (hi > n ? n : hi);
-    const int64_t per = (hi - lo + kCluster - 1) / kCluster;
+    const int64_t per = (hi - lo + CL - 1) / CL;
     const int64_t c0 = lo + min((int64_t)rank * per, hi - lo);
     const int64_t c1 = min(c0 + per, hi);
 
@@ -90,11 +93,22 @@ k_scale_stats(const float *__restrict__ s, const float *__restrict__ prev, int64
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) visit(a, v[u], p[u], r);
     }
-    for (; base < c1; base += kThreads) visit(a, s[base], prev ? prev[base] : __int_as_float(0x7FC00000), r);
+    {   // the ragged end: its loads also issued together
+        float v[kUnroll], p[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + u * kThreads;
+            v[u] = i < c1 ? __ldg(s + i) : 1.0f;
+            p[u] = (i < c1 && prev) ? __ldg(prev + i) : __int_as_float(0x7FC00000);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            if (base + u * kThreads < c1) visit(a, v[u], p[u], r);
+    }
 
     warp_reduce(a);
     __shared__ Acc part[kThreads / 32];
-    __shared__ Acc cta;   // this CTA's partial, read by the leading CTA
+    __shared__ Acc cta;   // this CTA's partial (read by the leading CTA of a cluster)
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) part[w] = a;
     __syncthreads();
@@ -103,20 +117,24 @@ k_scale_stats(const float *__restrict__ s, const float *__restrict__ prev, int64
         warp_reduce(a);
         if (lane == 0) cta = a;
     }
-    cluster.sync();   // every CTA's partial is published
-    if (rank == 0 && w == 0) {
-        a = lane < kCluster ? *cluster.map_shared_rank(&cta, lane) : Acc{0x7F800000u, 0u, 0.0, 0u, 0u, 0u};
-        warp_reduce(a);   // lanes >= kCluster hold the identity, so rank order fixes the sum
-        if (lane == 0) {
-            const bool any = a.nv != 0;
-            stats[3 * g + 0] = any ? __uint_as_float(a.mn) : 0.0f;
-            stats[3 * g + 1] = any ? __uint_as_float(a.mx) : 0.0f;
-            stats[3 * g + 2] = any ? (float)(a.sum / (double)a.nv) : 0.0f;
-            counts[2 * g + 0] = a.jumps;
-            counts[2 * g + 1] = a.invalid;
+    if (CL > 1) {
+        cg::this_cluster().sync();   // every CTA's partial is published
+        if (rank == 0 && w == 0) {
+            a = lane < CL ? *cg::this_cluster().map_shared_rank(&cta, lane) : Acc{0x7F800000u, 0u, 0.0, 0u, 0u, 0u};
+            warp_reduce(a);   // lanes >= CL hold the identity, so rank order fixes the sum
         }
+    } else {
+        __syncthreads();
     }
-    cluster.sync();   // no CTA leaves while the leading CTA may still read its partial
+    if (rank == 0 && threadIdx.x == 0) {
+        const bool any = a.nv != 0;
+        stats[3 * g + 0] = any ? __uint_as_float(a.mn) : 0.0f;
+        stats[3 * g + 1] = any ? __uint_as_float(a.mx) : 0.0f;
+        stats[3 * g + 2] = any ? (float)(a.sum / (double)a.nv) : 0.0f;
+        counts[2 * g + 0] = a.jumps;
+        counts[2 * g + 1] = a.invalid;
+    }
+    if (CL > 1) cg::this_cluster().sync();   // no CTA leaves while the leading CTA may read its partial
 }
 
 }  // namespace
@@ -129,13 +147,31 @@ extern "C" fp8_status fp8_scale_stats(const float *scales, const float *prev, in
     if (!stats || !counts || n < 0) return FP8_ERR_INVALID_ARG;
     if (n > 0 && !scales) return FP8_ERR_INVALID_ARG;
     if (!(jump_ratio >= 1.0f) || !(jump_ratio <= FLT_MAX)) return FP8_ERR_INVALID_ARG;
-    if (seg_offsets ? (num_segments < 1 || num_segments > 0x7FFFFFFF / kCluster) : num_segments != 1)
+    if (seg_offsets ? (num_segments < 1 || num_segments > 0x7FFFFFFF / kBigCluster) : num_segments != 1)
         return FP8_ERR_SHAPE;
     if (n > 0xFFFFFFFFll) return FP8_ERR_SHAPE;   // per-segment counters are 32-bit
     int sms;
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
-    k_scale_stats<<<(unsigned)(num_segments * kCluster), kThreads, 0, as_stream(stream)>>>(
-        scales, prev, n, seg_offsets, jump_ratio, stats, counts);
+    cudaStream_t cs = as_stream(stream);
+    if (n / num_segments > kBigSegment) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(num_segments * kBigCluster));
+        cfg.blockDim = dim3(kThreads);
+        cfg.stream = cs;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = kBigCluster;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, k_scale_stats<kBigCluster>, scales, prev, n, seg_offsets, jump_ratio, stats,
+                               counts) != cudaSuccess)
+            return FP8_ERR_CUDA;
+    } else {
+        k_scale_stats<1><<<(unsigned)num_segments, kThreads, 0, cs>>>(scales, prev, n, seg_offsets, jump_ratio,
+                                                                        stats, counts);
+    }
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }

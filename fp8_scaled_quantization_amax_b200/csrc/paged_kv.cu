@@ -15,10 +15,13 @@
 //
 // Write: a CTA takes kTok tokens; thread c owns elements [8c, 8c + 8) of every
 // one of them (one 16-byte load per token, all kTok in flight together).  A
-// head spans Dh/8 consecutive threads: when that is a power of two up to 32
+// head spans G = Dh/8 consecutive threads: when G is a power of two up to 32
 // its amax is a shuffle reduction inside the group, otherwise a shared-memory
-// max.  The codes leave as one 8-byte store per thread and token.
-// Gather: the mirror image, one CTA per kTok positions of one sequence.
+// max.  The kTok x H scales are then computed once each, by one thread per
+// (token, head) -- the correctly rounded divisions are the costliest step of
+// the kernel, and issuing them per 8-element chunk made it issue-bound --
+// and read back from shared memory for the cast.  The codes leave as one
+// 8-byte store per thread and token.
 #include "common.cuh"
 
 using namespace fp8q;
@@ -30,12 +33,15 @@ constexpr int kMaxRowElems = 8192;          // H * Dh per token
 constexpr int kMaxThreads = kMaxRowElems / 8;
 
 // G = Dh / 8 threads per head; SHFL: G is a power of two <= 32.
+// Dynamic shared memory: kTok * H uint32 head amax + kTok * H fp32 scales.
 template <int FMT, bool SHFL>
 __global__ void __launch_bounds__(kMaxThreads)
 k_paged_write(const uint4 *__restrict__ x, const int64_t *__restrict__ slot_mapping, int64_t T, int H,
               int G, int64_t num_slots, uint2 *__restrict__ cache, float *__restrict__ scale_cache) {
     constexpr float fm = fmax_of<FMT>();
-    __shared__ uint32_t head_amax[kTok][kMaxThreads];   // used when !SHFL (H <= kMaxThreads)
+    extern __shared__ uint32_t sm_paged[];
+    uint32_t *head_amax = sm_paged;                                   // [kTok][H]
+    float *head_scale = reinterpret_cast<float *>(sm_paged + kTok * H);   // [kTok][H]
     const int C = H * G;                                 // 8-element chunks per token
     const int c = threadIdx.x;
     const int64_t t0 = (int64_t)blockIdx.x * kTok;
@@ -52,40 +58,46 @@ k_paged_write(const uint4 *__restrict__ x, const int64_t *__restrict__ slot_mapp
 #pragma unroll
     for (int k = 0; k < kTok; ++k)
         if (slot[k] >= num_slots) slot[k] = -1;          // outside the cache: padding
-    uint32_t m[kTok];
+    if (!SHFL) {
+        for (int i = threadIdx.x; i < kTok * H; i += blockDim.x) head_amax[i] = 0u;
+        __syncthreads();
+    }
 #pragma unroll
     for (int k = 0; k < kTok; ++k) {
-        uint32_t bad = 0;
-        m[k] = amax_exact8(0u, v[k], bad);
-    }
-    if (SHFL) {
-#pragma unroll
-        for (int k = 0; k < kTok; ++k)
+        uint32_t m = amax_fast_final(amax_fast8(0u, v[k]));
+        if (m == 0xFFFFFFFFu) {   // a NaN or Inf among the eight: the exact, skipping form
+            uint32_t bad = 0;
+            m = amax_exact8(0u, v[k], bad);
+        }
+        if (SHFL) {
             for (int o = G >> 1; o > 0; o >>= 1) {
-                const uint32_t w = __shfl_xor_sync(0xFFFFFFFFu, m[k], o);
-                m[k] = w > m[k] ? w : m[k];
+                const uint32_t w = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+                m = w > m ? w : m;
             }
-    } else {
-        for (int i = threadIdx.x; i < kTok * H; i += blockDim.x) head_amax[i / H][i % H] = 0u;
-        __syncthreads();
-        if (c < C) {
-#pragma unroll
-            for (int k = 0; k < kTok; ++k) atomicMax(&head_amax[k][c / G], m[k]);
-        }
-        __syncthreads();
-        if (c < C) {
-#pragma unroll
-            for (int k = 0; k < kTok; ++k) m[k] = head_amax[k][c / G];
+            if (c < C && (c & (G - 1)) == 0) head_amax[k * H + c / G] = m;
+        } else if (c < C) {
+            atomicMax(&head_amax[k * H + c / G], m);
         }
     }
+    __syncthreads();
+    // one thread per (token, head): the scale, and 1/s into the cache
+    for (int i = threadIdx.x; i < kTok * H; i += blockDim.x) {
+        const int k = i / H, h = i - k * H;
+        const float s = scale_from_amax(bf16bits_to_float(head_amax[i]), fm);
+        head_scale[i] = s;
+        const int64_t t = t0 + k;
+        if (t < T) {
+            const int64_t sl = slot_mapping[t];
+            if (sl >= 0 && sl < num_slots) scale_cache[sl * H + h] = __fdiv_rn(1.0f, s);
+        }
+    }
+    __syncthreads();
     if (c >= C) return;
     const int h = c / G;
 #pragma unroll
     for (int k = 0; k < kTok; ++k) {
         if (slot[k] < 0) continue;
-        const float s = scale_from_amax(bf16bits_to_float(m[k]), fm);
-        cache[slot[k] * C + c] = cast8<FMT>(v[k], s);
-        if (c == h * G) scale_cache[slot[k] * H + h] = __fdiv_rn(1.0f, s);
+        cache[slot[k] * C + c] = cast8<FMT>(v[k], head_scale[k * H + h]);
     }
 }
 
@@ -168,12 +180,13 @@ extern "C" fp8_status fp8_paged_kv_write(const void *kv_bf16, const int64_t *slo
     cudaStream_t s = as_stream(stream);
     const uint4 *x = (const uint4 *)kv_bf16;
     uint2 *q = (uint2 *)cache;
+    const size_t sm = (size_t)kTok * H * 8;   // <= 32 KiB (H <= 1024)
     if (fmt == FP8_E4M3) {
-        if (shfl) k_paged_write<FP8_E4M3, true><<<grid, thr, 0, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
-        else k_paged_write<FP8_E4M3, false><<<grid, thr, 0, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
+        if (shfl) k_paged_write<FP8_E4M3, true><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
+        else k_paged_write<FP8_E4M3, false><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
     } else {
-        if (shfl) k_paged_write<FP8_E5M2, true><<<grid, thr, 0, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
-        else k_paged_write<FP8_E5M2, false><<<grid, thr, 0, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
+        if (shfl) k_paged_write<FP8_E5M2, true><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
+        else k_paged_write<FP8_E5M2, false><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
     }
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }

@@ -267,19 +267,20 @@ k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
 // iteration (the two half-warps take neighbouring blocks), so U 16-byte loads
 // per lane are in flight and no index division is needed.  scale_inv is
 // stored [kb][row].
-// E8M0 scale image (the operand layout of the hardware block-scaled MMA):
-// for K block kb and row r, the four bytes at
-//   ((kb * ceil(rows / 128) + r / 128) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4)
-// hold the biased exponent e of the dequantization factor 2^(e - 127), once
-// per 32-wide quarter of the 128-wide block (all four equal here).  For a
-// power-of-two scale s = 2^k the factor is 2^-k, so e = 127 - k
+// E8M0 scale image (the operand layout of the hardware block-scaled MMA,
+// which reads one byte per row for every 32-wide K slice; a 32-bit word holds
+// four such bytes).  Here a byte carries a whole 128-wide K block, so one word
+// covers four K blocks: for K block kb and row r the byte at
+//   ((kb / 4) * ceil(rows / 128) + r / 128) * 512 + (r % 32) * 16
+//     + ((r % 128) / 32) * 4 + kb % 4
+// holds the biased exponent e of the dequantization factor 2^(e - 127).  For
+// a power-of-two scale s = 2^k the factor is 2^-k, so e = 127 - k
 // = 254 - (biased exponent of s).
-__device__ __forceinline__ uint32_t e8m0_word_of_scale(float s) {
-    const uint32_t e = 254u - ((__float_as_uint(s) >> 23) & 0xFFu);
-    return e * 0x01010101u;
+__device__ __forceinline__ uint8_t e8m0_of_scale(float s) {
+    return (uint8_t)(254u - ((__float_as_uint(s) >> 23) & 0xFFu));
 }
 __device__ __forceinline__ int64_t e8m0_offset(int64_t kb, int64_t rt, int64_t r) {
-    return (kb * rt + (r >> 7)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+    return ((kb >> 2) * rt + (r >> 7)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (kb & 3);
 }
 
 // SF = false: fp32 scale_inv[kb * rows + row], s = fmax / amax.
@@ -328,7 +329,7 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
                 if (valid[u]) *reinterpret_cast<uint2 *>(qr + cidx[u]) = cast8<FMT>(v[u], s);
                 const int64_t kb = kb0 + 2 * u + half;
                 if (l16 == 0 && kb < nkb) {
-                    if (SF) *reinterpret_cast<uint32_t *>(sf_image + e8m0_offset(kb, rt, row)) = e8m0_word_of_scale(s);
+                    if (SF) sf_image[e8m0_offset(kb, rt, row)] = e8m0_of_scale(s);
                     else scale_inv[kb * rows + row] = __fdiv_rn(1.0f, s);
                 }
             }
@@ -340,8 +341,9 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
 // One CTA (256 threads) per 128x128 tile, the tile held in registers (8
 // vectors of 8 per thread: 16 threads across a 128-wide row, 16 rows per
 // pass, 8 passes).
-// SF = true: pow2 scale, the tile's 512-byte E8M0 image entry written by the
-// first 32 threads (every byte the tile's exponent).
+// SF = true: pow2 scale; the first 128 threads write the tile's exponent
+// into the E8M0 image byte of each of its 128 rows (rows past `rows`
+// included).
 template <int FMT, bool SF>
 __global__ void __launch_bounds__(256)
 k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
@@ -377,10 +379,7 @@ k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t l
             if (r < rows && c < cols) *reinterpret_cast<uint2 *>(q + r * cols + c) = cast8<FMT>(v[p], s);
         }
         if (SF) {
-            if (threadIdx.x < 32) {
-                const uint32_t w = e8m0_word_of_scale(s);
-                reinterpret_cast<uint4 *>(sf_image + (kb * nrb + rb) * 512)[threadIdx.x] = make_uint4(w, w, w, w);
-            }
+            if (threadIdx.x < 128) sf_image[e8m0_offset(kb, nrb, rb * 128 + threadIdx.x)] = e8m0_of_scale(s);
         } else if (threadIdx.x == 0) {
             scale_inv[rb * nkb + kb] = __fdiv_rn(1.0f, s);
         }

@@ -214,7 +214,7 @@ def fp8_gemm_block_e8m0(A, fa, B, fb, M, N, K, a_sf, b_sf, D, ldd, stream=None):
 
 
 def e8m0_image_bytes(rows: int, cols: int) -> int:
-    return ((cols + 127) // 128) * ((rows + 127) // 128) * 512
+    return ((cols + 511) // 512) * ((rows + 127) // 128) * 512
 
 
 def quantize_blockwise_e8m0(x, fmt, block_rows):

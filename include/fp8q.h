@@ -137,13 +137,15 @@ FP8Q_API fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int
  * s = the largest power of two with amax_block * s <= fmax (2^-126 ..
  * 2^127; amax 0 gives 1), q = sat_RNE(fp32(x) * s).
  *   q         [rows, cols] FP8, dense.
- *   sf_image  ceil(cols/128) * ceil(rows/128) * 512 bytes, 16-byte aligned.
- *             The dequantization factor of row r in K block kb is
- *             2^(e - 127) with e = sf_image[(kb * ceil(rows/128) + r/128) * 512
- *             + (r % 32) * 16 + ((r % 128) / 32) * 4 + j] for each of the
- *             four 32-wide slices j of the block (all four equal here).
- *             Rows past `rows` in the last 128-row group: e = 127 when
- *             block_rows == 1, the block's e when block_rows == 128.
+ *   sf_image  ceil(cols/512) * ceil(rows/128) * 512 bytes, 16-byte aligned.
+ *             The dequantization factor of row r in K block kb (128 wide) is
+ *             2^(e - 127) with e = sf_image[((kb / 4) * ceil(rows/128) + r/128)
+ *             * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4]: one
+ *             byte per row and K block, four K blocks per 32-bit word (the
+ *             block-scaled MMA's scale-factor layout).  Rows past `rows` in
+ *             the last 128-row group: e = 127 when block_rows == 1, the
+ *             block's e when block_rows == 128.  Bytes of K blocks past the
+ *             last one are not written.
  *   Shapes and errors: as fp8_quantize_blockwise.
  */
 FP8Q_API fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
@@ -195,8 +197,8 @@ FP8Q_API fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8
  *   two, without the per-block promotion in the epilogue.
  *   A [M, K], B [N, K] FP8, K contiguous (formats fa, fb).
  *   a_sf, b_sf: E8M0 scale images of A and B in the layout
- *   fp8_quantize_blockwise_e8m0 writes (a per-row or per-128-row-block
- *   exponent for every 128-wide K block), 16-byte aligned, device.
+ *   fp8_quantize_blockwise_e8m0 writes (an exponent per row and 128-wide K
+ *   block), 16-byte aligned, device.
  *   D [M, N] bf16, leading dimension ldd.  Deterministic (one fixed K order).
  *   Shapes: K % 16 == 0, N % 8 == 0, ldd % 8 == 0, ldd >= N; K == 0 writes
  *   zeros.  Errors as fp8_gemm_scaled.
