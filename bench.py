@@ -46,11 +46,13 @@ DEFAULT_STEPS = {"rowwise": 6000, "tensor": 6000, "blockmlp": 1500, "blockmlp_e8
 
 
 def peaks():
+    """(HBM GB/s, bf16 burst TFLOP/s, bf16 sustained TFLOP/s or None, source)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+        sus = d.get("bf16_tflops_sustained")
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), (float(sus) if sus else None), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, None, "fallback"
 
 
 def recorded_traffic(workload: str):
@@ -695,11 +697,17 @@ def main():
     e2e_value = world * wl.work() / (e2e_ms * 1e-3)
     assert fp8q.fp8_device_error(clear=True) == 0, "a kernel gave up a bounded wait"
 
-    hbm, bf16, src = peaks()
+    hbm, bf16, bf16_sus, src = peaks()
+    clocks = clk.summary()
     if wl.bound == "tensor":
-        peak = bf16 * FP8_OVER_BF16
-        peak_src = (f"FP8 dense peak = {src} bf16 burst {bf16} TFLOP/s x nominal fp8/bf16 ratio 2 "
-                    "(MEASURED_PEAKS.json)" if src == "measured" else f"fallback bf16 {bf16} x 2")
+        # the sustained (power-capped) figure when the timed region ran under
+        # the power cap, the burst figure otherwise
+        capped = "sw_power_cap" in clocks.get("reasons", []) and bf16_sus is not None
+        base = bf16_sus if capped else bf16
+        peak = base * FP8_OVER_BF16
+        peak_src = (f"FP8 dense peak = {src} bf16 {'sustained' if capped else 'burst'} {base} TFLOP/s x nominal "
+                    f"fp8/bf16 ratio 2 (MEASURED_PEAKS.json){'; sw_power_cap was active in the timed region' if capped else ''}"
+                    if src == "measured" else f"fallback bf16 {bf16} x 2")
     else:
         peak = hbm
         peak_src = f"{src} HBM copy bandwidth {hbm} GB/s"
@@ -736,7 +744,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": wl.launches * steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "wall_s_timed_region": t_wall,
     }
     print(json.dumps(line))

@@ -8,8 +8,8 @@
 // scale above a caller threshold, in either direction.
 //
 // One CTA of 512 threads per segment (a layer's scales), two CTAs per SM, a
-// thread's loads of both snapshots for a batch of 10 in flight together (a
-// larger batch spills at the 64 registers two CTAs per SM allow).
+// thread's loads of both snapshots for a batch of 16 in flight together: one
+// DRAM round trip covers 8192 scales.
 // Segments averaging more than 32768 scales get a cluster of 8 CTAs each,
 // every CTA reducing a contiguous eighth, combined by the leading CTA through
 // distributed shared memory in rank order.  The sum is kept in fp64 and every
@@ -26,7 +26,7 @@ using namespace fp8q;
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kUnroll = 10;
+constexpr int kUnroll = 16;
 constexpr int kBigCluster = 8;
 constexpr int64_t kBigSegment = 32768;   // average segment length above which clusters are used
 
@@ -36,16 +36,37 @@ struct Acc {
     uint32_t nv, jumps, invalid;
 };
 
+// "RN(v / p) > r" for positive finite v, p without the division (the
+// correctly rounded fp32 division is a long instruction sequence and made
+// this kernel issue-bound).  RN(q) > r exactly when q lies above the midpoint
+// mid = r + ulp(r)/2, or on it when the value above r has an even mantissa;
+// mid needs 25 significant bits and p 24, so mid * p is exact in fp64 and the
+// comparison with v is exact too.
+struct Ratio {
+    double mid;
+    bool tie_up;
+};
+__device__ __forceinline__ Ratio ratio_threshold(float r) {
+    const uint32_t rb = __float_as_uint(r);
+    const float up = __uint_as_float(rb + 1u);   // the next float above r (+inf above FLT_MAX)
+    const double ulp = isinf(up) ? 20282409603651670423947251286016.0 /* 2^104 */ : (double)up - (double)r;
+    return Ratio{(double)r + 0.5 * ulp, (rb & 1u) != 0u};
+}
+__device__ __forceinline__ bool ratio_above(float v, float p, const Ratio &t) {
+    const double x = (double)v, y = t.mid * (double)p;
+    return x > y || (x == y && t.tie_up);
+}
+
 // p is the previous snapshot's entry, or NaN when there is none (NaN fails
 // the validity test, so it never counts as a step change)
-__device__ __forceinline__ void visit(Acc &a, float v, float p, float r) {
+__device__ __forceinline__ void visit(Acc &a, float v, float p, const Ratio &t) {
     if (v > 0.0f && v <= FLT_MAX) {
         const uint32_t b = __float_as_uint(v);
         a.mn = b < a.mn ? b : a.mn;
         a.mx = b > a.mx ? b : a.mx;
         a.sum += (double)v;
         a.nv += 1;
-        if (p > 0.0f && p <= FLT_MAX && (__fdiv_rn(v, p) > r || __fdiv_rn(p, v) > r)) a.jumps += 1;
+        if (p > 0.0f && p <= FLT_MAX && (ratio_above(v, p, t) || ratio_above(p, v, t))) a.jumps += 1;
     } else {
         a.invalid += 1;
     }
@@ -81,6 +102,7 @@ k_scale_stats(const float *__restrict__ s, const float *__restrict__ prev, int64
     const int64_t c1 = min(c0 + per, hi);
 
     Acc a{0x7F800000u, 0u, 0.0, 0u, 0u, 0u};
+    const Ratio rt = ratio_threshold(r);
     const int64_t step = (int64_t)kThreads * kUnroll;
     int64_t base = c0 + threadIdx.x;
     for (; base + (kUnroll - 1) * kThreads < c1; base += step) {
@@ -91,7 +113,7 @@ k_scale_stats(const float *__restrict__ s, const float *__restrict__ prev, int64
             p[u] = prev ? __ldg(prev + base + u * kThreads) : __int_as_float(0x7FC00000);
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) visit(a, v[u], p[u], r);
+        for (int u = 0; u < kUnroll; ++u) visit(a, v[u], p[u], rt);
     }
     {   // the ragged end: its loads also issued together
         float v[kUnroll], p[kUnroll];
@@ -103,7 +125,7 @@ k_scale_stats(const float *__restrict__ s, const float *__restrict__ prev, int64
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u)
-            if (base + u * kThreads < c1) visit(a, v[u], p[u], r);
+            if (base + u * kThreads < c1) visit(a, v[u], p[u], rt);
     }
 
     warp_reduce(a);

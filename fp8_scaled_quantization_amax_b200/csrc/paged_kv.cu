@@ -15,9 +15,9 @@
 //
 // Write: a CTA takes kTok tokens; thread c owns elements [8c, 8c + 8) of every
 // one of them (one 16-byte load per token, all kTok in flight together).  A
-// head spans G = Dh/8 consecutive threads: when G is a power of two up to 32
-// its amax is a shuffle reduction inside the group, otherwise a shared-memory
-// max.  The kTok x H scales are then computed once each, by one thread per
+// head spans G = Dh/8 consecutive threads: for head sizes 64, 128 and 256
+// its amax is an unrolled shuffle reduction inside the group, otherwise a
+// shared-memory max.  The kTok x H scales are then computed once each, by one thread per
 // (token, head) -- the correctly rounded divisions are the costliest step of
 // the kernel, and issuing them per 8-element chunk made it issue-bound --
 // and read back from shared memory for the cast.  The codes leave as one
@@ -32,12 +32,16 @@ constexpr int kTok = 4;
 constexpr int kMaxRowElems = 8192;          // H * Dh per token
 constexpr int kMaxThreads = kMaxRowElems / 8;
 
-// G = Dh / 8 threads per head; SHFL: G is a power of two <= 32.
+// G = Dh / 8 threads per head.  GS = G when G is 8, 16 or 32 (head sizes 64,
+// 128, 256: the group reduction is an unrolled shuffle and the head index a
+// shift), GS = 0 otherwise (a shared-memory max, runtime division).
 // Dynamic shared memory: kTok * H uint32 head amax + kTok * H fp32 scales.
-template <int FMT, bool SHFL>
+template <int FMT, int GS>
 __global__ void __launch_bounds__(kMaxThreads)
 k_paged_write(const uint4 *__restrict__ x, const int64_t *__restrict__ slot_mapping, int64_t T, int H,
-              int G, int64_t num_slots, uint2 *__restrict__ cache, float *__restrict__ scale_cache) {
+              int G_rt, int64_t num_slots, uint2 *__restrict__ cache, float *__restrict__ scale_cache) {
+    constexpr bool SHFL = GS > 0;
+    const int G = SHFL ? GS : G_rt;
     constexpr float fm = fmax_of<FMT>();
     extern __shared__ uint32_t sm_paged[];
     uint32_t *head_amax = sm_paged;                                   // [kTok][H]
@@ -70,11 +74,12 @@ k_paged_write(const uint4 *__restrict__ x, const int64_t *__restrict__ slot_mapp
             m = amax_exact8(0u, v[k], bad);
         }
         if (SHFL) {
-            for (int o = G >> 1; o > 0; o >>= 1) {
+#pragma unroll
+            for (int o = GS >> 1; o > 0; o >>= 1) {
                 const uint32_t w = __shfl_xor_sync(0xFFFFFFFFu, m, o);
                 m = w > m ? w : m;
             }
-            if (c < C && (c & (G - 1)) == 0) head_amax[k * H + c / G] = m;
+            if (c < C && (c & (GS - 1)) == 0) head_amax[k * H + c / GS] = m;
         } else if (c < C) {
             atomicMax(&head_amax[k * H + c / G], m);
         }
@@ -174,20 +179,26 @@ extern "C" fp8_status fp8_paged_kv_write(const void *kv_bf16, const int64_t *slo
     st = check_device(&sms);
     if (st != FP8_OK) return st;
     const int G = (int)(Dh / 8);
-    const bool shfl = G <= 32 && (G & (G - 1)) == 0;
     const dim3 grid((unsigned)((T + kTok - 1) / kTok));
     const int thr = paged_threads(H, Dh);
     cudaStream_t s = as_stream(stream);
     const uint4 *x = (const uint4 *)kv_bf16;
     uint2 *q = (uint2 *)cache;
     const size_t sm = (size_t)kTok * H * 8;   // <= 32 KiB (H <= 1024)
+#define FP8Q_PAGED_WRITE(F, GS) \
+    k_paged_write<F, GS><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache)
     if (fmt == FP8_E4M3) {
-        if (shfl) k_paged_write<FP8_E4M3, true><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
-        else k_paged_write<FP8_E4M3, false><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
+        if (G == 16) FP8Q_PAGED_WRITE(FP8_E4M3, 16);
+        else if (G == 8) FP8Q_PAGED_WRITE(FP8_E4M3, 8);
+        else if (G == 32) FP8Q_PAGED_WRITE(FP8_E4M3, 32);
+        else FP8Q_PAGED_WRITE(FP8_E4M3, 0);
     } else {
-        if (shfl) k_paged_write<FP8_E5M2, true><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
-        else k_paged_write<FP8_E5M2, false><<<grid, thr, sm, s>>>(x, slot_mapping, T, (int)H, G, num_slots, q, scale_cache);
+        if (G == 16) FP8Q_PAGED_WRITE(FP8_E5M2, 16);
+        else if (G == 8) FP8Q_PAGED_WRITE(FP8_E5M2, 8);
+        else if (G == 32) FP8Q_PAGED_WRITE(FP8_E5M2, 32);
+        else FP8Q_PAGED_WRITE(FP8_E5M2, 0);
     }
+#undef FP8Q_PAGED_WRITE
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 

@@ -71,3 +71,21 @@ def test_offsets_beyond_the_array_are_clamped(orc):
     offs = torch.tensor([0, 600, 5000, 7000], dtype=torch.int64)
     stats, counts = fp8q.scale_stats(cur.cuda(), offs.cuda(), prev.cuda(), 4.0)
     _check(orc, cur.numpy(), prev.numpy(), [0, 600, 1000, 1000], 4.0, stats, counts)
+
+
+@pytest.mark.parametrize("r", [4.0, 1.0, 3.3, 1.0000001, 16777215.0])
+def test_step_change_decisions_at_the_threshold(orc, r):
+    """Ratios placed on and next to the threshold (one fp32 step either way,
+    both directions): the kernel's division-free test must take exactly the
+    decisions of the oracle's rounded fp32 division."""
+    rng = np.random.default_rng(int(r * 1000) % 2**31)
+    p = (2.0 ** rng.uniform(-20, 20, 6000)).astype(np.float32)
+    q = (p.astype(np.float64) * np.float64(np.float32(r))).astype(np.float32)
+    v = np.concatenate([q, np.nextafter(q, np.float32(np.inf)), np.nextafter(q, np.float32(0)),
+                        (p / np.float32(r)).astype(np.float32), np.nextafter(p / np.float32(r), np.float32(0))])
+    prev = np.concatenate([p] * 5)
+    ok = np.isfinite(v) & (v > 0)
+    v, prev = v[ok], prev[ok]
+    stats, counts = fp8q.scale_stats(torch.from_numpy(v).cuda(), prev=torch.from_numpy(prev).cuda(), jump_ratio=r)
+    _check(orc, v, prev, [0, len(v)], r, stats, counts)
+    assert 0 < int(to_np(counts)[0, 0]) < len(v)
