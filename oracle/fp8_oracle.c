@@ -521,3 +521,54 @@ void orc_paged_kv_gather(const uint8_t *cache, const float *scale_cache, const i
                 }
         }
 }
+
+/* ------------------------------------- backward operands and wgrad GEMM -- */
+
+/* Rowwise quantization of the transpose ("FP8训练与QAT量化感知训练：…用Soup
+ * 把大模型微调提速2倍", section "FP8 三种缩放配方怎么选": the rowwise recipes
+ * scale every row of each GEMM operand).  The backward GEMMs contract over a
+ * dimension that is not contiguous in memory -- tokens for the weight
+ * gradient dW = dY^T X, output channels for the data gradient dX = dY W --
+ * so their K-major operands are transposes: qT[c][r] = cast(x[r][c], s_c)
+ * with s_c from the amax of COLUMN c of x (a row of x^T), scale_inv[c] = 1/s_c.
+ * x [rows, cols] with leading dimension ld; qT [cols, rows]. */
+void orc_quantize_rowwise_transpose(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
+                                    int pow2, uint8_t *qT, float *scale_inv)
+{
+    float fm = (float)orc_fmax(fmt);
+    for (int64_t c = 0; c < cols; ++c) {
+        float amax = 0.0f;
+        for (int64_t r = 0; r < rows; ++r) {
+            uint16_t h = x[r * ld + c];
+            if (!bf16_finite(h)) continue;
+            float a = fabsf(bf16_to_f32(h));
+            if (a > amax) amax = a;
+        }
+        float s = pow2 ? orc_scale_pow2_from_amax(amax, fmt) : orc_scale_from_amax(amax, fmt);
+        for (int64_t r = 0; r < rows; ++r) qT[c * rows + r] = cast_one(x[r * ld + c], s, fmt, fm, NULL);
+        scale_inv[c] = orc_inverse(s);
+    }
+}
+
+/* Weight gradient kept in high precision (the same section: the
+ * rowwise_with_gw_hp recipe keeps the weight-gradient GEMM out of FP8):
+ *   dW[m][n] = sum_t dY[t][m] * X[t][n]   over the T token rows,
+ * from the bf16 tensors as stored (token-major, dY [T, M], X [T, N]); exact
+ * products summed in fp64.  mag[m][n] = sum_t |dY[t][m] * X[t][n]| (the
+ * tolerance basis).  Sampled at (idx_m[i], idx_n[i]). */
+void orc_gemm_bf16_wgrad_sampled(const uint16_t *dY, const uint16_t *X, int64_t T, int64_t M, int64_t N,
+                                 const int64_t *idx_m, const int64_t *idx_n, int64_t count, double *val,
+                                 double *mag)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        int64_t m = idx_m[i], n = idx_n[i];
+        double acc = 0.0, mg = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            double p = (double)bf16_to_f32(dY[t * M + m]) * (double)bf16_to_f32(X[t * N + n]);
+            acc += p;
+            mg += fabs(p);
+        }
+        val[i] = acc;
+        mag[i] = mg;
+    }
+}

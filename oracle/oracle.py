@@ -85,6 +85,10 @@ def lib():
         L.orc_paged_kv_write.argtypes = [P, P, I64, I64, I64, I64, I, P, P]
         L.orc_paged_kv_gather.restype = None
         L.orc_paged_kv_gather.argtypes = [P, P, P, P, I64, I64, I64, I64, I64, I64, I64, I, P]
+        L.orc_quantize_rowwise_transpose.restype = None
+        L.orc_quantize_rowwise_transpose.argtypes = [P, I64, I64, I64, I, I, P, P]
+        L.orc_gemm_bf16_wgrad_sampled.restype = None
+        L.orc_gemm_bf16_wgrad_sampled.argtypes = [P, P, I64, I64, I64, P, P, I64, P, P]
         L.orc_scale_stats.restype = None
         L.orc_scale_stats.argtypes = [P, P, I64, F, P, P]
         _lib = L
@@ -288,6 +292,44 @@ def kv_dequant(q: np.ndarray, scale_inv: np.ndarray, fmt: int = E4M3) -> np.ndar
     out = np.empty(q.shape, np.uint16)
     lib().orc_kv_dequant(_p(q), _p(sinv), B * H, S * Dh, fmt, _p(out))
     return out
+
+
+# ------------------------------------------ backward operands, wgrad GEMM --
+
+def quantize_rowwise_transpose(x_bits: np.ndarray, fmt: int, pow2: bool = True):
+    """x [rows, cols] -> (qT [cols, rows], scale_inv [cols]): rowwise
+    quantization of x^T (one scale per column of x)."""
+    x = _u16(x_bits)
+    rows, cols = x.shape
+    qT = np.empty((cols, rows), np.uint8)
+    sinv = np.empty(cols, np.float32)
+    lib().orc_quantize_rowwise_transpose(_p(x), rows, cols, cols, fmt, int(pow2), _p(qT), _p(sinv))
+    return qT, sinv
+
+
+def gemm_bf16_wgrad_sampled(dY_bits: np.ndarray, X_bits: np.ndarray, idx_m, idx_n):
+    """dW[m, n] = sum_t dY[t, m] X[t, n] (fp64) at the sampled (m, n)."""
+    dy = _u16(dY_bits)
+    x = _u16(X_bits)
+    T, M = dy.shape
+    T2, N = x.shape
+    assert T == T2
+    im = np.ascontiguousarray(idx_m, np.int64)
+    inn = np.ascontiguousarray(idx_n, np.int64)
+    val = np.empty(im.size, np.float64)
+    mag = np.empty(im.size, np.float64)
+    lib().orc_gemm_bf16_wgrad_sampled(_p(dy), _p(x), T, M, N, _p(im), _p(inn), im.size, _p(val), _p(mag))
+    return val, mag
+
+
+def gemm_bf16_wgrad(dY_bits: np.ndarray, X_bits: np.ndarray):
+    """Full dW [M, N] and magnitude (fp64)."""
+    T, M = np.asarray(dY_bits).shape
+    N = np.asarray(X_bits).shape[1]
+    im = np.repeat(np.arange(M), N)
+    inn = np.tile(np.arange(N), M)
+    v, g = gemm_bf16_wgrad_sampled(dY_bits, X_bits, im, inn)
+    return v.reshape(M, N), g.reshape(M, N)
 
 
 # --------------------------------------------------------- paged KV cache --

@@ -547,3 +547,69 @@ def test_paged_kv_write_and_gather(orc, fmt):
                 assert np.array_equal(out[b, t], ref[i]), (b, t)
             else:
                 assert not out[b, t].any(), (b, t)
+
+
+def _bf16_f64(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("pow2", [True, False])
+def test_rowwise_transpose_per_column(orc, fmt, pow2):
+    """Rowwise quantization of x^T (the Soup page's rowwise recipes applied to
+    the backward GEMMs' transposed operands), built independently: column
+    amax by torch over the finite entries, the scale from its closed form,
+    the cast by torch's float8 conversion of the clamped product."""
+    rows, cols = 45, 70
+    x = inputs.outlier_activations_bf16((rows, cols), seed=60 + fmt, frac=0.02)
+    bits = _bits(x).copy()
+    bits[3, 5] = 0x7FC0            # NaN: skipped by the amax, cast to NaN
+    bits[:, 9] = 0                 # an all-zero column: scale 1
+    qT, sinv = orc.quantize_rowwise_transpose(bits, fmt, pow2)
+    assert qT.shape == (cols, rows) and sinv.shape == (cols,)
+    xf = _bf16_f64(bits)
+    fm = orc.fmax(fmt)
+    for c in range(cols):
+        col = xf[:, c]
+        a = np.max(np.abs(col[np.isfinite(col)]), initial=0.0)
+        if a == 0:
+            s = 1.0
+        elif pow2:
+            k = math.floor(math.log2(fm / a))
+            while a * 2.0 ** (k + 1) <= fm:   # exact fix-ups of the float log
+                k += 1
+            while a * 2.0 ** k > fm:
+                k -= 1
+            s = 2.0 ** max(-126, min(127, k))
+        else:
+            s = float(np.float32(np.float32(fm) / np.float32(a)))
+        assert sinv[c] == np.float32(1.0) / np.float32(s), c
+        y = torch.from_numpy((col.astype(np.float32) * np.float32(s)).astype(np.float32))
+        ref = y.clamp(-fm, fm).to(TORCH_FP8[fmt]).view(torch.uint8).numpy()
+        fin = np.isfinite(col)
+        assert np.array_equal(qT[c][fin], ref[fin]), c
+        assert np.all(np.isin(qT[c][~fin], [0x7F, 0xFF, 0x7D, 0x7E, 0xFD, 0xFE]))
+    # the same numbers as the rowwise quantizer applied to the transpose
+    q2, s2 = orc.quantize_rowwise(np.ascontiguousarray(bits.T), fmt, pow2)
+    assert np.array_equal(q2, qT) and np.array_equal(s2, sinv)
+
+
+def test_bf16_wgrad_against_numpy(orc):
+    """dW = dY^T X from the bf16 tensors as stored (token-major), against
+    numpy's fp64 matmul of the same values on a non-square shape (a swapped
+    operand or index fails it), and exactly on small integers."""
+    T, M, N = 37, 24, 40
+    dy = _bits(inputs.lognormal_grads_bf16((T, M), seed=70))
+    x = _bits(inputs.normal_bf16((T, N), 1.0, seed=71))
+    D, mag = orc.gemm_bf16_wgrad(dy, x)
+    ref = _bf16_f64(dy).T @ _bf16_f64(x)
+    assert D.shape == (M, N)
+    assert np.allclose(D, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    assert np.allclose(mag, np.abs(_bf16_f64(dy)).T @ np.abs(_bf16_f64(x)), rtol=1e-12)
+    rng = np.random.default_rng(72)
+    ai = rng.integers(-8, 9, (T, M)).astype(np.float32)
+    bi = rng.integers(-8, 9, (T, N)).astype(np.float32)
+    abits = _bits(torch.from_numpy(ai).to(torch.bfloat16))
+    bbits = _bits(torch.from_numpy(bi).to(torch.bfloat16))
+    Di, _ = orc.gemm_bf16_wgrad(abits, bbits)
+    assert np.array_equal(Di, (ai.astype(np.int64).T @ bi.astype(np.int64)).astype(np.float64))
