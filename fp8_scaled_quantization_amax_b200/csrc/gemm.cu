@@ -859,18 +859,22 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
     return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-// The E8M0 GEMM's translation unit keeps its own error word (gemm_mx.cu).
+// The E8M0 and the bf16 weight-gradient GEMMs keep their own error words
+// (gemm_mx.cu, gemm_bf16.cu).
 fp8_status fp8q_mx_device_error(uint32_t *out, int clear);
+fp8_status fp8q_wgrad_device_error(uint32_t *out, int clear);
 
 extern "C" fp8_status fp8_device_error(uint32_t *host_out, int clear) {
     if (!host_out) return FP8_ERR_INVALID_ARG;
     if (cudaDeviceSynchronize() != cudaSuccess) return FP8_ERR_CUDA;
     unsigned int v = 0;
     if (cudaMemcpyFromSymbol(&v, g_gemm_error, sizeof(v)) != cudaSuccess) return FP8_ERR_CUDA;
-    uint32_t w = 0;
-    const fp8_status st = fp8q_mx_device_error(&w, clear);
+    uint32_t w = 0, g = 0;
+    fp8_status st = fp8q_mx_device_error(&w, clear);
     if (st != FP8_OK) return st;
-    *host_out = v | w;
+    st = fp8q_wgrad_device_error(&g, clear);
+    if (st != FP8_OK) return st;
+    *host_out = v | w | g;
     if (clear) {
         const unsigned int z = 0;
         if (cudaMemcpyToSymbol(g_gemm_error, &z, sizeof(z)) != cudaSuccess) return FP8_ERR_CUDA;

@@ -62,7 +62,7 @@ k_paged_write(const uint4 *__restrict__ x, const int64_t *__restrict__ slot_mapp
 #pragma unroll
     for (int k = 0; k < kTok; ++k)
         if (slot[k] >= num_slots) slot[k] = -1;          // outside the cache: padding
-    if (!SHFL) {
+    if constexpr (!SHFL) {
         for (int i = threadIdx.x; i < kTok * H; i += blockDim.x) head_amax[i] = 0u;
         __syncthreads();
     }
@@ -73,7 +73,7 @@ k_paged_write(const uint4 *__restrict__ x, const int64_t *__restrict__ slot_mapp
             uint32_t bad = 0;
             m = amax_exact8(0u, v[k], bad);
         }
-        if (SHFL) {
+        if constexpr (SHFL) {
 #pragma unroll
             for (int o = GS >> 1; o > 0; o >>= 1) {
                 const uint32_t w = __shfl_xor_sync(0xFFFFFFFFu, m, o);

@@ -182,6 +182,114 @@ k_cast_transpose(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64
     }
 }
 
+// ------------------------------------------- rowwise of the transpose ----
+// The backward GEMMs contract over a dimension that is not contiguous in
+// memory, so their K-major FP8 operands are transposes, quantized rowwise
+// (one scale per row of x^T = per column of x).  Two passes: k_colamax
+// reduces every column's amax over all rows into fp32 bits (atomicMax on
+// non-negative floats as integers: order-independent, so deterministic);
+// k_cast_transpose_col casts 64x64 tiles with per-column scales and writes
+// them transposed.  The second pass re-reads x, from L2 when x fits.
+constexpr int kColRows = 256;   // rows per k_colamax CTA
+
+// |x| of two bf16, non-finite halves replaced by 0 (so they never win a max)
+__device__ __forceinline__ uint32_t abs_finite2(uint32_t w) {
+    const uint32_t a = w & 0x7FFF7FFFu;
+    return a & __vcmpltu2(a, 0x7F807F80u);
+}
+
+__global__ void __launch_bounds__(256)
+k_colamax(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint32_t *__restrict__ amax_bits) {
+    __shared__ uint4 red[8][32];
+    const int cg = threadIdx.x & 31, sub = threadIdx.x >> 5;
+    const int64_t c = (int64_t)blockIdx.x * 256 + cg * 8;
+    const int64_t r0 = (int64_t)blockIdx.y * kColRows;
+    const int64_t r1 = min(r0 + kColRows, rows);
+    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;   // packed per-column maxima (bf16 magnitude bits)
+    if (c < cols) {
+        int64_t r = r0 + sub;
+        for (; r + 24 < r1; r += 32) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = ld_stream(reinterpret_cast<const uint4 *>(x + (r + 8 * u) * ld + c));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                m0 = __vmaxu2(m0, abs_finite2(v[u].x));
+                m1 = __vmaxu2(m1, abs_finite2(v[u].y));
+                m2 = __vmaxu2(m2, abs_finite2(v[u].z));
+                m3 = __vmaxu2(m3, abs_finite2(v[u].w));
+            }
+        }
+        for (; r < r1; r += 8) {
+            const uint4 v = ld_stream(reinterpret_cast<const uint4 *>(x + r * ld + c));
+            m0 = __vmaxu2(m0, abs_finite2(v.x));
+            m1 = __vmaxu2(m1, abs_finite2(v.y));
+            m2 = __vmaxu2(m2, abs_finite2(v.z));
+            m3 = __vmaxu2(m3, abs_finite2(v.w));
+        }
+    }
+    red[sub][cg] = make_uint4(m0, m1, m2, m3);
+    __syncthreads();
+    if (sub == 0 && c < cols) {
+#pragma unroll
+        for (int k = 1; k < 8; ++k) {
+            const uint4 o = red[k][cg];
+            m0 = __vmaxu2(m0, o.x);
+            m1 = __vmaxu2(m1, o.y);
+            m2 = __vmaxu2(m2, o.z);
+            m3 = __vmaxu2(m3, o.w);
+        }
+        const uint32_t w[4] = {m0, m1, m2, m3};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {   // bf16 magnitude bits << 16 = the fp32 bits of the same value
+            if ((w[j] & 0xFFFFu) != 0u) atomicMax(&amax_bits[c + 2 * j], (w[j] & 0xFFFFu) << 16);
+            if ((w[j] >> 16) != 0u) atomicMax(&amax_bits[c + 2 * j + 1], w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+// 64x64 tiles: the 64 column scales computed once per CTA into shared memory,
+// 16-byte loads of 8 bf16, the codes transposed through shared memory, 16-byte
+// stores of 16 codes along the output row.  Row tile 0 also writes 1/s.
+template <int FMT, bool POW2>
+__global__ void __launch_bounds__(256)
+k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t rows, int64_t cols,
+                     int64_t ld, const uint32_t *__restrict__ amax_bits, float *__restrict__ scale_inv) {
+    __shared__ __align__(16) uint8_t tile[64][64 + 16];
+    __shared__ float sc[64];
+    constexpr float fm = fmax_of<FMT>();
+    const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+    if (threadIdx.x < 64) {
+        const int64_t gc = c0 + threadIdx.x;
+        const float a = gc < cols ? __uint_as_float(amax_bits[gc]) : 0.0f;
+        const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
+        sc[threadIdx.x] = s;
+        if (blockIdx.y == 0 && gc < cols) scale_inv[gc] = __fdiv_rn(1.0f, s);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int u = threadIdx.x + h * 256;
+        const int row = u >> 3, cv = u & 7;
+        const int64_t gr = r0 + row, gc = c0 + cv * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (gr < rows && gc < cols) v = ld_stream(reinterpret_cast<const uint4 *>(x + gr * ld + gc));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t c2 = cvt2<FMT>(__fmul_rn(bf_lo(w[j]), sc[cv * 8 + 2 * j]),
+                                          __fmul_rn(bf_hi(w[j]), sc[cv * 8 + 2 * j + 1]));
+            tile[cv * 8 + 2 * j][row] = (uint8_t)(c2 & 0xFFu);
+            tile[cv * 8 + 2 * j + 1][row] = (uint8_t)(c2 >> 8);
+        }
+    }
+    __syncthreads();
+    const int oc = threadIdx.x >> 2, part = threadIdx.x & 3;
+    const int64_t go = c0 + oc, gi = r0 + part * 16;
+    if (go < cols && gi < rows)
+        *reinterpret_cast<uint4 *>(qt + go * rows + gi) = *reinterpret_cast<const uint4 *>(&tile[oc][part * 16]);
+}
+
 // --------------------------------------------------------------- rowwise --
 // A CTA (128 threads) quantizes R rows at a time, every row held in registers
 // (V vectors of 8 per thread) between its amax and its cast: one HBM read per
@@ -561,6 +669,36 @@ extern "C" fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, i
     cudaStream_t s = as_stream(stream);
     if (fmt == FP8_E4M3) launch_block<FP8_E4M3, false>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv, nullptr);
     else launch_block<FP8_E5M2, false>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv, nullptr);
+    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+extern "C" fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                                     fp8_format fmt, int pow2, uint8_t *qT, float *scale_inv,
+                                                     float *amax_out, void *stream) {
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols || (cols % 16) || (rows % 16)) return FP8_ERR_SHAPE;
+    if ((rows + 63) / 64 > 65535 || (rows + kColRows - 1) / kColRows > 65535) return FP8_ERR_SHAPE;
+    if (rows > 0 && cols > 0 && (!x_bf16 || !qT || !scale_inv || !amax_out)) return FP8_ERR_INVALID_ARG;
+    if (ld % 8) return FP8_ERR_ALIGNMENT;
+    if ((x_bf16 && !aligned16(x_bf16)) || (qT && !aligned16(qT))) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (rows == 0 || cols == 0) return FP8_OK;
+    cudaStream_t s = as_stream(stream);
+    uint32_t *amax_bits = reinterpret_cast<uint32_t *>(amax_out);
+    if (cudaMemsetAsync(amax_bits, 0, (size_t)cols * sizeof(uint32_t), s) != cudaSuccess) return FP8_ERR_CUDA;
+    const uint16_t *xs = static_cast<const uint16_t *>(x_bf16);
+    k_colamax<<<dim3((unsigned)((cols + 255) / 256), (unsigned)((rows + kColRows - 1) / kColRows)), 256, 0, s>>>(
+        xs, rows, cols, ld, amax_bits);
+    const dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+    if (fmt == FP8_E4M3) {
+        if (pow2) k_cast_transpose_col<FP8_E4M3, true><<<grid, 256, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+        else k_cast_transpose_col<FP8_E4M3, false><<<grid, 256, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+    } else {
+        if (pow2) k_cast_transpose_col<FP8_E5M2, true><<<grid, 256, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+        else k_cast_transpose_col<FP8_E5M2, false><<<grid, 256, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+    }
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 

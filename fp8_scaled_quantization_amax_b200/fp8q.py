@@ -44,6 +44,8 @@ SIGNATURES = {
     "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
     "fp8_quantize_blockwise_e8m0": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
+    "fp8_quantize_rowwise_transpose": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
+    "fp8_gemm_bf16_wgrad": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _I, _P]),
     "fp8_gemm_block_e8m0": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _P, _P, _P, _I64, _P]),
     "fp8_paged_kv_write": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_paged_kv_gather": (_S, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P]),
@@ -211,6 +213,38 @@ def fp8_gemm_block_e8m0(A, fa, B, fb, M, N, K, a_sf, b_sf, D, ldd, stream=None):
     _dev(a_sf, torch.uint8, "a_sf"); _dev(b_sf, torch.uint8, "b_sf")
     _check("fp8_gemm_block_e8m0", lib().fp8_gemm_block_e8m0(
         _ptr(A), fa, _ptr(B), fb, M, N, K, _ptr(a_sf), _ptr(b_sf), _ptr(D), ldd, _stream(stream)))
+
+
+def fp8_quantize_rowwise_transpose(x, rows, cols, ld, fmt, pow2, qT, scale_inv, amax_out, stream=None):
+    _dev(x, torch.bfloat16, "x"); _dev(qT, torch.uint8, "qT")
+    _dev(scale_inv, torch.float32, "scale_inv"); _dev(amax_out, torch.float32, "amax_out")
+    _check("fp8_quantize_rowwise_transpose", lib().fp8_quantize_rowwise_transpose(
+        _ptr(x), rows, cols, ld, fmt, int(pow2), _ptr(qT), _ptr(scale_inv), _ptr(amax_out), _stream(stream)))
+
+
+def quantize_rowwise_transpose(x, fmt, pow2=True):
+    """(qT [cols, rows], scale_inv [cols], amax [cols]) of x [rows, cols]."""
+    rows, cols = x.shape
+    qT = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+    sinv = torch.empty(cols, dtype=torch.float32, device=x.device)
+    am = torch.empty(cols, dtype=torch.float32, device=x.device)
+    fp8_quantize_rowwise_transpose(x, rows, cols, x.stride(0), fmt, pow2, qT, sinv, am)
+    return qT, sinv, am
+
+
+def fp8_gemm_bf16_wgrad(dY, X, T, M, N, ld_dy, ld_x, dW, ldd, accumulate=False, stream=None):
+    _dev(dY, torch.bfloat16, "dY"); _dev(X, torch.bfloat16, "X"); _dev(dW, torch.float32, "dW")
+    _check("fp8_gemm_bf16_wgrad", lib().fp8_gemm_bf16_wgrad(
+        _ptr(dY), _ptr(X), T, M, N, ld_dy, ld_x, _ptr(dW), ldd, int(accumulate), _stream(stream)))
+
+
+def gemm_bf16_wgrad(dY, X, out=None, accumulate=False):
+    """dW [M, N] fp32 = (dW if accumulate) + dY^T X for token-major dY [T, M], X [T, N]."""
+    T, M = dY.shape
+    N = X.shape[1]
+    dW = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=dY.device)
+    fp8_gemm_bf16_wgrad(dY, X, T, M, N, dY.stride(0), X.stride(0), dW, dW.stride(0), accumulate)
+    return dW
 
 
 def e8m0_image_bytes(rows: int, cols: int) -> int:

@@ -130,6 +130,27 @@ FP8Q_API fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int
                                   void *stream);
 
 /*
+ * Rowwise quantization of the transpose, for the backward GEMMs ([Soup]
+ * section "FP8 三种缩放配方怎么选": the rowwise recipes scale each row of
+ * every GEMM operand; the weight gradient dW = dY^T X contracts over tokens
+ * and the data gradient dX = dY W over output channels, so their K-major
+ * operands are dY^T, X^T and W^T).  x [rows, cols] bf16 (leading dimension
+ * ld); one scale per column c of x: pow2 != 0 gives the largest power of two
+ * with amax_c * s_c <= fmax, pow2 == 0 gives s_c = fmax / amax_c (amax over
+ * the finite entries of the column; 0 gives 1).
+ *   qT         [cols, rows] FP8, dense: qT[c][r] = sat_RNE(fp32(x[r][c]) * s_c).
+ *   scale_inv  [cols] fp32, 1 / s_c.
+ *   amax_out   [cols] fp32, the column amax (also used as the kernels'
+ *              reduction buffer; overwritten).
+ *   Shapes: rows % 16 == 0, cols % 16 == 0, ld % 8 == 0, ld >= cols,
+ *   ceil(rows / 64) <= 65535.  Three launches: a memset of amax_out, the
+ *   column reduction, the transposing cast.
+ */
+FP8Q_API fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                          fp8_format fmt, int pow2, uint8_t *qT, float *scale_inv,
+                                          float *amax_out, void *stream);
+
+/*
  * Per-block quantization with power-of-two scales written as an E8M0 scale
  * image, the operand format of the hardware block-scaled MMA
  * (fp8_gemm_block_e8m0).  Blocks as in fp8_quantize_blockwise ([DeepL] §2.3
@@ -187,6 +208,24 @@ FP8Q_API fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8
                            int64_t M, int64_t N, int64_t K, fp8_scale_mode mode,
                            const float *a_scale_inv, const float *b_scale_inv, void *D_bf16,
                            int64_t ldd, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Weight-gradient GEMM kept in high precision ([Soup] section "FP8 三种缩放
+ * 配方怎么选": the rowwise_with_gw_hp recipe keeps the weight gradient out of
+ * FP8):
+ *   dW[m, n] = (accumulate ? dW[m, n] : 0) + sum_t dY[t, m] * X[t, n],
+ *   bf16 products accumulated in fp32 on the tensor cores, fp32 output.
+ *   dY [T, M] bf16 (leading dimension ld_dy), X [T, N] bf16 (ld_x): the
+ *   token-major tensors of the layer's backward pass, read as stored (no
+ *   transpose pass).  dW [M, N] fp32, leading dimension ldd.
+ *   Deterministic (one fixed token order per output).
+ *   Shapes: M % 8 == 0, N % 8 == 0, ld_dy % 8 == 0, ld_x % 8 == 0,
+ *   ldd % 4 == 0; T == 0 writes zeros (or leaves dW when accumulating).
+ *   Pointers 16-byte aligned.
+ */
+FP8Q_API fp8_status fp8_gemm_bf16_wgrad(const void *dY_bf16, const void *X_bf16, int64_t T, int64_t M,
+                               int64_t N, int64_t ld_dy, int64_t ld_x, float *dW, int64_t ldd,
+                               int accumulate, void *stream);
 
 /*
  * FP8 GEMM with power-of-two block scales applied by the tensor core

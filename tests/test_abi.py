@@ -86,6 +86,12 @@ def test_validation_before_device_access():
     assert L.fp8_gemm_block_e8m0(FAKE, 2, FAKE, 0, 64, 64, 64, FAKE, FAKE, FAKE, 64, n) == INVALID
     assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 64, None, FAKE, FAKE, 64, n) == INVALID
     assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 64, FAKE_ODD, FAKE, FAKE, 64, n) == ALIGN
+    # backward operands and the bf16 weight gradient
+    assert L.fp8_quantize_rowwise_transpose(FAKE, 24, 32, 32, 0, 1, FAKE, FAKE, FAKE, n) == SHAPE   # rows % 16
+    assert L.fp8_quantize_rowwise_transpose(FAKE, 32, 32, 32, 0, 1, FAKE, FAKE, None, n) == INVALID
+    assert L.fp8_gemm_bf16_wgrad(FAKE, FAKE, 64, 12, 64, 12, 64, FAKE, 64, 0, n) == ALIGN    # M % 8
+    assert L.fp8_gemm_bf16_wgrad(FAKE, FAKE, 64, 64, 64, 64, 64, None, 64, 0, n) == INVALID
+    assert L.fp8_gemm_bf16_wgrad(FAKE, FAKE, 64, 64, 64, 32, 64, FAKE, 64, 0, n) == SHAPE    # ld_dy < M
     # paged KV cache
     assert L.fp8_paged_kv_write(FAKE, FAKE, 4, 2, 12, 64, 0, FAKE, FAKE, n) == SHAPE        # Dh % 8
     assert L.fp8_paged_kv_write(FAKE, FAKE, 4, 128, 128, 64, 0, FAKE, FAKE, n) == SHAPE     # H*Dh > 8192
