@@ -42,7 +42,7 @@ METRIC = "FP8 scaled GEMM TFLOP/s (% dense FP8 peak); quantize/KV GB/s (% HBM)"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_OVER_BF16 = 2.0     # nominal dense ratio: 4.5 PFLOP/s fp8 / 2.25 PFLOP/s bf16
-DEFAULT_STEPS = {"rowwise": 6000, "tensor": 6000, "blockmlp": 1500, "blockmlp_e8m0": 1500, "dgrad": 6000, "kv": 600, "paged": 600, "health": 6000}
+DEFAULT_STEPS = {"rowwise": 6000, "tensor": 6000, "blockmlp": 1500, "blockmlp_e8m0": 1500, "dgrad": 6000, "bwd_gw_hp": 2000, "kv": 600, "paged": 600, "health": 6000}
 
 
 def peaks():
@@ -328,6 +328,46 @@ class Workload:
             ev[1].record()
         self.hist.update(self.am)
 
+    # a linear layer's backward under the rowwise_with_gw_hp recipe
+    def _setup_bwd_gw_hp(self):
+        f, inp, d, s = self.f, self.inp, self.dev, self.seed
+        T, N_out, K_in = (2048 if self.profile else 8192), 4096, 4096
+        self.dY = inp.lognormal_grads_bf16((T, N_out), seed=s + 100, device=d)
+        self.X = inp.normal_bf16((T, K_in), 1.0, seed=s + 101, device=d)
+        self.W = inp.normal_bf16((N_out, K_in), 0.02, seed=s + 1, device=d)
+        self.qdy = torch.empty((T, N_out), dtype=torch.uint8, device=d)
+        self.sdy = torch.empty(T, dtype=torch.float32, device=d)
+        self.qwT = torch.empty((K_in, N_out), dtype=torch.uint8, device=d)
+        self.swT = torch.empty(K_in, dtype=torch.float32, device=d)
+        self.awT = torch.empty(K_in, dtype=torch.float32, device=d)
+        self.DX = torch.empty((T, K_in), dtype=torch.bfloat16, device=d)
+        self.DW = torch.empty((N_out, K_in), dtype=torch.float32, device=d)
+        self.dims = (T, N_out, K_in)
+        self.flops = 2 * 2.0 * T * N_out * K_in
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.peak_dtype = "bf16"   # the dominant kernel is the bf16 weight-gradient GEMM
+        self.launches = 5          # + one memset (the column-amax buffer), not a kernel
+        self.config = {"workload": "linear backward, rowwise_with_gw_hp (FP8 rowwise dgrad, bf16 wgrad)",
+                       "T": T, "N_out": N_out, "K_in": K_in,
+                       "dY": "|g| = 10^u, u ~ N(-2, (4/3)^2) clipped to [-6, 2], random sign; E5M2 per token",
+                       "W": "N(0,0.02) bf16; W^T E4M3 per input channel, requantized every step",
+                       "X": "N(0,1) bf16", "dW": "fp32, dY^T X from the bf16 tensors"}
+        self.host_inputs = [("dY", self.dY), ("X", self.X)]
+        self.host_output = self.DX
+
+    def _step_bwd_gw_hp(self, ev=None):
+        f = self.f
+        T, N_out, K_in = self.dims
+        f.fp8_quantize_rowwise(self.dY, T, N_out, N_out, f.E5M2, 1, self.qdy, self.sdy)
+        f.fp8_quantize_rowwise_transpose(self.W, N_out, K_in, K_in, f.E4M3, 1, self.qwT, self.swT, self.awT)
+        f.fp8_gemm_scaled(self.qdy, f.E5M2, self.qwT, f.E4M3, T, K_in, N_out, f.SCALE_ROW, self.sdy, self.swT,
+                          self.DX, K_in)
+        if ev:
+            ev[0].record()
+        f.fp8_gemm_bf16_wgrad(self.dY, self.X, T, N_out, K_in, N_out, K_in, self.DW, K_in)
+        if ev:
+            ev[1].record()
+
     # FP8 KV cache round trip
     def _setup_kv(self):
         f, inp, d, s = self.f, self.inp, self.dev, self.seed
@@ -452,6 +492,9 @@ class Workload:
             if self.name in ("blockmlp", "blockmlp_e8m0"):
                 M, Dm, F = self.dims
                 return 2.0 * M * Dm * F / 1e12
+            if self.name == "bwd_gw_hp":
+                T, N_out, K_in = self.dims
+                return 2.0 * T * N_out * K_in / 1e12
             return self.flops / 1e12
         return self.kernel_bytes / 1e9
 
@@ -465,6 +508,27 @@ def cpu_sample(name: str, seed: int = 0):
     from fp8_scaled_quantization_amax_b200 import inputs
     from oracle import oracle as orc
     orc.lib()
+    if name == "bwd_gw_hp":
+        T, N_out, K_in = 8192, 4096, 4096
+        r = 8
+        g = inputs.bf16_bits(inputs.lognormal_grads_bf16((T, N_out), seed=seed))
+        x = inputs.bf16_bits(inputs.normal_bf16((T, K_in), 1.0, seed=seed + 1))
+        w = inputs.bf16_bits(inputs.normal_bf16((N_out, K_in), 0.02, seed=seed + 2))
+        t0 = time.perf_counter()
+        qwT, swT = orc.quantize_rowwise_transpose(w, 0, True)
+        tw = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        qg, sg = orc.quantize_rowwise(g[:r], 1, True)
+        im = np.repeat(np.arange(r), 256)
+        inn = np.tile(np.arange(256), r)
+        orc.gemm_scaled_sampled(qg, 1, qwT, 0, 1, sg, swT, im, inn)
+        td = (time.perf_counter() - t0) * (T / r) * (K_in / 256)
+        t0 = time.perf_counter()
+        orc.gemm_bf16_wgrad_sampled(g, x, np.repeat(np.arange(2), 64), np.tile(np.arange(64), 2))
+        tg = (time.perf_counter() - t0) * (N_out * K_in / 128)
+        return 4.0 * T * N_out * K_in / (tw + td + tg) / 1e12, (
+            f"all of W^T quantized, {r} dY rows quantized and {r}x256 dX outputs (K=4096), 128 dW outputs "
+            "over all 8192 tokens; the dX and dW parts scaled to the full layer")
     if name == "blockmlp_e8m0":
         name = "blockmlp"   # the same per-block GEMM in the oracle (its cost does not depend on the scale rule)
     if name in ("rowwise", "tensor", "blockmlp", "dgrad"):
@@ -704,10 +768,16 @@ def main():
         # the power cap, the burst figure otherwise
         capped = "sw_power_cap" in clocks.get("reasons", []) and bf16_sus is not None
         base = bf16_sus if capped else bf16
-        peak = base * FP8_OVER_BF16
-        peak_src = (f"FP8 dense peak = {src} bf16 {'sustained' if capped else 'burst'} {base} TFLOP/s x nominal "
-                    f"fp8/bf16 ratio 2 (MEASURED_PEAKS.json){'; sw_power_cap was active in the timed region' if capped else ''}"
-                    if src == "measured" else f"fallback bf16 {bf16} x 2")
+        kind = 'sustained' if capped else 'burst'
+        note = '; sw_power_cap was active in the timed region' if capped else ''
+        if getattr(wl, "peak_dtype", "fp8") == "bf16":
+            peak = base
+            peak_src = (f"bf16 dense peak = {src} cuBLAS bf16 {kind} {base} TFLOP/s (MEASURED_PEAKS.json){note}"
+                        if src == "measured" else f"fallback bf16 {bf16}")
+        else:
+            peak = base * FP8_OVER_BF16
+            peak_src = (f"FP8 dense peak = {src} bf16 {kind} {base} TFLOP/s x nominal fp8/bf16 ratio 2 "
+                        f"(MEASURED_PEAKS.json){note}" if src == "measured" else f"fallback bf16 {bf16} x 2")
     else:
         peak = hbm
         peak_src = f"{src} HBM copy bandwidth {hbm} GB/s"
@@ -724,6 +794,7 @@ def main():
              "blockmlp": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate (per-128-K promotion) -> bf16",
              "blockmlp_e8m0": "fp8_e4m3 x fp8_e4m3, e8m0 block scales in the MMA -> f32 accumulate -> bf16",
              "dgrad": "fp8_e5m2 x fp8_e4m3 -> f32 accumulate -> bf16",
+             "bwd_gw_hp": "dgrad fp8_e5m2 x fp8_e4m3 -> bf16; wgrad bf16 x bf16 -> f32",
              "kv": "bf16 <-> fp8_e4m3 (f32 scale)",
              "paged": "bf16 <-> fp8_e4m3 (f32 scale per token and head)",
              "health": "f32 scales, f64 sums"}[args.workload]
@@ -737,7 +808,7 @@ def main():
                      "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "kernel": {"kv": "fp8_kv_quant", "paged": "fp8_paged_kv_write",
-                                "health": "fp8_scale_stats",
+                                "health": "fp8_scale_stats", "bwd_gw_hp": "fp8_gemm_bf16_wgrad",
                                 "blockmlp_e8m0": "fp8_gemm_block_e8m0"}.get(args.workload, "fp8_gemm_scaled"),
                      "kernel_ms": kern_avg_ms, "peak_source": peak_src},
         "cpu_baseline": cpu,

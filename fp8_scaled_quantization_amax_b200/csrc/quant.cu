@@ -206,12 +206,13 @@ k_colamax(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
     const int64_t r0 = (int64_t)blockIdx.y * kColRows;
     const int64_t r1 = min(r0 + kColRows, rows);
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;   // packed per-column maxima (bf16 magnitude bits)
+    const uint64_t keep = policy_evict_last();  // the cast pass reads x again, from L2 when it fits
     if (c < cols) {
         int64_t r = r0 + sub;
         for (; r + 24 < r1; r += 32) {
             uint4 v[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = ld_stream(reinterpret_cast<const uint4 *>(x + (r + 8 * u) * ld + c));
+            for (int u = 0; u < 4; ++u) v[u] = ld_hint(reinterpret_cast<const uint4 *>(x + (r + 8 * u) * ld + c), keep);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 m0 = __vmaxu2(m0, abs_finite2(v[u].x));
@@ -221,7 +222,7 @@ k_colamax(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
             }
         }
         for (; r < r1; r += 8) {
-            const uint4 v = ld_stream(reinterpret_cast<const uint4 *>(x + r * ld + c));
+            const uint4 v = ld_hint(reinterpret_cast<const uint4 *>(x + r * ld + c), keep);
             m0 = __vmaxu2(m0, abs_finite2(v.x));
             m1 = __vmaxu2(m1, abs_finite2(v.y));
             m2 = __vmaxu2(m2, abs_finite2(v.z));
@@ -248,14 +249,19 @@ k_colamax(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
     }
 }
 
-// 64x64 tiles: the 64 column scales computed once per CTA into shared memory,
-// 16-byte loads of 8 bf16, the codes transposed through shared memory, 16-byte
-// stores of 16 codes along the output row.  Row tile 0 also writes 1/s.
+// 64x64 tiles, 128 threads.  The 64 column scales are computed once per CTA
+// into shared memory.  Thread t loads rows 4(t/8) .. +3 of the 8 columns
+// 8(t%8) .. +7 (four 16-byte loads), casts them, and transposes the 4 x 8
+// bytes in registers (byte permutes) into eight 4-byte column words, stored
+// to shared memory as the tile's transposed lines (64 bytes per column; the
+// 16-byte chunk index XOR-swizzled by bits 3-4 of the column, so the eight
+// column groups of a warp spread over the banks).  Each thread then stores
+// two 16-byte chunks of output rows.  Row tile 0 also writes 1/s.
 template <int FMT, bool POW2>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t rows, int64_t cols,
                      int64_t ld, const uint32_t *__restrict__ amax_bits, float *__restrict__ scale_inv) {
-    __shared__ __align__(16) uint8_t tile[64][64 + 16];
+    __shared__ __align__(16) uint32_t tile[64 * 16];   // [column][16 words of 4 rows]
     __shared__ float sc[64];
     constexpr float fm = fmax_of<FMT>();
     const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
@@ -266,28 +272,58 @@ k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, i
         sc[threadIdx.x] = s;
         if (blockIdx.y == 0 && gc < cols) scale_inv[gc] = __fdiv_rn(1.0f, s);
     }
-    __syncthreads();
+    const int cv = threadIdx.x & 7, rg = threadIdx.x >> 3;
+    const int64_t gc = c0 + cv * 8;
+    const uint64_t drop = policy_evict_first();
+    uint4 v[4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int u = threadIdx.x + h * 256;
-        const int row = u >> 3, cv = u & 7;
-        const int64_t gr = r0 + row, gc = c0 + cv * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (gr < rows && gc < cols) v = ld_stream(reinterpret_cast<const uint4 *>(x + gr * ld + gc));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int k = 0; k < 4; ++k) {
+        const int64_t gr = r0 + rg * 4 + k;
+        v[k] = (gr < rows && gc < cols) ? ld_hint(reinterpret_cast<const uint4 *>(x + gr * ld + gc), drop)
+                                        : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();   // the scales
+    float s8[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t c2 = cvt2<FMT>(__fmul_rn(bf_lo(w[j]), sc[cv * 8 + 2 * j]),
-                                          __fmul_rn(bf_hi(w[j]), sc[cv * 8 + 2 * j + 1]));
-            tile[cv * 8 + 2 * j][row] = (uint8_t)(c2 & 0xFFu);
-            tile[cv * 8 + 2 * j + 1][row] = (uint8_t)(c2 >> 8);
-        }
+    for (int j = 0; j < 8; ++j) s8[j] = sc[cv * 8 + j];
+    uint32_t lo[4], hi[4];   // row k's codes of columns 0-3 and 4-7
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+        uint32_t c2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            c2[j] = cvt2<FMT>(__fmul_rn(bf_lo(w[j]), s8[2 * j]), __fmul_rn(bf_hi(w[j]), s8[2 * j + 1]));
+        lo[k] = c2[0] | (c2[1] << 16);
+        hi[k] = c2[2] | (c2[3] << 16);
+    }
+    // 4 rows x 4 bytes -> 4 columns x 4 rows, for the low and the high half
+    uint32_t colw[8];
+#pragma unroll
+    for (int hlf = 0; hlf < 2; ++hlf) {
+        const uint32_t *R = hlf ? hi : lo;
+        const uint32_t t01 = __byte_perm(R[0], R[1], 0x5140), t23 = __byte_perm(R[2], R[3], 0x5140);
+        const uint32_t u01 = __byte_perm(R[0], R[1], 0x7362), u23 = __byte_perm(R[2], R[3], 0x7362);
+        colw[4 * hlf + 0] = __byte_perm(t01, t23, 0x5410);
+        colw[4 * hlf + 1] = __byte_perm(t01, t23, 0x7632);
+        colw[4 * hlf + 2] = __byte_perm(u01, u23, 0x5410);
+        colw[4 * hlf + 3] = __byte_perm(u01, u23, 0x7632);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int col = cv * 8 + j;
+        const int chunk = (rg >> 2) ^ ((col >> 3) & 3);
+        tile[col * 16 + chunk * 4 + (rg & 3)] = colw[j];
     }
     __syncthreads();
-    const int oc = threadIdx.x >> 2, part = threadIdx.x & 3;
-    const int64_t go = c0 + oc, gi = r0 + part * 16;
-    if (go < cols && gi < rows)
-        *reinterpret_cast<uint4 *>(qt + go * rows + gi) = *reinterpret_cast<const uint4 *>(&tile[oc][part * 16]);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int q = threadIdx.x + 128 * i;
+        const int col = q >> 2, part = q & 3;
+        const int64_t go = c0 + col, gi = r0 + part * 16;
+        const uint4 o = *reinterpret_cast<const uint4 *>(&tile[col * 16 + ((part ^ ((col >> 3) & 3)) * 4)]);
+        if (go < cols && gi < rows) *reinterpret_cast<uint4 *>(qt + go * rows + gi) = o;
+    }
 }
 
 // --------------------------------------------------------------- rowwise --
@@ -693,11 +729,11 @@ extern "C" fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t
         xs, rows, cols, ld, amax_bits);
     const dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
     if (fmt == FP8_E4M3) {
-        if (pow2) k_cast_transpose_col<FP8_E4M3, true><<<grid, 256, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
-        else k_cast_transpose_col<FP8_E4M3, false><<<grid, 256, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+        if (pow2) k_cast_transpose_col<FP8_E4M3, true><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+        else k_cast_transpose_col<FP8_E4M3, false><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
     } else {
-        if (pow2) k_cast_transpose_col<FP8_E5M2, true><<<grid, 256, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
-        else k_cast_transpose_col<FP8_E5M2, false><<<grid, 256, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+        if (pow2) k_cast_transpose_col<FP8_E5M2, true><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+        else k_cast_transpose_col<FP8_E5M2, false><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
     }
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
