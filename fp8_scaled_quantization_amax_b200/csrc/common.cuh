@@ -159,6 +159,16 @@ __device__ __forceinline__ uint2 ld_stream_u2(const uint2 *p) {
     return r;
 }
 
+// Programmatic dependent launch.  A kernel launched with pdl_launch() may
+// start while the previous kernel in the stream is still running; it calls
+// pdl_wait() before its first global-memory access, which returns once that
+// kernel has completed and its writes are visible, so stream order is kept.
+// pdl_trigger() lets the next kernel be scheduled (it will wait in turn):
+// called once every CTA of this grid is resident, so a dependent grid never
+// takes an SM one of our CTAs still needs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t policy_evict_last() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -210,6 +220,23 @@ __device__ __forceinline__ uint32_t block_sum_u32(uint32_t v, uint32_t *smem) {
 
 // ------------------------------------------------------------- host side --
 namespace fp8q_host {
+// Launch with programmatic stream serialization allowed (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 
 // Current device must be compute capability 10.0 (B200, sm_100a); cached
 // per device ordinal.  Also returns the SM count.

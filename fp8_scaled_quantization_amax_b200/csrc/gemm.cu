@@ -43,6 +43,7 @@
 #include "tc.cuh"
 
 using namespace fp8q;
+using fp8q_host::pdl_launch;
 
 namespace {
 
@@ -105,6 +106,8 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();      // inputs of the previous kernel in the stream are visible from here on
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -340,6 +343,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int num_n = (N + BN - 1) / BN;
     int total_tiles = full_tiles;
     if constexpr (GROUPED) {
+        pdl_wait();   // the group offsets may come from the previous kernel
         total_tiles = 0;
         for (int e = 0; e < G; ++e) total_tiles += (int)((goff[e + 1] - goff[e] + 255) / 256) * num_n;
     }
@@ -406,6 +410,8 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     cluster_sync_all();   // both CTAs' barriers are initialised before any remote signal
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();      // inputs of the previous kernel in the stream are visible from here on
+    pdl_trigger();
     // BLOCK mode: each role branch resizes its own warpgroup's registers, so
     // the epilogue code is only reachable after the increase.
     if (warp == 0) {
@@ -671,9 +677,8 @@ cudaError_t launch_gemm(cudaStream_t st, int sms, const CUtensorMap &ta, const C
     if (attr_err != cudaSuccess) return attr_err;
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = std::max(1, std::min(tiles, sms));
-    k_gemm_fp8<MODE><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, M, N, K, idesc, sa, sb,
-                                                        static_cast<__nv_bfloat16 *>(D), ldd);
-    return cudaPeekAtLastError();
+    return pdl_launch(k_gemm_fp8<MODE>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, ta, tb, M, N, K, idesc, sa, sb,
+                      static_cast<__nv_bfloat16 *>(D), ldd);
 }
 
 // Pairs of the 2-SM kernel that fit on the device at once (cached per device).
@@ -739,10 +744,10 @@ cudaError_t launch_gemm_2sm(cudaStream_t st, const CUtensorMap &ta, const CUtens
     uint32_t *flags = plan.units ? reinterpret_cast<uint32_t *>(static_cast<char *>(ws) +
                                                                 (size_t)(plan.units / 2) * 2 * sm2::kSplitPartialFloats * sizeof(float))
                                  : nullptr;
-    k_gemm_fp8_2sm<MODE, BN, false><<<2 * pairs, sm2::THREADS, sm2::Cfg<BN>::SMEM, st>>>(
-        ta, tb, M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd,
-        plan.units ? plan.full_tiles : tiles, plan.units, part, flags, epoch, nullptr, 0);
-    return cudaPeekAtLastError();
+    return pdl_launch(k_gemm_fp8_2sm<MODE, BN, false>, dim3(2 * pairs), dim3(sm2::THREADS), sm2::Cfg<BN>::SMEM, st,
+                      ta, tb, M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd,
+                      plan.units ? plan.full_tiles : tiles, plan.units, part, flags, epoch,
+                      static_cast<const int64_t *>(nullptr), 0);
 }
 
 // Grouped launch: a persistent grid of every pair that fits; each pair
@@ -751,10 +756,9 @@ template <int MODE>
 cudaError_t launch_gemm_grouped(cudaStream_t st, const CUtensorMap &ta, const CUtensorMap &tb, int64_t total_M,
                                 int N, int K, uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd,
                                 const int64_t *goff, int G, int pairs_cap) {
-    k_gemm_fp8_2sm<MODE, 256, true><<<2 * pairs_cap, sm2::THREADS, sm2::Cfg<256>::SMEM, st>>>(
-        ta, tb, (int)total_M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd, 0, 0, nullptr, nullptr, 0,
-        goff, G);
-    return cudaPeekAtLastError();
+    return pdl_launch(k_gemm_fp8_2sm<MODE, 256, true>, dim3(2 * pairs_cap), dim3(sm2::THREADS), sm2::Cfg<256>::SMEM,
+                      st, ta, tb, (int)total_M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd, 0, 0,
+                      static_cast<float *>(nullptr), static_cast<uint32_t *>(nullptr), 0u, goff, G);
 }
 
 uint32_t make_idesc(fp8_format fa, fp8_format fb, int mma_m, int mma_n) {

@@ -29,6 +29,7 @@
 #include "tc.cuh"
 
 using namespace fp8q;
+using fp8q_host::pdl_launch;
 
 namespace {
 
@@ -116,6 +117,8 @@ k_gemm_bf16_wgrad_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     cluster_sync_all();   // both CTAs' barriers are initialised before any remote signal
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();      // inputs of the previous kernel in the stream are visible from here on
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -316,9 +319,10 @@ extern "C" fp8_status fp8_gemm_bf16_wgrad(const void *dY_bf16, const void *X_bf1
     if (cap <= 0) return FP8_ERR_CUDA;
     const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
-    k_gemm_bf16_wgrad_2sm<<<2 * pairs, sm2::THREADS, wg::SMEM, s>>>(ta, tb, (int)M, (int)N, (int)T,
-                                                                   make_idesc_bf16_mn(256, 256), dW, ldd, accumulate);
-    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    return pdl_launch(k_gemm_bf16_wgrad_2sm, dim3(2 * pairs), dim3(sm2::THREADS), wg::SMEM, s, ta, tb, (int)M,
+                      (int)N, (int)T, make_idesc_bf16_mn(256, 256), dW, ldd, accumulate) == cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_CUDA;
 }
 
 // This file's device error word (read and optionally cleared by

@@ -16,6 +16,7 @@
 #include "tc.cuh"
 
 using namespace fp8q;
+using fp8q_host::pdl_launch;
 
 namespace {
 
@@ -131,6 +132,8 @@ k_gemm_mx_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     cluster_sync_all();   // both CTAs' barriers are initialised before any remote signal
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();      // inputs of the previous kernel in the stream are visible from here on
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -353,10 +356,11 @@ extern "C" fp8_status fp8_gemm_block_e8m0(const uint8_t *A, fp8_format fa, const
     if (cap <= 0) return FP8_ERR_CUDA;
     const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
-    k_gemm_mx_2sm<<<2 * pairs, sm2::THREADS, mx::SMEM, s>>>(ta, tb, tsa, tsb, (int)M, (int)N, (int)K,
-                                                          make_idesc_mx(fa, fb, 256, 256),
-                                                          static_cast<__nv_bfloat16 *>(D_bf16), ldd);
-    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    return pdl_launch(k_gemm_mx_2sm, dim3(2 * pairs), dim3(sm2::THREADS), mx::SMEM, s, ta, tb, tsa, tsb, (int)M,
+                      (int)N, (int)K, make_idesc_mx(fa, fb, 256, 256), static_cast<__nv_bfloat16 *>(D_bf16), ldd) ==
+                   cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_CUDA;
 }
 
 // This file's device error word (read and optionally cleared by

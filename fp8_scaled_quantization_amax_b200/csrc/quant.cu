@@ -14,6 +14,7 @@
 #include "common.cuh"
 
 using namespace fp8q;
+using fp8q_host::pdl_launch;
 
 namespace {
 
@@ -26,6 +27,8 @@ __global__ void __launch_bounds__(kStreamThreads) k_amax(const uint4 *__restrict
                                                          const uint16_t *__restrict__ xs, int64_t n,
                                                          uint32_t *__restrict__ amax_bits,
                                                          uint32_t *__restrict__ counts) {
+    pdl_trigger();   // dependents are scheduled once all our CTAs have started
+    pdl_wait();
     __shared__ uint32_t red[32];
     const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -67,6 +70,8 @@ k_cast_tensor(const uint4 *__restrict__ xv, uint4 *__restrict__ qv, int64_t nuni
               const float *__restrict__ scale_in, const float *__restrict__ amax_in,
               float *__restrict__ scale_inv_out, uint32_t *__restrict__ amax_bits,
               uint32_t *__restrict__ nf_ctr, uint32_t *__restrict__ sat_ctr) {
+    pdl_trigger();   // dependents are scheduled once all our CTAs have started
+    pdl_wait();
     __shared__ uint32_t red[32];
     constexpr float fm = fmax_of<FMT>();
     const float s = scale_in ? *scale_in : scale_from_amax(*amax_in, fm);
@@ -137,6 +142,8 @@ k_cast_transpose(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64
                  const float *__restrict__ scale_in, const float *__restrict__ amax_in,
                  float *__restrict__ scale_inv_out, uint32_t *__restrict__ amax_bits,
                  uint32_t *__restrict__ nf_ctr, uint32_t *__restrict__ sat_ctr) {
+    pdl_trigger();   // dependents are scheduled once all our CTAs have started
+    pdl_wait();
     __shared__ __align__(16) uint8_t tile[64][64 + 16];
     __shared__ uint32_t red[32];
     constexpr float fm = fmax_of<FMT>();
@@ -336,6 +343,8 @@ template <int FMT, bool POW2, int V, int R>
 __global__ void __launch_bounds__(kRowThreads)
 k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
           uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
+    pdl_trigger();   // dependents are scheduled once all our CTAs have started
+    pdl_wait();
     __shared__ uint32_t red[R][32];
     constexpr float fm = fmax_of<FMT>();
     const int64_t ncv = cols / 8;
@@ -434,6 +443,8 @@ template <int FMT, int U, bool SF>
 __global__ void __launch_bounds__(256)
 k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
              uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image) {
+    pdl_trigger();   // dependents are scheduled once all our CTAs have started
+    pdl_wait();
     constexpr float fm = fmax_of<FMT>();
     const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
     const int64_t nkb = (cols + 127) / 128;
@@ -492,6 +503,8 @@ template <int FMT, bool SF>
 __global__ void __launch_bounds__(256)
 k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
            uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image) {
+    pdl_trigger();   // dependents are scheduled once all our CTAs have started
+    pdl_wait();
     __shared__ uint32_t red[32];
     constexpr float fm = fmax_of<FMT>();
     const int64_t nkb = (cols + 127) / 128, nrb = (rows + 127) / 128;
@@ -544,20 +557,20 @@ void launch_cast(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t 
     const uint16_t *xs = static_cast<const uint16_t *>(x);
     if (transpose_out) {
         dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
-        if (amax && count) k_cast_transpose<FMT, true, true><<<grid, 256, 0, st>>>(xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
-        else if (amax) k_cast_transpose<FMT, true, false><<<grid, 256, 0, st>>>(xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
-        else if (count) k_cast_transpose<FMT, false, true><<<grid, 256, 0, st>>>(xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
-        else k_cast_transpose<FMT, false, false><<<grid, 256, 0, st>>>(xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+        if (amax && count) pdl_launch(k_cast_transpose<FMT, true, true>, dim3(grid), dim3(256), 0, st, xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+        else if (amax) pdl_launch(k_cast_transpose<FMT, true, false>, dim3(grid), dim3(256), 0, st, xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+        else if (count) pdl_launch(k_cast_transpose<FMT, false, true>, dim3(grid), dim3(256), 0, st, xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+        else pdl_launch(k_cast_transpose<FMT, false, false>, dim3(grid), dim3(256), 0, st, xs, q, rows, cols, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
         return;
     }
     const int64_t n = rows * cols, nunit = n / 16;
     const int grid = stream_grid(sms, std::max<int64_t>(nunit / 2, 1), kStreamThreads);
     const uint4 *xv = static_cast<const uint4 *>(x);
     uint4 *qv = reinterpret_cast<uint4 *>(q);
-    if (amax && count) k_cast_tensor<FMT, true, true><<<grid, kStreamThreads, 0, st>>>(xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
-    else if (amax) k_cast_tensor<FMT, true, false><<<grid, kStreamThreads, 0, st>>>(xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
-    else if (count) k_cast_tensor<FMT, false, true><<<grid, kStreamThreads, 0, st>>>(xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
-    else k_cast_tensor<FMT, false, false><<<grid, kStreamThreads, 0, st>>>(xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+    if (amax && count) pdl_launch(k_cast_tensor<FMT, true, true>, dim3(grid), dim3(kStreamThreads), 0, st, xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+    else if (amax) pdl_launch(k_cast_tensor<FMT, true, false>, dim3(grid), dim3(kStreamThreads), 0, st, xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+    else if (count) pdl_launch(k_cast_tensor<FMT, false, true>, dim3(grid), dim3(kStreamThreads), 0, st, xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
+    else pdl_launch(k_cast_tensor<FMT, false, false>, dim3(grid), dim3(kStreamThreads), 0, st, xv, qv, nunit, xs, q, n, scale_in, amax_in, scale_inv, amax_bits, nf_ctr, sat_ctr);
 }
 
 template <int FMT, bool POW2>
@@ -572,17 +585,17 @@ void launch_rowwise(cudaStream_t st, int sms, const void *x, int64_t rows, int64
     const int R = two ? 2 : 1;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + R - 1) / R, slots));
     if (two) {
-        if (ncv <= T) k_rowwise<FMT, POW2, 1, 2><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-        else if (ncv <= 2 * T) k_rowwise<FMT, POW2, 2, 2><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-        else k_rowwise<FMT, POW2, 4, 2><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+        if (ncv <= T) pdl_launch(k_rowwise<FMT, POW2, 1, 2>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
+        else if (ncv <= 2 * T) pdl_launch(k_rowwise<FMT, POW2, 2, 2>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
+        else pdl_launch(k_rowwise<FMT, POW2, 4, 2>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
         return;
     }
-    if (ncv <= T) k_rowwise<FMT, POW2, 1, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 2 * T) k_rowwise<FMT, POW2, 2, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 4 * T) k_rowwise<FMT, POW2, 4, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 8 * T) k_rowwise<FMT, POW2, 8, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 16 * T) k_rowwise<FMT, POW2, 16, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
-    else k_rowwise<FMT, POW2, 0, 1><<<grid, T, 0, st>>>(xs, rows, cols, ld, q, scale_inv);
+    if (ncv <= T) pdl_launch(k_rowwise<FMT, POW2, 1, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 2 * T) pdl_launch(k_rowwise<FMT, POW2, 2, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 4 * T) pdl_launch(k_rowwise<FMT, POW2, 4, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 8 * T) pdl_launch(k_rowwise<FMT, POW2, 8, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
+    else if (ncv <= 16 * T) pdl_launch(k_rowwise<FMT, POW2, 16, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
+    else pdl_launch(k_rowwise<FMT, POW2, 0, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
 }
 
 template <int FMT, bool SF>
@@ -594,11 +607,11 @@ void launch_block(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t
         constexpr int U = 4;
         const int64_t r = SF ? (rows + 127) / 128 * 128 : rows;
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((r + 7) / 8, (int64_t)sms * 8));
-        k_block1x128<FMT, U, SF><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv, sf_image);
+        pdl_launch(k_block1x128<FMT, U, SF>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q, scale_inv, sf_image);
     } else {
         const int64_t tiles = ((rows + 127) / 128) * nkb;
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)sms * 8));
-        k_block128<FMT, SF><<<grid, 256, 0, st>>>(xs, rows, cols, ld, q, scale_inv, sf_image);
+        pdl_launch(k_block128<FMT, SF>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q, scale_inv, sf_image);
     }
 }
 
@@ -619,7 +632,7 @@ extern "C" fp8_status fp8_amax(const void *x_bf16, int64_t n, float *amax, uint3
     if (cudaMemsetAsync(amax, 0, sizeof(float), s) != cudaSuccess) return FP8_ERR_CUDA;
     const int64_t nvec = n / 8;
     const int grid = stream_grid(sms, std::max<int64_t>(nvec / 4, 1), kStreamThreads);
-    k_amax<<<grid, kStreamThreads, 0, s>>>(static_cast<const uint4 *>(x_bf16), nvec,
+    pdl_launch(k_amax, dim3(grid), dim3(kStreamThreads), 0, s, static_cast<const uint4 *>(x_bf16), nvec,
                                             static_cast<const uint16_t *>(x_bf16), n,
                                             reinterpret_cast<uint32_t *>(amax), counts);
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
