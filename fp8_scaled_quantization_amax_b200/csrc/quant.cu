@@ -339,17 +339,32 @@ k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, i
 // element, and all R rows' loads are issued before the first reduction.
 // V == 0: rows too long for registers, two passes (the second from L2).
 constexpr int kRowThreads = 128;
+// One tensor of a rowwise launch (a launch can quantize two, e.g. both GEMM
+// operands, which share the row length).
+struct RowJob {
+    const uint16_t *x;
+    int64_t rows, ld;
+    uint8_t *q;
+    float *scale_inv;
+};
 template <int FMT, bool POW2, int V, int R>
 __global__ void __launch_bounds__(kRowThreads)
-k_rowwise(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-          uint8_t *__restrict__ q, float *__restrict__ scale_inv) {
+k_rowwise(RowJob ja, RowJob jb, int64_t cols) {
     pdl_trigger();   // dependents are scheduled once all our CTAs have started
     pdl_wait();
     __shared__ uint32_t red[R][32];
     constexpr float fm = fmax_of<FMT>();
     const int64_t ncv = cols / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int64_t r0 = (int64_t)blockIdx.x * R; r0 < rows; r0 += (int64_t)gridDim.x * R) {
+    // groups of R rows: ja's first, then jb's
+    const int64_t ga = (ja.rows + R - 1) / R, gtot = ga + (jb.rows + R - 1) / R;
+    for (int64_t g = blockIdx.x; g < gtot; g += gridDim.x) {
+        const bool first = g < ga;
+        const uint16_t *x = first ? ja.x : jb.x;
+        const int64_t rows = first ? ja.rows : jb.rows, ld = first ? ja.ld : jb.ld;
+        uint8_t *q = first ? ja.q : jb.q;
+        float *scale_inv = first ? ja.scale_inv : jb.scale_inv;
+        const int64_t r0 = (first ? g : g - ga) * R;
         if constexpr (V > 0) {
             uint4 v[R][V];
             uint32_t m[R];
@@ -574,28 +589,26 @@ void launch_cast(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t 
 }
 
 template <int FMT, bool POW2>
-void launch_rowwise(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, int64_t ld,
-                    uint8_t *q, float *scale_inv) {
-    const uint16_t *xs = static_cast<const uint16_t *>(x);
+cudaError_t launch_rowwise(cudaStream_t st, int sms, const RowJob &ja, const RowJob &jb, int64_t cols) {
     const int64_t slots = (int64_t)sms * 16;   // resident 128-thread CTAs
     const int64_t ncv = cols / 8;
+    const int64_t rows = ja.rows + jb.rows;
     const int T = kRowThreads;
     // two rows per CTA when that lets one wave of CTAs cover every row
     const bool two = rows > slots && ncv <= 4 * T;
-    const int R = two ? 2 : 1;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + R - 1) / R, slots));
+    const int64_t groups = two ? (ja.rows + 1) / 2 + (jb.rows + 1) / 2 : rows;
+    const dim3 grid((unsigned)std::max<int64_t>(1, std::min<int64_t>(groups, slots))), block(T);
     if (two) {
-        if (ncv <= T) pdl_launch(k_rowwise<FMT, POW2, 1, 2>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
-        else if (ncv <= 2 * T) pdl_launch(k_rowwise<FMT, POW2, 2, 2>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
-        else pdl_launch(k_rowwise<FMT, POW2, 4, 2>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
-        return;
+        if (ncv <= T) return pdl_launch(k_rowwise<FMT, POW2, 1, 2>, grid, block, 0, st, ja, jb, cols);
+        if (ncv <= 2 * T) return pdl_launch(k_rowwise<FMT, POW2, 2, 2>, grid, block, 0, st, ja, jb, cols);
+        return pdl_launch(k_rowwise<FMT, POW2, 4, 2>, grid, block, 0, st, ja, jb, cols);
     }
-    if (ncv <= T) pdl_launch(k_rowwise<FMT, POW2, 1, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 2 * T) pdl_launch(k_rowwise<FMT, POW2, 2, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 4 * T) pdl_launch(k_rowwise<FMT, POW2, 4, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 8 * T) pdl_launch(k_rowwise<FMT, POW2, 8, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
-    else if (ncv <= 16 * T) pdl_launch(k_rowwise<FMT, POW2, 16, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
-    else pdl_launch(k_rowwise<FMT, POW2, 0, 1>, dim3(grid), dim3(T), 0, st, xs, rows, cols, ld, q, scale_inv);
+    if (ncv <= T) return pdl_launch(k_rowwise<FMT, POW2, 1, 1>, grid, block, 0, st, ja, jb, cols);
+    if (ncv <= 2 * T) return pdl_launch(k_rowwise<FMT, POW2, 2, 1>, grid, block, 0, st, ja, jb, cols);
+    if (ncv <= 4 * T) return pdl_launch(k_rowwise<FMT, POW2, 4, 1>, grid, block, 0, st, ja, jb, cols);
+    if (ncv <= 8 * T) return pdl_launch(k_rowwise<FMT, POW2, 8, 1>, grid, block, 0, st, ja, jb, cols);
+    if (ncv <= 16 * T) return pdl_launch(k_rowwise<FMT, POW2, 16, 1>, grid, block, 0, st, ja, jb, cols);
+    return pdl_launch(k_rowwise<FMT, POW2, 0, 1>, grid, block, 0, st, ja, jb, cols);
 }
 
 template <int FMT, bool SF>
@@ -674,6 +687,16 @@ extern "C" fp8_status fp8_quantize_tensorwise(const void *x_bf16, int64_t rows, 
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
+static fp8_status dispatch_rowwise(cudaStream_t s, int sms, fp8_format fmt, int pow2, const RowJob &ja,
+                                   const RowJob &jb, int64_t cols) {
+    cudaError_t e;
+    if (fmt == FP8_E4M3) e = pow2 ? launch_rowwise<FP8_E4M3, true>(s, sms, ja, jb, cols)
+                                  : launch_rowwise<FP8_E4M3, false>(s, sms, ja, jb, cols);
+    else e = pow2 ? launch_rowwise<FP8_E5M2, true>(s, sms, ja, jb, cols)
+                  : launch_rowwise<FP8_E5M2, false>(s, sms, ja, jb, cols);
+    return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
 extern "C" fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                            fp8_format fmt, int pow2, uint8_t *q, float *scale_inv,
                                            void *stream) {
@@ -691,15 +714,30 @@ extern "C" fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
     if (rows == 0) return FP8_OK;
-    cudaStream_t s = as_stream(stream);
-    if (fmt == FP8_E4M3) {
-        if (pow2) launch_rowwise<FP8_E4M3, true>(s, sms, x_bf16, rows, cols, ld, q, scale_inv);
-        else launch_rowwise<FP8_E4M3, false>(s, sms, x_bf16, rows, cols, ld, q, scale_inv);
-    } else {
-        if (pow2) launch_rowwise<FP8_E5M2, true>(s, sms, x_bf16, rows, cols, ld, q, scale_inv);
-        else launch_rowwise<FP8_E5M2, false>(s, sms, x_bf16, rows, cols, ld, q, scale_inv);
-    }
-    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    const RowJob ja{static_cast<const uint16_t *>(x_bf16), rows, ld, q, scale_inv}, jb{nullptr, 0, 0, nullptr, nullptr};
+    return dispatch_rowwise(as_stream(stream), sms, fmt, pow2, ja, jb, cols);
+}
+
+extern "C" fp8_status fp8_quantize_rowwise_pair(const void *a_bf16, int64_t rows_a, int64_t lda, uint8_t *qa,
+                                                float *sa, const void *b_bf16, int64_t rows_b, int64_t ldb,
+                                                uint8_t *qb, float *sb, int64_t cols, fp8_format fmt, int pow2,
+                                                void *stream) {
+    if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (rows_a < 0 || rows_b < 0 || cols < 0 || lda < cols || ldb < cols || (cols % 16)) return FP8_ERR_SHAPE;
+    if ((rows_a > 0 && (!sa || (cols > 0 && (!a_bf16 || !qa)))) ||
+        (rows_b > 0 && (!sb || (cols > 0 && (!b_bf16 || !qb)))))
+        return FP8_ERR_INVALID_ARG;
+    if (lda % 8 || ldb % 8) return FP8_ERR_ALIGNMENT;
+    if ((a_bf16 && !aligned16(a_bf16)) || (qa && !aligned16(qa)) || (b_bf16 && !aligned16(b_bf16)) ||
+        (qb && !aligned16(qb)))
+        return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (rows_a + rows_b == 0) return FP8_OK;
+    const RowJob ja{static_cast<const uint16_t *>(a_bf16), rows_a, lda, qa, sa};
+    const RowJob jb{static_cast<const uint16_t *>(b_bf16), rows_b, ldb, qb, sb};
+    return dispatch_rowwise(as_stream(stream), sms, fmt, pow2, ja, jb, cols);
 }
 
 extern "C" fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,

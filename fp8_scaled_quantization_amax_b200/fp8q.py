@@ -43,6 +43,7 @@ SIGNATURES = {
     "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
     "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
+    "fp8_quantize_rowwise_pair": (_S, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _P, _P, _I64, _I, _I, _P]),
     "fp8_quantize_blockwise_e8m0": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
     "fp8_quantize_rowwise_transpose": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
     "fp8_gemm_bf16_wgrad": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _I, _P]),
@@ -213,6 +214,27 @@ def fp8_gemm_block_e8m0(A, fa, B, fb, M, N, K, a_sf, b_sf, D, ldd, stream=None):
     _dev(a_sf, torch.uint8, "a_sf"); _dev(b_sf, torch.uint8, "b_sf")
     _check("fp8_gemm_block_e8m0", lib().fp8_gemm_block_e8m0(
         _ptr(A), fa, _ptr(B), fb, M, N, K, _ptr(a_sf), _ptr(b_sf), _ptr(D), ldd, _stream(stream)))
+
+
+def fp8_quantize_rowwise_pair(a, rows_a, lda, qa, sa, b, rows_b, ldb, qb, sb, cols, fmt, pow2, stream=None):
+    _dev(a, torch.bfloat16, "a"); _dev(qa, torch.uint8, "qa"); _dev(sa, torch.float32, "sa")
+    _dev(b, torch.bfloat16, "b"); _dev(qb, torch.uint8, "qb"); _dev(sb, torch.float32, "sb")
+    _check("fp8_quantize_rowwise_pair", lib().fp8_quantize_rowwise_pair(
+        _ptr(a), rows_a, lda, _ptr(qa), _ptr(sa), _ptr(b), rows_b, ldb, _ptr(qb), _ptr(sb), cols, fmt, int(pow2),
+        _stream(stream)))
+
+
+def quantize_rowwise_pair(a, b, fmt=E4M3, pow2=True):
+    """((qa, sa), (qb, sb)) of a [Ma, K] and b [Mb, K] in one launch."""
+    K = a.shape[1]
+    if b.shape[1] != K:
+        raise ValueError("both operands need the same row length")
+    qa = torch.empty(a.shape, dtype=torch.uint8, device=a.device)
+    qb = torch.empty(b.shape, dtype=torch.uint8, device=b.device)
+    sa = torch.empty(a.shape[0], dtype=torch.float32, device=a.device)
+    sb = torch.empty(b.shape[0], dtype=torch.float32, device=b.device)
+    fp8_quantize_rowwise_pair(a, a.shape[0], a.stride(0), qa, sa, b, b.shape[0], b.stride(0), qb, sb, K, fmt, pow2)
+    return (qa, sa), (qb, sb)
 
 
 def fp8_quantize_rowwise_transpose(x, rows, cols, ld, fmt, pow2, qT, scale_inv, amax_out, stream=None):

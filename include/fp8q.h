@@ -115,6 +115,18 @@ FP8Q_API fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int64
                                 void *stream);
 
 /*
+ * Both operands of a rowwise GEMM in one launch: fp8_quantize_rowwise of
+ * a [rows_a, cols] (leading dimension lda) into qa / sa and of b [rows_b,
+ * cols] (ldb) into qb / sb, with the same format and scale rule (the
+ * forward GEMM's activations and weights share K and E4M3).  One launch
+ * instead of two saves a launch gap and a ramp on short tensors.  Shapes,
+ * layouts and errors as fp8_quantize_rowwise; either count may be 0.
+ */
+FP8Q_API fp8_status fp8_quantize_rowwise_pair(const void *a_bf16, int64_t rows_a, int64_t lda, uint8_t *qa,
+                                     float *sa, const void *b_bf16, int64_t rows_b, int64_t ldb, uint8_t *qb,
+                                     float *sb, int64_t cols, fp8_format fmt, int pow2, void *stream);
+
+/*
  * Per-block quantization ([DeepL] §2.3: the tensor is cut into small blocks
  * with one scale each) of x [rows, cols] (leading dimension ld).  Blocks are
  * block_rows x 128: block_rows = 1 for activations (1x128), 128 for weights

@@ -78,6 +78,11 @@ def test_validation_before_device_access():
     assert L.fp8_amax_history_update(FAKE, FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
     assert L.fp8_amax_history_update(FAKE, FAKE, 2000, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
     assert L.fp8_amax_history_update(None, FAKE, 16, FAKE, 0, FAKE, FAKE, FAKE, n) == INVALID
+    # rowwise pair
+    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 32, FAKE, FAKE, 24, 0, 1, n) == SHAPE
+    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 16, FAKE, FAKE, 32, 0, 1, n) == SHAPE
+    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, None, 4, 32, FAKE, FAKE, 32, 0, 1, n) == INVALID
+    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 32, FAKE, FAKE, 32, 5, 1, n) == INVALID
     # E8M0 block scales
     assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 32, 32, 0, 64, FAKE, FAKE, n) == INVALID    # block_rows
     assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 24, 32, 0, 1, FAKE, FAKE, n) == SHAPE       # cols % 16

@@ -184,6 +184,25 @@ def test_rowwise_full_size_outlier_activations(orc):
     assert_f32_equal(to_np(sinv), rsinv)
 
 
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("shapes", [((300, 512), (257, 512)), ((1, 16), (0, 16)), ((0, 64), (33, 64)),
+                                    ((4096, 4096), (4096, 4096)), ((3000, 4096), (11008, 4096))])
+def test_rowwise_pair_one_launch(orc, fmt, shapes):
+    """Both GEMM operands in one launch: each bit-exact against the oracle's
+    per-tensor rowwise quantization (the tensors are read with their own
+    row counts; a zero count leaves that side alone)."""
+    (ra, k), (rb, _) = shapes
+    a = inputs.outlier_activations_bf16((max(ra, 1), k), seed=ra + 3)[:ra]
+    b = inputs.normal_bf16((max(rb, 1), k), 0.02, seed=rb + 4)[:rb]
+    (qa, sa), (qb, sb) = fp8q.quantize_rowwise_pair(_dev(a), _dev(b), fmt, True)
+    for q, s, t in ((qa, sa, a), (qb, sb, b)):
+        if t.shape[0] == 0:
+            continue
+        rq, rs = orc.quantize_rowwise(inputs.bf16_bits(t), fmt, True)
+        assert_codes_equal(to_np(q), rq, fmt)
+        assert_f32_equal(to_np(s), rs)
+
+
 # --------------------------------------------------------------- blockwise --
 
 @pytest.mark.parametrize("fmt", [0, 1])
