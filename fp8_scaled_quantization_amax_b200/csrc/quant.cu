@@ -597,7 +597,9 @@ cudaError_t launch_rowwise(cudaStream_t st, int sms, const RowJob &ja, const Row
     // two rows per CTA when that lets one wave of CTAs cover every row
     const bool two = rows > slots && ncv <= 4 * T;
     const int64_t groups = two ? (ja.rows + 1) / 2 + (jb.rows + 1) / 2 : rows;
-    const dim3 grid((unsigned)std::max<int64_t>(1, std::min<int64_t>(groups, slots))), block(T);
+    // the same number of row groups for every CTA (no half-empty last round)
+    const int64_t rounds = (groups + slots - 1) / slots;
+    const dim3 grid((unsigned)std::max<int64_t>(1, (groups + rounds - 1) / rounds)), block(T);
     if (two) {
         if (ncv <= T) return pdl_launch(k_rowwise<FMT, POW2, 1, 2>, grid, block, 0, st, ja, jb, cols);
         if (ncv <= 2 * T) return pdl_launch(k_rowwise<FMT, POW2, 2, 2>, grid, block, 0, st, ja, jb, cols);
