@@ -217,3 +217,32 @@ def test_gemm_split_k_long_k_sampled(orc):
     D = fp8q.gemm(_cuda(A), 0, _cuda(B), 0, 1, _cuda(da), _cuda(db), workspace=ws)
     _sampled_check(orc, D, A, 0, B, 0, 1, da, db, n=1024, seed=4)
     assert fp8q.fp8_gemm_workspace_size(4096, 4096, 4096, 1) == 0   # multi-wave: no split
+
+
+def test_launch_chain_keeps_stream_order(orc):
+    """The quantizers and GEMMs are launched with programmatic dependent
+    launch: each may start before its predecessor ends and waits for it
+    before touching memory.  Reusing the same FP8 buffers for two different
+    inputs back to back (quantize -> GEMM -> quantize over the same buffers
+    -> GEMM ...) must give every GEMM the operands quantized just before it
+    (a read-after-write and a write-after-read hazard on every step)."""
+    M, N, K = 512, 768, 1024
+    xs = [inputs.outlier_activations_bf16((M, K), seed=200 + i, device="cuda") for i in range(2)]
+    ws = [inputs.normal_bf16((N, K), 0.02, seed=210 + i, device="cuda") for i in range(2)]
+    refs = []
+    for i in range(2):
+        (qa, sa), (qb, sb) = fp8q.quantize_rowwise_pair(xs[i], ws[i], 0, True)
+        refs.append(fp8q.gemm(qa, 0, qb, 0, fp8q.SCALE_ROW, sa, sb).clone())
+    torch.cuda.synchronize()
+    qa = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    qb = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    sa = torch.empty(M, dtype=torch.float32, device="cuda")
+    sb = torch.empty(N, dtype=torch.float32, device="cuda")
+    outs = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(40)]
+    for j, out in enumerate(outs):
+        i = j % 2
+        fp8q.fp8_quantize_rowwise_pair(xs[i], M, K, qa, sa, ws[i], N, K, qb, sb, K, 0, True)
+        fp8q.fp8_gemm_scaled(qa, 0, qb, 0, M, N, K, fp8q.SCALE_ROW, sa, sb, out, N)
+    torch.cuda.synchronize()
+    for j, out in enumerate(outs):
+        assert torch.equal(out, refs[j % 2]), j
