@@ -130,3 +130,21 @@ def test_gemm_e8m0_mlp_up_sampled(orc):
     ref, mag = orc.gemm_scaled_sampled(A, 0, B, 0, orc.SCALE_BLOCK, da, db, im, inn)
     got = bf16_to_f64(D[_cuda(im), _cuda(inn)])
     assert_gemm_close(got, ref, mag, "e8m0 mlp up sampled")
+
+
+def test_gemm_e8m0_mlp_down_sampled(orc):
+    """[8192, 11008] x W_down[4096, 11008]^T, the block MLP's down projection
+    (the input a seeded bf16 tensor of the up projection's output shape):
+    2048 sampled outputs against the oracle."""
+    M, N, K = 8192, 4096, 11008
+    h = inputs.bf16_bits(inputs.normal_bf16((M, K), 1.0, seed=15, device="cuda"))
+    w = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, seed=16, device="cuda"))
+    A, da = orc.quantize_blockwise(h, 0, 1, pow2=True)
+    B, db = orc.quantize_blockwise(w, 0, 128, pow2=True)
+    D = fp8q.gemm_block_e8m0(_cuda(A), 0, _cuda(B), 0, _cuda(_image(da, M, K, 1)), _cuda(_image(db, N, K, 128)))
+    rng = np.random.default_rng(2)
+    im = np.concatenate([[0, M - 1, 255, 256], rng.integers(0, M, 2044)])
+    inn = np.concatenate([[0, N - 1, 255, 256], rng.integers(0, N, 2044)])
+    ref, mag = orc.gemm_scaled_sampled(A, 0, B, 0, orc.SCALE_BLOCK, da, db, im, inn)
+    got = bf16_to_f64(D[_cuda(im), _cuda(inn)])
+    assert_gemm_close(got, ref, mag, "e8m0 mlp down sampled")

@@ -118,3 +118,42 @@ def test_dgrad_delayed_scaling_loop(orc):
         assert_f32_equal(to_np(hist.scale), rh.scale)
         if t == 9:
             assert sat == 1
+
+
+def test_dgrad_full_size_delayed_scaling_sampled(orc):
+    """The dgrad workload at full size and in the bench's launch
+    configuration: dY_t [8192, 4096] (log-normal magnitudes, E5M2 with the
+    history's scale and fused amax) against W^T [4096, 4096] (E4M3
+    per-tensor, transposed cast), split-K workspace passed as the bench does,
+    16-step history; 5 steps, the third an x8 spike.  Codes and amax
+    bit-exact per step, 512 sampled outputs per step against the oracle."""
+    M, N_out, K_in = 8192, 4096, 4096
+    W = inputs.normal_bf16((N_out, K_in), 0.02, seed=300, device="cuda")
+    wq, wsinv, _ = fp8q.quantize_tensorwise(W, 0, transpose=True)
+    rwq, rwsinv, _, _ = orc.quantize_tensorwise(inputs.bf16_bits(W), 0, transpose_out=True)
+    assert_codes_equal(to_np(wq), rwq, 0)
+    hist = fp8q.AmaxHistory(16, 1)
+    rh = orc.AmaxHistory(16, 1)
+    ws = fp8q.gemm_workspace(M, K_in, N_out, fp8q.SCALE_TENSOR)
+    rng = np.random.default_rng(3)
+    for t in range(5):
+        g = inputs.lognormal_grads_bf16((M, N_out), seed=400 + t, device="cuda")
+        if t == 2:
+            g = (g.float() * 8).to(torch.bfloat16)
+        gb = inputs.bf16_bits(g)
+        q, sinv, am = fp8q.quantize_tensorwise(g, 1, scale_in=hist.scale)
+        rq, rsinv, ramax, _ = orc.quantize_tensorwise(gb, 1, scale_in=float(rh.scale[0]))
+        assert_codes_equal(to_np(q), rq, 1, f"dY8 step {t}")
+        assert_f32_equal(to_np(am), np.float32([ramax]))
+        D = fp8q.gemm(q, 1, wq, 0, 0, sinv, wsinv, workspace=ws)
+        im = np.concatenate([[0, M - 1], rng.integers(0, M, 510)])
+        inn = np.concatenate([[0, K_in - 1], rng.integers(0, K_in, 510)])
+        ref, mag = orc.gemm_scaled_sampled(rq, 1, rwq, 0, 0, np.float32([rsinv]), np.float32([rwsinv]), im, inn)
+        got = D.float().cpu().numpy().astype(np.float64)[im, inn]
+        assert_gemm_close(got, ref, mag, f"dX step {t}")
+        hist.update(am)
+        sat = rh.update(ramax)
+        assert int(hist.saturated) == sat
+        assert_f32_equal(to_np(hist.scale), rh.scale)
+        if t == 2:
+            assert sat == 1
