@@ -1,7 +1,7 @@
 // paged_kv.cu -- paged FP8 KV cache: write new tokens into fixed-size blocks,
 // read sequences back through their block tables.
 //
-// Sources: "FP8量化首次支持！ms-swift引领大模型低精度计算新浪潮" (vLLM's KV
+// Sources: "ms-swift全链路能力解析：训练、推理、评测、量化与部署一体化解决方案" (vLLM's KV
 // cache cut into fixed-size blocks handed out on demand) and
 // "DeepL押注FP8：大模型训练与推理统一精度实战解析" §3.1 (K and V stored in
 // FP8 halve the cache, dequantized when attention reads them).  Reading taken

@@ -350,8 +350,8 @@ FP8Q_API fp8_status fp8_kv_dequant(const uint8_t *q, const float *scale_inv, int
                           int64_t S, int64_t Dh, fp8_format fmt, void *out_bf16, void *stream);
 
 /*
- * Paged FP8 KV cache, write side ("FP8量化首次支持！ms-swift引领大模型低精度计算
- * 新浪潮": the KV cache is cut into fixed-size blocks allocated on demand;
+ * Paged FP8 KV cache, write side ("ms-swift全链路能力解析：训练、推理、评测、量化与
+ * 部署一体化解决方案": the KV cache is cut into fixed-size blocks allocated on demand;
  * [DeepL] §3.1: K and V stored in FP8).  Each (token, head) row of Dh
  * elements is quantized with its own scale s = fmax / amax(row) (tokens
  * arrive a few at a time, so a per-sequence amax is not known yet).

@@ -470,7 +470,7 @@ void orc_scale_stats(const float *s, const float *prev, int64_t n, float jump_ra
 /* ------------------------------------------------------- paged KV cache -- */
 
 /* Paged FP8 KV cache.  The cache is split into fixed-size blocks handed out on
- * demand ("FP8量化首次支持！ms-swift引领大模型低精度计算新浪潮", vLLM's block
+ * demand ("ms-swift全链路能力解析：训练、推理、评测、量化与部署一体化解决方案", vLLM's block
  * KV cache) and stores K / V in FP8 ([DeepL] §3.1).  Tokens arrive a few at a
  * time, so a scale over a whole (sequence, head) slice is not known when a
  * token is written: each (token, head) row of Dh elements gets its own scale.

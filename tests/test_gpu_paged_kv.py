@@ -1,6 +1,6 @@
 """GPU parity of the paged FP8 KV cache against the CPU oracle (bit-exact).
 
-Sources: "FP8量化首次支持！ms-swift引领大模型低精度计算新浪潮" (KV cache in
+Sources: "ms-swift全链路能力解析：训练、推理、评测、量化与部署一体化解决方案" (KV cache in
 fixed-size blocks allocated on demand) and "DeepL押注FP8：大模型训练与推理统一
 精度实战解析" §3.1 (K and V kept in FP8, dequantized when read).  Every case
 starts the device cache and the oracle's from the same stale bytes, so pages

@@ -489,7 +489,7 @@ def test_scale_stats_closed_forms(orc):
 
 @pytest.mark.parametrize("fmt", [0, 1])
 def test_paged_kv_write_and_gather(orc, fmt):
-    """Paged FP8 KV cache (block KV cache of the ms-swift page; FP8 KV of the
+    """Paged FP8 KV cache (block KV cache of "ms-swift全链路能力解析：训练、推理、评测、量化与部署一体化解决方案"; FP8 KV of the
     DeepL page §3.1), against torch built independently: per (token, head) the
     amax by torch, s = fmax / amax as one fp32 division, the cast by torch's
     float8 conversion of the clamped product, the read-back by torch's bf16
