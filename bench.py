@@ -130,6 +130,56 @@ class ClockSampler:
 
 # --------------------------------------------------------------- workloads --
 
+def config_of(name: str, profile: bool = False) -> dict:
+    """The workload description a bench line carries in "config" (both arms)."""
+    from fp8_scaled_quantization_amax_b200 import inputs as inp
+    small = 2048 if profile else 8192
+    if name == "rowwise":
+        return {"workload": "rowwise pow2 E4M3 GEMM", "M": 4096, "N": 4096, "K": 4096,
+                "A": "N(0,1) bf16, 0.1% entries x100", "B": "N(0,0.02) bf16",
+                "scales": "per-row A, per-row B (= per output column), powers of two"}
+    if name == "tensor":
+        return {"workload": "per-tensor E4M3 GEMM", "M": 256, "N": 256, "K": 256,
+                "A": "N(0,1) bf16", "B": "N(0,1) bf16", "scales": "s = 448/amax per tensor"}
+    if name == "blockmlp":
+        return {"workload": "block-scaled E4M3 MLP (up then down)", "M": small, "D": 4096, "F": 11008,
+                "X": "N(0,1) bf16", "W": "N(0,0.02) bf16",
+                "scales": "1x128 activation blocks, 128x128 weight blocks, fp32",
+                "chain": "H = up(X) in bf16 is requantized 1x128 for the down GEMM"}
+    if name == "blockmlp_e8m0":
+        return {"workload": "block-scaled E4M3 MLP (up then down), E8M0 scales in the MMA", "M": small,
+                "D": 4096, "F": 11008, "X": "N(0,1) bf16", "W": "N(0,0.02) bf16",
+                "scales": "1x128 activation blocks, 128x128 weight blocks, powers of two (E8M0)",
+                "chain": "H = up(X) in bf16 is requantized 1x128 for the down GEMM"}
+    if name == "dgrad":
+        return {"workload": "dgrad E5M2 x E4M3, delayed scaling", "M": small, "N_out": 4096, "K_in": 4096,
+                "dY": "|g| = 10^u, u ~ N(-2, (4/3)^2) clipped to [-6, 2], random sign, 16 seeded steps",
+                "W": "N(0,0.02) bf16, E4M3 per-tensor, transposed once", "history": 16}
+    if name == "bwd_gw_hp":
+        return {"workload": "linear backward, rowwise_with_gw_hp (FP8 rowwise dgrad, bf16 wgrad)",
+                "T": small, "N_out": 4096, "K_in": 4096,
+                "dY": "|g| = 10^u, u ~ N(-2, (4/3)^2) clipped to [-6, 2], random sign; E5M2 per token",
+                "W": "N(0,0.02) bf16; W^T E4M3 per input channel, requantized every step",
+                "X": "N(0,1) bf16", "dW": "fp32, dY^T X from the bf16 tensors"}
+    if name == "kv":
+        return {"workload": "FP8 KV cache quantize + dequantize", "B": 8 if profile else 32, "H": 32, "S": 8192,
+                "Dh": 128, "K,V": "N(0,1) bf16", "scale": "per (b, h): 448/amax, E4M3"}
+    if name == "paged":
+        P = inp.PAGED_KV
+        B = 8 if profile else P["B"]
+        return {"workload": "paged FP8 KV cache write + gather", "sequences": B, "tokens_per_seq": P["S"],
+                "H": P["H"], "Dh": P["Dh"], "block_size": P["block_size"],
+                "num_blocks": B * P["S"] // P["block_size"], "pages": "shuffled pool",
+                "K,V": "N(0,1) bf16", "scale": "per (token, head): 448/amax, E4M3"}
+    if name == "health":
+        L = inp.SCALE_HEALTH["layers"] * (8 if profile else 1)
+        return {"workload": "scale health check (min/max/mean + step changes)", "segments": L,
+                "scales_per_segment": inp.SCALE_HEALTH["per_layer"],
+                "scales": "log10 s ~ N(1, 0.25); next snapshot drifted, 0.1 % stepped x16 or /16",
+                "jump_ratio": 4.0}
+    raise ValueError(name)
+
+
 class Workload:
     """Inputs resident on the device and the step as a list of library calls."""
 
@@ -159,9 +209,7 @@ class Workload:
         self.flops = 2.0 * M * N * K
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.launches = 2
-        self.config = {"workload": "rowwise pow2 E4M3 GEMM", "M": M, "N": N, "K": K,
-                       "A": "N(0,1) bf16, 0.1% entries x100", "B": "N(0,0.02) bf16",
-                       "scales": "per-row A, per-row B (= per output column), powers of two"}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("A", self.A), ("B", self.B)]
         self.host_output = self.D
 
@@ -191,8 +239,7 @@ class Workload:
         self.flops = 2.0 * M * N * K
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.launches = 5
-        self.config = {"workload": "per-tensor E4M3 GEMM", "M": M, "N": N, "K": K,
-                       "A": "N(0,1) bf16", "B": "N(0,1) bf16", "scales": "s = 448/amax per tensor"}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("A", self.A), ("B", self.B)]
         self.host_output = self.D
 
@@ -229,10 +276,7 @@ class Workload:
         self.flops = 2 * 2.0 * M * Dm * F
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.launches = 6
-        self.config = {"workload": "block-scaled E4M3 MLP (up then down)", "M": M, "D": Dm, "F": F,
-                       "X": "N(0,1) bf16", "W": "N(0,0.02) bf16",
-                       "scales": "1x128 activation blocks, 128x128 weight blocks, fp32",
-                       "chain": "H = up(X) in bf16 is requantized 1x128 for the down GEMM"}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("X", self.X), ("W_up", self.Wu), ("W_down", self.Wd)]
         self.host_output = self.Y
 
@@ -268,10 +312,7 @@ class Workload:
         self.flops = 2 * 2.0 * M * Dm * F
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.launches = 6
-        self.config = {"workload": "block-scaled E4M3 MLP (up then down), E8M0 scales in the MMA", "M": M,
-                       "D": Dm, "F": F, "X": "N(0,1) bf16", "W": "N(0,0.02) bf16",
-                       "scales": "1x128 activation blocks, 128x128 weight blocks, powers of two (E8M0)",
-                       "chain": "H = up(X) in bf16 is requantized 1x128 for the down GEMM"}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("X", self.X), ("W_up", self.Wu), ("W_down", self.Wd)]
         self.host_output = self.Y
 
@@ -308,9 +349,7 @@ class Workload:
         self.flops = 2.0 * M * N_out * K_in
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.launches = 3
-        self.config = {"workload": "dgrad E5M2 x E4M3, delayed scaling", "M": M, "N_out": N_out, "K_in": K_in,
-                       "dY": "|g| = 10^u, u ~ N(-2, (4/3)^2) clipped to [-6, 2], random sign, 16 seeded steps",
-                       "W": "N(0,0.02) bf16, E4M3 per-tensor, transposed once", "history": 16}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("dY_t", self.G[0])]
         self.host_output = self.DX
 
@@ -347,11 +386,7 @@ class Workload:
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.peak_dtype = "bf16"   # the dominant kernel is the bf16 weight-gradient GEMM
         self.launches = 5          # + one memset (the column-amax buffer), not a kernel
-        self.config = {"workload": "linear backward, rowwise_with_gw_hp (FP8 rowwise dgrad, bf16 wgrad)",
-                       "T": T, "N_out": N_out, "K_in": K_in,
-                       "dY": "|g| = 10^u, u ~ N(-2, (4/3)^2) clipped to [-6, 2], random sign; E5M2 per token",
-                       "W": "N(0,0.02) bf16; W^T E4M3 per input channel, requantized every step",
-                       "X": "N(0,1) bf16", "dW": "fp32, dY^T X from the bf16 tensors"}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("dY", self.dY), ("X", self.X)]
         self.host_output = self.DX
 
@@ -386,8 +421,7 @@ class Workload:
         self.kernel_bytes = 3.0 * n + 4 * B * H       # one kv_quant launch
         self.unit, self.bound = "GB/s", "hbm"
         self.launches = 4
-        self.config = {"workload": "FP8 KV cache quantize + dequantize", "B": B, "H": H, "S": S, "Dh": Dh,
-                       "K,V": "N(0,1) bf16", "scale": "per (b, h): 448/amax, E4M3"}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("K", self.K), ("V", self.V)]
         self.host_output = self.Kd
 
@@ -429,9 +463,7 @@ class Workload:
         self.kernel_bytes = wbytes                                    # one fp8_paged_kv_write launch
         self.unit, self.bound = "GB/s", "hbm"
         self.launches = 4
-        self.config = {"workload": "paged FP8 KV cache write + gather", "sequences": B, "tokens_per_seq": S,
-                       "H": H, "Dh": Dh, "block_size": bs, "num_blocks": NB, "pages": "shuffled pool",
-                       "K,V": "N(0,1) bf16", "scale": "per (token, head): 448/amax, E4M3"}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("K", self.K), ("V", self.V)]
         self.host_output = self.Kd
 
@@ -466,9 +498,7 @@ class Workload:
         self.kernel_bytes = self.bytes
         self.unit, self.bound = "GB/s", "hbm"
         self.launches = 1
-        self.config = {"workload": "scale health check (min/max/mean + step changes)", "segments": L,
-                       "scales_per_segment": n, "scales": "log10 s ~ N(1, 0.25); next snapshot drifted, "
-                       "0.1 % stepped x16 or /16", "jump_ratio": 4.0}
+        self.config = config_of(self.name, self.profile)
         self.host_inputs = [("cur", self.cur)]
         self.host_output = self.stats
 
@@ -561,15 +591,17 @@ def cpu_sample(name: str, seed: int = 0):
             M = N = K = 256
             a = inputs.bf16_bits(inputs.normal_bf16((M, K), 1.0, seed=seed))
             b = inputs.bf16_bits(inputs.normal_bf16((N, K), 1.0, seed=seed + 1))
+            reps = 10
             t0 = time.perf_counter()
-            qa, sa, _, _ = orc.quantize_tensorwise(a, 0)
-            qb, sb, _, _ = orc.quantize_tensorwise(b, 0)
-            orc.gemm_scaled(qa, 0, qb, 0, 0, np.float32([sa]), np.float32([sb]))
-            t = time.perf_counter() - t0
-            return 2.0 * M * N * K / t / 1e12, "the whole 256^3 per-tensor step"
+            for _ in range(reps):
+                qa, sa, _, _ = orc.quantize_tensorwise(a, 0)
+                qb, sb, _, _ = orc.quantize_tensorwise(b, 0)
+                orc.gemm_scaled(qa, 0, qb, 0, 0, np.float32([sa]), np.float32([sb]))
+            t = (time.perf_counter() - t0) / reps
+            return 2.0 * M * N * K / t / 1e12, "the whole 256^3 per-tensor step, mean of 10"
         if name == "blockmlp":
             M, Dm, F = 8192, 4096, 11008
-            r = 4
+            r = 32
             x = inputs.bf16_bits(inputs.normal_bf16((r, Dm), 1.0, seed=seed))
             w = inputs.bf16_bits(inputs.normal_bf16((256, Dm), 0.02, seed=seed + 1))
             t0 = time.perf_counter()
@@ -586,7 +618,7 @@ def cpu_sample(name: str, seed: int = 0):
                 "scaled to both MLP GEMMs")
         if name == "dgrad":
             M, N_out, K_in = 8192, 4096, 4096
-            r = 16
+            r = 128
             g = inputs.bf16_bits(inputs.lognormal_grads_bf16((r, N_out), seed=seed))
             w = inputs.bf16_bits(inputs.normal_bf16((256, N_out), 0.02, seed=seed + 1))
             t0 = time.perf_counter()
@@ -616,22 +648,24 @@ def cpu_sample(name: str, seed: int = 0):
         L, n = inputs.SCALE_HEALTH["layers"], inputs.SCALE_HEALTH["per_layer"]
         prev, cur = inputs.scale_snapshots_f32(L * n, seed=seed + 7)
         p, c = prev.numpy(), cur.numpy()
+        reps = 20
         t0 = time.perf_counter()
-        for g in range(L):
-            orc.scale_stats(c[g * n:(g + 1) * n], p[g * n:(g + 1) * n], 4.0)
-        t = time.perf_counter() - t0
-        return (2 * 4.0 * L * n + 8 * (L + 1) + 20 * L) / t / 1e9, "the whole step (all 224 segments)"
+        for _ in range(reps):
+            for g in range(L):
+                orc.scale_stats(c[g * n:(g + 1) * n], p[g * n:(g + 1) * n], 4.0)
+        t = (time.perf_counter() - t0) / reps
+        return (2 * 4.0 * L * n + 8 * (L + 1) + 20 * L) / t / 1e9, "the whole step (all 224 segments), mean of 20"
     # kv
     B, H, S, Dh = 32, 32, 8192, 128
-    k = inputs.bf16_bits(inputs.normal_bf16((1, 2, S, Dh), 1.0, seed=seed))
+    k = inputs.bf16_bits(inputs.normal_bf16((1, 16, S, Dh), 1.0, seed=seed))
     t0 = time.perf_counter()
     q, s = orc.kv_quant(k, 0)
     orc.kv_dequant(q, s, 0)
     t = time.perf_counter() - t0
-    per_slice = t / 2
+    per_slice = t / 16
     n = B * H * S * Dh
     full = per_slice * B * H * 2
-    return 2 * (3.0 * n) * 2 / full / 1e9, "2 of the 2048 (b,h) slices of K/V quantized and dequantized; scaled"
+    return 2 * (3.0 * n) * 2 / full / 1e9, "16 of the 2048 (b,h) slices of K/V quantized and dequantized; scaled"
 
 
 # -------------------------------------------------------------------- main --
@@ -657,18 +691,22 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
+        # one untimed sample (the CPU oracle needs no more warm-up), then as many
+        # timed samples as --steps asks for within a ~2.5 minute budget
         vals = []
         desc = ""
-        for _ in range(warmup):
-            cpu_sample(args.workload)
-        for i in range(steps if args.steps is not None else 3):
+        t0 = time.perf_counter()
+        cpu_sample(args.workload)
+        per = max(time.perf_counter() - t0, 1e-3)
+        n = max(1, min(steps if args.steps is not None else 3, int(150.0 / per)))
+        for i in range(n):
             v, desc = cpu_sample(args.workload, seed=i)
             vals.append(v)
         v = statistics.mean(vals)
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
-                "steps": len(vals), "warmup": warmup, "higher_is_better": True, "scaling": "weak",
+                "steps": len(vals), "warmup": 1, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64 sums / fp32 scales (CPU oracle)", "data": "synthetic",
-                "config": {"workload": args.workload},
+                "config": config_of(args.workload),
                 "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle", "sample": desc},
                 "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
