@@ -580,6 +580,15 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     if (warp == 4 && lane == 0) {
                         if (wait_bar(part_bar, 0u, abort_flag, kErrSplit)) st_release_u32(flag, epoch);
                     }
+                } else if (wi.half == 1) {
+                    // consumed: once every epilogue warp has seen the flag and read its
+                    // share, clear it, so the workspace leaves this launch as it came
+                    // (a replayed CUDA graph reuses the epoch it was captured with)
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(part_bar);
+                    if (warp == 4 && lane == 0) {
+                        if (wait_bar(part_bar, 0u, abort_flag, kErrSplit)) st_release_u32(flag, 0u);
+                    }
                 }
             } else {
                 // fp32 accumulator of this thread's row, 128 columns as 64 packed pairs

@@ -207,9 +207,11 @@ FP8Q_API fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows
  *       long K) has each tile computed as two K halves on two CTA pairs, the
  *       first half handing its fp32 partial to the second through the
  *       workspace (TENSOR and ROW modes, M > 128).  The
- *       workspace must be zero-filled when first allocated; later calls leave
- *       it in a state the next call accepts.  Calls that share a workspace
- *       must not overlap on the device.  A workspace belongs to one device.
+ *       workspace must be zero-filled when first allocated; every call
+ *       leaves it as it found it (its hand-off flags cleared), so the call
+ *       may also be captured in a CUDA graph and replayed.  Calls that share
+ *       a workspace must not overlap on the device.  A workspace belongs to
+ *       one device.
  *   The result is deterministic: a fixed K order per tile and a fixed
  *   summation order for split tiles (second half + first half), so repeated
  *   calls with the same shapes and workspace setting are bit-identical.

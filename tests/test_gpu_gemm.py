@@ -246,3 +246,39 @@ def test_launch_chain_keeps_stream_order(orc):
     torch.cuda.synchronize()
     for j, out in enumerate(outs):
         assert torch.equal(out, refs[j % 2]), j
+
+
+def test_split_k_gemm_replays_in_a_cuda_graph(orc):
+    """A split-K GEMM (the workspace hand-off) captured in a CUDA graph and
+    replayed with new operands copied into the captured buffers: each replay
+    must match the eager call on the same operands (the launch clears its
+    hand-off flags, so a replay, which reuses the captured epoch, never sees
+    the previous replay's flag)."""
+    M, N, K = 512, 520, 1024
+    mode = fp8q.SCALE_ROW
+    ws = fp8q.gemm_workspace(M, N, K, mode)
+    assert ws is not None and ws.numel() > 0
+    ops = [_operands(orc, mode, M, N, K, seed=500 + i) for i in range(3)]
+    A_, da_ = _cuda(ops[0][0]), _cuda(ops[0][1])
+    B_, db_ = _cuda(ops[0][2]), _cuda(ops[0][3])
+    D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    fp8q.gemm(A_, 0, B_, 0, mode, da_, db_, out=D, workspace=ws)   # warm-up outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fp8q.gemm(A_, 0, B_, 0, mode, da_, db_, out=D, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    for rep in range(6):
+        A, da, B, db = ops[rep % 3]
+        A_.copy_(_cuda(A)); da_.copy_(_cuda(da)); B_.copy_(_cuda(B)); db_.copy_(_cuda(db))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = fp8q.gemm(_cuda(A), 0, _cuda(B), 0, mode, _cuda(da), _cuda(db), workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(D, ref), rep
+        oref, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
+        assert_gemm_close(bf16_to_f64(D), oref, mag)
+    del g
