@@ -6,13 +6,15 @@
 // "FP8 三种缩放配方怎么选" (tensorwise and rowwise scaled matmuls);
 // "DeepL押注FP8：大模型训练与推理统一精度实战解析" §2.3 (per-block scales),
 // §2.1 (E5M2 gradients against E4M3 weights), §5.3 (FP8 GEMM results depend
-// on the tiling; this kernel uses one fixed K order and no split-K, so it is
-// deterministic run to run).
+// on the tiling; here every tile has one fixed K order, and a tile split
+// along K sums its parts in one fixed order, so results are deterministic
+// run to run).
 //
 //   D[m, n] = bf16( epilogue( sum_k A[m, k] * B[n, k] ) )
 //   A [M, K], B [N, K]: FP8 codes, K contiguous; fp32 accumulation in TMEM.
 //
-// Design (one CTA per SM, persistent over 128x256 output tiles):
+// Design (one CTA per SM, persistent over 128x256 output tiles; for few
+// tiles, a cluster of CTAs per tile splitting K, see k_gemm_fp8's SPLIT):
 //   warp 0      TMA producer: 128x128 A and 256x128 B tiles (128-byte
 //               swizzle) into a 4-stage shared-memory ring, one mbarrier per
 //               stage carrying the transaction byte count.
@@ -44,6 +46,7 @@
 
 using namespace fp8q;
 using fp8q_host::pdl_launch;
+using fp8q_host::pdl_launch_cluster;
 
 namespace {
 
@@ -55,11 +58,73 @@ constexpr int EPI_WARPS = 8;
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
 constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, acc_full[2], acc_empty[2], drain
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_BARS * 8 + 16;
+// Split-K staging (SPLIT kernels): a CTA's fp32 partial tile, row-major with
+// a 260-float pitch (rows 16 B apart modulo the 32 banks, so the eight lanes
+// of a 16-byte store phase hit distinct banks), over the pipeline stages.
+constexpr int kStagePitch = BN + 4;
+static_assert((size_t)BM * kStagePitch * 4 <= (size_t)STAGES * STAGE_BYTES, "split-K stage exceeds the pipeline");
+constexpr int kMaxSplit = 8;   // K parts per tile (portable cluster size)
 
 enum { kModeTensor = 0, kModeRow = 1, kModeBlock = 2 };
 
-// ------------------------------------------------------------- kernel ----
+// SPLIT reduction: CTA q of the cluster owns float4 column groups
+// [q*64/S, (q+1)*64/S) of the tile; it sums that slice of every CTA's staged
+// partial in rank order (so the result does not depend on timing), applies
+// the output scales and stores bf16.  Threads 0..255 of the epilogue.
 template <int MODE>
+__device__ __forceinline__ void split_reduce_store(const float *stage, int S, int q, int et, int m_blk, int n_blk,
+                                                   int M, int N, const float *__restrict__ sa,
+                                                   const float *__restrict__ sb, __nv_bfloat16 *__restrict__ D,
+                                                   int64_t ldd) {
+    const int rows = min(M - m_blk * BM, BM);
+    const int g0 = q * (BN / 4) / S, g1 = (q + 1) * (BN / 4) / S, G = g1 - g0;
+    const uint32_t base = smem_u32(stage);
+    const float rs = (MODE == kModeTensor) ? __fmul_rn(sa[0], sb[0]) : 0.0f;
+    for (int i = et; i < rows * G; i += EPI_WARPS * 32) {
+        const int row = i / G, g = g0 + i % G;
+        const int n = n_blk * BN + g * 4;
+        if (n >= N) continue;   // N % 8 == 0: a group is wholly inside or outside
+        const uint32_t off = base + (uint32_t)(row * kStagePitch + g * 4) * 4u;
+        float4 p[kMaxSplit];
+#pragma unroll
+        for (int r = 0; r < kMaxSplit; ++r)
+            if (r < S) p[r] = ld_dsmem_f4(mapa_shared(off, (uint32_t)r));
+        float4 v = p[0];
+#pragma unroll
+        for (int r = 1; r < kMaxSplit; ++r) {
+            if (r < S) {
+                v.x = v.x + p[r].x;
+                v.y = v.y + p[r].y;
+                v.z = v.z + p[r].z;
+                v.w = v.w + p[r].w;
+            }
+        }
+        const int64_t m = (int64_t)m_blk * BM + row;
+        if (MODE == kModeRow) {
+            const float a = sa[m];
+            v.x = v.x * (a * sb[n + 0]);
+            v.y = v.y * (a * sb[n + 1]);
+            v.z = v.z * (a * sb[n + 2]);
+            v.w = v.w * (a * sb[n + 3]);
+        } else if (MODE == kModeTensor) {
+            v.x = v.x * rs;
+            v.y = v.y * rs;
+            v.z = v.z * rs;
+            v.w = v.w * rs;
+        }
+        uint2 o;
+        o.x = pack_bf16x2(v.x, v.y);
+        o.y = pack_bf16x2(v.z, v.w);
+        *reinterpret_cast<uint2 *>(D + m * ldd + n) = o;
+    }
+}
+
+// ------------------------------------------------------------- kernel ----
+// SPLIT: launched in clusters of S CTAs (S chosen at launch); the cluster
+// computes one output tile, CTA q accumulating K blocks [q*nk/S, (q+1)*nk/S),
+// and the K parts are summed through distributed shared memory
+// (split_reduce_store).  Otherwise the grid is persistent over whole tiles.
+template <int MODE, bool SPLIT>
 __global__ void __launch_bounds__(THREADS, 1)
 k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
            int K, uint32_t idesc, const float *__restrict__ sa, const float *__restrict__ sb,
@@ -74,6 +139,12 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
     const int num_tiles = num_m * num_n;
     const int nk = (K + BK - 1) / BK;
+    const int S = SPLIT ? (int)cluster_size() : 1;
+    const int q = SPLIT ? (int)cluster_rank() : 0;
+    const int t_first = SPLIT ? (int)blockIdx.x / S : (int)blockIdx.x;
+    const int t_step = SPLIT ? num_tiles : (int)gridDim.x;   // SPLIT: exactly one tile per CTA
+    const int k0 = (int)((int64_t)q * nk / S), k1 = (int)((int64_t)(q + 1) * nk / S);
+    float *stage = reinterpret_cast<float *>(smem);
 
     auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
     auto empty_bar = [&](int s) { return smem_u32(&bars[STAGES + s]); };
@@ -116,9 +187,9 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int tile = t_first; ok && tile < num_tiles; tile += t_step) {
                 const int m_blk = tile % num_m, n_blk = tile / num_m;
-                for (int kc = 0; kc < nk; ++kc, ++it) {
+                for (int kc = k0; kc < k1; ++kc, ++it) {
                     const int stage = it % STAGES;
                     const uint32_t round = it / STAGES;
                     if (!wait_bar(empty_bar(stage), (round & 1u) ^ 1u, abort_flag, kErrProducer)) {
@@ -143,7 +214,7 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         if (lane == 0) {
             uint32_t it = 0, lt = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++lt) {
+            for (int tile = t_first; ok && tile < num_tiles; tile += t_step, ++lt) {
                 uint32_t d_tmem = tmem;
                 if (MODE != kModeBlock) {
                     const uint32_t ab = lt & 1u, use = lt >> 1;
@@ -151,7 +222,7 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     tc_fence_after();
                     d_tmem = tmem + ab * BN;
                 }
-                for (int kc = 0; kc < nk; ++kc, ++it) {
+                for (int kc = k0; kc < k1; ++kc, ++it) {
                     const int stage = it % STAGES;
                     const uint32_t round = it / STAGES;
                     if (MODE == kModeBlock) {
@@ -167,7 +238,7 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) {
                         // +32 bytes along K inside the swizzled 128-byte row = +2 in the address field
-                        const uint32_t acc = (MODE == kModeBlock) ? (k > 0) : (kc > 0 || k > 0);
+                        const uint32_t acc = (MODE == kModeBlock) ? (k > 0) : (kc > k0 || k > 0);
                         tc_mma(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, acc);
                     }
                     tc_commit(empty_bar(stage));
@@ -188,9 +259,11 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
         uint32_t it = 0, lt = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++lt) {
+        for (int tile = t_first; ok && tile < num_tiles; tile += t_step, ++lt) {
             const int m_blk = tile % num_m, n_blk = tile / num_m;
             const int m = m_blk * BM + row_in_tile;
+            // SPLIT: rows of this tile to stage (the rest lie beyond M)
+            const bool stage_row = SPLIT && row_in_tile < M - m_blk * BM;
             const int n_base = n_blk * BN + ch * 128;
             __nv_bfloat16 *drow = D + (int64_t)m * ldd;
             if (MODE != kModeBlock) {
@@ -198,34 +271,59 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 float rs;
                 if (MODE == kModeRow) rs = (m < M) ? sa[m] : 0.0f;
                 else rs = __fmul_rn(sa[0], sb[0]);
+                // column scales (lane j: column n_base + 32c + j), fetched before the wait
+                float cbs[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int col = n_base + c * 32 + lane;
+                    cbs[c] = (MODE == kModeRow && col < N) ? sb[col] : 0.0f;
+                }
                 bool w = true;
                 if (lane == 0) w = wait_bar(accf_bar(ab), use & 1u, abort_flag, kErrEpilogue);
                 w = __shfl_sync(0xFFFFFFFFu, w, 0);
                 if (!w) break;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + ab * BN + ch * 128 + c * 32, v);
-                    const int col0 = n_base + c * 32;
-                    if (MODE == kModeRow) {
-                        const float cb = (col0 + lane < N) ? sb[col0 + lane] : 0.0f;
+                // two 32-column chunks per TMEM round trip
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = v[j] * (rs * __shfl_sync(0xFFFFFFFFu, cb, j));
-                    } else {
+                for (int c2 = 0; c2 < 4; c2 += 2) {
+                    uint32_t r[64];
+                    tmem_ld32_async(tmem + lane_base + ab * BN + ch * 128 + c2 * 32, r);
+                    tmem_ld32_async(tmem + lane_base + ab * BN + ch * 128 + c2 * 32 + 32, r + 32);
+                    tmem_wait64(r);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
-                    }
-                    if (m < M) {
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = c2 + cc;
+                        float v[32];
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            if (col0 + g * 8 < N) {
-                                uint4 o;
-                                o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-                                o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-                                o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-                                o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
-                                *reinterpret_cast<uint4 *>(drow + col0 + g * 8) = o;
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cc * 32 + j]);
+                        const int col0 = n_base + c * 32;
+                        if constexpr (SPLIT) {   // raw K-part partial to the stage; scaled after the sum
+                            if (stage_row) {
+                                float4 *dst = reinterpret_cast<float4 *>(stage + row_in_tile * kStagePitch + ch * 128 + c * 32);
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                            }
+                            continue;
+                        }
+                        if (MODE == kModeRow) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = v[j] * (rs * __shfl_sync(0xFFFFFFFFu, cbs[c], j));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
+                        }
+                        if (m < M) {
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                if (col0 + g * 8 < N) {
+                                    uint4 o;
+                                    o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+                                    o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+                                    o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+                                    o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+                                    *reinterpret_cast<uint4 *>(drow + col0 + g * 8) = o;
+                                }
                             }
                         }
                     }
@@ -240,9 +338,9 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 const int nkb_b = nk;                     // K blocks per row of sb
                 const int nb = n_base / 128;              // this half's 128-row block of B
                 const bool nb_ok = n_base < N;
-                float a_next = (m < M) ? sa[m] : 0.0f;
-                float b_next = nb_ok ? sb[(int64_t)nb * nkb_b] : 0.0f;
-                for (int kc = 0; kc < nk; ++kc, ++it) {
+                float a_next = (m < M) ? sa[(int64_t)k0 * M + m] : 0.0f;
+                float b_next = nb_ok ? sb[(int64_t)nb * nkb_b + k0] : 0.0f;
+                for (int kc = k0; kc < k1; ++kc, ++it) {
                     const uint32_t pb = it & 1u, use = it >> 1;
                     const float sc = __fmul_rn(a_next, b_next);
                     bool w = true;
@@ -258,7 +356,7 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(acce_bar(pb));
-                            if (kc + 1 < nk) {   // next block's scales, after the release (see the pair kernel)
+                            if (kc + 1 < k1) {   // next block's scales, after the release (see the pair kernel)
                                 a_next = (m < M) ? sa[(int64_t)(kc + 1) * M + m] : 0.0f;
                                 b_next = nb_ok ? sb[(int64_t)nb * nkb_b + kc + 1] : 0.0f;
                             }
@@ -268,6 +366,15 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     }
                 }
                 if (!ok) break;
+                if constexpr (SPLIT) {   // this K part's promoted sum to the stage
+                    if (stage_row) {
+                        float4 *dst = reinterpret_cast<float4 *>(stage + row_in_tile * kStagePitch + ch * 128);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+                    }
+                    continue;
+                }
                 if (m < M) {
 #pragma unroll
                     for (int g = 0; g < 16; ++g) {
@@ -286,6 +393,17 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         }
     }
 
+    if constexpr (SPLIT) {
+        // Every thread of the cluster takes both barriers, on the error paths
+        // too (a CTA's waits are all bounded, so each one gets here).
+        __syncwarp();
+        cluster_sync_all();   // every CTA has staged its K part
+        if (warp >= 2)
+            split_reduce_store<MODE>(stage, S, q, (int)threadIdx.x - 64, t_first % num_m, t_first / num_m, M, N, sa,
+                                     sb, D, ldd);
+        __syncwarp();         // the barrier below is warp-aligned
+        cluster_sync_all();   // no CTA leaves while a peer may still read its stage
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -512,6 +630,14 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 float rs;
                 if (MODE == kModeRow) rs = m_ok ? sa[m] : 0.0f;
                 else rs = __fmul_rn(sa[wi.e], sb[wi.e]);
+                // this warp's column scales (lane j holds column n_base + 32c + j),
+                // fetched while the accumulator is still being computed
+                float cbs[HALF / 32];
+#pragma unroll
+                for (int c = 0; c < HALF / 32; ++c) {
+                    const int col = n_base + c * 32 + lane;
+                    cbs[c] = (MODE == kModeRow && col < N) ? sbe[col] : 0.0f;
+                }
                 bool w = true;
                 if (lane == 0) w = wait_bar(accf_bar(ab), use & 1u, abort_flag, kErrEpilogue);
                 w = __shfl_sync(0xFFFFFFFFu, w, 0);
@@ -532,40 +658,51 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         (void)ld_acquire_u32(flag);   // acquire on every lane
                     }
                 }
-#pragma unroll 1
-                for (int c = 0; c < HALF / 32; ++c) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + ab * BN + ch * HALF + c * 32, v);
-                    const int col0 = n_base + c * 32;
-                    if (wi.half == 0) {   // first half: store the raw fp32 partial, no output
-                        float *pc = part + (size_t)(ch * HALF + c * 32) * 128;
+                // two 32-column chunks per TMEM round trip (unrolled: the scale
+                // array is indexed with constants only)
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) pc[(size_t)j * 128] = v[j];
-                        continue;
-                    }
-                    if (wi.half == 1) {   // second half: add the first half's partial (fixed order)
-                        const float *pc = part + (size_t)(ch * HALF + c * 32) * 128;
+                for (int c2 = 0; c2 < HALF / 32; c2 += 2) {
+                    uint32_t r[64];
+                    tmem_ld32_async(tmem + lane_base + ab * BN + ch * HALF + c2 * 32, r);
+                    tmem_ld32_async(tmem + lane_base + ab * BN + ch * HALF + c2 * 32 + 32, r + 32);
+                    tmem_wait64(r);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = v[j] + pc[(size_t)j * 128];
-                    }
-                    if (MODE == kModeRow) {
-                        const float cb = (col0 + lane < N) ? sbe[col0 + lane] : 0.0f;
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = c2 + cc;
+                        float v[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = v[j] * (rs * __shfl_sync(0xFFFFFFFFu, cb, j));
-                    } else {
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cc * 32 + j]);
+                        const int col0 = n_base + c * 32;
+                        if (wi.half == 0) {   // first half: store the raw fp32 partial, no output
+                            float *pc = part + (size_t)(ch * HALF + c * 32) * 128;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
-                    }
-                    if (m_ok) {
+                            for (int j = 0; j < 32; ++j) pc[(size_t)j * 128] = v[j];
+                            continue;
+                        }
+                        if (wi.half == 1) {   // second half: add the first half's partial (fixed order)
+                            const float *pc = part + (size_t)(ch * HALF + c * 32) * 128;
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            if (col0 + g * 8 < N) {
-                                uint4 o;
-                                o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-                                o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-                                o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-                                o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
-                                *reinterpret_cast<uint4 *>(drow + col0 + g * 8) = o;
+                            for (int j = 0; j < 32; ++j) v[j] = v[j] + pc[(size_t)j * 128];
+                        }
+                        if (MODE == kModeRow) {
+                            const float cb = cbs[c];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = v[j] * (rs * __shfl_sync(0xFFFFFFFFu, cb, j));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
+                        }
+                        if (m_ok) {
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                if (col0 + g * 8 < N) {
+                                    uint4 o;
+                                    o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+                                    o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+                                    o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+                                    o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+                                    *reinterpret_cast<uint4 *>(drow + col0 + g * 8) = o;
+                                }
                             }
                         }
                     }
@@ -675,19 +812,85 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
+// Per device: the 1-SM kernels' shared-memory opt-in done, and how many
+// split-K clusters of each size fit at once (0 = not asked yet, -1 = none).
+template <int MODE>
+struct OneSmState {
+    std::mutex mu;
+    bool attr_done[64] = {};
+    int cap[64][kMaxSplit + 1] = {};
+};
+template <int MODE>
+OneSmState<MODE> &one_sm_state() {
+    static OneSmState<MODE> st;
+    return st;
+}
+
+template <int MODE>
+cudaError_t one_sm_prepare(int dev) {
+    OneSmState<MODE> &g = one_sm_state<MODE>();
+    std::lock_guard<std::mutex> lk(g.mu);
+    if (g.attr_done[dev]) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_fp8<MODE, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_gemm_fp8<MODE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e == cudaSuccess) g.attr_done[dev] = true;
+    return e;
+}
+
+template <int MODE>
+int split_cluster_capacity(int dev, int S) {
+    OneSmState<MODE> &g = one_sm_state<MODE>();
+    std::lock_guard<std::mutex> lk(g.mu);
+    if (g.cap[dev][S] != 0) return g.cap[dev][S];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S * 16);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = S;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_fp8<MODE, true>, &cfg) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        n = -1;
+    }
+    g.cap[dev][S] = n;
+    return n;
+}
+
+// K parts per tile for the 1-SM kernel.  A problem of fewer tiles than half
+// the SMs leaves most tensor cores idle, so each tile is shared by a cluster
+// of S CTAs: the largest S (at most 8, with at least two K blocks per part)
+// for which every cluster is resident at once.  1 = no split.
+template <int MODE>
+int one_sm_split(int dev, int sms, int tiles, int nk) {
+    if (tiles * 2 > sms) return 1;
+    for (int S = std::min(kMaxSplit, nk / 2); S >= 2; --S)
+        if (tiles * S <= sms && split_cluster_capacity<MODE>(dev, S) >= tiles) return S;
+    return 1;
+}
+
 template <int MODE>
 cudaError_t launch_gemm(cudaStream_t st, int sms, const CUtensorMap &ta, const CUtensorMap &tb, int M, int N, int K,
                         uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd) {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(k_gemm_fp8<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    });
-    if (attr_err != cudaSuccess) return attr_err;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if ((e = one_sm_prepare<MODE>(dev)) != cudaSuccess) return e;
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int S = one_sm_split<MODE>(dev, sms, tiles, (K + BK - 1) / BK);
+    if (S > 1)
+        return pdl_launch_cluster(k_gemm_fp8<MODE, true>, dim3(tiles * S), dim3(THREADS), SMEM_BYTES, st, (unsigned)S,
+                                  ta, tb, M, N, K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D), ldd);
     const int grid = std::max(1, std::min(tiles, sms));
-    return pdl_launch(k_gemm_fp8<MODE>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, ta, tb, M, N, K, idesc, sa, sb,
-                      static_cast<__nv_bfloat16 *>(D), ldd);
+    return pdl_launch(k_gemm_fp8<MODE, false>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, ta, tb, M, N, K, idesc, sa,
+                      sb, static_cast<__nv_bfloat16 *>(D), ldd);
 }
 
 // Pairs of the 2-SM kernel that fit on the device at once (cached per device).

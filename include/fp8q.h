@@ -212,9 +212,17 @@ FP8Q_API fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows
  *       may also be captured in a CUDA graph and replayed.  Calls that share
  *       a workspace must not overlap on the device.  A workspace belongs to
  *       one device.
+ *   M <= 128 (decode-like shapes) needs no workspace for its split: when
+ *   the 128 x 256 tiles fill at most half of the SMs, each tile is computed
+ *   by a thread-block cluster of S = 2..8 CTAs, CTA q accumulating K blocks
+ *   [q*nk/S, (q+1)*nk/S) (nk = ceil(K/128)), and the partial tiles are summed
+ *   through distributed shared memory in rank order (all three modes).  S is
+ *   the largest value whose clusters are all resident at once, with at least
+ *   two K blocks per part.
  *   The result is deterministic: a fixed K order per tile and a fixed
- *   summation order for split tiles (second half + first half), so repeated
- *   calls with the same shapes and workspace setting are bit-identical.
+ *   summation order for split tiles (second half + first half; cluster ranks
+ *   in order), so repeated calls with the same shapes and workspace setting
+ *   on the same device are bit-identical.
  *   Shapes: M, N, K >= 0; K % 16 == 0; N % 8 == 0; ldd % 8 == 0, ldd >= N.
  *   K == 0 writes zeros.  workspace 16-byte aligned.
  */

@@ -282,3 +282,59 @@ def test_split_k_gemm_replays_in_a_cuda_graph(orc):
         oref, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
         assert_gemm_close(bf16_to_f64(D), oref, mag)
     del g
+
+
+# ------------------------------------ few-row GEMMs: K split over a cluster --
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("shape", [(1, 4096, 4096), (17, 2048, 2048), (100, 776, 1424), (64, 264, 528),
+                                   (128, 11008, 1024)])
+def test_gemm_few_rows_cluster_split_full_compare(orc, mode, shape):
+    """M <= 128 with few output tiles: each 128 x 256 tile is shared by a
+    cluster of CTAs, each accumulating a K range, and the partial tiles are
+    summed through distributed shared memory in rank order.  Ragged M, N and
+    K (a last K block of 16), 2 to 8 K parts; full compare with the oracle and
+    bit-identical repeats."""
+    M, N, K = shape
+    A, da, B, db = _operands(orc, mode, M, N, K, seed=M + 5 * N + K)
+    A_, B_, da_, db_ = _cuda(A), _cuda(B), _cuda(da), _cuda(db)
+    D = fp8q.gemm(A_, 0, B_, 0, mode, da_, db_)
+    ref, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
+    assert_gemm_close(bf16_to_f64(D), ref, mag)
+    for _ in range(2):
+        assert torch.equal(fp8q.gemm(A_, 0, B_, 0, mode, da_, db_), D)
+
+
+def test_gemm_few_rows_takes_the_cluster_split_and_replays_in_a_graph(orc):
+    """The decode-shaped GEMM (16 x 4096 x 4096) launches the cluster
+    split-K kernel (checked by kernel name in the profiler's trace), and the
+    launch, captured in a CUDA graph, replays to the eager result on new
+    operands copied into the captured buffers."""
+    from torch.profiler import ProfilerActivity, profile
+    M, N, K = 16, 4096, 4096
+    mode = fp8q.SCALE_ROW
+    ops = [_operands(orc, mode, M, N, K, seed=700 + i) for i in range(2)]
+    A_, da_, B_, db_ = (_cuda(x) for x in ops[0])
+    D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fp8q.gemm(A_, 0, B_, 0, mode, da_, db_, out=D)
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if "k_gemm_fp8" in e.name]
+    # k_gemm_fp8<MODE = 1, SPLIT = true>, demangled or not
+    assert names and all("k_gemm_fp8<1, true>" in n or "ILi1ELb1E" in n for n in names), names
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fp8q.gemm(A_, 0, B_, 0, mode, da_, db_, out=D)
+    torch.cuda.current_stream().wait_stream(s)
+    for rep in range(4):
+        A, da, B, db = ops[rep % 2]
+        A_.copy_(_cuda(A)); da_.copy_(_cuda(da)); B_.copy_(_cuda(B)); db_.copy_(_cuda(db))
+        g.replay()
+        torch.cuda.synchronize()
+        ref, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
+        assert_gemm_close(bf16_to_f64(D), ref, mag)
+        assert torch.equal(D, fp8q.gemm(_cuda(A), 0, _cuda(B), 0, mode, _cuda(da), _cuda(db))), rep
+    del g
