@@ -57,7 +57,9 @@ constexpr int STAGE_BYTES = A_TILE + B_TILE;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
 constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, acc_full[2], acc_empty[2], drain
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + NUM_BARS * 8 + 16;
+// after the pipeline and the barriers: one store_rows_coalesced buffer per epilogue warp
+constexpr size_t EPI_OFF = ((size_t)STAGES * STAGE_BYTES + NUM_BARS * 8 + 16 + 15) & ~(size_t)15;
+constexpr size_t SMEM_BYTES = 1024 + EPI_OFF + (size_t)EPI_WARPS * kEpiBufBytes;
 // Split-K staging (SPLIT kernels): a CTA's fp32 partial tile, row-major with
 // a 260-float pitch (rows 16 B apart modulo the 32 banks, so the eight lanes
 // of a 16-byte store phase hit distinct banks), over the pipeline stages.
@@ -265,7 +267,6 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             // SPLIT: rows of this tile to stage (the rest lie beyond M)
             const bool stage_row = SPLIT && row_in_tile < M - m_blk * BM;
             const int n_base = n_blk * BN + ch * 128;
-            __nv_bfloat16 *drow = D + (int64_t)m * ldd;
             if (MODE != kModeBlock) {
                 const uint32_t ab = lt & 1u, use = lt >> 1;
                 float rs;
@@ -283,20 +284,28 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 w = __shfl_sync(0xFFFFFFFFu, w, 0);
                 if (!w) break;
                 tc_fence_after();
-                // two 32-column chunks per TMEM round trip
+                // two 32-column chunks per TMEM round trip; the accumulator buffer is
+                // released once its last columns are in registers
+                uint8_t *ebuf = smem + EPI_OFF + (size_t)(warp - 2) * kEpiBufBytes;
+                const int64_t row0 = (int64_t)m_blk * BM + sp * 32;
 #pragma unroll
                 for (int c2 = 0; c2 < 4; c2 += 2) {
                     uint32_t r[64];
                     tmem_ld32_async(tmem + lane_base + ab * BN + ch * 128 + c2 * 32, r);
                     tmem_ld32_async(tmem + lane_base + ab * BN + ch * 128 + c2 * 32 + 32, r + 32);
                     tmem_wait64(r);
+                    if (c2 == 2) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acce_bar(ab));
+                    }
+                    uint32_t pk[32];
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const int c = c2 + cc;
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cc * 32 + j]);
-                        const int col0 = n_base + c * 32;
                         if constexpr (SPLIT) {   // raw K-part partial to the stage; scaled after the sum
                             if (stage_row) {
                                 float4 *dst = reinterpret_cast<float4 *>(stage + row_in_tile * kStagePitch + ch * 128 + c * 32);
@@ -313,24 +322,11 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 #pragma unroll
                             for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
                         }
-                        if (m < M) {
 #pragma unroll
-                            for (int g = 0; g < 4; ++g) {
-                                if (col0 + g * 8 < N) {
-                                    uint4 o;
-                                    o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-                                    o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-                                    o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-                                    o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
-                                    *reinterpret_cast<uint4 *>(drow + col0 + g * 8) = o;
-                                }
-                            }
-                        }
+                        for (int j = 0; j < 16; ++j) pk[cc * 16 + j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
                     }
+                    if constexpr (!SPLIT) store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, M, n_base + c2 * 32, N);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acce_bar(ab));
             } else {
                 float acc[128];
 #pragma unroll
@@ -375,19 +371,13 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                     }
                     continue;
                 }
-                if (m < M) {
+                uint8_t *ebuf = smem + EPI_OFF + (size_t)(warp - 2) * kEpiBufBytes;
 #pragma unroll
-                    for (int g = 0; g < 16; ++g) {
-                        const int col = n_base + g * 8;
-                        if (col < N) {
-                            uint4 o;
-                            o.x = pack_bf16x2(acc[g * 8 + 0], acc[g * 8 + 1]);
-                            o.y = pack_bf16x2(acc[g * 8 + 2], acc[g * 8 + 3]);
-                            o.z = pack_bf16x2(acc[g * 8 + 4], acc[g * 8 + 5]);
-                            o.w = pack_bf16x2(acc[g * 8 + 6], acc[g * 8 + 7]);
-                            *reinterpret_cast<uint4 *>(drow + col) = o;
-                        }
-                    }
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(acc[h2 * 64 + 2 * j], acc[h2 * 64 + 2 * j + 1]);
+                    store_rows_coalesced(ebuf, pk, lane, D, ldd, (int64_t)m_blk * BM + sp * 32, M, n_base + h2 * 64, N);
                 }
             }
         }
@@ -623,7 +613,6 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const int64_t m = wi.row0 + wi.m_blk * 256 + (int)rank * 128 + sp * 32 + lane;
             const bool m_ok = m < wi.row_end;
             const int n_base = n_blk * BN + ch * HALF;
-            __nv_bfloat16 *drow = D + m * ldd;
             const float *sbe = sb + (int64_t)wi.e * N;   // group e's column scales (ROW)
             if (MODE != kModeBlock) {
                 const uint32_t ab = lt % NBUF, use = lt / NBUF;
@@ -659,20 +648,28 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     }
                 }
                 // two 32-column chunks per TMEM round trip (unrolled: the scale
-                // array is indexed with constants only)
+                // array is indexed with constants only); the accumulator buffer is
+                // released as soon as its last columns are in registers
+                uint8_t *ebuf = smem + C::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
+                const int64_t row0 = wi.row0 + wi.m_blk * 256 + (int)rank * 128 + sp * 32;
 #pragma unroll
                 for (int c2 = 0; c2 < HALF / 32; c2 += 2) {
                     uint32_t r[64];
                     tmem_ld32_async(tmem + lane_base + ab * BN + ch * HALF + c2 * 32, r);
                     tmem_ld32_async(tmem + lane_base + ab * BN + ch * HALF + c2 * 32 + 32, r + 32);
                     tmem_wait64(r);
+                    if (c2 + 2 == HALF / 32) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(ab), 0));
+                    }
+                    uint32_t pk[32];
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const int c = c2 + cc;
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cc * 32 + j]);
-                        const int col0 = n_base + c * 32;
                         if (wi.half == 0) {   // first half: store the raw fp32 partial, no output
                             float *pc = part + (size_t)(ch * HALF + c * 32) * 128;
 #pragma unroll
@@ -692,24 +689,12 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
                             for (int j = 0; j < 32; ++j) v[j] = v[j] * rs;
                         }
-                        if (m_ok) {
 #pragma unroll
-                            for (int g = 0; g < 4; ++g) {
-                                if (col0 + g * 8 < N) {
-                                    uint4 o;
-                                    o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-                                    o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-                                    o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-                                    o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
-                                    *reinterpret_cast<uint4 *>(drow + col0 + g * 8) = o;
-                                }
-                            }
-                        }
+                        for (int j = 0; j < 16; ++j) pk[cc * 16 + j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
                     }
+                    if (wi.half != 0)
+                        store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, wi.row_end, n_base + c2 * 32, N);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(ab), 0));
                 if (wi.half == 0) {   // publish: every epilogue warp's stores, then the flag
                     __threadfence();
                     __syncwarp();
@@ -785,19 +770,16 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         if (ok && kc + i < nk && !promote(kc + i, as_[i], bs_[i])) ok = false;
                 }
                 if (!ok) break;
-                if (m_ok) {
+                uint8_t *ebuf = smem + C::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
+                const int64_t row0 = wi.row0 + wi.m_blk * 256 + (int)rank * 128 + sp * 32;
 #pragma unroll
-                    for (int g = 0; g < HALF / 8; ++g) {
-                        const int col = n_base + g * 8;
-                        if (col < N) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float((uint32_t)acc[g * 4 + 0]), __uint_as_float((uint32_t)(acc[g * 4 + 0] >> 32)));
-                            o.y = pack_bf16x2(__uint_as_float((uint32_t)acc[g * 4 + 1]), __uint_as_float((uint32_t)(acc[g * 4 + 1] >> 32)));
-                            o.z = pack_bf16x2(__uint_as_float((uint32_t)acc[g * 4 + 2]), __uint_as_float((uint32_t)(acc[g * 4 + 2] >> 32)));
-                            o.w = pack_bf16x2(__uint_as_float((uint32_t)acc[g * 4 + 3]), __uint_as_float((uint32_t)(acc[g * 4 + 3] >> 32)));
-                            *reinterpret_cast<uint4 *>(drow + col) = o;
-                        }
-                    }
+                for (int h2 = 0; h2 < HALF / 64; ++h2) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        pk[j] = pack_bf16x2(__uint_as_float((uint32_t)acc[h2 * 32 + j]),
+                                            __uint_as_float((uint32_t)(acc[h2 * 32 + j] >> 32)));
+                    store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, wi.row_end, n_base + h2 * 64, N);
                 }
             }
         }

@@ -40,7 +40,9 @@ constexpr int STAGE = 2 * HALF_TILE;      // this CTA's A half and B half
 constexpr int STAGES = 6;
 constexpr int NBUF = 2;
 constexpr int NBARS = 2 * STAGES + 2 * NBUF + 1;
-constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + NBARS * 8 + 16;
+// after the pipeline and the barriers: one store_rows_coalesced buffer per epilogue warp
+constexpr size_t EPI_OFF = ((size_t)STAGES * STAGE + NBARS * 8 + 16 + 15) & ~(size_t)15;
+constexpr size_t SMEM = 1024 + EPI_OFF + (size_t)sm2::EPI * kEpiBufBytes;
 }  // namespace wg
 
 // MN-major operand, 128-byte swizzle: 64-element (128-byte) rows, one per
@@ -202,33 +204,30 @@ k_gemm_bf16_wgrad_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             w = __shfl_sync(0xFFFFFFFFu, w, 0);
             if (!w) break;
             tc_fence_after();
-            float *drow = D + m * ldd;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float v[32];
-                tmem_ld32(tmem + lane_base + ab * 256 + ch * 128 + c * 32, v);
-                const int col0 = n_base + c * 32;
-                if (m < M) {
+            // two 32-column chunks per TMEM round trip; the buffer is released
+            // once its last columns are in registers
+            uint8_t *ebuf = smem + wg::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        if (col0 + g * 4 < N) {
-                            float4 o = make_float4(v[g * 4], v[g * 4 + 1], v[g * 4 + 2], v[g * 4 + 3]);
-                            float4 *dst = reinterpret_cast<float4 *>(drow + col0 + g * 4);
-                            if (accumulate) {
-                                const float4 p = *dst;
-                                o.x = p.x + o.x;
-                                o.y = p.y + o.y;
-                                o.z = p.z + o.z;
-                                o.w = p.w + o.w;
-                            }
-                            *dst = o;
-                        }
-                    }
+            for (int c2 = 0; c2 < 4; c2 += 2) {
+                uint32_t r[64];
+                tmem_ld32_async(tmem + lane_base + ab * 256 + ch * 128 + c2 * 32, r);
+                tmem_ld32_async(tmem + lane_base + ab * 256 + ch * 128 + c2 * 32 + 32, r + 32);
+                tmem_wait64(r);
+                if (c2 == 2) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(ab), 0));
+                }
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) pk[j] = r[cc * 32 + j];
+                    const int col0 = n_base + (c2 + cc) * 32;
+                    if (accumulate) store_rows_coalesced<float, true>(ebuf, pk, lane, D, ldd, m - lane, M, col0, N);
+                    else store_rows_coalesced<float, false>(ebuf, pk, lane, D, ldd, m - lane, M, col0, N);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(ab), 0));
         }
     }
 

@@ -51,7 +51,9 @@ constexpr int AB_STAGE = A_TILE + 128 * BK;       // this CTA's 128 rows of A an
 constexpr int SF_STAGE = SFA_BYTES + SFB_BYTES;
 constexpr int STAGES = 6;
 constexpr int NBARS = 2 * STAGES + 3;             // full, empty, acc full, acc empty, drain
-constexpr size_t SMEM = 1024 + (size_t)STAGES * (AB_STAGE + SF_STAGE) + NBARS * 8 + 16;
+// after the pipeline and the barriers: one store_rows_coalesced buffer per epilogue warp
+constexpr size_t EPI_OFF = ((size_t)STAGES * (AB_STAGE + SF_STAGE) + NBARS * 8 + 16 + 15) & ~(size_t)15;
+constexpr size_t SMEM = 1024 + EPI_OFF + (size_t)sm2::EPI * kEpiBufBytes;
 constexpr uint32_t SFA_COL = 256, SFB_COL = 260;  // TMEM columns after the accumulator
 static_assert(SMEM <= 232448, "shared memory per block");
 }  // namespace mx
@@ -241,21 +243,14 @@ k_gemm_mx_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar, 0));
-            if (m < M) {
-                __nv_bfloat16 *drow = D + m * ldd;
+            uint8_t *ebuf = smem + mx::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
 #pragma unroll
-                for (int g = 0; g < 16; ++g) {
-                    const int col = n_base + g * 8;
-                    const uint32_t *r = (g < 8) ? (r0 + g * 8) : (r1 + (g - 8) * 8);
-                    if (col < N) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                        o.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                        o.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                        o.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                        *reinterpret_cast<uint4 *>(drow + col) = o;
-                    }
-                }
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const uint32_t *r = h2 ? r1 : r0;
+                uint32_t pk[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                store_rows_coalesced(ebuf, pk, lane, D, ldd, m - lane, M, n_base + h2 * 64, N);
             }
         }
     }

@@ -208,6 +208,61 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t addr) {
     return d;
 }
 
+// Coalesced epilogue stores.  After tcgen05.ld a lane holds one output row,
+// so storing straight from registers makes every 16-byte store instruction
+// touch 32 rows (32 cache lines).  Instead a warp passes 128 bytes of each of
+// its 32 rows (64 bf16 or 32 fp32 columns, pk[] = the lane's row) through a
+// 16-row shared buffer in two passes: each lane of the half-warp writes its
+// row, then every lane reads 16 bytes, so that one global store instruction
+// writes 4 rows x 128 contiguous bytes (4 lines).  The 144-byte row pitch
+// keeps both shared accesses free of bank conflicts.  ACC (fp32 only) adds
+// the values already in D.  Warp-collective: all 32 lanes call it together.
+constexpr int kEpiRowPitch = 144;
+constexpr int kEpiBufBytes = 16 * kEpiRowPitch;   // per epilogue warp
+template <typename T, bool ACC = false>
+__device__ __forceinline__ void store_rows_coalesced(uint8_t *buf, const uint32_t (&pk)[32], int lane,
+                                                     T *__restrict__ D, int64_t ldd, int64_t row0, int64_t row_end,
+                                                     int col0, int N) {
+    constexpr int kPer16 = 16 / (int)sizeof(T);   // columns per 16 bytes
+    static_assert(!ACC || sizeof(T) == 4, "accumulation is for fp32 outputs");
+    const uint32_t sb = smem_u32(buf);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if ((lane >> 4) == h) {
+            const uint32_t dst = sb + (uint32_t)(lane & 15) * kEpiRowPitch;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16u * j), "r"(pk[4 * j]),
+                             "r"(pk[4 * j + 1]), "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
+                             : "memory");
+        }
+        __syncwarp();
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int rl = it * 4 + (lane >> 3), ck = lane & 7;
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(sb + (uint32_t)(rl * kEpiRowPitch + ck * 16))
+                         : "memory");
+            const int64_t row = row0 + h * 16 + rl;
+            const int col = col0 + ck * kPer16;
+            if (row < row_end && col < N) {
+                uint4 *dst = reinterpret_cast<uint4 *>(D + row * ldd + col);
+                if constexpr (ACC) {
+                    const float4 p = *reinterpret_cast<const float4 *>(dst);
+                    v.x = __float_as_uint(p.x + __uint_as_float(v.x));
+                    v.y = __float_as_uint(p.y + __uint_as_float(v.y));
+                    v.z = __float_as_uint(p.z + __uint_as_float(v.z));
+                    v.w = __float_as_uint(p.w + __uint_as_float(v.w));
+                }
+                *dst = v;
+            }
+        }
+        __syncwarp();   // the next pass overwrites the buffer
+    }
+}
+
 namespace sm2 {
 constexpr int EPI = 8;                 // epilogue warps 4..11 (warpgroups 1 and 2)
 constexpr int THREADS = 12 * 32;       // warpgroup 0: producer (warp 0), MMA (warp 1), two idle warps
@@ -225,7 +280,9 @@ struct Cfg {
     static constexpr int STAGES = (BN == 256) ? 6 : 8;
     static constexpr int NBUF = 512 / BN;
     static constexpr int NBARS = 2 * STAGES + 2 * NBUF + 2;   // + drain, + split partial written
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + NBARS * 8 + 16;
+    // epilogue store buffers (store_rows_coalesced), one per epilogue warp, 16-byte aligned
+    static constexpr size_t EPI_OFF = ((size_t)STAGES * STAGE + NBARS * 8 + 16 + 15) & ~(size_t)15;
+    static constexpr size_t SMEM = 1024 + EPI_OFF + (size_t)EPI * kEpiBufBytes;
 };
 // Split-K tail workspace: per split tile, per CTA of the pair, a 128 x 256
 // fp32 partial stored column-major (row index fastest, so a warp's lanes write
