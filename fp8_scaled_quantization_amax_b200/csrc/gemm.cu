@@ -857,6 +857,16 @@ int one_sm_split(int dev, int sms, int tiles, int nk) {
     return 1;
 }
 
+// Problems of any M whose 128 x 256 tiles fill at most a quarter of the SMs,
+// with at least 8 K blocks, run on the 1-SM kernel with each tile shared by a
+// cluster of S >= 4 CTAs (S from one_sm_split).  Measured (L2 flushed)
+// against the pair kernel: 256 x 4096 x 4096 19.5 us (pair 22.5),
+// 256 x 4096 x 16384 29.7 us (pair with its workspace split 41.0).
+inline bool one_sm_cluster_split(int64_t M, int64_t N, int64_t K, int sms) {
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    return tiles * 4 <= sms && (K + BK - 1) / BK >= 8;
+}
+
 template <int MODE>
 cudaError_t launch_gemm(cudaStream_t st, int sms, const CUtensorMap &ta, const CUtensorMap &tb, int M, int N, int K,
                         uint32_t idesc, const float *sa, const float *sb, void *D, int64_t ldd) {
@@ -916,12 +926,18 @@ int pair_capacity() {
 // half-empty last wave already runs uncontended and faster than a full one,
 // so the fp32 hand-off did not pay (63.5 vs 61.4 us): the plan splits only
 // single-wave problems.
+// The fp32 hand-off through global memory costs several microseconds, so a
+// pair split pays only for long K: measured on 16 tiles of 256 x 256, K =
+// 4096 (32 K blocks) ran 22.5 us unsplit and 24.6 split, K = 16384 53.2 and
+// 41.0.  Shorter-K problems with few tiles take the cluster split of the
+// 1-SM kernel instead (one_sm_cluster_split below) or run unsplit.
+constexpr int kPairSplitMinKBlocks = 64;
 struct SplitPlan { int full_tiles, units; size_t bytes; };
 SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int cap) {
     const int tiles = (int)(((M + 255) / 256) * ((N + 255) / 256));
     const int nk = (int)((K + BK - 1) / BK);
     const int r = tiles % cap;
-    if (cap <= 0 || nk < 2 || r == 0 || tiles >= cap || 2 * r > cap) return SplitPlan{tiles, 0, 0};
+    if (cap <= 0 || nk < kPairSplitMinKBlocks || r == 0 || tiles >= cap || 2 * r > cap) return SplitPlan{tiles, 0, 0};
     const size_t flags_off = (size_t)r * 2 * sm2::kSplitPartialFloats * sizeof(float);
     return SplitPlan{tiles - r, 2 * r, flags_off + (((size_t)r * 2 * sizeof(uint32_t) + 255) & ~(size_t)255)};
 }
@@ -977,7 +993,7 @@ extern "C" fp8_status fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, f
     int sms;
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
-    if (mode == FP8_SCALE_BLOCK || M <= BM || N == 0 || K == 0) return FP8_OK;
+    if (mode == FP8_SCALE_BLOCK || M <= BM || N == 0 || K == 0 || one_sm_cluster_split(M, N, K, sms)) return FP8_OK;
     const int cap = (mode == FP8_SCALE_TENSOR) ? pair_capacity<kModeTensor, 256>() : pair_capacity<kModeRow, 256>();
     if (cap <= 0) return FP8_ERR_CUDA;
     *bytes = split_plan(M, N, K, cap).bytes;
@@ -1010,8 +1026,10 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
         return cudaMemset2DAsync(D_bf16, (size_t)ldd * 2, 0, (size_t)N * 2, (size_t)M, s) == cudaSuccess ? FP8_OK
                                                                                                        : FP8_ERR_CUDA;
     }
-    // M > 128: a CTA pair per 256-row tile (2-SM MMA); otherwise one CTA per 128-row tile.
-    if (M > BM) {
+    // M > 128: a CTA pair per 256-row tile (2-SM MMA), unless the problem has
+    // so few tiles that the cluster split-K of the 1-SM kernel applies;
+    // otherwise one CTA per 128-row tile.
+    if (M > BM && !one_sm_cluster_split(M, N, K, sms)) {
         CUtensorMap ta, tb;
         if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
         const uint32_t idesc = make_idesc(fa, fb, 256, 256);

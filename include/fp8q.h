@@ -202,9 +202,10 @@ FP8Q_API fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows
  *                an fp32 register accumulator with its two scales).
  *   D  [M, N] bf16 with leading dimension ldd (elements).
  *   workspace / workspace_bytes: optional device scratch (NULL, 0 = none).
- *       With at least fp8_gemm_workspace_size() bytes, a problem whose
- *       256 x 256 tiles fill at most half of the GPU's CTA pairs (few tiles,
- *       long K) has each tile computed as two K halves on two CTA pairs, the
+ *       With at least fp8_gemm_workspace_size() bytes, a long-K problem
+ *       (at least 64 K blocks of 128) whose 256 x 256 tiles fill at most half
+ *       of the GPU's CTA pairs, and that the cluster split below does not
+ *       take, has each tile computed as two K halves on two CTA pairs, the
  *       first half handing its fp32 partial to the second through the
  *       workspace (TENSOR and ROW modes, M > 128).  The
  *       workspace must be zero-filled when first allocated; every call
@@ -212,13 +213,14 @@ FP8Q_API fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows
  *       may also be captured in a CUDA graph and replayed.  Calls that share
  *       a workspace must not overlap on the device.  A workspace belongs to
  *       one device.
- *   M <= 128 (decode-like shapes) needs no workspace for its split: when
- *   the 128 x 256 tiles fill at most half of the SMs, each tile is computed
- *   by a thread-block cluster of S = 2..8 CTAs, CTA q accumulating K blocks
- *   [q*nk/S, (q+1)*nk/S) (nk = ceil(K/128)), and the partial tiles are summed
- *   through distributed shared memory in rank order (all three modes).  S is
- *   the largest value whose clusters are all resident at once, with at least
- *   two K blocks per part.
+ *   Few-tile problems split K without a workspace: when the 128 x 256
+ *   tiles fill at most a quarter of the SMs and K has at least 8 blocks
+ *   (any M), or at most half of them (M <= 128, decode-like shapes), each
+ *   tile is computed by a thread-block cluster of S = 2..8 CTAs, CTA q
+ *   accumulating K blocks [q*nk/S, (q+1)*nk/S) (nk = ceil(K/128)), and the
+ *   partial tiles are summed through distributed shared memory in rank
+ *   order (all three modes).  S is the largest value whose clusters are all
+ *   resident at once, with at least two K blocks per part.
  *   The result is deterministic: a fixed K order per tile and a fixed
  *   summation order for split tiles (second half + first half; cluster ranks
  *   in order), so repeated calls with the same shapes and workspace setting
@@ -293,7 +295,8 @@ FP8Q_API fp8_status fp8_gemm_grouped(const uint8_t *A, fp8_format fa, const uint
 
 /*
  * Bytes of workspace fp8_gemm_scaled can use for this shape on the current
- * device (0: the shape fills whole waves, or the mode takes none).
+ * device (0: no pair split applies -- the shape fills whole waves, K is
+ * short, the cluster split takes it, or the mode takes none).
  */
 FP8Q_API fp8_status fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8_scale_mode mode,
                                             size_t *bytes);

@@ -38,7 +38,7 @@ def _noalloc_via_c_abi(A, fa, B, fb, mode, da, db, D):
     assert st == 0, L.fp8_status_string(st)
 
 
-@pytest.mark.parametrize("shape", [(1024, 1024, 16384), (300, 272, 400), (4096, 4096, 4096)])
+@pytest.mark.parametrize("shape", [(1000, 1288, 8208), (1024, 1024, 16384), (300, 272, 400), (4096, 4096, 4096)])
 def test_noalloc_gemm_matches_workspace_entry_point(orc, shape):
     need_gpu()
     M, N, K = shape
