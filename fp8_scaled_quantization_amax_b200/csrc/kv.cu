@@ -214,13 +214,7 @@ extern "C" fp8_status fp8_kv_quant(const void *kv_bf16, int64_t B, int64_t H, in
     cudaStream_t s = as_stream(stream);
     const int active = fmt == FP8_E4M3 ? max_active_clusters<FP8_E4M3>() : max_active_clusters<FP8_E5M2>();
     if (active <= 0) return FP8_ERR_CUDA;
-    // Slices are dealt to the clusters in turn.  With R = ceil(BH / active)
-    // slices per cluster, the fewest clusters that still need only R keep the
-    // clusters evenly loaded: 1024 slices on 33 resident clusters become 32
-    // clusters x 32 slices, instead of one cluster finishing a 32nd slice
-    // alone after the others are done.
-    const int64_t per_cluster = (BH + active - 1) / active;
-    const int clusters = (int)std::max<int64_t>(1, (BH + per_cluster - 1) / per_cluster);
+    const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(BH, active));
     const dim3 grid(clusters * kClusterCtas);
     if (fmt == FP8_E4M3)
         k_kv_quant<FP8_E4M3><<<grid, kKvThreads, 0, s>>>(static_cast<const uint4 *>(kv_bf16), reinterpret_cast<uint4 *>(q), BH, nunit, scale_inv);
