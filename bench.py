@@ -205,7 +205,8 @@ class Workload:
         self.sa = torch.empty(M, dtype=torch.float32, device=d)
         self.sb = torch.empty(N, dtype=torch.float32, device=d)
         self.D = torch.empty((M, N), dtype=torch.bfloat16, device=d)
-        self.ws = f.gemm_workspace(M, N, K, f.SCALE_ROW, device=d)   # split-K tail of the last wave
+        # the library's split-K workspace, as a caller would pass it (0 bytes, so None, for 4096^3)
+        self.ws = f.gemm_workspace(M, N, K, f.SCALE_ROW, device=d)
         self.flops = 2.0 * M * N * K
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.launches = 2
