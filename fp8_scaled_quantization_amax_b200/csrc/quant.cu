@@ -133,6 +133,78 @@ k_cast_tensor(const uint4 *__restrict__ xv, uint4 *__restrict__ qv, int64_t nuni
     }
 }
 
+// ------------------------------------ small tensors: amax + cast fused --
+// Current scaling of a small tensor (at most kSmallTensor elements) in one
+// launch: a single 1024-thread CTA loads the whole tensor into registers
+// (thread t holds the 8-element vectors t, t + 1024, ..., all loads in
+// flight at once), takes the exact amax (the k_amax arithmetic), derives the
+// scale and casts from the registers (the k_cast_tensor arithmetic), so HBM
+// is read once.  The memset, amax and cast launches of the general path
+// cost more than the work here.  Outputs and counters are the general
+// path's: amax_out = max |x| over the finite elements, nf_ctr += non-finite
+// count, sat_ctr += saturated count.
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallVecs = 8;   // 8-element vectors per thread
+constexpr int64_t kSmallTensor = (int64_t)kSmallThreads * kSmallVecs * 8;
+template <int FMT>
+__global__ void __launch_bounds__(kSmallThreads)
+k_quant_tensor_small(const uint4 *__restrict__ xv, const uint16_t *__restrict__ xs, int64_t n,
+                     uint8_t *__restrict__ q, uint32_t *__restrict__ amax_bits, float *__restrict__ scale_inv_out,
+                     uint32_t *__restrict__ nf_ctr, uint32_t *__restrict__ sat_ctr) {
+    pdl_trigger();
+    pdl_wait();
+    __shared__ uint32_t red[32];
+    constexpr float fm = fmax_of<FMT>();
+    const int tid = threadIdx.x;
+    const int nvec = (int)(n / 8);
+    uint4 v[kSmallVecs];
+#pragma unroll
+    for (int k = 0; k < kSmallVecs; ++k) {
+        const int i = tid + k * kSmallThreads;
+        v[k] = i < nvec ? ld_stream(xv + i) : make_uint4(0, 0, 0, 0);   // zeros do not move the max
+    }
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int k = 0; k < kSmallVecs; ++k) m2 = amax_fast8(m2, v[k]);
+    uint32_t m = amax_fast_final(m2), bad = 0;
+    if (m == 0xFFFFFFFFu) {   // a NaN or Inf among this thread's elements: exact pass
+        m = 0;
+#pragma unroll
+        for (int k = 0; k < kSmallVecs; ++k) m = amax_exact8(m, v[k], bad);
+    }
+    for (int64_t j = (int64_t)nvec * 8 + tid; j < n; j += kSmallThreads) {   // tail (< 8 elements)
+        uint32_t h = xs[j] & 0x7FFFu;
+        if (h < 0x7F80u) m = h > m ? h : m; else ++bad;
+    }
+    m = block_max_u32(m, red);
+    if (nf_ctr) bad = block_sum_u32(bad, red);
+    const float s = scale_from_amax(__uint_as_float(m << 16), fm);
+    if (tid == 0) {
+        *amax_bits = m << 16;
+        *scale_inv_out = __fdiv_rn(1.0f, s);
+        if (nf_ctr && bad) atomicAdd(nf_ctr, bad);
+    }
+    uint32_t sat = 0;
+#pragma unroll
+    for (int k = 0; k < kSmallVecs; ++k) {
+        const int i = tid + k * kSmallThreads;
+        if (i < nvec) {
+            *reinterpret_cast<uint2 *>(q + (int64_t)i * 8) = cast8<FMT>(v[k], s);
+            if (sat_ctr) sat += count_sat8(v[k], s, fm);
+        }
+    }
+    for (int64_t j = (int64_t)nvec * 8 + tid; j < n; j += kSmallThreads) {   // tail, exact and scalar
+        uint32_t h = xs[j];
+        float y = __fmul_rn(__uint_as_float(h << 16), s);
+        q[j] = (uint8_t)(cvt2<FMT>(y, 0.0f) & 0xFFu);
+        if (fabsf(y) > fm) ++sat;
+    }
+    if (sat_ctr) {
+        sat = block_sum_u32(sat, red);
+        if (tid == 0 && sat) atomicAdd(sat_ctr, sat);
+    }
+}
+
 // ---------------------------------------- tensorwise cast with transpose --
 // 64x64 tiles: coalesced 16-byte bf16 loads, the FP8 codes written transposed
 // into shared memory, then coalesced 16-byte stores of the [cols, rows] output.
@@ -671,6 +743,18 @@ extern "C" fp8_status fp8_quantize_tensorwise(const void *x_bf16, int64_t rows, 
     uint32_t *amax_bits = reinterpret_cast<uint32_t *>(amax_out);
     const float *amax_in = nullptr;
     uint32_t *nf_ctr = counts, *sat_ctr = counts ? counts + 1 : nullptr;
+    if (!scale_in && !transpose_out && n > 0 && n <= kSmallTensor) {   // one launch for a small tensor
+        if ((reinterpret_cast<uintptr_t>(amax_out) & 3u) || (counts && (reinterpret_cast<uintptr_t>(counts) & 3u)))
+            return FP8_ERR_ALIGNMENT;
+        const uint16_t *xs = static_cast<const uint16_t *>(x_bf16);
+        const uint4 *xv = static_cast<const uint4 *>(x_bf16);
+        cudaError_t e = (fmt == FP8_E4M3)
+            ? pdl_launch(k_quant_tensor_small<FP8_E4M3>, dim3(1), dim3(kSmallThreads), 0, s, xv, xs, n, q,
+                         amax_bits, scale_inv_out, nf_ctr, sat_ctr)
+            : pdl_launch(k_quant_tensor_small<FP8_E5M2>, dim3(1), dim3(kSmallThreads), 0, s, xv, xs, n, q,
+                         amax_bits, scale_inv_out, nf_ctr, sat_ctr);
+        return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    }
     if (!scale_in) {
         // Current scaling: an amax pass first (fills amax_out and counts the
         // non-finite inputs), then the cast pass reads the amax back.

@@ -83,6 +83,10 @@ FP8Q_API fp8_status fp8_amax(const void *x_bf16, int64_t n, float *amax, uint32_
  *   scale_in == NULL : current scaling.  amax_out receives amax(x) and
  *                      s = fmax / amax (amax == 0 gives 1; overflow clamps
  *                      to FLT_MAX).  amax_out is REQUIRED in this mode.
+ *                      Up to 65536 elements (without transpose_out) the
+ *                      amax and the cast run in one launch (one CTA holding
+ *                      the tensor in registers); larger tensors take an amax
+ *                      launch, then a cast launch.
  *   scale_in != NULL : delayed scaling ([DeepL] §2.3): s = *scale_in (from
  *                      the amax history); amax_out (may be NULL) receives this
  *                      tensor's amax for the next history update.
