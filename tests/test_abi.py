@@ -122,3 +122,22 @@ def test_valid_call_without_device_fails_loudly():
     assert st in (UNSUPPORTED, CUDA)
     with pytest.raises((fp8q.Fp8Error, RuntimeError, ValueError)):
         fp8q.amax(torch.zeros(64, dtype=torch.bfloat16))
+
+
+@pytest.mark.parametrize("lang", ["c", "c++"])
+def test_header_compiles_as_plain_c_and_cpp(tmp_path, lang):
+    """The boundary is a C ABI: the header must compile as strict C99 (no C++
+    types or overloads in the signatures) and as C++ (extern "C" guards)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "fp8q.h"\n'
+                   "int main(void) { fp8_status s = FP8_OK; fp8_format f = FP8_E5M2;\n"
+                   "  fp8_scale_mode m = FP8_SCALE_BLOCK; (void)s; (void)f; (void)m; return 0; }\n")
+    std = ["-std=c99", "-pedantic", "-x", "c"] if lang == "c" else ["-std=c++17", "-x", "c++"]
+    r = subprocess.run([cc, *std, "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), "-c",
+                        str(src), "-o", str(tmp_path / "use_header.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
