@@ -379,6 +379,48 @@ void orc_gemm_scaled_sampled(const uint8_t *A, int fa, const uint8_t *B, int fb,
         gemm_one(A, fa, B, fb, M, N, K, mode, da, db, idx_m[i], idx_n[i], &val[i], &mag[i]);
 }
 
+/* The same GEMM accumulated the naive way in fp32 (kept to report how far
+ * the tensor cores' fp32 accumulation sits from the plain sequential fp32
+ * sum; the fp64 functions above stay the reference).  Each product of two
+ * FP8 values is exact in fp32 (at most 4 x 4 significant bits, exponents in
+ * range); the sum runs over k in order with one fp32 rounding per addition;
+ * block mode sums each 128-wide K block alone, then adds sc * part (sc =
+ * da * db rounded to fp32; multiply and add rounded separately); tensor and
+ * row modes multiply the whole sum by the fp32 product of the two scales.
+ * Returned as fp64 values of the fp32 results. */
+static double gemm_one_f32(const uint8_t *A, int fa, const uint8_t *B, int fb, int64_t M, int64_t K,
+                           int mode, const float *da, const float *db, int64_t m, int64_t n)
+{
+    int64_t nkb = (K + 127) / 128;
+    float acc = 0.0f;
+    if (mode == ORC_SCALE_BLOCK) {
+        for (int64_t kb = 0; kb < nkb; ++kb) {
+            float part = 0.0f;
+            int64_t k1 = (kb + 1) * 128 < K ? (kb + 1) * 128 : K;
+            for (int64_t k = kb * 128; k < k1; ++k)
+                part += (float)(orc_decode(A[m * K + k], fa) * orc_decode(B[n * K + k], fb));
+            float sc = da[kb * M + m] * db[(n / 128) * nkb + kb];
+            float t = sc * part;
+            acc = acc + t;
+        }
+    } else {
+        for (int64_t k = 0; k < K; ++k)
+            acc += (float)(orc_decode(A[m * K + k], fa) * orc_decode(B[n * K + k], fb));
+        float sc = (mode == ORC_SCALE_ROW) ? da[m] * db[n] : da[0] * db[0];
+        acc = acc * sc;
+    }
+    return (double)acc;
+}
+
+void orc_gemm_scaled_f32acc_sampled(const uint8_t *A, int fa, const uint8_t *B, int fb, int64_t M,
+                                    int64_t N, int64_t K, int mode, const float *da, const float *db,
+                                    const int64_t *idx_m, const int64_t *idx_n, int64_t count, double *val)
+{
+    (void)N;
+    for (int64_t i = 0; i < count; ++i)
+        val[i] = gemm_one_f32(A, fa, B, fb, M, K, mode, da, db, idx_m[i], idx_n[i]);
+}
+
 /* ------------------------------------------------------- delayed scaling -- */
 
 /* Delayed-scaling update ([DeepL] §2.3: the scale for this step is predicted

@@ -75,6 +75,8 @@ def lib():
         L.orc_gemm_scaled.argtypes = [P, I, P, I, I64, I64, I64, I, P, P, P, P]
         L.orc_gemm_scaled_sampled.restype = None
         L.orc_gemm_scaled_sampled.argtypes = [P, I, P, I, I64, I64, I64, I, P, P, P, P, I64, P, P]
+        L.orc_gemm_scaled_f32acc_sampled.restype = None
+        L.orc_gemm_scaled_f32acc_sampled.argtypes = [P, I, P, I, I64, I64, I64, I, P, P, P, P, I64, P]
         L.orc_amax_history_update.restype = None
         L.orc_amax_history_update.argtypes = [P, P, I, F, I, P, P, P]
         L.orc_kv_quant.restype = None
@@ -172,27 +174,38 @@ def quantize_tensorwise(x_bits: np.ndarray, fmt: int, scale_in: float | None = N
     return q, float(sinv[0]), float(am[0]), (int(counts[0]), int(counts[1]))
 
 
-def quantize_rowwise(x_bits: np.ndarray, fmt: int, pow2: bool = True):
+def _rows_cols_ld(x: np.ndarray, cols):
+    """A [rows, ld] array read as [rows, cols] rows of a wider buffer."""
+    rows, ld = x.shape
+    cols = ld if cols is None else int(cols)
+    assert 0 <= cols <= ld
+    return rows, cols, ld
+
+
+def quantize_rowwise(x_bits: np.ndarray, fmt: int, pow2: bool = True, cols=None):
+    """x [rows, ld] (the first ``cols`` columns of each row are the tensor;
+    cols=None: all) -> (q [rows, cols], scale_inv [rows])."""
     x = _u16(x_bits)
-    rows, cols = x.shape
+    rows, cols, ld = _rows_cols_ld(x, cols)
     q = np.empty((rows, cols), np.uint8)
     sinv = np.empty(rows, np.float32)
-    lib().orc_quantize_rowwise(_p(x), rows, cols, cols, fmt, int(pow2), _p(q), _p(sinv))
+    lib().orc_quantize_rowwise(_p(x), rows, cols, ld, fmt, int(pow2), _p(q), _p(sinv))
     return q, sinv
 
 
-def quantize_blockwise(x_bits: np.ndarray, fmt: int, block_rows: int, pow2: bool = False):
-    """block_rows 1: scales [ceil(cols/128), rows]; block_rows 128: scales
-    [ceil(rows/128), ceil(cols/128)]."""
+def quantize_blockwise(x_bits: np.ndarray, fmt: int, block_rows: int, pow2: bool = False, cols=None):
+    """x [rows, ld] (the first ``cols`` columns of each row are the tensor;
+    cols=None: all) -> (q [rows, cols], scales).  block_rows 1: scales
+    [ceil(cols/128), rows]; block_rows 128: scales [ceil(rows/128), ceil(cols/128)]."""
     x = _u16(x_bits)
-    rows, cols = x.shape
+    rows, cols, ld = _rows_cols_ld(x, cols)
     nkb = (cols + 127) // 128
     q = np.empty((rows, cols), np.uint8)
     if block_rows == 1:
         sinv = np.empty((nkb, rows), np.float32)
     else:
         sinv = np.empty(((rows + block_rows - 1) // block_rows, nkb), np.float32)
-    lib().orc_quantize_blockwise(_p(x), rows, cols, cols, fmt, block_rows, int(pow2), _p(q), _p(sinv))
+    lib().orc_quantize_blockwise(_p(x), rows, cols, ld, fmt, block_rows, int(pow2), _p(q), _p(sinv))
     return q, sinv
 
 
@@ -229,6 +242,33 @@ def gemm_scaled_sampled(A: np.ndarray, fa: int, B: np.ndarray, fb: int, mode: in
     lib().orc_gemm_scaled_sampled(_p(A), fa, _p(B), fb, M, N, K, mode, _p(da), _p(db),
                                   _p(im), _p(inn), im.size, _p(val), _p(mag))
     return val, mag
+
+
+def gemm_scaled_f32acc_sampled(A: np.ndarray, fa: int, B: np.ndarray, fb: int, mode: int,
+                               da: np.ndarray, db: np.ndarray, idx_m: np.ndarray, idx_n: np.ndarray):
+    """The naive sequential fp32-accumulate GEMM at the listed outputs (fp64
+    values of fp32 results, before any bf16 rounding)."""
+    A = np.ascontiguousarray(A, np.uint8)
+    B = np.ascontiguousarray(B, np.uint8)
+    M, K = A.shape
+    N, _ = B.shape
+    da = np.ascontiguousarray(da, np.float32)
+    db = np.ascontiguousarray(db, np.float32)
+    im = np.ascontiguousarray(idx_m, np.int64)
+    inn = np.ascontiguousarray(idx_n, np.int64)
+    val = np.empty(im.size, np.float64)
+    lib().orc_gemm_scaled_f32acc_sampled(_p(A), fa, _p(B), fb, M, N, K, mode, _p(da), _p(db),
+                                         _p(im), _p(inn), im.size, _p(val))
+    return val
+
+
+def gemm_scaled_f32acc(A: np.ndarray, fa: int, B: np.ndarray, fb: int, mode: int,
+                       da: np.ndarray, db: np.ndarray):
+    """Full [M, N] naive fp32-accumulate GEMM (fp64 values of fp32 results)."""
+    M, N = np.asarray(A).shape[0], np.asarray(B).shape[0]
+    im = np.repeat(np.arange(M), N)
+    inn = np.tile(np.arange(N), M)
+    return gemm_scaled_f32acc_sampled(A, fa, B, fb, mode, da, db, im, inn).reshape(M, N)
 
 
 def gemm_grouped(A: np.ndarray, fa: int, B: np.ndarray, fb: int, offsets, mode: int,

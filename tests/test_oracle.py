@@ -293,6 +293,74 @@ def test_blockwise_layout_and_invariants(orc, block_rows):
     assert np.all(dpad.reshape(nrb, block_rows, nkb, 128).max(axis=(1, 3)) == 448.0)
 
 
+def _pow2_scale_by_comparison(a, fm):
+    """Largest 2^k (k clamped to [-126, 127]) with a * 2^k <= fm, by exact
+    fp64 comparisons (a * 2^k is exact); 1 for a == 0."""
+    if a == 0:
+        return 1.0
+    k = math.floor(math.log2(fm / a))
+    while a * 2.0 ** (k + 1) <= fm:
+        k += 1
+    while a * 2.0 ** k > fm:
+        k -= 1
+    return 2.0 ** min(max(k, -126), 127)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("block_rows", [1, 128])
+@pytest.mark.parametrize("pow2", [False, True])
+def test_blockwise_every_code_against_torch(orc, fmt, block_rows, pow2):
+    """Every code and scale of the per-block quantizer (the DeepL page §2.3:
+    the tensor is cut into blocks, each with its own scale; power-of-two
+    block scales follow the Soup page's rowwise rule), recomputed
+    independently: the block amax by numpy over the block's finite valid
+    elements, s = fmax / amax as an fp32 division (or the largest power of
+    two with amax * s <= fmax, by exact comparisons), and the codes by
+    torch's float8 conversion of clamp(fp32(x) * s, -fmax, fmax).  The input
+    lives in a wider buffer (ld > cols) whose padding holds huge values and
+    NaN, so reading a padding element, or indexing the input with the
+    output's row pitch, changes a scale or a code.  Blocks differ in
+    magnitude by up to 10^+-3; one NaN and one -Inf sit in valid blocks
+    (NaN stays NaN, -Inf saturates to -fmax, neither counts in the amax)."""
+    rows, cols = (200, 300) if block_rows == 128 else (7, 400)
+    ld = cols + 40
+    fm = orc.fmax(fmt)
+    rng = np.random.default_rng(20 + 4 * fmt + 2 * (block_rows == 128) + pow2)
+    nrb, nkb = -(-rows // block_rows), -(-cols // 128)
+    xf = rng.standard_normal((rows, cols)).astype(np.float32)
+    mult = 10.0 ** rng.integers(-3, 4, (nrb, nkb))
+    xf *= np.kron(mult, np.ones((block_rows, 128)))[:rows, :cols].astype(np.float32)
+    x = torch.from_numpy(xf).to(torch.bfloat16)
+    bits = _bits(x).copy()
+    bits[1, 5] = 0x7FC0                      # NaN
+    bits[rows - 1, cols - 3] = 0xFF80        # -Inf
+    wide = np.full((rows, ld), 0x7F00, np.uint16)   # 1.7e38 in the padding
+    wide[:, cols + 1] = 0x7FC0                       # and NaN
+    wide[:, :cols] = bits
+    q, sinv = orc.quantize_blockwise(wide, fmt, block_rows, pow2=pow2, cols=cols)
+    assert q.shape == (rows, cols)
+
+    xv = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    fin = np.where(np.isfinite(xv), np.abs(xv), 0.0)
+    pad = np.zeros((nrb * block_rows, nkb * 128), np.float32)
+    pad[:rows, :cols] = fin
+    bam = pad.reshape(nrb, block_rows, nkb, 128).max(axis=(1, 3))
+    if pow2:
+        s = np.array([[_pow2_scale_by_comparison(float(a), fm) for a in r] for r in bam], np.float32)
+    else:
+        s = np.where(bam > 0, np.float32(fm) / np.maximum(bam, np.float32(1e-38)).astype(np.float32),
+                     np.float32(1.0)).astype(np.float32)
+    s_full = np.kron(s, np.ones((block_rows, 128), np.float32))[:rows, :cols]
+    y = np.clip((xv * s_full).astype(np.float32), -fm, fm)
+    ref = torch.from_numpy(y).to(TORCH_FP8[fmt]).view(torch.uint8).numpy()
+    nan = np.isnan(xv)
+    assert np.all(np.isnan(orc.decode_table(fmt)[q[nan]]))
+    assert np.array_equal(q[~nan], ref[~nan])
+    assert orc.decode_table(fmt)[q[rows - 1, cols - 3]] == -fm
+    inv = (np.float32(1.0) / s).astype(np.float32)
+    assert np.array_equal(sinv, inv.T if block_rows == 1 else inv)
+
+
 # -------------------------------------------------------------------- GEMM --
 
 def _int_codes(rng, shape, fmt):
@@ -353,6 +421,50 @@ def test_gemm_random_codes_against_numpy(orc):
     inn = rng.integers(0, N, 50)
     v, mg = orc.gemm_scaled_sampled(A, 0, B, 0, orc.SCALE_ROW, da, db, im, inn)
     assert np.array_equal(v, D[im, inn]) and np.array_equal(mg, mag[im, inn])
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_gemm_f32acc_variant_exact_on_integers_and_within_the_summation_bound(orc, mode):
+    """The naive fp32-accumulate variant: on small-integer codes with
+    power-of-two scales every sum is exact in fp32, so it equals the fp64
+    GEMM (and the int64 matmul); on random codes it stays within the
+    classical bound of sequential fp32 summation, (K + 2) u sum|scaled
+    products| with u = 2^-24."""
+    rng = np.random.default_rng(30 + mode)
+    M, N, K = 9, 260, 300
+    nkb = -(-K // 128)
+    va, A = _int_codes(rng, (M, K), 0)
+    vb, B = _int_codes(rng, (N, K), 0)
+    if mode == orc.SCALE_TENSOR:
+        da, db = np.float32([0.25]), np.float32([2.0])
+    elif mode == orc.SCALE_ROW:
+        da = np.exp2(rng.integers(-2, 3, M)).astype(np.float32)
+        db = np.exp2(rng.integers(-2, 3, N)).astype(np.float32)
+    else:
+        da = np.exp2(rng.integers(-1, 2, (nkb, M))).astype(np.float32)
+        db = np.exp2(rng.integers(-1, 2, (-(-N // 128), nkb))).astype(np.float32)
+    D, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
+    F = orc.gemm_scaled_f32acc(A, 0, B, 0, mode, da, db)
+    assert np.array_equal(F, D)
+    if mode != orc.SCALE_BLOCK:
+        sa = da if mode == orc.SCALE_ROW else np.repeat(da, M)
+        sb = db if mode == orc.SCALE_ROW else np.repeat(db, N)
+        exact = (va.astype(np.int64) @ vb.astype(np.int64).T).astype(np.float64)
+        assert np.array_equal(D, exact * sa[:, None].astype(np.float64) * sb[None, :].astype(np.float64))
+    t = orc.decode_table(0)
+    fin = np.where(np.isfinite(t))[0]
+    A = rng.choice(fin, (M, K)).astype(np.uint8)
+    B = rng.choice(fin, (N, K)).astype(np.uint8)
+    if mode == orc.SCALE_BLOCK:
+        da = rng.uniform(0.1, 3, (nkb, M)).astype(np.float32)
+        db = rng.uniform(0.1, 3, (-(-N // 128), nkb)).astype(np.float32)
+    elif mode == orc.SCALE_ROW:
+        da = rng.uniform(0.5, 2, M).astype(np.float32)
+        db = rng.uniform(0.5, 2, N).astype(np.float32)
+    D, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
+    F = orc.gemm_scaled_f32acc(A, 0, B, 0, mode, da, db)
+    assert np.all(np.abs(F - D) <= (K + 2) * 2.0 ** -24 * mag)
+    assert not np.array_equal(F, D)   # the rounding is really fp32
 
 
 def test_gemm_blockwise_against_numpy(orc):
