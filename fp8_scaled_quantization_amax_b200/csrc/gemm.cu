@@ -859,7 +859,9 @@ int one_sm_split(int dev, int sms, int tiles, int nk) {
 
 // Problems of any M whose 128 x 256 tiles fill at most a quarter of the SMs,
 // with at least 8 K blocks, run on the 1-SM kernel with each tile shared by a
-// cluster of S >= 4 CTAs (S from one_sm_split).  Measured (L2 flushed)
+// cluster of S CTAs: one_sm_split takes the largest S from min(8, nk / 2)
+// down to 2 whose clusters are all resident at once (for M <= 128 the split
+// also applies up to half the SMs).  Measured (L2 flushed)
 // against the pair kernel: 256 x 4096 x 4096 19.5 us (pair 22.5),
 // 256 x 4096 x 16384 29.7 us (pair with its workspace split 41.0).
 inline bool one_sm_cluster_split(int64_t M, int64_t N, int64_t K, int sms) {
@@ -981,6 +983,11 @@ uint32_t make_idesc(fp8_format fa, fp8_format fb, int mma_m, int mma_n) {
 
 using namespace fp8q_host;
 
+// The block-scaled GEMM on CTA pairs lives in gemm_block.cu.
+fp8_status fp8q_gemm_block_pair(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int64_t M,
+                                int64_t N, int64_t K, const float *sa, const float *sb, void *D_bf16, int64_t ldd,
+                                cudaStream_t s);
+
 namespace {
 std::atomic<uint32_t> g_split_epoch[64];   // per device; a split launch publishes with a fresh value
 }
@@ -1030,6 +1037,8 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
     // so few tiles that the cluster split-K of the 1-SM kernel applies;
     // otherwise one CTA per 128-row tile.
     if (M > BM && !one_sm_cluster_split(M, N, K, sms)) {
+        if (mode == FP8_SCALE_BLOCK)
+            return fp8q_gemm_block_pair(A, fa, B, fb, M, N, K, a_scale_inv, b_scale_inv, D_bf16, ldd, s);
         CUtensorMap ta, tb;
         if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
         const uint32_t idesc = make_idesc(fa, fb, 256, 256);
@@ -1075,10 +1084,11 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
     return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-// The E8M0 and the bf16 weight-gradient GEMMs keep their own error words
-// (gemm_mx.cu, gemm_bf16.cu).
+// The E8M0, the block-scaled pair and the bf16 weight-gradient GEMMs keep
+// their own error words (gemm_mx.cu, gemm_block.cu, gemm_bf16.cu).
 fp8_status fp8q_mx_device_error(uint32_t *out, int clear);
 fp8_status fp8q_wgrad_device_error(uint32_t *out, int clear);
+fp8_status fp8q_block_device_error(uint32_t *out, int clear);
 
 extern "C" fp8_status fp8_device_error(uint32_t *host_out, int clear) {
     if (!host_out) return FP8_ERR_INVALID_ARG;
@@ -1090,7 +1100,10 @@ extern "C" fp8_status fp8_device_error(uint32_t *host_out, int clear) {
     if (st != FP8_OK) return st;
     st = fp8q_wgrad_device_error(&g, clear);
     if (st != FP8_OK) return st;
-    *host_out = v | w | g;
+    uint32_t b = 0;
+    st = fp8q_block_device_error(&b, clear);
+    if (st != FP8_OK) return st;
+    *host_out = v | w | g | b;
     if (clear) {
         const unsigned int z = 0;
         if (cudaMemcpyToSymbol(g_gemm_error, &z, sizeof(z)) != cudaSuccess) return FP8_ERR_CUDA;
@@ -1153,8 +1166,10 @@ void *g_noalloc_ptr[64];   // device address of g_noalloc_scratch, per device
 }
 
 // One-time set-up per device (with that device current): look up the
-// array's device address and clear it on the caller's stream.
-static fp8_status noalloc_scratch(cudaStream_t stream, void **out) {
+// array's device address.  The array needs no clearing: a __device__ array
+// without an initializer is zero when the module loads, and the split-K
+// schedule leaves its hand-off flags at zero after every call.
+static fp8_status noalloc_scratch(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return FP8_ERR_CUDA;
     if (dev >= 64) return FP8_ERR_UNSUPPORTED_DEVICE;
@@ -1162,7 +1177,6 @@ static fp8_status noalloc_scratch(cudaStream_t stream, void **out) {
     if (!g_noalloc_ptr[dev]) {
         void *ptr = nullptr;
         if (cudaGetSymbolAddress((void **)&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return FP8_ERR_CUDA;
-        if (cudaMemsetAsync(ptr, 0, kNoAllocScratchBytes, stream) != cudaSuccess) return FP8_ERR_CUDA;
         g_noalloc_ptr[dev] = ptr;
     }
     *out = g_noalloc_ptr[dev];
@@ -1179,7 +1193,7 @@ extern "C" fp8_status fp8_gemm_scaled_noalloc(const uint8_t *A, fp8_format fa, c
     if (need > kNoAllocScratchBytes) return FP8_ERR_SHAPE;   // the split needs more than the built-in scratch
     void *scratch = nullptr;
     if (need > 0) {
-        st = noalloc_scratch(as_stream(stream), &scratch);
+        st = noalloc_scratch(&scratch);
         if (st != FP8_OK) return st;
     }
     return fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D_bf16, ldd, scratch, need, stream);

@@ -1,0 +1,351 @@
+// gemm_block.cu -- FP8 GEMM with full fp32 per-block scales (1x128 blocks of
+// A, 128x128 blocks of B), promoted per 128-wide K block on the CTA pairs.
+//
+// Sources: "DeepL押注FP8：大模型训练与推理统一精度实战解析" §2.3 (per-block
+// scales: the tensor is cut into small blocks, each with its own scale),
+// §5.3 (a fixed summation order per output, so results do not change run to
+// run); "H100 FP8加速实测：新一代计算架构的飞跃" (the multiply-accumulate runs
+// on the 8-bit floats in the tensor cores).
+//
+//   D[m, n] = bf16( sum_kb sa[kb, m] * sb[n / 128, kb] * sum_{k in kb} A[m, k] B[n, k] )
+//
+// The scales change every 128 elements of K, so no single epilogue scale
+// exists: each K block's product is accumulated alone in tensor memory and
+// the epilogue warps add it, scaled, into an fp32 register accumulator.
+// What bounds this loop on sm_100a (measured with clock stamps and probes):
+//   * an mbarrier signal takes ~200 cycles from arrive to the waiter's wake-up
+//     and a tcgen05.commit ~400 cycles from the MMAs' completion to the wake-up,
+//     so releasing a TMEM buffer and seeing the next MMA's result in it costs
+//     ~1.3k cycles however fast the epilogue computes;
+//   * a 256-row CTA-pair MMA runs at the same rate per flop for N = 128 as
+//     for N = 256 (65 vs 131 cycles per K = 32 step).
+// So each K block is issued as two 256 x 128 halves (tile columns 0-127 and
+// 128-255, each one 128-row block of B and therefore one B scale) into four
+// 128-column TMEM buffers, buffer 2 * (kb % 2) + half.  Three other halves
+// (768 MMA cycles) run while one is promoted, instead of one K block (512
+// cycles) with two 256-column buffers, and the two halves' epilogue warps run
+// half a K block apart, so one warp's TMEM round trip overlaps the other's
+// FMAs on the same SM sub-partition.
+//
+// Layout per CTA of the pair (M = 256 rows per tile, 128 per CTA):
+//   warp 0      TMA producer: per stage this CTA's 128 rows of A (16 KiB) and
+//               its 64-row share of each half's 128 rows of B (2 x 8 KiB);
+//   warp 1      TMEM allocator; in the even CTA the MMA issuer;
+//   warps 4-11  epilogue: warp w promotes TMEM lane quarter w % 4 (32 rows)
+//               of half (w - 4) / 4 (128 columns) -- two 64-column round
+//               trips, scalar fp32 FMAs (fma.rn, one rounding per term);
+//               then bf16 RNE and coalesced stores.
+// Summation order per output is fixed (K blocks in order, each block's
+// partial from the tensor core, then one FMA), so results are bit-identical
+// run to run.  Every mbarrier wait is bounded (about one second, see tc.cuh);
+// on expiry the kernel records a bit in this file's device error word, stops
+// issuing, drains its copies and MMAs, frees TMEM and returns.
+#include <algorithm>
+#include <mutex>
+
+#include "tc.cuh"
+
+using namespace fp8q;
+using fp8q_host::pdl_launch;
+
+namespace {
+
+namespace blk {
+constexpr int STAGES = 6;
+constexpr int B_SUB = 64 * BK;                  // this CTA's 64 rows of one half of B (8 KiB)
+constexpr int STAGE = A_TILE + 2 * B_SUB;       // 32 KiB per stage and CTA
+constexpr int NBUF = 4;                         // 128-column TMEM partial buffers
+constexpr int NBARS = 2 * STAGES + 2 * NBUF + 1;   // full, empty, partial full / free, drain
+constexpr size_t EPI_OFF = ((size_t)STAGES * STAGE + NBARS * 8 + 16 + 15) & ~(size_t)15;
+constexpr size_t SMEM = 1024 + EPI_OFF + (size_t)sm2::EPI * kEpiBufBytes;
+constexpr int PF = 2;                           // scale prefetch distance in K blocks
+static_assert(SMEM <= 232448, "shared memory per block");
+}  // namespace blk
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
+k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                 int K, uint32_t idesc, const float *__restrict__ sa, const float *__restrict__ sb,
+                 __nv_bfloat16 *__restrict__ D, int64_t ldd) {
+    constexpr int STG = blk::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)STG * blk::STAGE);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + blk::NBARS);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = (rank == 0);
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int num_m = (M + 255) / 256, num_n = (N + 255) / 256;
+    const int tiles = num_m * num_n;
+    const int nk = (K + BK - 1) / BK;
+    const int n_items = (pair < tiles) ? (tiles - 1 - pair) / npairs + 1 : 0;
+
+    auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+    auto empty_bar = [&](int s) { return smem_u32(&bars[STG + s]); };
+    auto accf_bar = [&](int q) { return smem_u32(&bars[2 * STG + q]); };
+    auto acce_bar = [&](int q) { return smem_u32(&bars[2 * STG + blk::NBUF + q]); };
+    const uint32_t drain_bar = smem_u32(&bars[2 * STG + 2 * blk::NBUF]);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STG; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int q = 0; q < blk::NBUF; ++q) {
+            mbar_init(accf_bar(q), 1);
+            mbar_init(acce_bar(q), 2 * (sm2::EPI / 2));   // both CTAs' four warps of that half
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();   // both CTAs' barriers are initialised before any remote signal
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();      // inputs of the previous kernel in the stream are visible from here on
+    pdl_trigger();
+
+    // Each role branch resizes its own warpgroup's registers (the epilogue
+    // holds a 128-wide fp32 accumulator row per thread); the launch pool is
+    // checked on the host.
+    if (warp == 0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            int last_round[STG];
+            for (int s = 0; s < STG; ++s) last_round[s] = -1;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < n_items; ++i) {
+                const int t = pair + i * npairs;
+                const int m_blk = t % num_m, n_blk = t / num_m;
+                const int a_row = m_blk * 256 + (int)rank * 128;
+                // an N = 128 pair MMA takes rows [0, 64) of its B operand from
+                // the even CTA and [64, 128) from the odd one
+                const int b_row = n_blk * 256 + (int)rank * 64;
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const int stage = it % STG;
+                    const uint32_t round = it / STG;
+                    if (!wait_bar(empty_bar(stage), (round & 1u) ^ 1u, abort_flag, kErrProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_leader = mapa_shared(full_bar(stage), 0);
+                    if (leader) mbar_expect_tx(full_bar(stage), 2 * blk::STAGE);
+                    const uint32_t a_dst = smem_u32(smem + (size_t)stage * blk::STAGE);
+                    tma_load_2d_pair(a_dst, &tmA, full_leader, kc * BK, a_row);
+                    tma_load_2d_pair(a_dst + A_TILE, &tmB, full_leader, kc * BK, b_row);
+                    tma_load_2d_pair(a_dst + A_TILE + blk::B_SUB, &tmB, full_leader, kc * BK, b_row + 128);
+                    last_round[stage] = (int)round;
+                }
+            }
+            if (leader && (!ok || *abort_flag)) {   // copies in flight must land before the CTA exits
+                for (int s = 0; s < STG; ++s)
+                    if (last_round[s] >= 0) wait_bar_drain(full_bar(s), (uint32_t)last_round[s] & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
+        // ------------------------------------- MMA issuer (leader only) --
+        if (leader && lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < n_items; ++i) {
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const int stage = it % STG;
+                    const uint32_t round = it / STG;
+                    if (!wait_bar(full_bar(stage), round & 1u, abort_flag, kErrMma)) { ok = false; break; }
+                    const uint32_t a_addr = smem_u32(smem + (size_t)stage * blk::STAGE);
+                    const uint64_t adesc = sdesc_k_sw128(a_addr);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int q = 2 * (int)(it & 1u) + h;
+                        if (!wait_bar(acce_bar(q), ((it >> 1) & 1u) ^ 1u, abort_flag, kErrMma)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint64_t bdesc = sdesc_k_sw128(a_addr + A_TILE + h * blk::B_SUB);
+#pragma unroll
+                        for (int k = 0; k < BK / 32; ++k)   // +32 bytes along K = +2 in the address field
+                            tc_mma_pair(tmem + q * 128, adesc + 2u * k, bdesc + 2u * k, idesc, k > 0 ? 1u : 0u);
+                        tc_commit_pair_both(accf_bar(q));
+                    }
+                    if (!ok) break;
+                    tc_commit_pair_both(empty_bar(stage));
+                }
+            }
+            // all MMAs issued by this thread complete before TMEM is freed
+            tc_commit_pair_self(drain_bar);
+            wait_bar_drain(drain_bar, 0u);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(sm2::REGS_HIGH));
+        // --------------------------------------------------- epilogue ----
+        const int sp = warp & 3;
+        const int h = (warp - 4) >> 2;                  // half of the tile: columns h*128 .. +127
+        const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+        const uint32_t release_to = leader ? 0u : mapa_shared(acce_bar(0), 0);   // rank 1: the leader's barriers
+        uint32_t it = 0;
+        bool ok = true;
+        for (int i = 0; ok && i < n_items; ++i) {
+            const int t = pair + i * npairs;
+            const int m_blk = t % num_m, n_blk = t / num_m;
+            const int64_t row0 = (int64_t)m_blk * 256 + (int)rank * 128 + sp * 32;
+            const int64_t m = row0 + lane;
+            const bool m_ok = m < M;
+            const int n_base = n_blk * 256 + h * 128;
+            const int nb = n_blk * 2 + h;               // this half's 128-row block of B
+            const bool nb_ok = n_base < N;
+            float acc[128];
+#pragma unroll
+            for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+            // Scales run PF K blocks ahead in PF register sets (the K loop is
+            // unrolled by PF, so no register copy waits on a load).
+            float as_[blk::PF], bs_[blk::PF];
+#pragma unroll
+            for (int p = 0; p < blk::PF; ++p) {
+                as_[p] = (p < nk && m_ok) ? sa[(int64_t)p * M + m] : 0.0f;
+                bs_[p] = (p < nk && nb_ok) ? sb[(int64_t)nb * nk + p] : 0.0f;
+            }
+            // one K block: wait for this half's partial, promote it, release it
+            auto promote = [&](int kc, float &as, float &bs) -> bool {
+                const int q = 2 * (int)(it & 1u) + h;
+                const float sc = __fmul_rn(as, bs);
+                bool w = true;
+                if (lane == 0) w = wait_bar(accf_bar(q), (it >> 1) & 1u, abort_flag, kErrEpilogue);
+                w = __shfl_sync(0xFFFFFFFFu, w, 0);
+                if (!w) return false;
+                tc_fence_after();
+                const uint32_t src = tmem + lane_base + q * 128;
+                uint32_t r[64];
+                tmem_ld32_async(src, r);
+                tmem_ld32_async(src + 32, r + 32);
+                tmem_wait64(r);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) acc[j] = fmaf(__uint_as_float(r[j]), sc, acc[j]);
+                tmem_ld32_async(src + 64, r);
+                tmem_ld32_async(src + 96, r + 32);
+                tmem_wait64(r);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {   // the partial is in registers: hand the buffer back to the MMA
+                    if (leader) mbar_arrive(acce_bar(q));
+                    else mbar_arrive_cluster(release_to + (uint32_t)(q * 8));
+                }
+                if (kc + blk::PF < nk) {   // block kc + PF's scales, after the release
+                    as = m_ok ? sa[(int64_t)(kc + blk::PF) * M + m] : 0.0f;
+                    bs = nb_ok ? sb[(int64_t)nb * nk + kc + blk::PF] : 0.0f;
+                }
+#pragma unroll
+                for (int j = 0; j < 64; ++j) acc[64 + j] = fmaf(__uint_as_float(r[j]), sc, acc[64 + j]);
+                ++it;
+                return true;
+            };
+            for (int kc = 0; ok && kc < nk; kc += blk::PF) {
+#pragma unroll
+                for (int p = 0; p < blk::PF; ++p)
+                    if (ok && kc + p < nk && !promote(kc + p, as_[p], bs_[p])) ok = false;
+            }
+            if (!ok) break;
+            uint8_t *ebuf = smem + blk::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(acc[h2 * 64 + 2 * j], acc[h2 * 64 + 2 * j + 1]);
+                store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, (int64_t)M, n_base + h2 * 64, N);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();   // every TMEM read and MMA of both CTAs is done
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// Pairs of the block-scaled kernel that fit on the device at once (cached per
+// device); 0 when the kernel cannot be launched as the register split needs.
+int block_pair_capacity() {
+    static int cache[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev] > 0) return cache[dev];
+    if (cudaFuncSetAttribute(k_gemm_block_2sm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)blk::SMEM) !=
+        cudaSuccess)
+        return 0;
+    cudaFuncAttributes fa;   // the setmaxnreg split assumes this launch register count
+    if (cudaFuncGetAttributes(&fa, k_gemm_block_2sm) != cudaSuccess || fa.numRegs != sm2::REGS_LAUNCH) return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 64);
+    cfg.blockDim = dim3(sm2::THREADS);
+    cfg.dynamicSmemBytes = blk::SMEM;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_block_2sm, &cfg) != cudaSuccess) return 0;
+    cache[dev] = n;
+    return n;
+}
+
+}  // namespace
+
+using namespace fp8q_host;
+
+// The block-scaled GEMM on CTA pairs (M > 128 rows); arguments validated by
+// fp8_gemm_scaled.  Returns FP8_ERR_CUDA when a map cannot be encoded or the
+// launch fails.
+fp8_status fp8q_gemm_block_pair(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int64_t M,
+                                int64_t N, int64_t K, const float *sa, const float *sb, void *D_bf16, int64_t ldd,
+                                cudaStream_t s) {
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 64)) return FP8_ERR_CUDA;
+    const int cap = block_pair_capacity();
+    if (cap <= 0) return FP8_ERR_CUDA;
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
+    // fp32 accumulator, A/B formats, K-major A and B, N = 128 (>> 3), M = 256 (>> 4)
+    const uint32_t idesc = (1u << 4) | ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(128 >> 3) << 17) |
+                           ((uint32_t)(256 >> 4) << 24);
+    return pdl_launch(k_gemm_block_2sm, dim3(2 * pairs), dim3(sm2::THREADS), blk::SMEM, s, ta, tb, (int)M, (int)N,
+                      (int)K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D_bf16), ldd) == cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_CUDA;
+}
+
+// This file's device error word (read and optionally cleared by
+// fp8_device_error together with the other GEMM files').
+fp8_status fp8q_block_device_error(uint32_t *out, int clear) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_gemm_error, sizeof(v)) != cudaSuccess) return FP8_ERR_CUDA;
+    *out = v;
+    if (clear) {
+        const unsigned int z = 0;
+        if (cudaMemcpyToSymbol(g_gemm_error, &z, sizeof(z)) != cudaSuccess) return FP8_ERR_CUDA;
+    }
+    return FP8_OK;
+}

@@ -317,9 +317,12 @@ FP8Q_API fp8_status fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8
  *   caller still passes A, B, the scales and D.
  *   Returns FP8_ERR_SHAPE when the shape's split needs more scratch than the
  *   10 MiB (fp8_gemm_workspace_size() > 10 MiB); nothing is enqueued then.
+ *   On a 148-SM B200 the largest split needs 9.25 MiB (37 tiles of two
+ *   128 x 256 fp32 partials), so every shape runs there.
  *   The first call on a device that needs the scratch does a one-time
- *   set-up (looks up the array's device address, clears it on `stream`);
- *   make that first call before any stream capture.
+ *   set-up: it looks up the array's device address (the array starts
+ *   zeroed when the library's module loads, and each call leaves its
+ *   hand-off flags zeroed); make that first call before any stream capture.
  *   Allocates nothing: no cudaMalloc / cudaFree or allocating library call.
  *   All calls on a device share the one array and it keeps the last call's
  *   contents; calls that overlap on the GPU (other streams, other threads)
