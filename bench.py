@@ -4,15 +4,19 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One "step" is one pass of the whole hot path over one batch of synthetic
-input already resident in HBM.  Default workload ``rowwise``: per-row
-power-of-two E4M3 quantization of activations A [4096, 4096] (N(0,1) with 0.1 %
-x100 outliers) and weights B [4096, 4096] (N(0, 0.02)), then the rowwise-scaled
-FP8 GEMM D = A8 x B8^T (fp32 accumulate, bf16 out).  Other workloads:
-``tensor`` (per-tensor E4M3, 256^3), ``blockmlp`` (1x128 / 128x128 block
-scales, X[8192, 4096] -> W_up[11008, 4096] -> W_down[4096, 11008]),
-``dgrad`` (E5M2 gradients [8192, 4096] x E4M3 W^T [4096, 4096] with delayed
-scaling over a 16-step history) and ``kv`` (FP8 KV cache K, V [32, 32, 8192,
-128] quantize + dequantize, GB/s).
+input already resident in HBM.  Default workload ``blockmlp``: the
+block-scaled E4M3 MLP of a 7B-style layer -- X [8192, 4096] (N(0,1)) quantized
+with 1x128 scales, W_up [11008, 4096] and W_down [4096, 11008] (N(0, 0.02))
+with 128x128 scales, H = X8 W_up8^T in bf16 (fp32 accumulate, fp32 scales
+promoted per 128-wide K block), H requantized 1x128, D = H8 W_down8^T.
+Other workloads: ``rowwise`` (per-row power-of-two E4M3 quantization of A
+[4096, 4096] with 0.1 % x100 outliers and B [4096, 4096], then the
+rowwise-scaled GEMM), ``tensor`` (per-tensor E4M3, 256^3),
+``blockmlp_e8m0`` (the MLP with power-of-two block scales applied in the
+MMA), ``dgrad`` (E5M2 gradients [8192, 4096] x E4M3 W^T [4096, 4096] with
+delayed scaling over a 16-step history), ``bwd_gw_hp`` (a layer's backward
+under the rowwise_with_gw_hp recipe), ``kv`` (FP8 KV cache K, V [32, 32,
+8192, 128] quantize + dequantize, GB/s), ``paged`` and ``health``.
 
 Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then K steps
 bracketed by a barrier and a device synchronize; each step's kernels are
@@ -20,7 +24,9 @@ timed with CUDA events on the launching stream, L2 is flushed (a 256 MiB write
 and a 256 MiB read)
 before every step outside the events; multi-GPU takes the max over ranks.
 ``--impl reference`` times the CPU oracle (the only reference this project
-has) on a bounded sample of the same workload.
+has) on a bounded sample of the same workload, on every host thread this
+process may use; the GPU line's ``cpu_baseline`` gives that figure and the
+one-thread figure of the same sample.
 """
 from __future__ import annotations
 
@@ -539,134 +545,202 @@ class Workload:
 
 # --------------------------------------------------------- CPU (oracle) arm --
 
-def cpu_sample(name: str, seed: int = 0):
-    """Time the CPU oracle, as it stands, on a bounded sample of the workload;
-    returns (value in the workload's unit for a full step, sample description)."""
+def host_cores() -> int:
+    """Host threads this process may run on (its CPU affinity)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class _Phases:
+    """Timed phases of the oracle sample.  Each phase is a list of independent
+    jobs (oracle calls on disjoint rows, columns, outputs, slices or
+    segments); the oracle is C called through ctypes, which releases the GIL,
+    so a thread pool runs the jobs on separate cores.  A phase's wall time,
+    times the phase's extrapolation factor, adds to the full-step estimate."""
+
+    def __init__(self, pool):
+        self.pool = pool
+        self.total = 0.0
+
+    def run(self, factor, jobs):
+        t0 = time.perf_counter()
+        out = [j() for j in jobs] if self.pool is None else list(self.pool.map(lambda j: j(), jobs))
+        self.total += factor * (time.perf_counter() - t0)
+        return out
+
+
+def _chunks(n: int, parts: int):
+    parts = max(1, min(n, parts))
+    b = [n * i // parts for i in range(parts + 1)]
+    return [(b[i], b[i + 1]) for i in range(parts) if b[i + 1] > b[i]]
+
+
+def cpu_sample(name: str, seed: int = 0, pool=None, threads: int = 1):
+    """Time the CPU oracle, as it stands, on a bounded sample of the workload,
+    on `threads` host threads (pool: a ThreadPoolExecutor of that size, or
+    None for one thread); returns (value in the workload's unit for a full
+    step, sample description)."""
     import numpy as np
     from fp8_scaled_quantization_amax_b200 import inputs
     from oracle import oracle as orc
     orc.lib()
+    ph = _Phases(pool)
+    parts = 4 * threads
+    C = np.ascontiguousarray
+
+    def rows_job(fn, x, r0, r1, *a):
+        piece = C(x[r0:r1])
+        return lambda: fn(piece, *a)
+
+    def gemm_jobs(A, fa, B, fb, mode, da, db, im, inn):
+        return [(lambda lo=lo, hi=hi: orc.gemm_scaled_sampled(A, fa, B, fb, mode, da, db, im[lo:hi], inn[lo:hi]))
+                for lo, hi in _chunks(im.size, parts)]
+
     if name == "bwd_gw_hp":
         T, N_out, K_in = 8192, 4096, 4096
         r = 8
         g = inputs.bf16_bits(inputs.lognormal_grads_bf16((T, N_out), seed=seed))
         x = inputs.bf16_bits(inputs.normal_bf16((T, K_in), 1.0, seed=seed + 1))
         w = inputs.bf16_bits(inputs.normal_bf16((N_out, K_in), 0.02, seed=seed + 2))
-        t0 = time.perf_counter()
-        qwT, swT = orc.quantize_rowwise_transpose(w, 0, True)
-        tw = time.perf_counter() - t0
-        t0 = time.perf_counter()
-        qg, sg = orc.quantize_rowwise(g[:r], 1, True)
-        im = np.repeat(np.arange(r), 256)
-        inn = np.tile(np.arange(256), r)
-        orc.gemm_scaled_sampled(qg, 1, qwT, 0, 1, sg, swT, im, inn)
-        td = (time.perf_counter() - t0) * (T / r) * (K_in / 256)
-        t0 = time.perf_counter()
-        orc.gemm_bf16_wgrad_sampled(g, x, np.repeat(np.arange(2), 64), np.tile(np.arange(64), 2))
-        tg = (time.perf_counter() - t0) * (N_out * K_in / 128)
-        return 4.0 * T * N_out * K_in / (tw + td + tg) / 1e12, (
+        cols = [C(w[:, c0:c1]) for c0, c1 in _chunks(K_in, parts)]
+        res = ph.run(1.0, [(lambda p=p: orc.quantize_rowwise_transpose(p, 0, True)) for p in cols])
+        qwT, swT = np.concatenate([q for q, _ in res]), np.concatenate([s_ for _, s_ in res])
+        res = ph.run((T / r) * (K_in / 256), [rows_job(orc.quantize_rowwise, g, i, i + 1, 1, True) for i in range(r)])
+        qg, sg = np.concatenate([q for q, _ in res]), np.concatenate([s_ for _, s_ in res])
+        im, inn = np.repeat(np.arange(r), 256), np.tile(np.arange(256), r)
+        ph.run((T / r) * (K_in / 256), gemm_jobs(qg, 1, qwT, 0, 1, sg, swT, im, inn))
+        wm, wn = np.repeat(np.arange(2), 64), np.tile(np.arange(64), 2)
+        ph.run(N_out * K_in / 128, [(lambda lo=lo, hi=hi: orc.gemm_bf16_wgrad_sampled(g, x, wm[lo:hi], wn[lo:hi]))
+                                    for lo, hi in _chunks(wm.size, parts)])
+        return 4.0 * T * N_out * K_in / ph.total / 1e12, (
             f"all of W^T quantized, {r} dY rows quantized and {r}x256 dX outputs (K=4096), 128 dW outputs "
             "over all 8192 tokens; the dX and dW parts scaled to the full layer")
     if name == "blockmlp_e8m0":
         name = "blockmlp"   # the same per-block GEMM in the oracle (its cost does not depend on the scale rule)
-    if name in ("rowwise", "tensor", "blockmlp", "dgrad"):
-        if name == "rowwise":
-            M = N = K = 4096
-            r = 8
-            a = inputs.bf16_bits(inputs.outlier_activations_bf16((r, K), seed=seed))
-            b = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, seed=seed + 1))
-            t0 = time.perf_counter()
-            qb, sb = orc.quantize_rowwise(b, 0, True)
-            tb = time.perf_counter() - t0
-            t0 = time.perf_counter()
-            qa, sa = orc.quantize_rowwise(a, 0, True)
-            im = np.repeat(np.arange(r), N)
-            inn = np.tile(np.arange(N), r)
-            orc.gemm_scaled_sampled(qa, 0, qb, 0, 1, sa, sb, im, inn)
-            tr = time.perf_counter() - t0
-            full = tb + tr * (M / r)
-            return 2.0 * M * N * K / full / 1e12, (
-                f"rowwise-quantize all of B [4096,4096] + {r} rows of A, then those {r}x4096 outputs "
-                f"(fp64 sums); full step extrapolated as t_B + (4096/{r}) x t_rows")
-        if name == "tensor":
-            M = N = K = 256
-            a = inputs.bf16_bits(inputs.normal_bf16((M, K), 1.0, seed=seed))
-            b = inputs.bf16_bits(inputs.normal_bf16((N, K), 1.0, seed=seed + 1))
-            reps = 10
-            t0 = time.perf_counter()
-            for _ in range(reps):
-                qa, sa, _, _ = orc.quantize_tensorwise(a, 0)
-                qb, sb, _, _ = orc.quantize_tensorwise(b, 0)
-                orc.gemm_scaled(qa, 0, qb, 0, 0, np.float32([sa]), np.float32([sb]))
-            t = (time.perf_counter() - t0) / reps
-            return 2.0 * M * N * K / t / 1e12, "the whole 256^3 per-tensor step, mean of 10"
-        if name == "blockmlp":
-            M, Dm, F = 8192, 4096, 11008
-            r = 32
-            x = inputs.bf16_bits(inputs.normal_bf16((r, Dm), 1.0, seed=seed))
-            w = inputs.bf16_bits(inputs.normal_bf16((256, Dm), 0.02, seed=seed + 1))
-            t0 = time.perf_counter()
-            qw, sw = orc.quantize_blockwise(w, 0, 128)
-            tw = (time.perf_counter() - t0) * (F / 256) * 2
-            t0 = time.perf_counter()
-            qx, sx = orc.quantize_blockwise(x, 0, 1)
-            im = np.repeat(np.arange(r), 256)
-            inn = np.tile(np.arange(256), r)
-            orc.gemm_scaled_sampled(qx, 0, qw, 0, 2, sx, sw, im, inn)
-            tr = (time.perf_counter() - t0) * (M / r) * (F / 256) * 2
-            return 4.0 * M * Dm * F / (tw + tr) / 1e12, (
-                f"blockwise-quantize 256 W rows and {r} X rows, then {r}x256 outputs at K=4096; "
-                "scaled to both MLP GEMMs")
-        if name == "dgrad":
-            M, N_out, K_in = 8192, 4096, 4096
-            r = 128
-            g = inputs.bf16_bits(inputs.lognormal_grads_bf16((r, N_out), seed=seed))
-            w = inputs.bf16_bits(inputs.normal_bf16((256, N_out), 0.02, seed=seed + 1))
-            t0 = time.perf_counter()
-            qw, sw, _, _ = orc.quantize_tensorwise(w, 0)
-            qg, sg, _, _ = orc.quantize_tensorwise(g, 1, scale_in=1.0)
-            im = np.repeat(np.arange(r), 256)
-            inn = np.tile(np.arange(256), r)
-            orc.gemm_scaled_sampled(qg, 1, qw, 0, 0, np.float32([sg]), np.float32([sw]), im, inn)
-            t = (time.perf_counter() - t0) * (M / r) * (K_in / 256)
-            return 2.0 * M * N_out * K_in / t / 1e12, (
-                f"quantize {r} gradient rows (E5M2) + 256 weight rows, then {r}x256 outputs; scaled to the step")
+    if name == "rowwise":
+        M = N = K = 4096
+        r = 8
+        a = inputs.bf16_bits(inputs.outlier_activations_bf16((r, K), seed=seed))
+        b = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, seed=seed + 1))
+        res = ph.run(1.0, [rows_job(orc.quantize_rowwise, b, r0, r1, 0, True) for r0, r1 in _chunks(N, parts)])
+        qb, sb = np.concatenate([q for q, _ in res]), np.concatenate([s_ for _, s_ in res])
+        res = ph.run(M / r, [rows_job(orc.quantize_rowwise, a, i, i + 1, 0, True) for i in range(r)])
+        qa, sa = np.concatenate([q for q, _ in res]), np.concatenate([s_ for _, s_ in res])
+        im, inn = np.repeat(np.arange(r), N), np.tile(np.arange(N), r)
+        ph.run(M / r, gemm_jobs(qa, 0, qb, 0, 1, sa, sb, im, inn))
+        return 2.0 * M * N * K / ph.total / 1e12, (
+            f"rowwise-quantize all of B [4096,4096] + {r} rows of A, then those {r}x4096 outputs "
+            f"(fp64 sums); full step extrapolated as t_B + (4096/{r}) x t_rows")
+    if name == "tensor":
+        M = N = K = 256
+        a = inputs.bf16_bits(inputs.normal_bf16((M, K), 1.0, seed=seed))
+        b = inputs.bf16_bits(inputs.normal_bf16((N, K), 1.0, seed=seed + 1))
+        reps = 10
+        im, inn = np.repeat(np.arange(M), N), np.tile(np.arange(N), M)
+        for _ in range(reps):
+            (qa, sa, _, _), (qb, sb, _, _) = ph.run(1.0 / reps, [lambda: orc.quantize_tensorwise(a, 0),
+                                                                 lambda: orc.quantize_tensorwise(b, 0)])
+            ph.run(1.0 / reps, gemm_jobs(qa, 0, qb, 0, 0, np.float32([sa]), np.float32([sb]), im, inn))
+        return 2.0 * M * N * K / ph.total / 1e12, "the whole 256^3 per-tensor step, mean of 10"
+    if name == "blockmlp":
+        M, Dm, F = 8192, 4096, 11008
+        r = 32
+        wrows = 128 * max(2, min(threads, 86))
+        x = inputs.bf16_bits(inputs.normal_bf16((r, Dm), 1.0, seed=seed))
+        w = inputs.bf16_bits(inputs.normal_bf16((wrows, Dm), 0.02, seed=seed + 1))
+        res = ph.run((F / wrows) * 2, [rows_job(orc.quantize_blockwise, w, r0, r0 + 128, 0, 128)
+                                       for r0 in range(0, wrows, 128)])
+        qw, sw = np.concatenate([q for q, _ in res]), np.concatenate([s_ for _, s_ in res])
+        res = ph.run((M / r) * (F / 256) * 2, [rows_job(orc.quantize_blockwise, x, i, i + 1, 0, 1) for i in range(r)])
+        qx, sx = np.concatenate([q for q, _ in res]), np.concatenate([s_ for _, s_ in res], axis=1)
+        im, inn = np.repeat(np.arange(r), 256), np.tile(np.arange(256), r)
+        ph.run((M / r) * (F / 256) * 2, gemm_jobs(qx, 0, qw, 0, 2, C(sx), sw, im, inn))
+        return 4.0 * M * Dm * F / ph.total / 1e12, (
+            f"blockwise-quantize {wrows} W rows and {r} X rows, then {r}x256 outputs at K=4096; "
+            "scaled to both MLP GEMMs")
+    if name == "dgrad":
+        M, N_out, K_in = 8192, 4096, 4096
+        r = 128
+        g = inputs.bf16_bits(inputs.lognormal_grads_bf16((r, N_out), seed=seed))
+        w = inputs.bf16_bits(inputs.normal_bf16((256, N_out), 0.02, seed=seed + 1))
+        f = (M / r) * (K_in / 256)
+        jobs = [lambda: orc.quantize_tensorwise(w, 0)] + [
+            (lambda p=C(g[r0:r1]): orc.quantize_tensorwise(p, 1, scale_in=1.0)) for r0, r1 in _chunks(r, parts)]
+        res = ph.run(f, jobs)
+        qw, sw = res[0][0], res[0][1]
+        qg, sg = np.concatenate([q[0] for q in res[1:]]), res[1][1]
+        im, inn = np.repeat(np.arange(r), 256), np.tile(np.arange(256), r)
+        ph.run(f, gemm_jobs(qg, 1, qw, 0, 0, np.float32([sg]), np.float32([sw]), im, inn))
+        return 2.0 * M * N_out * K_in / ph.total / 1e12, (
+            f"quantize {r} gradient rows (E5M2) + 256 weight rows, then {r}x256 outputs; scaled to the step")
     if name == "paged":
         P = inputs.PAGED_KV
         B, S, H, Dh, bs = P["B"], P["S"], P["H"], P["Dh"], P["block_size"]
-        r = 2048
+        per = 256
+        nseq = max(8, min(2 * threads, 128))
+        r = per * nseq
         x = inputs.bf16_bits(inputs.normal_bf16((r, H, Dh), 1.0, seed=seed))
-        table, slots = inputs.paged_layout([r], bs, r // bs, seed=seed + 3)
-        t0 = time.perf_counter()
-        c, sc = orc.paged_kv_write(x, slots.numpy(), np.zeros((r // bs, bs, H, Dh), np.uint8),
-                                   np.zeros((r // bs, bs, H), np.float32), 0)
-        orc.paged_kv_gather(c, sc, table.numpy(), np.array([r], np.int32), r, 0)
-        t = (time.perf_counter() - t0) * (B * S / r) * 2
+        subs = []
+        for i in range(nseq):
+            table, slots = inputs.paged_layout([per], bs, per // bs, seed=seed + 3 + i)
+            subs.append((C(x[i * per:(i + 1) * per]), slots.numpy(), table.numpy()))
+
+        def one(xi, sl, tb):
+            c, sc = orc.paged_kv_write(xi, sl, np.zeros((per // bs, bs, H, Dh), np.uint8),
+                                       np.zeros((per // bs, bs, H), np.float32), 0)
+            orc.paged_kv_gather(c, sc, tb, np.array([per], np.int32), per, 0)
+
+        ph.run((B * S / r) * 2, [(lambda t=t: one(*t)) for t in subs])
         T = B * S
         full = 2 * (2 * (3.0 * T * H * Dh + 4.0 * T * H) + 8.0 * T + 4.0 * T / bs + 4.0 * B)
-        return full / t / 1e9, f"{r} tokens of K written and gathered; scaled to K and V of all {B}x{S} tokens"
+        return full / ph.total / 1e9, (f"{r} tokens of K ({nseq} sequences of {per}) written and gathered; "
+                                       f"scaled to K and V of all {B}x{S} tokens")
     if name == "health":
         L, n = inputs.SCALE_HEALTH["layers"], inputs.SCALE_HEALTH["per_layer"]
         prev, cur = inputs.scale_snapshots_f32(L * n, seed=seed + 7)
         p, c = prev.numpy(), cur.numpy()
         reps = 20
-        t0 = time.perf_counter()
+        segs = [(C(c[g * n:(g + 1) * n]), C(p[g * n:(g + 1) * n])) for g in range(L)]
+
+        def some(g0, g1):   # a job takes several segments: one is too little work for a thread hand-off
+            for a, b in segs[g0:g1]:
+                orc.scale_stats(a, b, 4.0)
+
+        groups = _chunks(L, threads)
         for _ in range(reps):
-            for g in range(L):
-                orc.scale_stats(c[g * n:(g + 1) * n], p[g * n:(g + 1) * n], 4.0)
-        t = (time.perf_counter() - t0) / reps
-        return (2 * 4.0 * L * n + 8 * (L + 1) + 20 * L) / t / 1e9, "the whole step (all 224 segments), mean of 20"
+            ph.run(1.0 / reps, [(lambda g0=g0, g1=g1: some(g0, g1)) for g0, g1 in groups])
+        return (2 * 4.0 * L * n + 8 * (L + 1) + 20 * L) / ph.total / 1e9, "the whole step (all 224 segments), mean of 20"
     # kv
     B, H, S, Dh = 32, 32, 8192, 128
-    k = inputs.bf16_bits(inputs.normal_bf16((1, 16, S, Dh), 1.0, seed=seed))
-    t0 = time.perf_counter()
-    q, s = orc.kv_quant(k, 0)
-    orc.kv_dequant(q, s, 0)
-    t = time.perf_counter() - t0
-    per_slice = t / 16
+    ns = max(16, min(2 * threads, 256))
+    k = inputs.bf16_bits(inputs.normal_bf16((1, ns, S, Dh), 1.0, seed=seed))
+    slices = [C(k[:, i:i + 1]) for i in range(ns)]
+
+    def kv_one(sl):
+        q, sc = orc.kv_quant(sl, 0)
+        orc.kv_dequant(q, sc, 0)
+
+    ph.run(B * H * 2 / ns, [(lambda sl=sl: kv_one(sl)) for sl in slices])
     n = B * H * S * Dh
-    full = per_slice * B * H * 2
-    return 2 * (3.0 * n) * 2 / full / 1e9, "16 of the 2048 (b,h) slices of K/V quantized and dequantized; scaled"
+    return 2 * (3.0 * n) * 2 / ph.total / 1e9, f"{ns} of the 2048 (b,h) slices of K/V quantized and dequantized; scaled"
+
+
+def cpu_baseline(name: str, seed: int = 0):
+    """The oracle on all host threads this process may use and on one thread,
+    on the same bounded sample: (value, threads, one-thread value,
+    description), where value and threads are the faster of the two runs (a
+    sample of many tiny oracle calls can run slower on many threads, whose
+    hand-offs go through the interpreter lock)."""
+    import concurrent.futures as cf
+    threads = host_cores()
+    v1, desc = cpu_sample(name, seed)
+    if threads == 1:
+        return v1, 1, v1, desc
+    with cf.ThreadPoolExecutor(max_workers=threads) as pool:
+        vall, desc = cpu_sample(name, seed, pool=pool, threads=threads)
+    return (vall, threads, v1, desc) if vall >= v1 else (v1, 1, v1, desc)
 
 
 # -------------------------------------------------------------------- main --
@@ -676,7 +750,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="rowwise", choices=list(DEFAULT_STEPS))
+    ap.add_argument("--workload", default="blockmlp", choices=list(DEFAULT_STEPS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
@@ -694,21 +768,24 @@ def main():
             return
         # one untimed sample (the CPU oracle needs no more warm-up), then as many
         # timed samples as --steps asks for within a ~2.5 minute budget
+        import concurrent.futures as cf
+        threads = host_cores()
         vals = []
         desc = ""
-        t0 = time.perf_counter()
-        cpu_sample(args.workload)
-        per = max(time.perf_counter() - t0, 1e-3)
-        n = max(1, min(steps if args.steps is not None else 3, int(150.0 / per)))
-        for i in range(n):
-            v, desc = cpu_sample(args.workload, seed=i)
-            vals.append(v)
+        with cf.ThreadPoolExecutor(max_workers=threads) as pool:
+            t0 = time.perf_counter()
+            cpu_sample(args.workload, pool=pool, threads=threads)
+            per = max(time.perf_counter() - t0, 1e-3)
+            n = max(1, min(steps if args.steps is not None else 3, int(150.0 / per)))
+            for i in range(n):
+                v, desc = cpu_sample(args.workload, seed=i, pool=pool, threads=threads)
+                vals.append(v)
         v = statistics.mean(vals)
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
                 "steps": len(vals), "warmup": 1, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64 sums / fp32 scales (CPU oracle)", "data": "synthetic",
                 "config": config_of(args.workload),
-                "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle", "sample": desc},
+                "cpu_baseline": {"value": v, "unit": unit, "cores": threads, "kind": "oracle", "sample": desc},
                 "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return
@@ -863,8 +940,9 @@ def main():
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        v, desc = cpu_sample(args.workload)
-        cpu = {"value": v, "unit": wl.unit, "cores": 1, "kind": "oracle", "sample": desc}
+        v, threads, v1, desc = cpu_baseline(args.workload)
+        cpu = {"value": v, "unit": wl.unit, "cores": threads, "kind": "oracle", "sample": desc,
+               "value_1_core": v1}
     dtype = {"rowwise": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate -> bf16",
              "tensor": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate -> bf16",
              "blockmlp": "fp8_e4m3 x fp8_e4m3 -> f32 accumulate (per-128-K promotion) -> bf16",

@@ -416,8 +416,8 @@ k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 //     free, accumulator / partial ready);
 //   * both CTAs' epilogue warps release a TMEM buffer by arriving on the
 //     leader's barrier (count 2 x 8 warps).
-// BLOCK mode uses BN = 128 and four 128-column TMEM partial buffers, so the
-// MMA can run three K chunks ahead of the promotion.
+// Tensor and row scales only: the block-scaled GEMM on CTA pairs is the
+// kernel in gemm_block.cu.
 template <int MODE, int BN, bool GROUPED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
 k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
@@ -429,6 +429,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     constexpr int STG = C::STAGES, NBUF = C::NBUF;
     constexpr int HALF = BN / 2;             // columns per epilogue warp
     static_assert(BN == 256, "the pair kernel runs 256 x 256 tiles");
+    static_assert(MODE != kModeBlock, "block scales on CTA pairs: gemm_block.cu");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)STG * C::STAGE);
@@ -520,10 +521,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
     pdl_wait();      // inputs of the previous kernel in the stream are visible from here on
     pdl_trigger();
-    // BLOCK mode: each role branch resizes its own warpgroup's registers, so
-    // the epilogue code is only reachable after the increase.
     if (warp == 0) {
-        if constexpr (MODE == kModeBlock) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             int last_round[STG];
@@ -556,56 +554,41 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         __syncwarp();
     } else if (warp == 1) {
-        if constexpr (MODE == kModeBlock) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
         // ------------------------------------- MMA issuer (leader only) --
         if (leader && lane == 0) {
             uint32_t it = 0, lt = 0;
             bool ok = true;
             for (int i = 0; ok && i < n_items; ++i, ++lt) {
                 const Item w = item(i);
-                uint32_t d_tmem = tmem;
-                if (MODE != kModeBlock) {
-                    const uint32_t ab = lt % NBUF, use = lt / NBUF;
-                    if (!wait_bar(acce_bar(ab), (use & 1u) ^ 1u, abort_flag, kErrMma)) break;
-                    tc_fence_after();
-                    d_tmem = tmem + ab * BN;
-                }
+                const uint32_t ab = lt % NBUF, use = lt / NBUF;
+                if (!wait_bar(acce_bar(ab), (use & 1u) ^ 1u, abort_flag, kErrMma)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + ab * BN;
                 for (int kc = w.k0; kc < w.k1; ++kc, ++it) {
                     const int stage = it % STG;
                     const uint32_t round = it / STG;
-                    if (MODE == kModeBlock) {
-                        const uint32_t pb = it % NBUF, use = it / NBUF;
-                        if (!wait_bar(acce_bar(pb), (use & 1u) ^ 1u, abort_flag, kErrMma)) { ok = false; break; }
-                        d_tmem = tmem + pb * BN;
-                    }
                     if (!wait_bar(full_bar(stage), round & 1u, abort_flag, kErrMma)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + (size_t)stage * C::STAGE);
                     const uint64_t adesc = sdesc_k_sw128(a_addr);
                     const uint64_t bdesc = sdesc_k_sw128(a_addr + A_TILE);
 #pragma unroll
-                    for (int k = 0; k < BK / 32; ++k) {
-                        const uint32_t acc = (MODE == kModeBlock) ? (k > 0) : (kc > w.k0 || k > 0);
-                        tc_mma_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, acc);
-                    }
+                    for (int k = 0; k < BK / 32; ++k)
+                        tc_mma_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kc > w.k0 || k > 0) ? 1u : 0u);
                     tc_commit_pair_both(empty_bar(stage));
-                    if (MODE == kModeBlock) tc_commit_pair_both(accf_bar(it % NBUF));
                 }
-                if (ok && MODE != kModeBlock) tc_commit_pair_both(accf_bar(lt % NBUF));
+                if (ok) tc_commit_pair_both(accf_bar(lt % NBUF));
             }
             tc_commit_pair_self(drain_bar);
             wait_bar_drain(drain_bar, 0u);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        if constexpr (MODE == kModeBlock) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
-    } else {
-        if constexpr (MODE == kModeBlock) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(sm2::REGS_HIGH));
+    } else if (warp >= 4) {
         // --------------------------------------------------- epilogue ----
         const int sp = warp & 3;
         const int ch = (warp - 4) >> 2;
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-        uint32_t it = 0, lt = 0;
+        uint32_t lt = 0;
         bool ok = true;
         for (int i = 0; ok && i < n_items; ++i, ++lt) {
             const Item wi = item(i);
@@ -614,7 +597,7 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const bool m_ok = m < wi.row_end;
             const int n_base = n_blk * BN + ch * HALF;
             const float *sbe = sb + (int64_t)wi.e * N;   // group e's column scales (ROW)
-            if (MODE != kModeBlock) {
+            {
                 const uint32_t ab = lt % NBUF, use = lt / NBUF;
                 float rs;
                 if (MODE == kModeRow) rs = m_ok ? sa[m] : 0.0f;
@@ -711,75 +694,6 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     if (warp == 4 && lane == 0) {
                         if (wait_bar(part_bar, 0u, abort_flag, kErrSplit)) st_release_u32(flag, 0u);
                     }
-                }
-            } else {
-                // fp32 accumulator of this thread's row, 128 columns as 64 packed pairs
-                uint64_t acc[HALF / 2];
-#pragma unroll
-                for (int j = 0; j < HALF / 2; ++j) acc[j] = 0ull;
-                const int nb = n_base / 128;
-                const bool nb_ok = n_base < N;
-                // Scales run PF K blocks ahead in PF register sets (the K loop
-                // unrolled by PF so no register copy waits on a load): block
-                // kc + PF's pair is fetched right after block kc's partial is
-                // released, well before its use.
-                constexpr int PF = 2;   // scale prefetch distance in K blocks (= unroll)
-                float as_[PF], bs_[PF];
-#pragma unroll
-                for (int i = 0; i < PF; ++i) {
-                    as_[i] = (i < nk && m_ok) ? sa[(int64_t)i * M + m] : 0.0f;
-                    bs_[i] = (i < nk && nb_ok) ? sb[(int64_t)nb * nk + i] : 0.0f;
-                }
-                // one K block: wait for its partial, promote it, release it
-                auto promote = [&](int kc, float &as, float &bs) -> bool {
-                    const uint32_t pb = it % NBUF, use = it / NBUF;
-                    const float sc = __fmul_rn(as, bs);
-                    const uint64_t sc2 = pack_f32x2(__float_as_uint(sc), __float_as_uint(sc));
-                    bool w = true;
-                    if (lane == 0) w = wait_bar(accf_bar(pb), use & 1u, abort_flag, kErrEpilogue);
-                    w = __shfl_sync(0xFFFFFFFFu, w, 0);
-                    if (!w) return false;
-                    tc_fence_after();
-                    const uint32_t src = tmem + lane_base + pb * BN + ch * HALF;
-                    // two 64-column halves, one TMEM round trip each
-                    uint32_t r[64];
-                    tmem_ld32_async(src, r);
-                    tmem_ld32_async(src + 32, r + 32);
-                    tmem_wait64(r);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[j] = fma_f32x2(pack_f32x2(r[2 * j], r[2 * j + 1]), sc2, acc[j]);
-                    tmem_ld32_async(src + 64, r);
-                    tmem_ld32_async(src + 96, r + 32);
-                    tmem_wait64(r);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(pb), 0));
-                    if (kc + PF < nk) {   // block kc + PF's scales, after the release
-                        as = m_ok ? sa[(int64_t)(kc + PF) * M + m] : 0.0f;
-                        bs = nb_ok ? sb[(int64_t)nb * nk + kc + PF] : 0.0f;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        acc[32 + j] = fma_f32x2(pack_f32x2(r[2 * j], r[2 * j + 1]), sc2, acc[32 + j]);
-                    ++it;
-                    return true;
-                };
-                for (int kc = 0; ok && kc < nk; kc += PF) {
-#pragma unroll
-                    for (int i = 0; i < PF; ++i)
-                        if (ok && kc + i < nk && !promote(kc + i, as_[i], bs_[i])) ok = false;
-                }
-                if (!ok) break;
-                uint8_t *ebuf = smem + C::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
-                const int64_t row0 = wi.row0 + wi.m_blk * 256 + (int)rank * 128 + sp * 32;
-#pragma unroll
-                for (int h2 = 0; h2 < HALF / 64; ++h2) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        pk[j] = pack_bf16x2(__uint_as_float((uint32_t)acc[h2 * 32 + j]),
-                                            __uint_as_float((uint32_t)(acc[h2 * 32 + j] >> 32)));
-                    store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, wi.row_end, n_base + h2 * 64, N);
                 }
             }
         }
@@ -899,11 +813,6 @@ int pair_capacity() {
     if (cudaFuncSetAttribute(k_gemm_fp8_2sm<MODE, BN, GROUPED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm2::Cfg<BN>::SMEM) != cudaSuccess)
         return 0;
-    if (MODE == kModeBlock) {   // the setmaxnreg split assumes this launch register count
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, k_gemm_fp8_2sm<MODE, BN, GROUPED>) != cudaSuccess || fa.numRegs != sm2::REGS_LAUNCH)
-            return 0;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 64);
     cfg.blockDim = dim3(sm2::THREADS);
@@ -1044,12 +953,11 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
         const uint32_t idesc = make_idesc(fa, fb, 256, 256);
         cudaError_t e = cudaErrorUnknown;
         int cap;
-        const int dev_cap = (mode == FP8_SCALE_TENSOR) ? pair_capacity<kModeTensor, 256>()
-                            : (mode == FP8_SCALE_ROW) ? pair_capacity<kModeRow, 256>() : pair_capacity<kModeBlock, 256>();
+        const int dev_cap = (mode == FP8_SCALE_TENSOR) ? pair_capacity<kModeTensor, 256>() : pair_capacity<kModeRow, 256>();
         if (dev_cap <= 0) return FP8_ERR_CUDA;
         SplitPlan plan{(int)(((M + 255) / 256) * ((N + 255) / 256)), 0, 0};
         uint32_t epoch = 0;
-        if (mode != FP8_SCALE_BLOCK && workspace) {
+        if (workspace) {
             const SplitPlan sp = split_plan(M, N, K, dev_cap);
             if (sp.units > 0 && workspace_bytes >= sp.bytes) {
                 int dev = 0;
@@ -1062,12 +970,9 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
         if (mode == FP8_SCALE_TENSOR) {
             if ((cap = pair_capacity<kModeTensor, 256>()) > 0)
                 e = launch_gemm_2sm<kModeTensor, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap, plan, workspace, epoch);
-        } else if (mode == FP8_SCALE_ROW) {
+        } else {
             if ((cap = pair_capacity<kModeRow, 256>()) > 0)
                 e = launch_gemm_2sm<kModeRow, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap, plan, workspace, epoch);
-        } else {
-            if ((cap = pair_capacity<kModeBlock, 256>()) > 0)
-                e = launch_gemm_2sm<kModeBlock, 256>(s, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd, cap, plan, workspace, epoch);
         }
         return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
     }

@@ -31,6 +31,11 @@
 //   warp 0      TMA producer: per stage this CTA's 128 rows of A (16 KiB) and
 //               its 64-row share of each half's 128 rows of B (2 x 8 KiB);
 //   warp 1      TMEM allocator; in the even CTA the MMA issuer;
+//   warps 2-3   release warps of the two halves: they return a partial
+//               buffer to the MMA issuer once the half's four epilogue warps
+//               have read it (named barrier), so the epilogue warps never
+//               stall on the mbarrier arrive (~200 cycles when it completes
+//               a phase someone waits on);
 //   warps 4-11  epilogue: warp w promotes TMEM lane quarter w % 4 (32 rows)
 //               of half (w - 4) / 4 (128 columns) -- two 64-column round
 //               trips, scalar fp32 FMAs (fma.rn, one rounding per term);
@@ -60,7 +65,36 @@ constexpr size_t EPI_OFF = ((size_t)STAGES * STAGE + NBARS * 8 + 16 + 15) & ~(si
 constexpr size_t SMEM = 1024 + EPI_OFF + (size_t)sm2::EPI * kEpiBufBytes;
 constexpr int PF = 2;                           // scale prefetch distance in K blocks
 static_assert(SMEM <= 232448, "shared memory per block");
+// Named barriers 1-4: the four epilogue warps of half h hand K block kb's
+// finished reads to that half's release warp (warp 2 + h) through barrier
+// 1 + 2h + kb % 2 (4 x 32 arriving threads + the 32 of the release warp).
+constexpr int kReleaseThreads = 5 * 32;
 }  // namespace blk
+
+// 32 lanes x 64 consecutive fp32 columns in one load; valid after tmem_wait64.
+__device__ __forceinline__ void tmem_ld64_async(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void named_arrive(int id, int threads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
 k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
@@ -95,7 +129,7 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         for (int q = 0; q < blk::NBUF; ++q) {
             mbar_init(accf_bar(q), 1);
-            mbar_init(acce_bar(q), 2 * (sm2::EPI / 2));   // both CTAs' four warps of that half
+            mbar_init(acce_bar(q), 2);   // both CTAs' release warps of that half
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0u;
@@ -192,13 +226,30 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
     } else if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
+        // ------------------------------------------- release warp of half h --
+        // An mbarrier arrive that completes a phase a thread is waiting on
+        // stalls the arriving thread ~200 cycles; this warp takes that stall
+        // off the epilogue warps, which only arrive on a named barrier.  Every
+        // epilogue warp arrives once per K block on every path (the error path
+        // included), so each bar.sync here returns.
+        const int h = warp - 2;
+        const uint32_t release_to = leader ? 0u : mapa_shared(acce_bar(0), 0);
+        const uint32_t total = (uint32_t)n_items * (uint32_t)nk;
+        for (uint32_t it = 0; it < total; ++it) {
+            named_sync(1 + 2 * h + (int)(it & 1u), blk::kReleaseThreads);
+            if (lane == 0) {
+                const int q = 2 * (int)(it & 1u) + h;
+                if (leader) mbar_arrive(acce_bar(q));
+                else mbar_arrive_cluster(release_to + (uint32_t)(q * 8));
+            }
+            __syncwarp();
+        }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(sm2::REGS_HIGH));
         // --------------------------------------------------- epilogue ----
         const int sp = warp & 3;
         const int h = (warp - 4) >> 2;                  // half of the tile: columns h*128 .. +127
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-        const uint32_t release_to = leader ? 0u : mapa_shared(acce_bar(0), 0);   // rank 1: the leader's barriers
         uint32_t it = 0;
         bool ok = true;
         for (int i = 0; ok && i < n_items; ++i) {
@@ -232,20 +283,15 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tc_fence_after();
                 const uint32_t src = tmem + lane_base + q * 128;
                 uint32_t r[64];
-                tmem_ld32_async(src, r);
-                tmem_ld32_async(src + 32, r + 32);
+                tmem_ld64_async(src, r);
                 tmem_wait64(r);
 #pragma unroll
                 for (int j = 0; j < 64; ++j) acc[j] = fmaf(__uint_as_float(r[j]), sc, acc[j]);
-                tmem_ld32_async(src + 64, r);
-                tmem_ld32_async(src + 96, r + 32);
+                tmem_ld64_async(src + 64, r);
                 tmem_wait64(r);
+                // the partial is in registers: the release warp hands the buffer back to the MMA
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {   // the partial is in registers: hand the buffer back to the MMA
-                    if (leader) mbar_arrive(acce_bar(q));
-                    else mbar_arrive_cluster(release_to + (uint32_t)(q * 8));
-                }
+                named_arrive(1 + 2 * h + (int)(it & 1u), blk::kReleaseThreads);
                 if (kc + blk::PF < nk) {   // block kc + PF's scales, after the release
                     as = m_ok ? sa[(int64_t)(kc + blk::PF) * M + m] : 0.0f;
                     bs = nb_ok ? sb[(int64_t)nb * nk + kc + blk::PF] : 0.0f;
@@ -260,7 +306,11 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 for (int p = 0; p < blk::PF; ++p)
                     if (ok && kc + p < nk && !promote(kc + p, as_[p], bs_[p])) ok = false;
             }
-            if (!ok) break;
+            if (!ok) {   // the release warp still expects one arrival per K block
+                for (const uint32_t total = (uint32_t)n_items * (uint32_t)nk; it < total; ++it)
+                    named_arrive(1 + 2 * h + (int)(it & 1u), blk::kReleaseThreads);
+                break;
+            }
             uint8_t *ebuf = smem + blk::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {

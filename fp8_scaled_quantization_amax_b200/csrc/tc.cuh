@@ -266,8 +266,8 @@ __device__ __forceinline__ void store_rows_coalesced(uint8_t *buf, const uint32_
 namespace sm2 {
 constexpr int EPI = 8;                 // epilogue warps 4..11 (warpgroups 1 and 2)
 constexpr int THREADS = 12 * 32;       // warpgroup 0: producer (warp 0), MMA (warp 1), two idle warps
-// BLOCK mode moves registers from warpgroup 0 to the epilogue warpgroups,
-// which hold a 128-wide fp32 accumulator row per thread.  The split must
+// The block-scaled pair kernel moves registers from warpgroup 0 to the
+// epilogue warpgroups, which hold a 128-wide fp32 accumulator row per thread.  The split must
 // not exceed the launch pool: 128 * 56 + 256 * 224 = 64512 = 384 * 168,
 // so the kernel must launch at exactly 168 registers per thread (checked on
 // the host before the first launch).

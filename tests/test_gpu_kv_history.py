@@ -85,6 +85,43 @@ def test_history_sequence_bit_exact(orc, fmt):
         assert int(dev.saturated) == sat
 
 
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_history_checkpoint_resume_on_device(orc, fmt):
+    """The delayed-scaling state (history ring, position, scale) is the whole
+    checkpoint ("DeepL押注FP8" §2.3: the scale of a step is predicted from
+    the previous steps' statistics).  Run 8 steps on the device, save the
+    state to the host, reload it into fresh device buffers and run 12 more:
+    every step after the reload must equal, bit for bit, an uninterrupted
+    device run and the oracle."""
+    rng = np.random.default_rng(17 + fmt)
+    amaxes = rng.uniform(0.25, 8.0, 20).astype(np.float32)
+    amaxes[11] = 500.0 if fmt == 0 else 6e4          # a spike after the reload
+    cur = torch.empty(1, dtype=torch.float32, device="cuda")
+    full = fp8q.AmaxHistory(16, fmt)
+    part = fp8q.AmaxHistory(16, fmt)
+    ref = orc.AmaxHistory(16, fmt)
+    for a in amaxes[:8]:
+        cur.fill_(float(a))
+        full.update(cur)
+        part.update(cur)
+        ref.update(float(a))
+    saved = {k: getattr(part, k).cpu().clone() for k in ("history", "pos", "scale", "scale_inv")}
+    del part
+    resumed = fp8q.AmaxHistory(16, fmt)
+    for k, v in saved.items():
+        getattr(resumed, k).copy_(v.to("cuda"))
+    for a in amaxes[8:]:
+        cur.fill_(float(a))
+        full.update(cur)
+        resumed.update(cur)
+        sat = ref.update(float(a))
+        for k in ("history", "scale", "scale_inv"):
+            assert_f32_equal(to_np(getattr(resumed, k)), to_np(getattr(full, k)), k)
+            assert_f32_equal(to_np(getattr(resumed, k)), getattr(ref, k), k)
+        assert int(resumed.pos) == int(full.pos) == int(ref.pos[0])
+        assert int(resumed.saturated) == int(full.saturated) == sat
+
+
 def test_dgrad_delayed_scaling_loop(orc):
     """Data-gradient GEMM with delayed scaling, reduced to [512, 256] x
     W[256, 384]: per step quantize dY_t (E5M2, scale from the history, amax

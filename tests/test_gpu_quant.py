@@ -81,6 +81,30 @@ def test_tensorwise_current_scaling(orc, fmt, shape):
 
 
 @pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("n", [65535, 65536, 65537, 65544, 8, 9])
+def test_tensorwise_small_tensor_path_boundary(orc, fmt, n):
+    """Current scaling of up to 65536 elements runs in one launch (the whole
+    tensor in one CTA's registers); longer tensors take the amax pass and the
+    cast pass.  Both sides of the boundary, with an element count that is
+    not a multiple of 8 inside the small path (65535, 9: the scalar tail),
+    a NaN and an Inf in the tensor and a huge element so that the scale is
+    set by it: codes, amax, scale and both counters against the oracle."""
+    bits = _special_values(n, 40 + n % 7, huge=False) if n >= 64 else inputs.bf16_bits(
+        inputs.normal_bf16((n,), 2.0, seed=n)).copy()
+    bits[n // 2] = 0x7FC0            # NaN
+    bits[n - 1] = 0xFF80             # -Inf, in the tail when n % 8 != 0
+    bits[n // 3] = 0x4700            # 32768: the amax
+    x = inputs.from_bf16_bits(bits, "cuda")
+    counts = torch.zeros(2, dtype=torch.int32, device="cuda")
+    q, sinv, am = fp8q.quantize_tensorwise(x, fmt, counts=counts)
+    rq, rsinv, ramax, (nf, sat) = orc.quantize_tensorwise(bits, fmt)
+    assert_codes_equal(to_np(q).reshape(rq.shape), rq, fmt)
+    assert_f32_equal(to_np(sinv), np.float32([rsinv]), "scale_inv")
+    assert_f32_equal(to_np(am), np.float32([ramax]), "amax")
+    assert (int(counts[0]), int(counts[1])) == (nf, sat) and nf == 2
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
 def test_tensorwise_edge_values(orc, fmt):
     bits = _special_values(50_000, 5 + fmt, huge=False).reshape(500, 100)
     bits[3, 4] = 0x7FC0       # NaN
