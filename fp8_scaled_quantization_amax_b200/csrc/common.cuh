@@ -143,6 +143,36 @@ __device__ __forceinline__ uint32_t count_sat8(uint4 v, float s, float fm) {
     return c;
 }
 
+// Non-finite elements among 8 bf16 (NaN or +-Inf: every exponent bit set).
+__device__ __forceinline__ uint32_t count_nonfinite8(uint4 v) {
+    uint32_t c = 0;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        c += ((w[i] & 0x7F80u) == 0x7F80u) ? 1u : 0u;
+        c += ((w[i] & 0x7F800000u) == 0x7F800000u) ? 1u : 0u;
+    }
+    return c;
+}
+
+// Counters of the quantizers (counts[0] non-finite inputs, counts[1]
+// saturated elements = |fp32(x) * s| > fmax, NaN excluded, +-Inf included):
+// a unit (row, block, slice) can only have saturated elements when it holds
+// a non-finite value or when fp32(amax) * s rounds above fmax, so the
+// kernels count exactly only then.  The warp's per-thread counts are summed
+// and added by lane 0 (warp-collective: all 32 lanes call it).
+__device__ __forceinline__ bool may_saturate(bool nonfinite_seen, float amax, float s, float fm) {
+    return nonfinite_seen || __fmul_rn(amax, s) > fm;
+}
+__device__ __forceinline__ void flush_counts(uint32_t *counts, uint32_t nf, uint32_t sat) {
+    nf = __reduce_add_sync(0xFFFFFFFFu, nf);
+    sat = __reduce_add_sync(0xFFFFFFFFu, sat);
+    if ((threadIdx.x & 31) == 0) {
+        if (nf) atomicAdd(counts, nf);
+        if (sat) atomicAdd(counts + 1, sat);
+    }
+}
+
 // Streaming 16-byte load that does not allocate in L1.
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
     uint4 r;

@@ -34,10 +34,12 @@ namespace {
 constexpr int kClusterCtas = 8;
 constexpr int kKvThreads = 512;
 
-template <int FMT>
+// COUNT: the non-finite / saturated counters (a separate instantiation, so
+// the plain path keeps its registers).
+template <int FMT, bool COUNT>
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kKvThreads, 2)
 k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64_t nunit,
-           float *__restrict__ scale_inv) {
+           float *__restrict__ scale_inv, uint32_t *__restrict__ counts) {
     __shared__ uint32_t red[32];
     __shared__ uint32_t slot[2];        // this CTA's partial amax, double-buffered by slice parity
     __shared__ uint32_t slice_amax;
@@ -49,6 +51,7 @@ k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64
     const int64_t u0 = min((int64_t)rank * per, nunit);
     const int64_t u1 = min(u0 + per, nunit);
     const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+    uint32_t nf = 0, sat = 0;   // counters (counts != NULL)
     int it = 0;
     for (int64_t sl = cid; sl < BH; sl += ncl, ++it) {
         const uint4 *xs = x + 2 * sl * nunit;   // a unit is 16 elements = two uint4 of bf16
@@ -69,7 +72,8 @@ k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64
         for (; u < u1; u += kKvThreads)
             m2 = amax_fast8(amax_fast8(m2, ld_hint(xs + 2 * u, keep)), ld_hint(xs + 2 * u + 1, keep));
         uint32_t m = amax_fast_final(m2);
-        if (m == 0xFFFFFFFFu) {
+        const bool nonfin = m == 0xFFFFFFFFu;
+        if (nonfin) {
             uint32_t bad = 0;
             m = 0;
             for (int64_t j = u0 + threadIdx.x; j < u1; j += kKvThreads)
@@ -87,6 +91,8 @@ k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64
         __syncthreads();
         const float s = scale_from_amax(bf16bits_to_float(slice_amax), fm);
         if (rank == 0 && threadIdx.x == 0) scale_inv[sl] = __fdiv_rn(1.0f, s);
+        // exact counts where this thread saw a non-finite value or the slice may saturate
+        const bool cnt = COUNT && may_saturate(nonfin, bf16bits_to_float(slice_amax), s, fm);
         // pass 2: cast (the re-read hits L2)
         int64_t j = u0 + threadIdx.x;
         for (; j + 3 * kKvThreads < u1; j += 4 * kKvThreads) {
@@ -100,14 +106,23 @@ k_kv_quant(const uint4 *__restrict__ x, uint4 *__restrict__ q, int64_t BH, int64
             for (int k = 0; k < 4; ++k) {
                 uint2 c0 = cast8<FMT>(v[2 * k], s), c1 = cast8<FMT>(v[2 * k + 1], s);
                 st_hint(qs + j + k * kKvThreads, make_uint4(c0.x, c0.y, c1.x, c1.y), drop);
+                if (COUNT && cnt) {
+                    nf += count_nonfinite8(v[2 * k]) + count_nonfinite8(v[2 * k + 1]);
+                    sat += count_sat8(v[2 * k], s, fm) + count_sat8(v[2 * k + 1], s, fm);
+                }
             }
         }
         for (; j < u1; j += kKvThreads) {
             uint4 a0 = ld_hint(xs + 2 * j, drop), a1 = ld_hint(xs + 2 * j + 1, drop);
             uint2 c0 = cast8<FMT>(a0, s), c1 = cast8<FMT>(a1, s);
             st_hint(qs + j, make_uint4(c0.x, c0.y, c1.x, c1.y), drop);
+            if (COUNT && cnt) {
+                nf += count_nonfinite8(a0) + count_nonfinite8(a1);
+                sat += count_sat8(a0, s, fm) + count_sat8(a1, s, fm);
+            }
         }
     }
+    if (COUNT) flush_counts(counts, nf, sat);
     cluster.sync();   // no CTA leaves while a peer may still read its slots
 }
 
@@ -169,7 +184,7 @@ using namespace fp8q_host;
 // whole number of 8-SM clusters, so this is below sm_count / 8); cached per
 // device.  The grid never exceeds it, so no cluster waits for another to
 // finish before it can start.
-template <int FMT>
+template <int FMT, bool COUNT>
 static int max_active_clusters() {
     static int cache[64];
     int dev = 0;
@@ -187,7 +202,7 @@ static int max_active_clusters() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_kv_quant<FMT>, &cfg) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_kv_quant<FMT, COUNT>, &cfg) != cudaSuccess) return 0;
     cache[dev] = n;
     return n;
 }
@@ -200,26 +215,34 @@ static fp8_status kv_check(int64_t B, int64_t H, int64_t S, int64_t Dh) {
 }
 
 extern "C" fp8_status fp8_kv_quant(const void *kv_bf16, int64_t B, int64_t H, int64_t S, int64_t Dh,
-                                   fp8_format fmt, uint8_t *q, float *scale_inv, void *stream) {
+                                   fp8_format fmt, uint8_t *q, float *scale_inv, uint32_t *counts, void *stream) {
     if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     fp8_status c = kv_check(B, H, S, Dh);
     if (c != FP8_OK) return c;
     const int64_t BH = B * H, nunit = S * Dh / 16;
     if (BH > 0 && (!scale_inv || (nunit > 0 && (!kv_bf16 || !q)))) return FP8_ERR_INVALID_ARG;
     if ((kv_bf16 && !aligned16(kv_bf16)) || (q && !aligned16(q))) return FP8_ERR_ALIGNMENT;
+    if (counts && (reinterpret_cast<uintptr_t>(counts) & 3u)) return FP8_ERR_ALIGNMENT;
     int sms;
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
     if (BH == 0) return FP8_OK;
     cudaStream_t s = as_stream(stream);
-    const int active = fmt == FP8_E4M3 ? max_active_clusters<FP8_E4M3>() : max_active_clusters<FP8_E5M2>();
+    const bool cnt = counts != nullptr;
+    const int active = fmt == FP8_E4M3 ? (cnt ? max_active_clusters<FP8_E4M3, true>() : max_active_clusters<FP8_E4M3, false>())
+                                       : (cnt ? max_active_clusters<FP8_E5M2, true>() : max_active_clusters<FP8_E5M2, false>());
     if (active <= 0) return FP8_ERR_CUDA;
     const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(BH, active));
     const dim3 grid(clusters * kClusterCtas);
-    if (fmt == FP8_E4M3)
-        k_kv_quant<FP8_E4M3><<<grid, kKvThreads, 0, s>>>(static_cast<const uint4 *>(kv_bf16), reinterpret_cast<uint4 *>(q), BH, nunit, scale_inv);
-    else
-        k_kv_quant<FP8_E5M2><<<grid, kKvThreads, 0, s>>>(static_cast<const uint4 *>(kv_bf16), reinterpret_cast<uint4 *>(q), BH, nunit, scale_inv);
+    const uint4 *xv = static_cast<const uint4 *>(kv_bf16);
+    uint4 *qv = reinterpret_cast<uint4 *>(q);
+    if (fmt == FP8_E4M3) {
+        if (cnt) k_kv_quant<FP8_E4M3, true><<<grid, kKvThreads, 0, s>>>(xv, qv, BH, nunit, scale_inv, counts);
+        else k_kv_quant<FP8_E4M3, false><<<grid, kKvThreads, 0, s>>>(xv, qv, BH, nunit, scale_inv, counts);
+    } else {
+        if (cnt) k_kv_quant<FP8_E5M2, true><<<grid, kKvThreads, 0, s>>>(xv, qv, BH, nunit, scale_inv, counts);
+        else k_kv_quant<FP8_E5M2, false><<<grid, kKvThreads, 0, s>>>(xv, qv, BH, nunit, scale_inv, counts);
+    }
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 

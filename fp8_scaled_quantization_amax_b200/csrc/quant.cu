@@ -339,9 +339,11 @@ k_colamax(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
 template <int FMT, bool POW2>
 __global__ void __launch_bounds__(128)
 k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t rows, int64_t cols,
-                     int64_t ld, const uint32_t *__restrict__ amax_bits, float *__restrict__ scale_inv) {
+                     int64_t ld, const uint32_t *__restrict__ amax_bits, float *__restrict__ scale_inv,
+                     uint32_t *__restrict__ counts) {
     __shared__ __align__(16) uint32_t tile[64 * 16];   // [column][16 words of 4 rows]
     __shared__ float sc[64];
+    __shared__ uint32_t maysat[2];   // bit j of word w: column c0 + 32w + j has fp32(amax) * s > fmax
     constexpr float fm = fmax_of<FMT>();
     const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
     if (threadIdx.x < 64) {
@@ -350,6 +352,8 @@ k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, i
         const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
         sc[threadIdx.x] = s;
         if (blockIdx.y == 0 && gc < cols) scale_inv[gc] = __fdiv_rn(1.0f, s);
+        const uint32_t b = __ballot_sync(0xFFFFFFFFu, __fmul_rn(a, s) > fm);
+        if ((threadIdx.x & 31) == 0) maysat[threadIdx.x >> 5] = b;
     }
     const int cv = threadIdx.x & 7, rg = threadIdx.x >> 3;
     const int64_t gc = c0 + cv * 8;
@@ -365,6 +369,23 @@ k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, i
     float s8[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) s8[j] = sc[cv * 8 + j];
+    uint32_t nf = 0, sat = 0;
+    if (counts) {   // exact counts where a column may saturate or a value is not finite
+        const uint32_t cols8 = (maysat[cv >> 2] >> ((cv & 3) * 8)) & 0xFFu;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t bad = count_nonfinite8(v[k]);
+            nf += bad;
+            if (bad || cols8) {
+                const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    sat += fabsf(__fmul_rn(bf_lo(w[j]), s8[2 * j])) > fm ? 1u : 0u;
+                    sat += fabsf(__fmul_rn(bf_hi(w[j]), s8[2 * j + 1])) > fm ? 1u : 0u;
+                }
+            }
+        }
+    }
     uint32_t lo[4], hi[4];   // row k's codes of columns 0-3 and 4-7
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -403,6 +424,7 @@ k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, i
         const uint4 o = *reinterpret_cast<const uint4 *>(&tile[col * 16 + ((part ^ ((col >> 3) & 3)) * 4)]);
         if (go < cols && gi < rows) *reinterpret_cast<uint4 *>(qt + go * rows + gi) = o;
     }
+    if (counts) flush_counts(counts, nf, sat);
 }
 
 // --------------------------------------------------------------- rowwise --
@@ -421,11 +443,12 @@ struct RowJob {
 };
 template <int FMT, bool POW2, int V, int R>
 __global__ void __launch_bounds__(kRowThreads)
-k_rowwise(RowJob ja, RowJob jb, int64_t cols) {
+k_rowwise(RowJob ja, RowJob jb, int64_t cols, uint32_t *__restrict__ counts) {
     pdl_trigger();   // dependents are scheduled once all our CTAs have started
     pdl_wait();
     __shared__ uint32_t red[R][32];
     constexpr float fm = fmax_of<FMT>();
+    uint32_t nf = 0, sat = 0;   // counters (counts != NULL)
     const int64_t ncv = cols / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // groups of R rows: ja's first, then jb's
@@ -440,6 +463,7 @@ k_rowwise(RowJob ja, RowJob jb, int64_t cols) {
         if constexpr (V > 0) {
             uint4 v[R][V];
             uint32_t m[R];
+            bool nonfin[R];
 #pragma unroll
             for (int rr = 0; rr < R; ++rr) {
                 const uint4 *xr = reinterpret_cast<const uint4 *>(x + (r0 + rr) * ld);
@@ -456,7 +480,8 @@ k_rowwise(RowJob ja, RowJob jb, int64_t cols) {
 #pragma unroll
                 for (int j = 0; j < V; ++j) m2 = amax_fast8(m2, v[rr][j]);
                 m[rr] = amax_fast_final(m2);
-                if (m[rr] == 0xFFFFFFFFu) {
+                nonfin[rr] = m[rr] == 0xFFFFFFFFu;
+                if (nonfin[rr]) {
                     uint32_t bad = 0;
                     m[rr] = 0;
 #pragma unroll
@@ -480,6 +505,13 @@ k_rowwise(RowJob ja, RowJob jb, int64_t cols) {
                         if (cv < ncv) qr[cv] = cast8<FMT>(v[rr][j], s);
                     }
                     if (threadIdx.x == 0) scale_inv[r0 + rr] = __fdiv_rn(1.0f, s);
+                    if (counts && may_saturate(nonfin[rr], a, s, fm)) {   // vectors past the row are zeros
+#pragma unroll
+                        for (int j = 0; j < V; ++j) {
+                            nf += count_nonfinite8(v[rr][j]);
+                            sat += count_sat8(v[rr][j], s, fm);
+                        }
+                    }
                 }
             }
             __syncthreads();   // red[] is reused by the next rows
@@ -493,12 +525,19 @@ k_rowwise(RowJob ja, RowJob jb, int64_t cols) {
                 mm = block_max_u32(mm, red[0]);
                 const float a = bf16bits_to_float(mm);
                 const float s = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
-                for (int64_t cv = threadIdx.x; cv < ncv; cv += kRowThreads) qr[cv] = cast8<FMT>(xr[cv], s);
+                const bool cnt = counts && may_saturate(bad > 0, a, s, fm);
+                nf += bad;
+                for (int64_t cv = threadIdx.x; cv < ncv; cv += kRowThreads) {
+                    const uint4 w = xr[cv];
+                    qr[cv] = cast8<FMT>(w, s);
+                    if (cnt) sat += count_sat8(w, s, fm);
+                }
                 if (threadIdx.x == 0) scale_inv[r] = __fdiv_rn(1.0f, s);
                 __syncthreads();
             }
         }
     }
+    if (counts) flush_counts(counts, nf, sat);
 }
 
 // ---------------------------------------------------------- block 1x128 --
@@ -529,10 +568,12 @@ __device__ __forceinline__ int64_t e8m0_offset(int64_t kb, int64_t rt, int64_t r
 template <int FMT, int U, bool SF>
 __global__ void __launch_bounds__(256)
 k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-             uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image) {
+             uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image,
+             uint32_t *__restrict__ counts) {
     pdl_trigger();   // dependents are scheduled once all our CTAs have started
     pdl_wait();
     constexpr float fm = fmax_of<FMT>();
+    uint32_t nf = 0, sat = 0;   // counters (counts != NULL)
     const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
     const int64_t nkb = (cols + 127) / 128;
     const int64_t rt = (rows + 127) / 128;
@@ -557,7 +598,8 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 uint32_t m = amax_fast_final(amax_fast8(0u, v[u]));
-                if (m == 0xFFFFFFFFu) {
+                const bool nonfin = m == 0xFFFFFFFFu;
+                if (nonfin) {
                     uint32_t bad = 0;
                     m = amax_exact8(0u, v[u], bad);
                 }
@@ -569,6 +611,10 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
                 const float s = SF ? pow2_scale_from_amax(bf16bits_to_float(m), fm)
                                    : scale_from_amax(bf16bits_to_float(m), fm);
                 if (valid[u]) *reinterpret_cast<uint2 *>(qr + cidx[u]) = cast8<FMT>(v[u], s);
+                if (counts && valid[u] && may_saturate(nonfin, bf16bits_to_float(m), s, fm)) {
+                    nf += count_nonfinite8(v[u]);
+                    sat += count_sat8(v[u], s, fm);
+                }
                 const int64_t kb = kb0 + 2 * u + half;
                 if (l16 == 0 && kb < nkb) {
                     if (SF) sf_image[e8m0_offset(kb, rt, row)] = e8m0_of_scale(s);
@@ -577,6 +623,7 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
             }
         }
     }
+    if (counts) flush_counts(counts, nf, sat);
 }
 
 // -------------------------------------------------------- block 128x128 --
@@ -589,11 +636,13 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
 template <int FMT, bool SF>
 __global__ void __launch_bounds__(256)
 k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-           uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image) {
+           uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image,
+           uint32_t *__restrict__ counts) {
     pdl_trigger();   // dependents are scheduled once all our CTAs have started
     pdl_wait();
     __shared__ uint32_t red[32];
     constexpr float fm = fmax_of<FMT>();
+    uint32_t nf = 0, sat = 0;   // counters (counts != NULL)
     const int64_t nkb = (cols + 127) / 128, nrb = (rows + 127) / 128;
     const int rsub = threadIdx.x >> 4, cv = threadIdx.x & 15;
     for (int64_t t = blockIdx.x; t < nrb * nkb; t += gridDim.x) {
@@ -609,7 +658,8 @@ k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t l
             m2 = amax_fast8(m2, v[p]);
         }
         uint32_t m = amax_fast_final(m2);
-        if (m == 0xFFFFFFFFu) {
+        const bool nonfin = m == 0xFFFFFFFFu;
+        if (nonfin) {
             uint32_t bad = 0;
             m = 0;
 #pragma unroll
@@ -622,12 +672,20 @@ k_block128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t l
             const int64_t r = rb * 128 + p * 16 + rsub;
             if (r < rows && c < cols) *reinterpret_cast<uint2 *>(q + r * cols + c) = cast8<FMT>(v[p], s);
         }
+        if (counts && may_saturate(nonfin, bf16bits_to_float(m), s, fm)) {   // out-of-range vectors are zeros
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                nf += count_nonfinite8(v[p]);
+                sat += count_sat8(v[p], s, fm);
+            }
+        }
         if (SF) {
             if (threadIdx.x < 128) sf_image[e8m0_offset(kb, nrb, rb * 128 + threadIdx.x)] = e8m0_of_scale(s);
         } else if (threadIdx.x == 0) {
             scale_inv[rb * nkb + kb] = __fdiv_rn(1.0f, s);
         }
     }
+    if (counts) flush_counts(counts, nf, sat);
 }
 
 int stream_grid(int sms, int64_t work_units, int threads) {
@@ -661,7 +719,8 @@ void launch_cast(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t 
 }
 
 template <int FMT, bool POW2>
-cudaError_t launch_rowwise(cudaStream_t st, int sms, const RowJob &ja, const RowJob &jb, int64_t cols) {
+cudaError_t launch_rowwise(cudaStream_t st, int sms, const RowJob &ja, const RowJob &jb, int64_t cols,
+                           uint32_t *counts) {
     const int64_t slots = (int64_t)sms * 16;   // resident 128-thread CTAs
     const int64_t ncv = cols / 8;
     const int64_t rows = ja.rows + jb.rows;
@@ -673,32 +732,34 @@ cudaError_t launch_rowwise(cudaStream_t st, int sms, const RowJob &ja, const Row
     const int64_t rounds = (groups + slots - 1) / slots;
     const dim3 grid((unsigned)std::max<int64_t>(1, (groups + rounds - 1) / rounds)), block(T);
     if (two) {
-        if (ncv <= T) return pdl_launch(k_rowwise<FMT, POW2, 1, 2>, grid, block, 0, st, ja, jb, cols);
-        if (ncv <= 2 * T) return pdl_launch(k_rowwise<FMT, POW2, 2, 2>, grid, block, 0, st, ja, jb, cols);
-        return pdl_launch(k_rowwise<FMT, POW2, 4, 2>, grid, block, 0, st, ja, jb, cols);
+        if (ncv <= T) return pdl_launch(k_rowwise<FMT, POW2, 1, 2>, grid, block, 0, st, ja, jb, cols, counts);
+        if (ncv <= 2 * T) return pdl_launch(k_rowwise<FMT, POW2, 2, 2>, grid, block, 0, st, ja, jb, cols, counts);
+        return pdl_launch(k_rowwise<FMT, POW2, 4, 2>, grid, block, 0, st, ja, jb, cols, counts);
     }
-    if (ncv <= T) return pdl_launch(k_rowwise<FMT, POW2, 1, 1>, grid, block, 0, st, ja, jb, cols);
-    if (ncv <= 2 * T) return pdl_launch(k_rowwise<FMT, POW2, 2, 1>, grid, block, 0, st, ja, jb, cols);
-    if (ncv <= 4 * T) return pdl_launch(k_rowwise<FMT, POW2, 4, 1>, grid, block, 0, st, ja, jb, cols);
-    if (ncv <= 8 * T) return pdl_launch(k_rowwise<FMT, POW2, 8, 1>, grid, block, 0, st, ja, jb, cols);
-    if (ncv <= 16 * T) return pdl_launch(k_rowwise<FMT, POW2, 16, 1>, grid, block, 0, st, ja, jb, cols);
-    return pdl_launch(k_rowwise<FMT, POW2, 0, 1>, grid, block, 0, st, ja, jb, cols);
+    if (ncv <= T) return pdl_launch(k_rowwise<FMT, POW2, 1, 1>, grid, block, 0, st, ja, jb, cols, counts);
+    if (ncv <= 2 * T) return pdl_launch(k_rowwise<FMT, POW2, 2, 1>, grid, block, 0, st, ja, jb, cols, counts);
+    if (ncv <= 4 * T) return pdl_launch(k_rowwise<FMT, POW2, 4, 1>, grid, block, 0, st, ja, jb, cols, counts);
+    if (ncv <= 8 * T) return pdl_launch(k_rowwise<FMT, POW2, 8, 1>, grid, block, 0, st, ja, jb, cols, counts);
+    if (ncv <= 16 * T) return pdl_launch(k_rowwise<FMT, POW2, 16, 1>, grid, block, 0, st, ja, jb, cols, counts);
+    return pdl_launch(k_rowwise<FMT, POW2, 0, 1>, grid, block, 0, st, ja, jb, cols, counts);
 }
 
 template <int FMT, bool SF>
-void launch_block(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, int64_t ld,
-                  int block_rows, uint8_t *q, float *scale_inv, uint8_t *sf_image) {
+cudaError_t launch_block(cudaStream_t st, int sms, const void *x, int64_t rows, int64_t cols, int64_t ld,
+                         int block_rows, uint8_t *q, float *scale_inv, uint8_t *sf_image, uint32_t *counts) {
     const uint16_t *xs = static_cast<const uint16_t *>(x);
     const int64_t nkb = (cols + 127) / 128;
     if (block_rows == 1) {
         constexpr int U = 4;
         const int64_t r = SF ? (rows + 127) / 128 * 128 : rows;
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((r + 7) / 8, (int64_t)sms * 8));
-        pdl_launch(k_block1x128<FMT, U, SF>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q, scale_inv, sf_image);
+        return pdl_launch(k_block1x128<FMT, U, SF>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q, scale_inv,
+                          sf_image, counts);
     } else {
         const int64_t tiles = ((rows + 127) / 128) * nkb;
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)sms * 8));
-        pdl_launch(k_block128<FMT, SF>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q, scale_inv, sf_image);
+        return pdl_launch(k_block128<FMT, SF>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q, scale_inv,
+                          sf_image, counts);
     }
 }
 
@@ -773,19 +834,21 @@ extern "C" fp8_status fp8_quantize_tensorwise(const void *x_bf16, int64_t rows, 
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
+static bool counts_ok(const uint32_t *counts) { return !counts || !(reinterpret_cast<uintptr_t>(counts) & 3u); }
+
 static fp8_status dispatch_rowwise(cudaStream_t s, int sms, fp8_format fmt, int pow2, const RowJob &ja,
-                                   const RowJob &jb, int64_t cols) {
+                                   const RowJob &jb, int64_t cols, uint32_t *counts) {
     cudaError_t e;
-    if (fmt == FP8_E4M3) e = pow2 ? launch_rowwise<FP8_E4M3, true>(s, sms, ja, jb, cols)
-                                  : launch_rowwise<FP8_E4M3, false>(s, sms, ja, jb, cols);
-    else e = pow2 ? launch_rowwise<FP8_E5M2, true>(s, sms, ja, jb, cols)
-                  : launch_rowwise<FP8_E5M2, false>(s, sms, ja, jb, cols);
+    if (fmt == FP8_E4M3) e = pow2 ? launch_rowwise<FP8_E4M3, true>(s, sms, ja, jb, cols, counts)
+                                  : launch_rowwise<FP8_E4M3, false>(s, sms, ja, jb, cols, counts);
+    else e = pow2 ? launch_rowwise<FP8_E5M2, true>(s, sms, ja, jb, cols, counts)
+                  : launch_rowwise<FP8_E5M2, false>(s, sms, ja, jb, cols, counts);
     return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 extern "C" fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                            fp8_format fmt, int pow2, uint8_t *q, float *scale_inv,
-                                           void *stream) {
+                                           uint32_t *counts, void *stream) {
     if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0 || ld < cols) return FP8_ERR_SHAPE;
     if (cols % 16) return FP8_ERR_SHAPE;
@@ -795,19 +858,19 @@ extern "C" fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int
         return FP8_ERR_INVALID_ARG;
     }
     if (ld % 8) return FP8_ERR_ALIGNMENT;
-    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q))) return FP8_ERR_ALIGNMENT;
+    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q)) || !counts_ok(counts)) return FP8_ERR_ALIGNMENT;
     int sms;
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
     if (rows == 0) return FP8_OK;
     const RowJob ja{static_cast<const uint16_t *>(x_bf16), rows, ld, q, scale_inv}, jb{nullptr, 0, 0, nullptr, nullptr};
-    return dispatch_rowwise(as_stream(stream), sms, fmt, pow2, ja, jb, cols);
+    return dispatch_rowwise(as_stream(stream), sms, fmt, pow2, ja, jb, cols, counts);
 }
 
 extern "C" fp8_status fp8_quantize_rowwise_pair(const void *a_bf16, int64_t rows_a, int64_t lda, uint8_t *qa,
                                                 float *sa, const void *b_bf16, int64_t rows_b, int64_t ldb,
                                                 uint8_t *qb, float *sb, int64_t cols, fp8_format fmt, int pow2,
-                                                void *stream) {
+                                                uint32_t *counts, void *stream) {
     if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     if (rows_a < 0 || rows_b < 0 || cols < 0 || lda < cols || ldb < cols || (cols % 16)) return FP8_ERR_SHAPE;
     if ((rows_a > 0 && (!sa || (cols > 0 && (!a_bf16 || !qa)))) ||
@@ -815,7 +878,7 @@ extern "C" fp8_status fp8_quantize_rowwise_pair(const void *a_bf16, int64_t rows
         return FP8_ERR_INVALID_ARG;
     if (lda % 8 || ldb % 8) return FP8_ERR_ALIGNMENT;
     if ((a_bf16 && !aligned16(a_bf16)) || (qa && !aligned16(qa)) || (b_bf16 && !aligned16(b_bf16)) ||
-        (qb && !aligned16(qb)))
+        (qb && !aligned16(qb)) || !counts_ok(counts))
         return FP8_ERR_ALIGNMENT;
     int sms;
     fp8_status st = check_device(&sms);
@@ -823,37 +886,39 @@ extern "C" fp8_status fp8_quantize_rowwise_pair(const void *a_bf16, int64_t rows
     if (rows_a + rows_b == 0) return FP8_OK;
     const RowJob ja{static_cast<const uint16_t *>(a_bf16), rows_a, lda, qa, sa};
     const RowJob jb{static_cast<const uint16_t *>(b_bf16), rows_b, ldb, qb, sb};
-    return dispatch_rowwise(as_stream(stream), sms, fmt, pow2, ja, jb, cols);
+    return dispatch_rowwise(as_stream(stream), sms, fmt, pow2, ja, jb, cols, counts);
 }
 
 extern "C" fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                              fp8_format fmt, int block_rows, uint8_t *q, float *scale_inv,
-                                             void *stream) {
+                                             uint32_t *counts, void *stream) {
     if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     if (block_rows != 1 && block_rows != 128) return FP8_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0 || ld < cols || (cols % 16)) return FP8_ERR_SHAPE;
     if (rows > 0 && cols > 0 && (!x_bf16 || !q || !scale_inv)) return FP8_ERR_INVALID_ARG;
     if (ld % 8) return FP8_ERR_ALIGNMENT;
-    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q))) return FP8_ERR_ALIGNMENT;
+    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q)) || !counts_ok(counts)) return FP8_ERR_ALIGNMENT;
     int sms;
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
     if (rows == 0 || cols == 0) return FP8_OK;
     cudaStream_t s = as_stream(stream);
-    if (fmt == FP8_E4M3) launch_block<FP8_E4M3, false>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv, nullptr);
-    else launch_block<FP8_E5M2, false>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv, nullptr);
-    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    const cudaError_t e =
+        (fmt == FP8_E4M3)
+            ? launch_block<FP8_E4M3, false>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv, nullptr, counts)
+            : launch_block<FP8_E5M2, false>(s, sms, x_bf16, rows, cols, ld, block_rows, q, scale_inv, nullptr, counts);
+    return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 extern "C" fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                                      fp8_format fmt, int pow2, uint8_t *qT, float *scale_inv,
-                                                     float *amax_out, void *stream) {
+                                                     float *amax_out, uint32_t *counts, void *stream) {
     if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0 || ld < cols || (cols % 16) || (rows % 16)) return FP8_ERR_SHAPE;
     if ((rows + 63) / 64 > 65535 || (rows + kColRows - 1) / kColRows > 65535) return FP8_ERR_SHAPE;
     if (rows > 0 && cols > 0 && (!x_bf16 || !qT || !scale_inv || !amax_out)) return FP8_ERR_INVALID_ARG;
     if (ld % 8) return FP8_ERR_ALIGNMENT;
-    if ((x_bf16 && !aligned16(x_bf16)) || (qT && !aligned16(qT))) return FP8_ERR_ALIGNMENT;
+    if ((x_bf16 && !aligned16(x_bf16)) || (qT && !aligned16(qT)) || !counts_ok(counts)) return FP8_ERR_ALIGNMENT;
     int sms;
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
@@ -866,31 +931,34 @@ extern "C" fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t
         xs, rows, cols, ld, amax_bits);
     const dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
     if (fmt == FP8_E4M3) {
-        if (pow2) k_cast_transpose_col<FP8_E4M3, true><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
-        else k_cast_transpose_col<FP8_E4M3, false><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+        if (pow2) k_cast_transpose_col<FP8_E4M3, true><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv, counts);
+        else k_cast_transpose_col<FP8_E4M3, false><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv, counts);
     } else {
-        if (pow2) k_cast_transpose_col<FP8_E5M2, true><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
-        else k_cast_transpose_col<FP8_E5M2, false><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv);
+        if (pow2) k_cast_transpose_col<FP8_E5M2, true><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv, counts);
+        else k_cast_transpose_col<FP8_E5M2, false><<<grid, 128, 0, s>>>(xs, qT, rows, cols, ld, amax_bits, scale_inv, counts);
     }
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 extern "C" fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                                   fp8_format fmt, int block_rows, uint8_t *q, uint8_t *sf_image,
-                                                  void *stream) {
+                                                  uint32_t *counts, void *stream) {
     if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
     if (block_rows != 1 && block_rows != 128) return FP8_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0 || ld < cols || (cols % 16)) return FP8_ERR_SHAPE;
     if (rows > 0 && cols > 0 && (!x_bf16 || !q || !sf_image)) return FP8_ERR_INVALID_ARG;
     if (ld % 8) return FP8_ERR_ALIGNMENT;
-    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q)) || (sf_image && !aligned16(sf_image)))
+    if ((x_bf16 && !aligned16(x_bf16)) || (q && !aligned16(q)) || (sf_image && !aligned16(sf_image)) ||
+        !counts_ok(counts))
         return FP8_ERR_ALIGNMENT;
     int sms;
     fp8_status st = check_device(&sms);
     if (st != FP8_OK) return st;
     if (rows == 0 || cols == 0) return FP8_OK;
     cudaStream_t s = as_stream(stream);
-    if (fmt == FP8_E4M3) launch_block<FP8_E4M3, true>(s, sms, x_bf16, rows, cols, ld, block_rows, q, nullptr, sf_image);
-    else launch_block<FP8_E5M2, true>(s, sms, x_bf16, rows, cols, ld, block_rows, q, nullptr, sf_image);
-    return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    const cudaError_t e =
+        (fmt == FP8_E4M3)
+            ? launch_block<FP8_E4M3, true>(s, sms, x_bf16, rows, cols, ld, block_rows, q, nullptr, sf_image, counts)
+            : launch_block<FP8_E5M2, true>(s, sms, x_bf16, rows, cols, ld, block_rows, q, nullptr, sf_image, counts);
+    return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }

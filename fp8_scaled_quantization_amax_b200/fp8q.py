@@ -34,18 +34,18 @@ SIGNATURES = {
     "fp8_status_string": (ctypes.c_char_p, [_S]),
     "fp8_amax": (_S, [_P, _I64, _P, _P, _P]),
     "fp8_quantize_tensorwise": (_S, [_P, _I64, _I64, _I, _P, _P, _I, _P, _P, _P, _P]),
-    "fp8_quantize_rowwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
-    "fp8_quantize_blockwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
+    "fp8_quantize_rowwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
+    "fp8_quantize_blockwise": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
     "fp8_gemm_scaled": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P, ctypes.c_size_t, _P]),
     "fp8_gemm_workspace_size": (_S, [_I64, _I64, _I64, _I, _P]),
     "fp8_gemm_grouped": (_S, [_P, _I, _P, _I, _I, _P, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
     "fp8_gemm_scaled_noalloc": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
     "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
-    "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
+    "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P, _P]),
     "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
-    "fp8_quantize_rowwise_pair": (_S, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _P, _P, _I64, _I, _I, _P]),
-    "fp8_quantize_blockwise_e8m0": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
-    "fp8_quantize_rowwise_transpose": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
+    "fp8_quantize_rowwise_pair": (_S, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _P, _P, _I64, _I, _I, _P, _P]),
+    "fp8_quantize_blockwise_e8m0": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
+    "fp8_quantize_rowwise_transpose": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P]),
     "fp8_gemm_bf16_wgrad": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _I, _P]),
     "fp8_gemm_block_e8m0": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _P, _P, _P, _I64, _P]),
     "fp8_paged_kv_write": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
@@ -134,16 +134,18 @@ def fp8_quantize_tensorwise(x, rows, cols, fmt, scale_in, q, transpose_out, scal
         _ptr(amax_out), _ptr(counts), _stream(stream)))
 
 
-def fp8_quantize_rowwise(x, rows, cols, ld, fmt, pow2, q, scale_inv, stream=None):
+def fp8_quantize_rowwise(x, rows, cols, ld, fmt, pow2, q, scale_inv, counts=None, stream=None):
     _dev(x, torch.bfloat16, "x"); _dev(q, torch.uint8, "q"); _dev(scale_inv, torch.float32, "scale_inv")
+    _dev(counts, torch.int32, "counts")
     _check("fp8_quantize_rowwise", lib().fp8_quantize_rowwise(
-        _ptr(x), rows, cols, ld, fmt, int(pow2), _ptr(q), _ptr(scale_inv), _stream(stream)))
+        _ptr(x), rows, cols, ld, fmt, int(pow2), _ptr(q), _ptr(scale_inv), _ptr(counts), _stream(stream)))
 
 
-def fp8_quantize_blockwise(x, rows, cols, ld, fmt, block_rows, q, scale_inv, stream=None):
+def fp8_quantize_blockwise(x, rows, cols, ld, fmt, block_rows, q, scale_inv, counts=None, stream=None):
     _dev(x, torch.bfloat16, "x"); _dev(q, torch.uint8, "q"); _dev(scale_inv, torch.float32, "scale_inv")
+    _dev(counts, torch.int32, "counts")
     _check("fp8_quantize_blockwise", lib().fp8_quantize_blockwise(
-        _ptr(x), rows, cols, ld, fmt, block_rows, _ptr(q), _ptr(scale_inv), _stream(stream)))
+        _ptr(x), rows, cols, ld, fmt, block_rows, _ptr(q), _ptr(scale_inv), _ptr(counts), _stream(stream)))
 
 
 def fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, ldd, workspace=None,
@@ -191,9 +193,10 @@ def fp8_amax_history_update(history, pos, amax_cur, fmt, scale, scale_inv, satur
         _ptr(saturated), _stream(stream)))
 
 
-def fp8_kv_quant(kv, B, H, S, Dh, fmt, q, scale_inv, stream=None):
+def fp8_kv_quant(kv, B, H, S, Dh, fmt, q, scale_inv, counts=None, stream=None):
     _dev(kv, torch.bfloat16, "kv"); _dev(q, torch.uint8, "q"); _dev(scale_inv, torch.float32, "scale_inv")
-    _check("fp8_kv_quant", lib().fp8_kv_quant(_ptr(kv), B, H, S, Dh, fmt, _ptr(q), _ptr(scale_inv),
+    _dev(counts, torch.int32, "counts")
+    _check("fp8_kv_quant", lib().fp8_kv_quant(_ptr(kv), B, H, S, Dh, fmt, _ptr(q), _ptr(scale_inv), _ptr(counts),
                                               _stream(stream)))
 
 
@@ -203,10 +206,11 @@ def fp8_kv_dequant(q, scale_inv, B, H, S, Dh, fmt, out, stream=None):
                                                   _stream(stream)))
 
 
-def fp8_quantize_blockwise_e8m0(x, rows, cols, ld, fmt, block_rows, q, sf_image, stream=None):
+def fp8_quantize_blockwise_e8m0(x, rows, cols, ld, fmt, block_rows, q, sf_image, counts=None, stream=None):
     _dev(x, torch.bfloat16, "x"); _dev(q, torch.uint8, "q"); _dev(sf_image, torch.uint8, "sf_image")
+    _dev(counts, torch.int32, "counts")
     _check("fp8_quantize_blockwise_e8m0", lib().fp8_quantize_blockwise_e8m0(
-        _ptr(x), rows, cols, ld, fmt, block_rows, _ptr(q), _ptr(sf_image), _stream(stream)))
+        _ptr(x), rows, cols, ld, fmt, block_rows, _ptr(q), _ptr(sf_image), _ptr(counts), _stream(stream)))
 
 
 def fp8_gemm_block_e8m0(A, fa, B, fb, M, N, K, a_sf, b_sf, D, ldd, stream=None):
@@ -216,15 +220,17 @@ def fp8_gemm_block_e8m0(A, fa, B, fb, M, N, K, a_sf, b_sf, D, ldd, stream=None):
         _ptr(A), fa, _ptr(B), fb, M, N, K, _ptr(a_sf), _ptr(b_sf), _ptr(D), ldd, _stream(stream)))
 
 
-def fp8_quantize_rowwise_pair(a, rows_a, lda, qa, sa, b, rows_b, ldb, qb, sb, cols, fmt, pow2, stream=None):
+def fp8_quantize_rowwise_pair(a, rows_a, lda, qa, sa, b, rows_b, ldb, qb, sb, cols, fmt, pow2, counts=None,
+                              stream=None):
     _dev(a, torch.bfloat16, "a"); _dev(qa, torch.uint8, "qa"); _dev(sa, torch.float32, "sa")
     _dev(b, torch.bfloat16, "b"); _dev(qb, torch.uint8, "qb"); _dev(sb, torch.float32, "sb")
+    _dev(counts, torch.int32, "counts")
     _check("fp8_quantize_rowwise_pair", lib().fp8_quantize_rowwise_pair(
         _ptr(a), rows_a, lda, _ptr(qa), _ptr(sa), _ptr(b), rows_b, ldb, _ptr(qb), _ptr(sb), cols, fmt, int(pow2),
-        _stream(stream)))
+        _ptr(counts), _stream(stream)))
 
 
-def quantize_rowwise_pair(a, b, fmt=E4M3, pow2=True):
+def quantize_rowwise_pair(a, b, fmt=E4M3, pow2=True, counts=None):
     """((qa, sa), (qb, sb)) of a [Ma, K] and b [Mb, K] in one launch."""
     K = a.shape[1]
     if b.shape[1] != K:
@@ -233,24 +239,28 @@ def quantize_rowwise_pair(a, b, fmt=E4M3, pow2=True):
     qb = torch.empty(b.shape, dtype=torch.uint8, device=b.device)
     sa = torch.empty(a.shape[0], dtype=torch.float32, device=a.device)
     sb = torch.empty(b.shape[0], dtype=torch.float32, device=b.device)
-    fp8_quantize_rowwise_pair(a, a.shape[0], a.stride(0), qa, sa, b, b.shape[0], b.stride(0), qb, sb, K, fmt, pow2)
+    fp8_quantize_rowwise_pair(a, a.shape[0], a.stride(0), qa, sa, b, b.shape[0], b.stride(0), qb, sb, K, fmt, pow2,
+                              counts)
     return (qa, sa), (qb, sb)
 
 
-def fp8_quantize_rowwise_transpose(x, rows, cols, ld, fmt, pow2, qT, scale_inv, amax_out, stream=None):
+def fp8_quantize_rowwise_transpose(x, rows, cols, ld, fmt, pow2, qT, scale_inv, amax_out, counts=None,
+                                   stream=None):
     _dev(x, torch.bfloat16, "x"); _dev(qT, torch.uint8, "qT")
     _dev(scale_inv, torch.float32, "scale_inv"); _dev(amax_out, torch.float32, "amax_out")
+    _dev(counts, torch.int32, "counts")
     _check("fp8_quantize_rowwise_transpose", lib().fp8_quantize_rowwise_transpose(
-        _ptr(x), rows, cols, ld, fmt, int(pow2), _ptr(qT), _ptr(scale_inv), _ptr(amax_out), _stream(stream)))
+        _ptr(x), rows, cols, ld, fmt, int(pow2), _ptr(qT), _ptr(scale_inv), _ptr(amax_out), _ptr(counts),
+        _stream(stream)))
 
 
-def quantize_rowwise_transpose(x, fmt, pow2=True):
+def quantize_rowwise_transpose(x, fmt, pow2=True, counts=None):
     """(qT [cols, rows], scale_inv [cols], amax [cols]) of x [rows, cols]."""
     rows, cols = x.shape
     qT = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
     sinv = torch.empty(cols, dtype=torch.float32, device=x.device)
     am = torch.empty(cols, dtype=torch.float32, device=x.device)
-    fp8_quantize_rowwise_transpose(x, rows, cols, x.stride(0), fmt, pow2, qT, sinv, am)
+    fp8_quantize_rowwise_transpose(x, rows, cols, x.stride(0), fmt, pow2, qT, sinv, am, counts)
     return qT, sinv, am
 
 
@@ -273,12 +283,12 @@ def e8m0_image_bytes(rows: int, cols: int) -> int:
     return ((cols + 511) // 512) * ((rows + 127) // 128) * 512
 
 
-def quantize_blockwise_e8m0(x, fmt, block_rows):
+def quantize_blockwise_e8m0(x, fmt, block_rows, counts=None):
     """(q, sf_image) of x [rows, cols] with power-of-two block scales."""
     rows, cols = x.shape
     q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     img = torch.empty(e8m0_image_bytes(rows, cols), dtype=torch.uint8, device=x.device)
-    fp8_quantize_blockwise_e8m0(x, rows, cols, x.stride(0), fmt, block_rows, q, img)
+    fp8_quantize_blockwise_e8m0(x, rows, cols, x.stride(0), fmt, block_rows, q, img, counts)
     return q, img
 
 
@@ -342,15 +352,17 @@ def quantize_tensorwise(x, fmt=E4M3, scale_in=None, transpose=False, counts=None
     return q, sinv, am
 
 
-def quantize_rowwise(x, fmt=E4M3, pow2=True):
+def quantize_rowwise(x, fmt=E4M3, pow2=True, counts=None):
+    """(q, scale_inv) of x [rows, cols]; counts: an int32 [2] device tensor
+    the non-finite and saturated counts are added to, or None."""
     rows, cols = x.shape
     q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     sinv = torch.empty(rows, dtype=torch.float32, device=x.device)
-    fp8_quantize_rowwise(x, rows, cols, x.stride(0), fmt, pow2, q, sinv)
+    fp8_quantize_rowwise(x, rows, cols, x.stride(0), fmt, pow2, q, sinv, counts)
     return q, sinv
 
 
-def quantize_blockwise(x, fmt=E4M3, block_rows=1):
+def quantize_blockwise(x, fmt=E4M3, block_rows=1, counts=None):
     rows, cols = x.shape
     nkb = (cols + 127) // 128
     q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
@@ -358,7 +370,7 @@ def quantize_blockwise(x, fmt=E4M3, block_rows=1):
         sinv = torch.empty((nkb, rows), dtype=torch.float32, device=x.device)
     else:
         sinv = torch.empty(((rows + block_rows - 1) // block_rows, nkb), dtype=torch.float32, device=x.device)
-    fp8_quantize_blockwise(x, rows, cols, x.stride(0), fmt, block_rows, q, sinv)
+    fp8_quantize_blockwise(x, rows, cols, x.stride(0), fmt, block_rows, q, sinv, counts)
     return q, sinv
 
 
@@ -386,11 +398,11 @@ def gemm_grouped(A, fa, B, fb, group_offsets, mode, a_scale_inv, b_scale_inv, ou
     return D
 
 
-def kv_quant(kv, fmt=E4M3):
+def kv_quant(kv, fmt=E4M3, counts=None):
     B, H, S, Dh = kv.shape
     q = torch.empty(kv.shape, dtype=torch.uint8, device=kv.device)
     sinv = torch.empty(B * H, dtype=torch.float32, device=kv.device)
-    fp8_kv_quant(kv, B, H, S, Dh, fmt, q, sinv)
+    fp8_kv_quant(kv, B, H, S, Dh, fmt, q, sinv, counts)
     return q, sinv
 
 

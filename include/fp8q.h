@@ -112,11 +112,16 @@ FP8Q_API fp8_status fp8_quantize_tensorwise(const void *x_bf16, int64_t rows, in
  * amax_r * s_r <= fmax; pow2 == 0: s_r = fmax / amax_r.
  *   q          [rows, cols] FP8, dense.
  *   scale_inv  [rows] fp32, d_r = 1 / s_r.
+ *   counts     [2] uint32 or NULL: [0] += non-finite inputs (NaN, +-Inf),
+ *              [1] += saturated elements (|fp32(x) * s| > fmax: +-Inf and
+ *              values whose scaled magnitude rounds past fmax; NaN is not
+ *              saturated) -- [DeepL] §5.1: overflow and NaN are the failures
+ *              to detect.  Added to, never reset; 4-byte aligned.
  *   Shapes: cols % 16 == 0, ld % 8 == 0, ld >= cols.
  */
 FP8Q_API fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                 fp8_format fmt, int pow2, uint8_t *q, float *scale_inv,
-                                void *stream);
+                                uint32_t *counts, void *stream);
 
 /*
  * Both operands of a rowwise GEMM in one launch: fp8_quantize_rowwise of
@@ -125,10 +130,12 @@ FP8Q_API fp8_status fp8_quantize_rowwise(const void *x_bf16, int64_t rows, int64
  * forward GEMM's activations and weights share K and E4M3).  One launch
  * instead of two saves a launch gap and a ramp on short tensors.  Shapes,
  * layouts and errors as fp8_quantize_rowwise; either count may be 0.
+ * counts (as fp8_quantize_rowwise) adds both tensors' counts.
  */
 FP8Q_API fp8_status fp8_quantize_rowwise_pair(const void *a_bf16, int64_t rows_a, int64_t lda, uint8_t *qa,
                                      float *sa, const void *b_bf16, int64_t rows_b, int64_t ldb, uint8_t *qb,
-                                     float *sb, int64_t cols, fp8_format fmt, int pow2, void *stream);
+                                     float *sb, int64_t cols, fp8_format fmt, int pow2, uint32_t *counts,
+                                     void *stream);
 
 /*
  * Per-block quantization ([DeepL] §2.3: the tensor is cut into small blocks
@@ -139,11 +146,16 @@ FP8Q_API fp8_status fp8_quantize_rowwise_pair(const void *a_bf16, int64_t rows_a
  *   scale_inv  block_rows == 1  : [ceil(cols/128), rows]  (row index fastest,
  *                                  the layout the GEMM reads per K block);
  *              block_rows == 128: [ceil(rows/128), ceil(cols/128)].
+ *   counts     [2] uint32 or NULL: [0] += non-finite inputs (NaN, +-Inf),
+ *              [1] += saturated elements (|fp32(x) * s| > fmax: +-Inf and
+ *              values whose scaled magnitude rounds past fmax; NaN is not
+ *              saturated) -- [DeepL] §5.1: overflow and NaN are the failures
+ *              to detect.  Added to, never reset; 4-byte aligned.
  *   Shapes: cols % 16 == 0, ld % 8 == 0, ld >= cols.
  */
 FP8Q_API fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                   fp8_format fmt, int block_rows, uint8_t *q, float *scale_inv,
-                                  void *stream);
+                                  uint32_t *counts, void *stream);
 
 /*
  * Rowwise quantization of the transpose, for the backward GEMMs ([Soup]
@@ -158,13 +170,18 @@ FP8Q_API fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int
  *   scale_inv  [cols] fp32, 1 / s_c.
  *   amax_out   [cols] fp32, the column amax (also used as the kernels'
  *              reduction buffer; overwritten).
+ *   counts     [2] uint32 or NULL: [0] += non-finite inputs (NaN, +-Inf),
+ *              [1] += saturated elements (|fp32(x) * s| > fmax: +-Inf and
+ *              values whose scaled magnitude rounds past fmax; NaN is not
+ *              saturated) -- [DeepL] §5.1: overflow and NaN are the failures
+ *              to detect.  Added to, never reset; 4-byte aligned.
  *   Shapes: rows % 16 == 0, cols % 16 == 0, ld % 8 == 0, ld >= cols,
  *   ceil(rows / 64) <= 65535.  Three launches: a memset of amax_out, the
  *   column reduction, the transposing cast.
  */
 FP8Q_API fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                           fp8_format fmt, int pow2, uint8_t *qT, float *scale_inv,
-                                          float *amax_out, void *stream);
+                                          float *amax_out, uint32_t *counts, void *stream);
 
 /*
  * Per-block quantization with power-of-two scales written as an E8M0 scale
@@ -183,11 +200,12 @@ FP8Q_API fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t r
  *             the last 128-row group: e = 127 when block_rows == 1, the
  *             block's e when block_rows == 128.  Bytes of K blocks past the
  *             last one are not written.
+ *   counts    as fp8_quantize_blockwise.
  *   Shapes and errors: as fp8_quantize_blockwise.
  */
 FP8Q_API fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                        fp8_format fmt, int block_rows, uint8_t *q, uint8_t *sf_image,
-                                       void *stream);
+                                       uint32_t *counts, void *stream);
 
 /*
  * FP8 scaled GEMM ([H100]: the multiply-accumulate runs on FP8 operands on
@@ -355,10 +373,12 @@ FP8Q_API fp8_status fp8_amax_history_update(float *history, int32_t *pos, int le
  * cache).  kv [B, H, S, Dh] bf16; each (b, h) slice of S*Dh elements gets a
  * per-tensor scale s = fmax / amax(slice).
  *   q          [B, H, S, Dh] FP8.   scale_inv [B*H] fp32.
+ *   counts     [2] uint32 or NULL: [0] += non-finite inputs, [1] += saturated
+ *              elements (as fp8_quantize_rowwise); 4-byte aligned.
  *   Shapes: (S*Dh) % 16 == 0, B*H <= 65535.
  */
 FP8Q_API fp8_status fp8_kv_quant(const void *kv_bf16, int64_t B, int64_t H, int64_t S, int64_t Dh,
-                        fp8_format fmt, uint8_t *q, float *scale_inv, void *stream);
+                        fp8_format fmt, uint8_t *q, float *scale_inv, uint32_t *counts, void *stream);
 
 /*
  * FP8 KV-cache dequantization when the cache is read ([DeepL] §3.1):

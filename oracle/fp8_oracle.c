@@ -262,18 +262,23 @@ void orc_quantize_tensorwise(const uint16_t *x, int64_t rows, int64_t cols, int 
 
 /* One scale per row of a [rows, cols] tensor (leading dimension ld)
  * ([DeepL] §2.3 per-row; [Soup] rowwise recipe, pow2 scales when pow2 != 0).
- * q is dense [rows, cols]; scale_inv[r] = 1 / s_r. */
+ * q is dense [rows, cols]; scale_inv[r] = 1 / s_r.  counts (may be NULL):
+ * counts[0] += non-finite inputs, counts[1] += saturated elements, as the
+ * tensorwise quantizer counts them ([DeepL] §5.1: overflow and NaN are the
+ * failures to watch). */
 void orc_quantize_rowwise(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
-                          int fmt, int pow2, uint8_t *q, float *scale_inv)
+                          int fmt, int pow2, uint8_t *q, float *scale_inv, uint64_t *counts)
 {
     float fm = (float)orc_fmax(fmt);
+    uint64_t nf = 0, sat = 0;
     for (int64_t r = 0; r < rows; ++r) {
         const uint16_t *row = x + r * ld;
-        float amax = orc_amax_bf16(row, cols, NULL);
+        float amax = orc_amax_bf16(row, cols, &nf);
         float s = pow2 ? orc_scale_pow2_from_amax(amax, fmt) : orc_scale_from_amax(amax, fmt);
-        for (int64_t c = 0; c < cols; ++c) q[r * cols + c] = cast_one(row[c], s, fmt, fm, NULL);
+        for (int64_t c = 0; c < cols; ++c) q[r * cols + c] = cast_one(row[c], s, fmt, fm, &sat);
         scale_inv[r] = orc_inverse(s);
     }
+    if (counts) { counts[0] += nf; counts[1] += sat; }
 }
 
 /* -------------------------------------------------- blockwise quantize -- */
@@ -284,11 +289,14 @@ void orc_quantize_rowwise(const uint16_t *x, int64_t rows, int64_t cols, int64_t
  * elements.  q is dense [rows, cols].
  * Scale layout (the GEMM's):
  *   block_rows == 1  : scale_inv[kb * rows + r]            ([ceil(cols/128), rows])
- *   block_rows == 128: scale_inv[rb * ceil(cols/128) + kb] ([ceil(rows/128), ceil(cols/128)]) */
+ *   block_rows == 128: scale_inv[rb * ceil(cols/128) + kb] ([ceil(rows/128), ceil(cols/128)])
+ * counts (may be NULL): non-finite inputs and saturated elements, added. */
 void orc_quantize_blockwise(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
-                            int fmt, int block_rows, int pow2, uint8_t *q, float *scale_inv)
+                            int fmt, int block_rows, int pow2, uint8_t *q, float *scale_inv,
+                            uint64_t *counts)
 {
     float fm = (float)orc_fmax(fmt);
+    uint64_t nf = 0, sat = 0;
     int64_t nkb = (cols + 127) / 128;
     int64_t nrb = (rows + block_rows - 1) / block_rows;
     for (int64_t rb = 0; rb < nrb; ++rb)
@@ -299,15 +307,16 @@ void orc_quantize_blockwise(const uint16_t *x, int64_t rows, int64_t cols, int64
             if (c1 > cols) c1 = cols;
             float amax = 0.0f;
             for (int64_t r = r0; r < r1; ++r) {
-                float a = orc_amax_bf16(x + r * ld + c0, c1 - c0, NULL);
+                float a = orc_amax_bf16(x + r * ld + c0, c1 - c0, &nf);
                 if (a > amax) amax = a;
             }
             float s = pow2 ? orc_scale_pow2_from_amax(amax, fmt) : orc_scale_from_amax(amax, fmt);
             for (int64_t r = r0; r < r1; ++r)
-                for (int64_t c = c0; c < c1; ++c) q[r * cols + c] = cast_one(x[r * ld + c], s, fmt, fm, NULL);
+                for (int64_t c = c0; c < c1; ++c) q[r * cols + c] = cast_one(x[r * ld + c], s, fmt, fm, &sat);
             if (block_rows == 1) scale_inv[kb * rows + rb] = orc_inverse(s);
             else scale_inv[rb * nkb + kb] = orc_inverse(s);
         }
+    if (counts) { counts[0] += nf; counts[1] += sat; }
 }
 
 /* ------------------------------------------------------------------ GEMM -- */
@@ -448,17 +457,21 @@ void orc_amax_history_update(float *history, int32_t *pos, int len, float amax_c
 
 /* FP8 KV cache ([DeepL] §3.1: K and V stored in FP8, halving memory).
  * x is [B, H, S, Dh] bf16; every (b, h) slice of S*Dh elements gets its own
- * per-tensor scale.  q is the same layout, scale_inv[b*H + h] = 1/s. */
-void orc_kv_quant(const uint16_t *x, int64_t BH, int64_t SD, int fmt, uint8_t *q, float *scale_inv)
+ * per-tensor scale.  q is the same layout, scale_inv[b*H + h] = 1/s.
+ * counts (may be NULL): non-finite inputs and saturated elements, added. */
+void orc_kv_quant(const uint16_t *x, int64_t BH, int64_t SD, int fmt, uint8_t *q, float *scale_inv,
+                  uint64_t *counts)
 {
     float fm = (float)orc_fmax(fmt);
+    uint64_t nf = 0, sat = 0;
     for (int64_t i = 0; i < BH; ++i) {
         const uint16_t *sl = x + i * SD;
-        float amax = orc_amax_bf16(sl, SD, NULL);
+        float amax = orc_amax_bf16(sl, SD, &nf);
         float s = orc_scale_from_amax(amax, fmt);
-        for (int64_t j = 0; j < SD; ++j) q[i * SD + j] = cast_one(sl[j], s, fmt, fm, NULL);
+        for (int64_t j = 0; j < SD; ++j) q[i * SD + j] = cast_one(sl[j], s, fmt, fm, &sat);
         scale_inv[i] = orc_inverse(s);
     }
+    if (counts) { counts[0] += nf; counts[1] += sat; }
 }
 
 /* Dequantization when the cache is read: x_hat = bf16(fp32(dec(q)) * d). */
@@ -573,23 +586,26 @@ void orc_paged_kv_gather(const uint8_t *cache, const float *scale_cache, const i
  * gradient dW = dY^T X, output channels for the data gradient dX = dY W --
  * so their K-major operands are transposes: qT[c][r] = cast(x[r][c], s_c)
  * with s_c from the amax of COLUMN c of x (a row of x^T), scale_inv[c] = 1/s_c.
- * x [rows, cols] with leading dimension ld; qT [cols, rows]. */
+ * x [rows, cols] with leading dimension ld; qT [cols, rows].
+ * counts (may be NULL): non-finite inputs and saturated elements, added. */
 void orc_quantize_rowwise_transpose(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
-                                    int pow2, uint8_t *qT, float *scale_inv)
+                                    int pow2, uint8_t *qT, float *scale_inv, uint64_t *counts)
 {
     float fm = (float)orc_fmax(fmt);
+    uint64_t nf = 0, sat = 0;
     for (int64_t c = 0; c < cols; ++c) {
         float amax = 0.0f;
         for (int64_t r = 0; r < rows; ++r) {
             uint16_t h = x[r * ld + c];
-            if (!bf16_finite(h)) continue;
+            if (!bf16_finite(h)) { ++nf; continue; }
             float a = fabsf(bf16_to_f32(h));
             if (a > amax) amax = a;
         }
         float s = pow2 ? orc_scale_pow2_from_amax(amax, fmt) : orc_scale_from_amax(amax, fmt);
-        for (int64_t r = 0; r < rows; ++r) qT[c * rows + r] = cast_one(x[r * ld + c], s, fmt, fm, NULL);
+        for (int64_t r = 0; r < rows; ++r) qT[c * rows + r] = cast_one(x[r * ld + c], s, fmt, fm, &sat);
         scale_inv[c] = orc_inverse(s);
     }
+    if (counts) { counts[0] += nf; counts[1] += sat; }
 }
 
 /* Weight gradient kept in high precision (the same section: the

@@ -68,9 +68,9 @@ def lib():
         L.orc_quantize_tensorwise.restype = None
         L.orc_quantize_tensorwise.argtypes = [P, I64, I64, I, P, I, P, P, P, P]
         L.orc_quantize_rowwise.restype = None
-        L.orc_quantize_rowwise.argtypes = [P, I64, I64, I64, I, I, P, P]
+        L.orc_quantize_rowwise.argtypes = [P, I64, I64, I64, I, I, P, P, P]
         L.orc_quantize_blockwise.restype = None
-        L.orc_quantize_blockwise.argtypes = [P, I64, I64, I64, I, I, I, P, P]
+        L.orc_quantize_blockwise.argtypes = [P, I64, I64, I64, I, I, I, P, P, P]
         L.orc_gemm_scaled.restype = None
         L.orc_gemm_scaled.argtypes = [P, I, P, I, I64, I64, I64, I, P, P, P, P]
         L.orc_gemm_scaled_sampled.restype = None
@@ -80,7 +80,7 @@ def lib():
         L.orc_amax_history_update.restype = None
         L.orc_amax_history_update.argtypes = [P, P, I, F, I, P, P, P]
         L.orc_kv_quant.restype = None
-        L.orc_kv_quant.argtypes = [P, I64, I64, I, P, P]
+        L.orc_kv_quant.argtypes = [P, I64, I64, I, P, P, P]
         L.orc_kv_dequant.restype = None
         L.orc_kv_dequant.argtypes = [P, P, I64, I64, I, P]
         L.orc_paged_kv_write.restype = None
@@ -88,7 +88,7 @@ def lib():
         L.orc_paged_kv_gather.restype = None
         L.orc_paged_kv_gather.argtypes = [P, P, P, P, I64, I64, I64, I64, I64, I64, I64, I, P]
         L.orc_quantize_rowwise_transpose.restype = None
-        L.orc_quantize_rowwise_transpose.argtypes = [P, I64, I64, I64, I, I, P, P]
+        L.orc_quantize_rowwise_transpose.argtypes = [P, I64, I64, I64, I, I, P, P, P]
         L.orc_gemm_bf16_wgrad_sampled.restype = None
         L.orc_gemm_bf16_wgrad_sampled.argtypes = [P, P, I64, I64, I64, P, P, I64, P, P]
         L.orc_scale_stats.restype = None
@@ -182,20 +182,28 @@ def _rows_cols_ld(x: np.ndarray, cols):
     return rows, cols, ld
 
 
-def quantize_rowwise(x_bits: np.ndarray, fmt: int, pow2: bool = True, cols=None):
+def _with_counts(res, counts, want):
+    return (*res, (int(counts[0]), int(counts[1]))) if want else res
+
+
+def quantize_rowwise(x_bits: np.ndarray, fmt: int, pow2: bool = True, cols=None, counts: bool = False):
     """x [rows, ld] (the first ``cols`` columns of each row are the tensor;
-    cols=None: all) -> (q [rows, cols], scale_inv [rows])."""
+    cols=None: all) -> (q [rows, cols], scale_inv [rows]) and, with
+    counts=True, (non-finite inputs, saturated elements)."""
     x = _u16(x_bits)
     rows, cols, ld = _rows_cols_ld(x, cols)
     q = np.empty((rows, cols), np.uint8)
     sinv = np.empty(rows, np.float32)
-    lib().orc_quantize_rowwise(_p(x), rows, cols, ld, fmt, int(pow2), _p(q), _p(sinv))
-    return q, sinv
+    c = np.zeros(2, np.uint64)
+    lib().orc_quantize_rowwise(_p(x), rows, cols, ld, fmt, int(pow2), _p(q), _p(sinv), _p(c))
+    return _with_counts((q, sinv), c, counts)
 
 
-def quantize_blockwise(x_bits: np.ndarray, fmt: int, block_rows: int, pow2: bool = False, cols=None):
+def quantize_blockwise(x_bits: np.ndarray, fmt: int, block_rows: int, pow2: bool = False, cols=None,
+                       counts: bool = False):
     """x [rows, ld] (the first ``cols`` columns of each row are the tensor;
-    cols=None: all) -> (q [rows, cols], scales).  block_rows 1: scales
+    cols=None: all) -> (q [rows, cols], scales) and, with counts=True,
+    (non-finite inputs, saturated elements).  block_rows 1: scales
     [ceil(cols/128), rows]; block_rows 128: scales [ceil(rows/128), ceil(cols/128)]."""
     x = _u16(x_bits)
     rows, cols, ld = _rows_cols_ld(x, cols)
@@ -205,8 +213,9 @@ def quantize_blockwise(x_bits: np.ndarray, fmt: int, block_rows: int, pow2: bool
         sinv = np.empty((nkb, rows), np.float32)
     else:
         sinv = np.empty(((rows + block_rows - 1) // block_rows, nkb), np.float32)
-    lib().orc_quantize_blockwise(_p(x), rows, cols, ld, fmt, block_rows, int(pow2), _p(q), _p(sinv))
-    return q, sinv
+    c = np.zeros(2, np.uint64)
+    lib().orc_quantize_blockwise(_p(x), rows, cols, ld, fmt, block_rows, int(pow2), _p(q), _p(sinv), _p(c))
+    return _with_counts((q, sinv), c, counts)
 
 
 # -------------------------------------------------------------------- GEMM --
@@ -315,14 +324,16 @@ class AmaxHistory:
 
 # ---------------------------------------------------------------- KV cache --
 
-def kv_quant(x_bits: np.ndarray, fmt: int = E4M3):
-    """x [B, H, S, Dh] bf16 bits -> (q same shape, scale_inv [B*H])."""
+def kv_quant(x_bits: np.ndarray, fmt: int = E4M3, counts: bool = False):
+    """x [B, H, S, Dh] bf16 bits -> (q same shape, scale_inv [B*H]) and, with
+    counts=True, (non-finite inputs, saturated elements)."""
     x = _u16(x_bits)
     B, H, S, Dh = x.shape
     q = np.empty(x.shape, np.uint8)
     sinv = np.empty(B * H, np.float32)
-    lib().orc_kv_quant(_p(x), B * H, S * Dh, fmt, _p(q), _p(sinv))
-    return q, sinv
+    c = np.zeros(2, np.uint64)
+    lib().orc_kv_quant(_p(x), B * H, S * Dh, fmt, _p(q), _p(sinv), _p(c))
+    return _with_counts((q, sinv), c, counts)
 
 
 def kv_dequant(q: np.ndarray, scale_inv: np.ndarray, fmt: int = E4M3) -> np.ndarray:
@@ -336,15 +347,17 @@ def kv_dequant(q: np.ndarray, scale_inv: np.ndarray, fmt: int = E4M3) -> np.ndar
 
 # ------------------------------------------ backward operands, wgrad GEMM --
 
-def quantize_rowwise_transpose(x_bits: np.ndarray, fmt: int, pow2: bool = True):
+def quantize_rowwise_transpose(x_bits: np.ndarray, fmt: int, pow2: bool = True, counts: bool = False):
     """x [rows, cols] -> (qT [cols, rows], scale_inv [cols]): rowwise
-    quantization of x^T (one scale per column of x)."""
+    quantization of x^T (one scale per column of x); with counts=True also
+    (non-finite inputs, saturated elements)."""
     x = _u16(x_bits)
     rows, cols = x.shape
     qT = np.empty((cols, rows), np.uint8)
     sinv = np.empty(cols, np.float32)
-    lib().orc_quantize_rowwise_transpose(_p(x), rows, cols, cols, fmt, int(pow2), _p(qT), _p(sinv))
-    return qT, sinv
+    c = np.zeros(2, np.uint64)
+    lib().orc_quantize_rowwise_transpose(_p(x), rows, cols, cols, fmt, int(pow2), _p(qT), _p(sinv), _p(c))
+    return _with_counts((qT, sinv), c, counts)
 
 
 def gemm_bf16_wgrad_sampled(dY_bits: np.ndarray, X_bits: np.ndarray, idx_m, idx_n):

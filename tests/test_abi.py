@@ -59,10 +59,12 @@ def test_validation_before_device_access():
     assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, -1, 64, 64, 0, FAKE, FAKE, FAKE, 64, None, 0, n) == SHAPE
     assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 64, 64, 64, 0, FAKE, FAKE, FAKE, 32, None, 0, n) == SHAPE  # ldd < N
     # quantizers
-    assert L.fp8_quantize_rowwise(FAKE, 4, 24, 32, 0, 1, FAKE, FAKE, n) == SHAPE
-    assert L.fp8_quantize_rowwise(FAKE, 4, 16, 20, 0, 1, FAKE, FAKE, n) == ALIGN
-    assert L.fp8_quantize_rowwise(FAKE, 4, 16, 16, 2, 1, FAKE, FAKE, n) == INVALID
-    assert L.fp8_quantize_blockwise(FAKE, 4, 32, 32, 0, 64, FAKE, FAKE, n) == INVALID
+    assert L.fp8_quantize_rowwise(FAKE, 4, 24, 32, 0, 1, FAKE, FAKE, None, n) == SHAPE
+    assert L.fp8_quantize_rowwise(FAKE, 4, 16, 20, 0, 1, FAKE, FAKE, None, n) == ALIGN
+    assert L.fp8_quantize_rowwise(FAKE, 4, 16, 16, 2, 1, FAKE, FAKE, None, n) == INVALID
+    assert L.fp8_quantize_rowwise(FAKE, 4, 16, 16, 0, 1, FAKE, FAKE, FAKE_ODD, n) == ALIGN   # counts
+    assert L.fp8_quantize_blockwise(FAKE, 4, 32, 32, 0, 64, FAKE, FAKE, None, n) == INVALID
+    assert L.fp8_quantize_blockwise(FAKE, 4, 32, 32, 0, 1, FAKE, FAKE, FAKE_ODD, n) == ALIGN  # counts
     assert L.fp8_quantize_tensorwise(FAKE, 4, 32, 0, None, FAKE, 0, FAKE, None, None, n) == INVALID
     assert L.fp8_quantize_tensorwise(FAKE, 4, 40, 0, FAKE, FAKE, 1, FAKE, None, None, n) == SHAPE
     assert L.fp8_gemm_scaled(FAKE, 0, FAKE, 0, 256, 256, 256, 0, FAKE, FAKE, FAKE, 256, FAKE_ODD, 1024, n) == ALIGN
@@ -73,27 +75,28 @@ def test_validation_before_device_access():
     assert L.fp8_amax(FAKE, -1, FAKE, None, n) == SHAPE
     assert L.fp8_amax(FAKE, 10, None, None, n) == INVALID
     # KV cache and history
-    assert L.fp8_kv_quant(FAKE, 2, 2, 3, 5, 0, FAKE, FAKE, n) == SHAPE
+    assert L.fp8_kv_quant(FAKE, 2, 2, 3, 5, 0, FAKE, FAKE, None, n) == SHAPE
+    assert L.fp8_kv_quant(FAKE, 2, 2, 16, 8, 0, FAKE, FAKE, FAKE_ODD, n) == ALIGN   # counts
     assert L.fp8_kv_dequant(FAKE, FAKE, 2, 2, 16, 8, 7, FAKE, n) == INVALID
     assert L.fp8_amax_history_update(FAKE, FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
     assert L.fp8_amax_history_update(FAKE, FAKE, 2000, FAKE, 0, FAKE, FAKE, FAKE, n) == SHAPE
     assert L.fp8_amax_history_update(None, FAKE, 16, FAKE, 0, FAKE, FAKE, FAKE, n) == INVALID
     # rowwise pair
-    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 32, FAKE, FAKE, 24, 0, 1, n) == SHAPE
-    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 16, FAKE, FAKE, 32, 0, 1, n) == SHAPE
-    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, None, 4, 32, FAKE, FAKE, 32, 0, 1, n) == INVALID
-    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 32, FAKE, FAKE, 32, 5, 1, n) == INVALID
+    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 32, FAKE, FAKE, 24, 0, 1, None, n) == SHAPE
+    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 16, FAKE, FAKE, 32, 0, 1, None, n) == SHAPE
+    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, None, 4, 32, FAKE, FAKE, 32, 0, 1, None, n) == INVALID
+    assert L.fp8_quantize_rowwise_pair(FAKE, 4, 32, FAKE, FAKE, FAKE, 4, 32, FAKE, FAKE, 32, 5, 1, None, n) == INVALID
     # E8M0 block scales
-    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 32, 32, 0, 64, FAKE, FAKE, n) == INVALID    # block_rows
-    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 24, 32, 0, 1, FAKE, FAKE, n) == SHAPE       # cols % 16
-    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 32, 32, 0, 1, FAKE, FAKE_ODD, n) == ALIGN
+    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 32, 32, 0, 64, FAKE, FAKE, None, n) == INVALID    # block_rows
+    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 24, 32, 0, 1, FAKE, FAKE, None, n) == SHAPE       # cols % 16
+    assert L.fp8_quantize_blockwise_e8m0(FAKE, 4, 32, 32, 0, 1, FAKE, FAKE_ODD, None, n) == ALIGN
     assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 40, FAKE, FAKE, FAKE, 64, n) == SHAPE   # K % 16
     assert L.fp8_gemm_block_e8m0(FAKE, 2, FAKE, 0, 64, 64, 64, FAKE, FAKE, FAKE, 64, n) == INVALID
     assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 64, None, FAKE, FAKE, 64, n) == INVALID
     assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 64, FAKE_ODD, FAKE, FAKE, 64, n) == ALIGN
     # backward operands and the bf16 weight gradient
-    assert L.fp8_quantize_rowwise_transpose(FAKE, 24, 32, 32, 0, 1, FAKE, FAKE, FAKE, n) == SHAPE   # rows % 16
-    assert L.fp8_quantize_rowwise_transpose(FAKE, 32, 32, 32, 0, 1, FAKE, FAKE, None, n) == INVALID
+    assert L.fp8_quantize_rowwise_transpose(FAKE, 24, 32, 32, 0, 1, FAKE, FAKE, FAKE, None, n) == SHAPE   # rows % 16
+    assert L.fp8_quantize_rowwise_transpose(FAKE, 32, 32, 32, 0, 1, FAKE, FAKE, None, None, n) == INVALID
     assert L.fp8_gemm_bf16_wgrad(FAKE, FAKE, 64, 12, 64, 12, 64, FAKE, 64, 0, n) == ALIGN    # M % 8
     assert L.fp8_gemm_bf16_wgrad(FAKE, FAKE, 64, 64, 64, 64, 64, None, 64, 0, n) == INVALID
     assert L.fp8_gemm_bf16_wgrad(FAKE, FAKE, 64, 64, 64, 32, 64, FAKE, 64, 0, n) == SHAPE    # ld_dy < M

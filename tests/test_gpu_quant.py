@@ -287,3 +287,89 @@ def test_quantize_tensorwise_global_single_rank(orc):
     assert_codes_equal(to_np(q), rq, 0)
     assert_f32_equal(to_np(sinv), np.float32([rsinv]))
     assert_f32_equal(to_np(am), np.float32([ramax]))
+
+
+# ------------------------------------------- non-finite / saturation counters --
+
+def _with_nonfinite(bits, seed, k=12):
+    """Copy of bf16 bits with NaN, +Inf and -Inf written at seeded positions
+    (one whole row NaN when the tensor has more than 4 rows)."""
+    b = bits.copy()
+    flat = b.reshape(-1)
+    rng = np.random.default_rng(seed)
+    pos = rng.choice(flat.size, k, replace=False)
+    flat[pos] = np.resize(np.array([0x7FC0, 0x7F80, 0xFF80, 0xFFC1], np.uint16), k)
+    if b.ndim == 2 and b.shape[0] > 4:
+        b[3, :] = 0x7FC0
+    return b
+
+
+def _counts_dev():
+    return torch.zeros(2, dtype=torch.int32, device="cuda")
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("shape", [(300, 400), (2048, 4096), (7, 8192), (5, 16400)])
+def test_counts_rowwise_pair_and_transpose(orc, fmt, shape):
+    """Non-finite and saturated counts of the per-row quantizer (pow2 and fp32
+    scales), the two-tensor launch and the transposed per-row quantizer equal
+    the oracle's ("DeepL押注FP8" §5.1: overflow and NaN are what a run must
+    catch); codes and scales stay bit-exact on these inputs."""
+    rows, cols = shape
+    bits = _with_nonfinite(inputs.bf16_bits(inputs.outlier_activations_bf16(shape, seed=rows + fmt)), rows)
+    x = inputs.from_bf16_bits(bits, "cuda")
+    for pow2 in (True, False):
+        c = _counts_dev()
+        q, sinv = fp8q.quantize_rowwise(x, fmt, pow2, counts=c)
+        rq, rs, rc = orc.quantize_rowwise(bits, fmt, pow2, counts=True)
+        assert_codes_equal(to_np(q), rq, fmt)
+        assert_f32_equal(to_np(sinv), rs)
+        assert (int(c[0]), int(c[1])) == rc and rc[0] >= cols
+    bits_b = _with_nonfinite(inputs.bf16_bits(inputs.normal_bf16((96, cols), 0.02, seed=5)), 9, k=5)
+    c = _counts_dev()
+    (qa, sa), (qb, sb) = fp8q.quantize_rowwise_pair(x, inputs.from_bf16_bits(bits_b, "cuda"), fmt, True, counts=c)
+    ra, rb = orc.quantize_rowwise(bits, fmt, True, counts=True), orc.quantize_rowwise(bits_b, fmt, True, counts=True)
+    assert_codes_equal(to_np(qb), rb[0], fmt)
+    assert (int(c[0]), int(c[1])) == (ra[2][0] + rb[2][0], ra[2][1] + rb[2][1])
+    if rows % 16 == 0:
+        c = _counts_dev()
+        qT, sT, _ = fp8q.quantize_rowwise_transpose(x, fmt, True, counts=c)
+        rqT, rsT, rcT = orc.quantize_rowwise_transpose(bits, fmt, True, counts=True)
+        assert_codes_equal(to_np(qT), rqT, fmt)
+        assert (int(c[0]), int(c[1])) == rcT
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("block_rows", [1, 128])
+@pytest.mark.parametrize("shape", [(300, 400), (1024, 4096)])
+def test_counts_blockwise_and_e8m0(orc, fmt, block_rows, shape):
+    """Counts of the per-block quantizers (fp32 scales and power-of-two scales
+    written as E8M0) against the oracle, codes bit-exact."""
+    bits = _with_nonfinite(inputs.bf16_bits(inputs.normal_bf16(shape, 1.0, seed=shape[0] + block_rows)), 77)
+    x = inputs.from_bf16_bits(bits, "cuda")
+    c = _counts_dev()
+    q, sinv = fp8q.quantize_blockwise(x, fmt, block_rows, counts=c)
+    rq, rs, rc = orc.quantize_blockwise(bits, fmt, block_rows, counts=True)
+    assert_codes_equal(to_np(q), rq, fmt)
+    assert_f32_equal(to_np(sinv), rs)
+    assert (int(c[0]), int(c[1])) == rc and rc[0] > 0 and rc[1] > 0
+    c = _counts_dev()
+    q, _ = fp8q.quantize_blockwise_e8m0(x, fmt, block_rows, counts=c)
+    rq, _, rc = orc.quantize_blockwise(bits, fmt, block_rows, pow2=True, counts=True)
+    assert_codes_equal(to_np(q), rq, fmt)
+    assert (int(c[0]), int(c[1])) == rc
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_counts_kv_quant(orc, fmt):
+    """Counts of the per-(b, h) KV quantizer against the oracle, codes bit-exact;
+    a NaN-only slice quantizes with scale 1."""
+    kv = inputs.normal_bf16((2, 4, 512, 128), 1.0, seed=13 + fmt)
+    bits = _with_nonfinite(inputs.bf16_bits(kv).reshape(8, -1), 21, k=20).reshape(2, 4, 512, 128)
+    bits[1, 2] = 0x7FC0
+    c = _counts_dev()
+    q, sinv = fp8q.kv_quant(inputs.from_bf16_bits(bits, "cuda"), fmt, counts=c)
+    rq, rs, rc = orc.kv_quant(bits, fmt, counts=True)
+    assert_codes_equal(to_np(q), rq, fmt)
+    assert_f32_equal(to_np(sinv), rs)
+    assert (int(c[0]), int(c[1])) == rc and rc[0] >= 512 * 128

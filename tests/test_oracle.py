@@ -359,6 +359,54 @@ def test_blockwise_every_code_against_torch(orc, fmt, block_rows, pow2):
     assert orc.decode_table(fmt)[q[rows - 1, cols - 3]] == -fm
     inv = (np.float32(1.0) / s).astype(np.float32)
     assert np.array_equal(sinv, inv.T if block_rows == 1 else inv)
+    # counts: the NaN and the -Inf are non-finite; saturated = |fp32(x) * s| > fmax (the -Inf among them)
+    _, _, (nf, sat) = orc.quantize_blockwise(wide, fmt, block_rows, pow2=pow2, cols=cols, counts=True)
+    with np.errstate(invalid="ignore", over="ignore"):
+        y = (xv * s_full).astype(np.float32)
+    assert nf == 2 and sat == int(np.sum(np.abs(y) > fm)) >= 1
+
+
+def _counts_reference(xv, s_full, fm):
+    """(non-finite inputs, elements with |fp32(x) * s| > fmax): NaN is not
+    saturated, +-Inf is."""
+    with np.errstate(invalid="ignore", over="ignore"):
+        y = (xv * s_full).astype(np.float32)
+    return int(np.sum(~np.isfinite(xv))), int(np.sum(np.abs(y) > fm))
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_rowwise_kv_transpose_counts(orc, fmt):
+    """Non-finite and saturation counts of the per-row, per-(b,h)-slice and
+    per-column quantizers ("DeepL押注FP8" §5.1: overflow and NaN are the
+    failures a run must notice) against numpy on inputs with NaN and +-Inf
+    (an element whose fp32(x) * s rounds above fmax counts as saturated on
+    both sides); the scales are recomputed independently (numpy maxima, the
+    fp32 division or the exact power-of-two comparison)."""
+    fm = orc.fmax(fmt)
+    rng = np.random.default_rng(70 + fmt)
+    xf = rng.standard_normal((24, 96)).astype(np.float32)
+    bits = _bits(torch.from_numpy(xf).to(torch.bfloat16)).copy()
+    bits[2, 5], bits[7, 1], bits[7, 2], bits[20, 95] = 0x7FC0, 0x7F80, 0xFF80, 0xFFC0
+    xv = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    fin = np.where(np.isfinite(xv), np.abs(xv), 0.0)
+
+    def s_of(a, pow2):
+        if pow2:
+            return np.float32(_pow2_scale_by_comparison(float(a), fm))
+        return np.float32(1.0) if a == 0 else np.float32(fm) / np.float32(a)
+
+    for pow2 in (False, True):
+        _, _, c = orc.quantize_rowwise(bits, fmt, pow2, counts=True)
+        s_full = np.array([s_of(a, pow2) for a in fin.max(axis=1)], np.float32)[:, None] * np.ones((1, 96), np.float32)
+        assert c == _counts_reference(xv, s_full, fm)
+        _, _, c = orc.quantize_rowwise_transpose(bits, fmt, pow2, counts=True)
+        s_full = np.ones((24, 1), np.float32) * np.array([s_of(a, pow2) for a in fin.max(axis=0)], np.float32)[None, :]
+        assert c == _counts_reference(xv, s_full, fm)
+    kv = bits.reshape(2, 3, 4, 96)
+    _, _, c = orc.kv_quant(kv, fmt, counts=True)
+    sl = fin.reshape(6, -1).max(axis=1)
+    s_full = np.repeat(np.array([s_of(a, False) for a in sl], np.float32), 4 * 96).reshape(24, 96)
+    assert c == _counts_reference(xv, s_full, fm) and c[0] == 4
 
 
 # -------------------------------------------------------------------- GEMM --
