@@ -541,11 +541,15 @@ k_rowwise(RowJob ja, RowJob jb, int64_t cols, uint32_t *__restrict__ counts) {
 }
 
 // ---------------------------------------------------------- block 1x128 --
-// A half-warp per 1x128 block (16 lanes x 8 elements).  A warp walks rows
-// (warp, warp + nwarps, ...) and, inside a row, U pairs of blocks per
-// iteration (the two half-warps take neighbouring blocks), so U 16-byte loads
-// per lane are in flight and no index division is needed.  scale_inv is
-// stored [kb][row].
+// Four lanes per 1x128 block, 32 elements each: a warp walks rows (warp,
+// warp + nwarps, ...) and takes 8 blocks of a row per step, lanes 4g .. 4g+3
+// block g, lane j its 16-byte pieces j, j+4, j+8, j+12 (each load instruction
+// reads 64 contiguous bytes per block, each store writes 32).  Two steps'
+// loads (8 x 16 bytes per lane) are issued before the first reduction.  The
+// per-block work -- a two-shuffle max, the scale division, the scale store --
+// is shared by four lanes' 32 elements (with 16 lanes of 8 elements it cost
+// as many instructions as the cast itself: 15 per element against 5 now).
+// scale_inv is stored [kb][row].
 // E8M0 scale image (the operand layout of the hardware block-scaled MMA,
 // which reads one byte per row for every 32-wide K slice; a 32-bit word holds
 // four such bytes).  Here a byte carries a whole 128-wide K block, so one word
@@ -565,7 +569,8 @@ __device__ __forceinline__ int64_t e8m0_offset(int64_t kb, int64_t rt, int64_t r
 // SF = false: fp32 scale_inv[kb * rows + row], s = fmax / amax.
 // SF = true:  E8M0 image (sf_image), s the pow2 rule; the image's padding rows
 //             (up to a multiple of 128) get e = 127 (factor 1).
-template <int FMT, int U, bool SF>
+// COUNT: the non-finite / saturated counters.
+template <int FMT, bool SF, bool COUNT>
 __global__ void __launch_bounds__(256)
 k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
              uint8_t *__restrict__ q, float *__restrict__ scale_inv, uint8_t *__restrict__ sf_image,
@@ -573,57 +578,64 @@ k_block1x128(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t
     pdl_trigger();   // dependents are scheduled once all our CTAs have started
     pdl_wait();
     constexpr float fm = fmax_of<FMT>();
-    uint32_t nf = 0, sat = 0;   // counters (counts != NULL)
-    const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
+    constexpr int STEPS = 2;                 // 8-block steps whose loads are in flight together
+    const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
     const int64_t nkb = (cols + 127) / 128;
     const int64_t rt = (rows + 127) / 128;
     const int64_t row_end = SF ? rt * 128 : rows;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    uint32_t nf = 0, sat = 0;
     for (int64_t row = warp; row < row_end; row += nwarps) {
         const bool live = row < rows;
         const uint16_t *xr = x + (live ? row : 0) * ld;
         uint8_t *qr = q + row * cols;
-        for (int64_t kb0 = 0; kb0 < nkb; kb0 += 2 * U) {
-            uint4 v[U];
-            int64_t cidx[U];
-            bool valid[U];
+        for (int64_t kb0 = 0; kb0 < nkb; kb0 += 8 * STEPS) {
+            uint4 v[STEPS][4];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int64_t kb = kb0 + 2 * u + half;
-                cidx[u] = kb * 128 + l16 * 8;
-                valid[u] = live && (kb < nkb) && (cidx[u] < cols);
-                v[u] = valid[u] ? ld_stream(reinterpret_cast<const uint4 *>(xr + cidx[u])) : make_uint4(0, 0, 0, 0);
+            for (int t = 0; t < STEPS; ++t) {
+                const int64_t c0 = (kb0 + 8 * t + g) * 128;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int64_t c = c0 + (j + 4 * p) * 8;
+                    v[t][p] = (live && c < cols) ? ld_stream(reinterpret_cast<const uint4 *>(xr + c))
+                                                 : make_uint4(0, 0, 0, 0);
+                }
             }
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                uint32_t m = amax_fast_final(amax_fast8(0u, v[u]));
+            for (int t = 0; t < STEPS; ++t) {
+                const int64_t kb = kb0 + 8 * t + g;
+                uint32_t m = amax_fast_final(amax_fast8(amax_fast8(amax_fast8(amax_fast8(0u, v[t][0]), v[t][1]), v[t][2]), v[t][3]));
                 const bool nonfin = m == 0xFFFFFFFFu;
                 if (nonfin) {
                     uint32_t bad = 0;
-                    m = amax_exact8(0u, v[u], bad);
+                    m = amax_exact8(amax_exact8(amax_exact8(amax_exact8(0u, v[t][0], bad), v[t][1], bad), v[t][2], bad),
+                                    v[t][3], bad);
                 }
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                const float amax = bf16bits_to_float(m);
+                const float s = SF ? pow2_scale_from_amax(amax, fm) : scale_from_amax(amax, fm);
 #pragma unroll
-                for (int o = 8; o >= 1; o >>= 1) {
-                    const uint32_t t = __shfl_xor_sync(0xFFFFFFFFu, m, o);
-                    m = t > m ? t : m;
+                for (int p = 0; p < 4; ++p) {
+                    const int64_t c = kb * 128 + (j + 4 * p) * 8;
+                    if (live && c < cols) *reinterpret_cast<uint2 *>(qr + c) = cast8<FMT>(v[t][p], s);
                 }
-                const float s = SF ? pow2_scale_from_amax(bf16bits_to_float(m), fm)
-                                   : scale_from_amax(bf16bits_to_float(m), fm);
-                if (valid[u]) *reinterpret_cast<uint2 *>(qr + cidx[u]) = cast8<FMT>(v[u], s);
-                if (counts && valid[u] && may_saturate(nonfin, bf16bits_to_float(m), s, fm)) {
-                    nf += count_nonfinite8(v[u]);
-                    sat += count_sat8(v[u], s, fm);
-                }
-                const int64_t kb = kb0 + 2 * u + half;
-                if (l16 == 0 && kb < nkb) {
-                    if (SF) sf_image[e8m0_offset(kb, rt, row)] = e8m0_of_scale(s);
+                if (j == 0 && kb < nkb) {
+                    if (SF) sf_image[e8m0_offset(kb, rt, row)] = live ? e8m0_of_scale(s) : (uint8_t)127;
                     else scale_inv[kb * rows + row] = __fdiv_rn(1.0f, s);
+                }
+                if (COUNT && live && may_saturate(nonfin, amax, s, fm)) {   // pieces past the row are zeros
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        nf += count_nonfinite8(v[t][p]);
+                        sat += count_sat8(v[t][p], s, fm);
+                    }
                 }
             }
         }
     }
-    if (counts) flush_counts(counts, nf, sat);
+    if (COUNT) flush_counts(counts, nf, sat);
 }
 
 // -------------------------------------------------------- block 128x128 --
@@ -750,10 +762,12 @@ cudaError_t launch_block(cudaStream_t st, int sms, const void *x, int64_t rows, 
     const uint16_t *xs = static_cast<const uint16_t *>(x);
     const int64_t nkb = (cols + 127) / 128;
     if (block_rows == 1) {
-        constexpr int U = 4;
         const int64_t r = SF ? (rows + 127) / 128 * 128 : rows;
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((r + 7) / 8, (int64_t)sms * 8));
-        return pdl_launch(k_block1x128<FMT, U, SF>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q, scale_inv,
+        if (counts)
+            return pdl_launch(k_block1x128<FMT, SF, true>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q,
+                              scale_inv, sf_image, counts);
+        return pdl_launch(k_block1x128<FMT, SF, false>, dim3(grid), dim3(256), 0, st, xs, rows, cols, ld, q, scale_inv,
                           sf_image, counts);
     } else {
         const int64_t tiles = ((rows + 127) / 128) * nkb;
