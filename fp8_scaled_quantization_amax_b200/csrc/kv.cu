@@ -16,10 +16,10 @@
 // launch, with no scratch memory and no grid-wide wait.
 //
 // Dequantize: each CTA streams a contiguous 256 KiB of FP8 codes (16 codes
-// in per 16-byte load, 16 bf16 out as two 16-byte stores); contiguous
-// per-CTA chunks keep the write-heavy stream at DRAM-page locality (a
-// grid-stride layout measured ~20 % slower).  One scale per (b, h) from the
-// grid's y index.
+// in per 16-byte load); the bf16 results go through shared memory and leave
+// in 32 KiB bulk copies.  Contiguous per-CTA chunks keep the write-heavy
+// stream at DRAM-page locality (a grid-stride layout measured ~20 % slower).
+// One scale per (b, h) from the grid's y index.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -142,38 +142,64 @@ __device__ __forceinline__ void dequant16(uint4 c, float d, uint4 &o0, uint4 &o1
 }
 
 // A CTA dequantizes the contiguous units [blockIdx.x * per, +per) of slice
-// blockIdx.y: four 16-byte loads in flight per thread, then eight 16-byte
-// stores.
+// blockIdx.y (a unit = 16 codes = 32 bytes of bf16 out).  Per round each of
+// the 256 threads loads four units' codes (16 KiB per CTA in flight), writes
+// their bf16 values into one of two 32 KiB shared-memory buffers, and one
+// thread sends the buffer to global memory with a single bulk copy
+// (cp.async.bulk), so the write stream -- two thirds of the traffic -- costs
+// no per-thread global stores: with two 16-byte stores per unit the
+// load/store queue throttled the kernel (ncu: lg_throttle the top stall).
 constexpr int64_t kDequantUnitsPerCta = 16384;   // 256 KiB of FP8 codes
+constexpr int kDqThreads = 256;
+constexpr int kDqRound = 4 * kDqThreads;          // units per round
+constexpr int kDqBuf = kDqRound * 32;             // bytes of bf16 per round
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
 template <int FMT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kDqThreads)
 k_kv_dequant(const uint4 *__restrict__ q, const float *__restrict__ scale_inv, int64_t nunit,
              uint4 *__restrict__ out) {
+    extern __shared__ __align__(128) uint8_t dq_smem[];   // two buffers of kDqBuf bytes
     const int64_t sl = blockIdx.y;
     const float d = scale_inv[sl];
     const uint4 *qs = q + sl * nunit;
     uint4 *os = out + 2 * sl * nunit;
     const int64_t u0 = blockIdx.x * kDequantUnitsPerCta;
     const int64_t u1 = min(u0 + kDequantUnitsPerCta, nunit);
-    int64_t u = u0 + threadIdx.x;
-    for (; u + 3 * 256 < u1; u += 4 * 256) {
+    int buf = 0;
+    for (int64_t r0 = u0; r0 < u1; r0 += kDqRound, buf ^= 1) {
         uint4 c[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) c[k] = ld_stream(qs + u + k * 256);
+        for (int k = 0; k < 4; ++k) {
+            const int64_t u = r0 + threadIdx.x + k * kDqThreads;
+            c[k] = u < u1 ? ld_stream(qs + u) : make_uint4(0, 0, 0, 0);
+        }
+        // the bulk copy issued from this buffer two rounds ago has read it
+        if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        __syncthreads();
+        const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(dq_smem)) + (uint32_t)(buf * kDqBuf);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             uint4 o0, o1;
             dequant16<FMT>(c[k], d, o0, o1);
-            os[2 * (u + k * 256)] = o0;
-            os[2 * (u + k * 256) + 1] = o1;
+            const uint32_t a = base + (uint32_t)(threadIdx.x + k * kDqThreads) * 32u;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o0.x), "r"(o0.y), "r"(o0.z), "r"(o0.w)
+                         : "memory");
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a + 16), "r"(o1.x), "r"(o1.y), "r"(o1.z),
+                         "r"(o1.w)
+                         : "memory");
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the bulk copy
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const int64_t n = min((int64_t)kDqRound, u1 - r0);
+            bulk_store(os + 2 * r0, base, (uint32_t)(n * 32));
         }
     }
-    for (; u < u1; u += 256) {
-        uint4 o0, o1;
-        dequant16<FMT>(ld_stream(qs + u), d, o0, o1);
-        os[2 * u] = o0;
-        os[2 * u + 1] = o1;
-    }
+    if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 }  // namespace
@@ -262,9 +288,19 @@ extern "C" fp8_status fp8_kv_dequant(const uint8_t *q, const float *scale_inv, i
     const int64_t per_slice = (nunit + kDequantUnitsPerCta - 1) / kDequantUnitsPerCta;
     if (per_slice > 2147483647LL) return FP8_ERR_SHAPE;
     const dim3 grid((unsigned)per_slice, (unsigned)BH);
+    static bool attr_set[64][2];   // per device: the 64 KiB of shared memory needs the opt-in
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
+    if (!attr_set[dev][fmt]) {
+        const cudaError_t e = (fmt == FP8_E4M3)
+            ? cudaFuncSetAttribute(k_kv_dequant<FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * kDqBuf)
+            : cudaFuncSetAttribute(k_kv_dequant<FP8_E5M2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * kDqBuf);
+        if (e != cudaSuccess) return FP8_ERR_CUDA;
+        attr_set[dev][fmt] = true;
+    }
     if (fmt == FP8_E4M3)
-        k_kv_dequant<FP8_E4M3><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(q), scale_inv, nunit, static_cast<uint4 *>(out_bf16));
+        k_kv_dequant<FP8_E4M3><<<grid, kDqThreads, 2 * kDqBuf, s>>>(reinterpret_cast<const uint4 *>(q), scale_inv, nunit, static_cast<uint4 *>(out_bf16));
     else
-        k_kv_dequant<FP8_E5M2><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(q), scale_inv, nunit, static_cast<uint4 *>(out_bf16));
+        k_kv_dequant<FP8_E5M2><<<grid, kDqThreads, 2 * kDqBuf, s>>>(reinterpret_cast<const uint4 *>(q), scale_inv, nunit, static_cast<uint4 *>(out_bf16));
     return cudaPeekAtLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
