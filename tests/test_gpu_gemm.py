@@ -101,6 +101,29 @@ def test_gemm_integer_values_exact(orc):
     assert np.array_equal(D.float().cpu().numpy(), bf)
 
 
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_gemm_against_the_naive_fp32_sum(orc, mode):
+    """How far the tensor cores' accumulation sits from the naive sequential
+    fp32 sum (the oracle's fp32-accumulate variant), both against the fp64
+    reference: the GPU's worst error relative to max |ref| is no larger than
+    that of the naive fp32 sum rounded to bf16 the same way (both are
+    dominated by the output's bf16 rounding), and the two bf16 results agree
+    on almost every output (they can differ where an fp32 rounding
+    difference lands on a bf16 rounding boundary).  The figures are logged
+    with the other GEMM error figures."""
+    M, N, K = 520, 776, 640
+    A, da, B, db = _operands(orc, mode, M, N, K, seed=90 + mode)
+    D = _run(A, 0, B, 0, mode, da, db)
+    ref, mag = orc.gemm_scaled(A, 0, B, 0, mode, da, db)
+    f32 = orc.gemm_scaled_f32acc(A, 0, B, 0, mode, da, db)
+    naive = torch.from_numpy(f32.astype(np.float32)).to(torch.bfloat16)
+    got = D.cpu()
+    e_gpu = assert_gemm_close(bf16_to_f64(D), ref, mag, f"gpu mode {mode}")
+    e_naive = assert_gemm_close(naive.double().numpy(), ref, mag, f"naive fp32 sum mode {mode}")
+    assert e_gpu <= 1.5 * e_naive + 1e-12
+    assert float((got != naive).float().mean()) < 0.01
+
+
 def test_gemm_identity_weight(orc):
     K = 256
     A, da, _, _ = orc.quantize_tensorwise(inputs.bf16_bits(inputs.normal_bf16((200, K), 1.0, seed=9)), 0)
