@@ -12,34 +12,30 @@
 // The scales change every 128 elements of K, so no single epilogue scale
 // exists: each K block's product is accumulated alone in tensor memory and
 // the epilogue warps add it, scaled, into an fp32 register accumulator.
-// What bounds this loop on sm_100a (measured with clock stamps and probes):
-//   * an mbarrier signal takes ~200 cycles from arrive to the waiter's wake-up
-//     and a tcgen05.commit ~400 cycles from the MMAs' completion to the wake-up,
-//     so releasing a TMEM buffer and seeing the next MMA's result in it costs
-//     ~1.3k cycles however fast the epilogue computes;
-//   * a 256-row CTA-pair MMA runs at the same rate per flop for N = 128 as
-//     for N = 256 (65 vs 131 cycles per K = 32 step).
-// So each K block is issued as two 256 x 128 halves (tile columns 0-127 and
-// 128-255, each one 128-row block of B and therefore one B scale) into four
-// 128-column TMEM buffers, buffer 2 * (kb % 2) + half.  Three other halves
-// (768 MMA cycles) run while one is promoted, instead of one K block (512
-// cycles) with two 256-column buffers, and the two halves' epilogue warps run
-// half a K block apart, so one warp's TMEM round trip overlaps the other's
-// FMAs on the same SM sub-partition.
-//
+// What bounds this loop on sm_100a (measured with clock stamps):
+//   * a CTA-pair MMA instruction (M = 256, K = 32) occupies the tensor core
+//     ~190 cycles in a TMA-fed loop whether N is 128 or 256, so each K block
+//     is issued as four N = 256 MMAs (splitting N doubles the MMA time);
+//   * an mbarrier signal takes ~200 cycles from arrive to the waiter's
+//     wake-up and a tcgen05.commit ~400 cycles from the MMAs' completion.
+// Two 256-column TMEM buffers alternate by K-block parity: the MMAs of block
+// kb + 1 run while block kb is read out, and the buffer goes back to the MMA
+// as soon as the epilogue warps hold their columns in registers (before the
+// second half of the FMAs).
 // Layout per CTA of the pair (M = 256 rows per tile, 128 per CTA):
 //   warp 0      TMA producer: per stage this CTA's 128 rows of A (16 KiB) and
-//               its 64-row share of each half's 128 rows of B (2 x 8 KiB);
+//               its 128 rows of the tile's 256 rows of B (16 KiB);
 //   warp 1      TMEM allocator; in the even CTA the MMA issuer;
-//   warps 2-3   release warps of the two halves: they return a partial
-//               buffer to the MMA issuer once the half's four epilogue warps
+//   warps 2-3   release warps of the two buffers: they return a partial
+//               buffer to the MMA issuer once all eight epilogue warps
 //               have read it (named barrier), so the epilogue warps never
 //               stall on the mbarrier arrive (~200 cycles when it completes
 //               a phase someone waits on);
 //   warps 4-11  epilogue: warp w promotes TMEM lane quarter w % 4 (32 rows)
-//               of half (w - 4) / 4 (128 columns) -- two 64-column round
-//               trips, scalar fp32 FMAs (fma.rn, one rounding per term);
-//               then bf16 RNE and coalesced stores.
+//               and column half g = (w - 4) / 4 (tile columns g * 128 .. +
+//               127, one 128-row block of B, so one B scale) -- two 64-column
+//               round trips, scalar fp32 FMAs (fma.rn, one rounding per
+//               term); then bf16 RNE and coalesced stores.
 // Summation order per output is fixed (K blocks in order, each block's
 // partial from the tensor core, then one FMA), so results are bit-identical
 // run to run.  Every mbarrier wait is bounded (about one second, see tc.cuh);
@@ -57,18 +53,18 @@ namespace {
 
 namespace blk {
 constexpr int STAGES = 6;
-constexpr int B_SUB = 64 * BK;                  // this CTA's 64 rows of one half of B (8 KiB)
-constexpr int STAGE = A_TILE + 2 * B_SUB;       // 32 KiB per stage and CTA
-constexpr int NBUF = 4;                         // 128-column TMEM partial buffers
+constexpr int B_TILE = 128 * BK;                // this CTA's 128 rows of B (16 KiB)
+constexpr int STAGE = A_TILE + B_TILE;          // 32 KiB per stage and CTA
+constexpr int NBUF = 2;                         // 256-column TMEM partial buffers
 constexpr int NBARS = 2 * STAGES + 2 * NBUF + 1;   // full, empty, partial full / free, drain
 constexpr size_t EPI_OFF = ((size_t)STAGES * STAGE + NBARS * 8 + 16 + 15) & ~(size_t)15;
 constexpr size_t SMEM = 1024 + EPI_OFF + (size_t)sm2::EPI * kEpiBufBytes;
-constexpr int PF = 2;                           // scale prefetch distance in K blocks
+constexpr int PF = 1;                           // scale prefetch distance in K blocks
 static_assert(SMEM <= 232448, "shared memory per block");
-// Named barriers 1-4: the four epilogue warps of half h hand K block kb's
-// finished reads to that half's release warp (warp 2 + h) through barrier
-// 1 + 2h + kb % 2 (4 x 32 arriving threads + the 32 of the release warp).
-constexpr int kReleaseThreads = 5 * 32;
+// Named barriers 1-2: the eight epilogue warps hand K block kb's finished
+// reads to the release warp of buffer kb % 2 (warp 2 + kb % 2) through
+// barrier 1 + kb % 2 (8 x 32 arriving threads + the 32 of the release warp).
+constexpr int kReleaseThreads = 9 * 32;
 }  // namespace blk
 
 // 32 lanes x 64 consecutive fp32 columns in one load; valid after tmem_wait64.
@@ -166,9 +162,7 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const int t = pair + i * npairs;
                 const int m_blk = t % num_m, n_blk = t / num_m;
                 const int a_row = m_blk * 256 + (int)rank * 128;
-                // an N = 128 pair MMA takes rows [0, 64) of its B operand from
-                // the even CTA and [64, 128) from the odd one
-                const int b_row = n_blk * 256 + (int)rank * 64;
+                const int b_row = n_blk * 256 + (int)rank * 128;
                 for (int kc = 0; kc < nk; ++kc, ++it) {
                     const int stage = it % STG;
                     const uint32_t round = it / STG;
@@ -181,7 +175,6 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const uint32_t a_dst = smem_u32(smem + (size_t)stage * blk::STAGE);
                     tma_load_2d_pair(a_dst, &tmA, full_leader, kc * BK, a_row);
                     tma_load_2d_pair(a_dst + A_TILE, &tmB, full_leader, kc * BK, b_row);
-                    tma_load_2d_pair(a_dst + A_TILE + blk::B_SUB, &tmB, full_leader, kc * BK, b_row + 128);
                     last_round[stage] = (int)round;
                 }
             }
@@ -204,18 +197,14 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     if (!wait_bar(full_bar(stage), round & 1u, abort_flag, kErrMma)) { ok = false; break; }
                     const uint32_t a_addr = smem_u32(smem + (size_t)stage * blk::STAGE);
                     const uint64_t adesc = sdesc_k_sw128(a_addr);
+                    const uint64_t bdesc = sdesc_k_sw128(a_addr + A_TILE);
+                    const int q = (int)(it & 1u);
+                    if (!wait_bar(acce_bar(q), ((it >> 1) & 1u) ^ 1u, abort_flag, kErrMma)) { ok = false; break; }
+                    tc_fence_after();
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int q = 2 * (int)(it & 1u) + h;
-                        if (!wait_bar(acce_bar(q), ((it >> 1) & 1u) ^ 1u, abort_flag, kErrMma)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint64_t bdesc = sdesc_k_sw128(a_addr + A_TILE + h * blk::B_SUB);
-#pragma unroll
-                        for (int k = 0; k < BK / 32; ++k)   // +32 bytes along K = +2 in the address field
-                            tc_mma_pair(tmem + q * 128, adesc + 2u * k, bdesc + 2u * k, idesc, k > 0 ? 1u : 0u);
-                        tc_commit_pair_both(accf_bar(q));
-                    }
-                    if (!ok) break;
+                    for (int k = 0; k < BK / 32; ++k)   // +32 bytes along K = +2 in the address field
+                        tc_mma_pair(tmem + q * 256, adesc + 2u * k, bdesc + 2u * k, idesc, k > 0 ? 1u : 0u);
+                    tc_commit_pair_both(accf_bar(q));
                     tc_commit_pair_both(empty_bar(stage));
                 }
             }
@@ -226,7 +215,7 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
     } else if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(sm2::REGS_LOW));
-        // ------------------------------------------- release warp of half h --
+        // ---------------------------------------- release warp of buffer h --
         // An mbarrier arrive that completes a phase a thread is waiting on
         // stalls the arriving thread ~200 cycles; this warp takes that stall
         // off the epilogue warps, which only arrive on a named barrier.  Every
@@ -235,12 +224,11 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int h = warp - 2;
         const uint32_t release_to = leader ? 0u : mapa_shared(acce_bar(0), 0);
         const uint32_t total = (uint32_t)n_items * (uint32_t)nk;
-        for (uint32_t it = 0; it < total; ++it) {
-            named_sync(1 + 2 * h + (int)(it & 1u), blk::kReleaseThreads);
+        for (uint32_t it = (uint32_t)h; it < total; it += 2) {
+            named_sync(1 + h, blk::kReleaseThreads);
             if (lane == 0) {
-                const int q = 2 * (int)(it & 1u) + h;
-                if (leader) mbar_arrive(acce_bar(q));
-                else mbar_arrive_cluster(release_to + (uint32_t)(q * 8));
+                if (leader) mbar_arrive(acce_bar(h));
+                else mbar_arrive_cluster(release_to + (uint32_t)(h * 8));
             }
             __syncwarp();
         }
@@ -248,19 +236,21 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(sm2::REGS_HIGH));
         // --------------------------------------------------- epilogue ----
         const int sp = warp & 3;
-        const int h = (warp - 4) >> 2;                  // half of the tile: columns h*128 .. +127
-        const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+        const int g = (warp - 4) >> 2;                  // column half: tile columns g * 128 .. + 127
+        const uint32_t tsrc = tmem + ((uint32_t)(sp * 32) << 16) + (uint32_t)(g * 128);   // this warp's lanes and columns
         uint32_t it = 0;
         bool ok = true;
         for (int i = 0; ok && i < n_items; ++i) {
             const int t = pair + i * npairs;
             const int m_blk = t % num_m, n_blk = t / num_m;
             const int64_t row0 = (int64_t)m_blk * 256 + (int)rank * 128 + sp * 32;
-            const int64_t m = row0 + lane;
-            const bool m_ok = m < M;
-            const int n_base = n_blk * 256 + h * 128;
-            const int nb = n_blk * 2 + h;               // this half's 128-row block of B
-            const bool nb_ok = n_base < N;
+            // Scale loads are unconditional, from addresses clamped into the
+            // arrays: rows past M and columns past N are never stored, so their
+            // scales do not matter, and a load whose value is selected at once
+            // would stall the warp until it lands.
+            const int nbn = (N + 127) / 128;
+            const float *sap = sa + min(row0 + lane, (int64_t)M - 1);          // + kc * M: block kc
+            const float *sbp = sb + (int64_t)min(n_blk * 2 + g, nbn - 1) * nk;  // [kc]
             float acc[128];
 #pragma unroll
             for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
@@ -269,55 +259,60 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             float as_[blk::PF], bs_[blk::PF];
 #pragma unroll
             for (int p = 0; p < blk::PF; ++p) {
-                as_[p] = (p < nk && m_ok) ? sa[(int64_t)p * M + m] : 0.0f;
-                bs_[p] = (p < nk && nb_ok) ? sb[(int64_t)nb * nk + p] : 0.0f;
+                const int64_t kb = min(p, nk - 1);
+                as_[p] = sap[kb * M];
+                bs_[p] = sbp[kb];
             }
-            // one K block: wait for this half's partial, promote it, release it
-            auto promote = [&](int kc, float &as, float &bs) -> bool {
-                const int q = 2 * (int)(it & 1u) + h;
+            // One K block: wait for the partial, read this warp's 128 columns
+            // in two round trips, hand the buffer back, promote.  A failed wait
+            // (the kernel is aborting) only clears ok_tile: the tile runs to
+            // its end on whatever TMEM holds, so the hot loop has no early
+            // exit and every named-barrier arrival happens; its stores are
+            // skipped.
+            bool ok_tile = true;
+            auto promote = [&](int kc, float &as, float &bs) {
                 const float sc = __fmul_rn(as, bs);
+                if (kc + blk::PF < nk) {   // block kc + PF's scales
+                    as = sap[(int64_t)(kc + blk::PF) * M];
+                    bs = sbp[kc + blk::PF];
+                }
+                const int q = (int)(it & 1u);
                 bool w = true;
                 if (lane == 0) w = wait_bar(accf_bar(q), (it >> 1) & 1u, abort_flag, kErrEpilogue);
-                w = __shfl_sync(0xFFFFFFFFu, w, 0);
-                if (!w) return false;
+                ok_tile = __shfl_sync(0xFFFFFFFFu, w, 0) && ok_tile;
                 tc_fence_after();
-                const uint32_t src = tmem + lane_base + q * 128;
                 uint32_t r[64];
-                tmem_ld64_async(src, r);
+                tmem_ld64_async(tsrc + q * 256, r);
                 tmem_wait64(r);
 #pragma unroll
                 for (int j = 0; j < 64; ++j) acc[j] = fmaf(__uint_as_float(r[j]), sc, acc[j]);
-                tmem_ld64_async(src + 64, r);
+                tmem_ld64_async(tsrc + q * 256 + 64, r);
                 tmem_wait64(r);
                 // the partial is in registers: the release warp hands the buffer back to the MMA
                 tc_fence_before();
-                named_arrive(1 + 2 * h + (int)(it & 1u), blk::kReleaseThreads);
-                if (kc + blk::PF < nk) {   // block kc + PF's scales, after the release
-                    as = m_ok ? sa[(int64_t)(kc + blk::PF) * M + m] : 0.0f;
-                    bs = nb_ok ? sb[(int64_t)nb * nk + kc + blk::PF] : 0.0f;
-                }
+                named_arrive(1 + q, blk::kReleaseThreads);
 #pragma unroll
                 for (int j = 0; j < 64; ++j) acc[64 + j] = fmaf(__uint_as_float(r[j]), sc, acc[64 + j]);
                 ++it;
-                return true;
             };
-            for (int kc = 0; ok && kc < nk; kc += blk::PF) {
+            for (int kc = 0; kc < nk; kc += blk::PF) {
 #pragma unroll
                 for (int p = 0; p < blk::PF; ++p)
-                    if (ok && kc + p < nk && !promote(kc + p, as_[p], bs_[p])) ok = false;
+                    if (kc + p < nk) promote(kc + p, as_[p], bs_[p]);
             }
-            if (!ok) {   // the release warp still expects one arrival per K block
+            if (!ok_tile) {   // aborting: the release warps still expect one arrival per K block
+                ok = false;
                 for (const uint32_t total = (uint32_t)n_items * (uint32_t)nk; it < total; ++it)
-                    named_arrive(1 + 2 * h + (int)(it & 1u), blk::kReleaseThreads);
+                    named_arrive(1 + (int)(it & 1u), blk::kReleaseThreads);
                 break;
             }
             uint8_t *ebuf = smem + blk::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
+            for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(acc[h2 * 64 + 2 * j], acc[h2 * 64 + 2 * j + 1]);
-                store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, (int64_t)M, n_base + h2 * 64, N);
+                for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(acc[h * 64 + 2 * j], acc[h * 64 + 2 * j + 1]);
+                store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, (int64_t)M, n_blk * 256 + g * 128 + h * 64, N);
             }
         }
     }
@@ -373,13 +368,13 @@ fp8_status fp8q_gemm_block_pair(const uint8_t *A, fp8_format fa, const uint8_t *
                                 int64_t N, int64_t K, const float *sa, const float *sb, void *D_bf16, int64_t ldd,
                                 cudaStream_t s) {
     CUtensorMap ta, tb;
-    if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 64)) return FP8_ERR_CUDA;
+    if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
     const int cap = block_pair_capacity();
     if (cap <= 0) return FP8_ERR_CUDA;
     const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
-    // fp32 accumulator, A/B formats, K-major A and B, N = 128 (>> 3), M = 256 (>> 4)
-    const uint32_t idesc = (1u << 4) | ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(128 >> 3) << 17) |
+    // fp32 accumulator, A/B formats, K-major A and B, N = 256 (>> 3), M = 256 (>> 4)
+    const uint32_t idesc = (1u << 4) | ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(256 >> 3) << 17) |
                            ((uint32_t)(256 >> 4) << 24);
     return pdl_launch(k_gemm_block_2sm, dim3(2 * pairs), dim3(sm2::THREADS), blk::SMEM, s, ta, tb, (int)M, (int)N,
                       (int)K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D_bf16), ldd) == cudaSuccess

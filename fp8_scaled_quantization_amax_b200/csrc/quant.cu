@@ -11,6 +11,8 @@
 // the amax and the cast, so each element is read from HBM exactly once).
 #include <algorithm>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 using namespace fp8q;
@@ -328,6 +330,57 @@ k_colamax(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld
     }
 }
 
+// Four rows x eight columns of bf16 (v[k] = row k), cast with the columns'
+// scales s8 and transposed in registers: colw[j] holds column j's four codes,
+// row 0 in the low byte.
+template <int FMT>
+__device__ __forceinline__ void cast_transpose_4x8(const uint4 (&v)[4], const float (&s8)[8], uint32_t (&colw)[8]) {
+    uint32_t lo[4], hi[4];   // row k's codes of columns 0-3 and 4-7
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+        uint32_t c2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            c2[j] = cvt2<FMT>(__fmul_rn(bf_lo(w[j]), s8[2 * j]), __fmul_rn(bf_hi(w[j]), s8[2 * j + 1]));
+        lo[k] = c2[0] | (c2[1] << 16);
+        hi[k] = c2[2] | (c2[3] << 16);
+    }
+    // 4 rows x 4 bytes -> 4 columns x 4 rows, for the low and the high half
+#pragma unroll
+    for (int hlf = 0; hlf < 2; ++hlf) {
+        const uint32_t *R = hlf ? hi : lo;
+        const uint32_t t01 = __byte_perm(R[0], R[1], 0x5140), t23 = __byte_perm(R[2], R[3], 0x5140);
+        const uint32_t u01 = __byte_perm(R[0], R[1], 0x7362), u23 = __byte_perm(R[2], R[3], 0x7362);
+        colw[4 * hlf + 0] = __byte_perm(t01, t23, 0x5410);
+        colw[4 * hlf + 1] = __byte_perm(t01, t23, 0x7632);
+        colw[4 * hlf + 2] = __byte_perm(u01, u23, 0x5410);
+        colw[4 * hlf + 3] = __byte_perm(u01, u23, 0x7632);
+    }
+}
+
+// Counters of the same 4 x 8 elements: non-finite inputs always, saturated
+// elements exactly where a value is not finite or a column may saturate
+// (bit j of cols8: column j has fp32(amax) * s > fmax).
+template <int FMT>
+__device__ __forceinline__ void count_4x8(const uint4 (&v)[4], const float (&s8)[8], uint32_t cols8, uint32_t &nf,
+                                          uint32_t &sat) {
+    constexpr float fm = fmax_of<FMT>();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t bad = count_nonfinite8(v[k]);
+        nf += bad;
+        if (bad || cols8) {
+            const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                sat += fabsf(__fmul_rn(bf_lo(w[j]), s8[2 * j])) > fm ? 1u : 0u;
+                sat += fabsf(__fmul_rn(bf_hi(w[j]), s8[2 * j + 1])) > fm ? 1u : 0u;
+            }
+        }
+    }
+}
+
 // 64x64 tiles, 128 threads.  The 64 column scales are computed once per CTA
 // into shared memory.  Thread t loads rows 4(t/8) .. +3 of the 8 columns
 // 8(t%8) .. +7 (four 16-byte loads), casts them, and transposes the 4 x 8
@@ -370,45 +423,9 @@ k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, i
 #pragma unroll
     for (int j = 0; j < 8; ++j) s8[j] = sc[cv * 8 + j];
     uint32_t nf = 0, sat = 0;
-    if (counts) {   // exact counts where a column may saturate or a value is not finite
-        const uint32_t cols8 = (maysat[cv >> 2] >> ((cv & 3) * 8)) & 0xFFu;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t bad = count_nonfinite8(v[k]);
-            nf += bad;
-            if (bad || cols8) {
-                const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    sat += fabsf(__fmul_rn(bf_lo(w[j]), s8[2 * j])) > fm ? 1u : 0u;
-                    sat += fabsf(__fmul_rn(bf_hi(w[j]), s8[2 * j + 1])) > fm ? 1u : 0u;
-                }
-            }
-        }
-    }
-    uint32_t lo[4], hi[4];   // row k's codes of columns 0-3 and 4-7
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-        uint32_t c2[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            c2[j] = cvt2<FMT>(__fmul_rn(bf_lo(w[j]), s8[2 * j]), __fmul_rn(bf_hi(w[j]), s8[2 * j + 1]));
-        lo[k] = c2[0] | (c2[1] << 16);
-        hi[k] = c2[2] | (c2[3] << 16);
-    }
-    // 4 rows x 4 bytes -> 4 columns x 4 rows, for the low and the high half
+    if (counts) count_4x8<FMT>(v, s8, (maysat[cv >> 2] >> ((cv & 3) * 8)) & 0xFFu, nf, sat);
     uint32_t colw[8];
-#pragma unroll
-    for (int hlf = 0; hlf < 2; ++hlf) {
-        const uint32_t *R = hlf ? hi : lo;
-        const uint32_t t01 = __byte_perm(R[0], R[1], 0x5140), t23 = __byte_perm(R[2], R[3], 0x5140);
-        const uint32_t u01 = __byte_perm(R[0], R[1], 0x7362), u23 = __byte_perm(R[2], R[3], 0x7362);
-        colw[4 * hlf + 0] = __byte_perm(t01, t23, 0x5410);
-        colw[4 * hlf + 1] = __byte_perm(t01, t23, 0x7632);
-        colw[4 * hlf + 2] = __byte_perm(u01, u23, 0x5410);
-        colw[4 * hlf + 3] = __byte_perm(u01, u23, 0x7632);
-    }
+    cast_transpose_4x8<FMT>(v, s8, colw);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int col = cv * 8 + j;
@@ -425,6 +442,180 @@ k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, i
         if (go < cols && gi < rows) *reinterpret_cast<uint4 *>(qt + go * rows + gi) = o;
     }
     if (counts) flush_counts(counts, nf, sat);
+}
+
+// Single pass over x for the transposed rowwise quantizer: a cluster of
+// kQtCtas CTAs owns a strip of 64 columns, CTA rank r a contiguous range of
+// 128-row tiles of it.  Pass 1 reads the CTA's rows (loads kept in L2) and
+// reduces the 64 column maxima of the finite magnitudes; the partial maxima
+// are combined through distributed shared memory behind one cluster barrier;
+// pass 2 re-reads the same rows (an L2 hit: the strip was read microseconds
+// earlier) and casts and transposes them in 128 x 64 tiles.  x crosses HBM
+// once; clusters loop over strips.  The grid is capped so that the strips
+// in flight fit in L2 together.
+constexpr int kQtCtas = 8;
+constexpr int kQtThreads = 256;
+constexpr int kQtTile = 128;                      // rows per cast tile (4 per thread)
+constexpr int64_t kQtMaxRows = 16384;             // strip of 2 MiB at most; longer columns take two passes
+
+template <int FMT, bool POW2>
+__global__ void __cluster_dims__(kQtCtas, 1, 1) __launch_bounds__(kQtThreads, 4)
+k_qt_strip(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t rows, int64_t cols, int64_t ld,
+           float *__restrict__ scale_inv, float *__restrict__ amax_out, uint32_t *__restrict__ counts) {
+    __shared__ __align__(16) uint32_t tile[64 * 32];   // [column][32 words = 128 rows of codes], swizzled
+    __shared__ uint4 red[32][8];                       // per row lane: packed maxima of 8 x 8 columns
+    __shared__ uint32_t part[2][64];                   // this CTA's column maxima (fp32 bits), by strip parity
+    __shared__ float sc[64];
+    __shared__ uint32_t maysat[2];
+    constexpr float fm = fmax_of<FMT>();
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned rank = cluster.block_rank();
+    const int64_t cid = blockIdx.x / kQtCtas, ncl = gridDim.x / kQtCtas;
+    const int64_t nstrips = (cols + 63) / 64;
+    const int64_t ntiles = (rows + kQtTile - 1) / kQtTile, tpc = (ntiles + kQtCtas - 1) / kQtCtas;
+    const int64_t rb = min((int64_t)rank * tpc, ntiles) * kQtTile;
+    const int64_t re = min(min((int64_t)rank * tpc + tpc, ntiles) * kQtTile, rows);
+    const int cv = threadIdx.x & 7, rr = threadIdx.x >> 3;   // 8 columns x (rows rr, rr + 32, ...)
+    const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+    uint32_t nf = 0, sat = 0;
+    int it = 0;
+    for (int64_t strip = cid; strip < nstrips; strip += ncl, ++it) {
+        const int64_t c0 = strip * 64, gc = c0 + cv * 8;
+        const bool cok = gc < cols;   // cols % 16 == 0: a vector of 8 columns is all in or all out
+        // pass 1: column maxima of this CTA's rows
+        uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+        if (cok) {
+            const uint16_t *xc = x + gc;
+            int64_t r = rb + rr;
+            for (; r + 7 * 32 < re; r += 8 * 32) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = ld_hint(reinterpret_cast<const uint4 *>(xc + (r + 32 * u) * ld), keep);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    m0 = __vmaxu2(m0, abs_finite2(v[u].x));
+                    m1 = __vmaxu2(m1, abs_finite2(v[u].y));
+                    m2 = __vmaxu2(m2, abs_finite2(v[u].z));
+                    m3 = __vmaxu2(m3, abs_finite2(v[u].w));
+                }
+            }
+            for (; r < re; r += 32) {
+                const uint4 v = ld_hint(reinterpret_cast<const uint4 *>(xc + r * ld), keep);
+                m0 = __vmaxu2(m0, abs_finite2(v.x));
+                m1 = __vmaxu2(m1, abs_finite2(v.y));
+                m2 = __vmaxu2(m2, abs_finite2(v.z));
+                m3 = __vmaxu2(m3, abs_finite2(v.w));
+            }
+        }
+        red[rr][cv] = make_uint4(m0, m1, m2, m3);
+        __syncthreads();
+        if (threadIdx.x < 64) {   // column j = 8 * (j >> 3) + (j & 7): word (j & 7) >> 1, half j & 1
+            const int j = threadIdx.x, sh = (j & 1) * 16;
+            uint32_t m = 0;
+#pragma unroll 8
+            for (int k = 0; k < 32; ++k) {
+                const uint4 w = red[k][j >> 3];
+                const uint32_t wj = ((j & 7) >> 1) == 0 ? w.x : ((j & 7) >> 1) == 1 ? w.y : ((j & 7) >> 1) == 2 ? w.z : w.w;
+                m = max(m, (wj >> sh) & 0xFFFFu);
+            }
+            part[it & 1][j] = m << 16;   // bf16 magnitude bits << 16 = the fp32 bits of the same value
+        }
+        cluster.sync();   // every CTA's column maxima of this strip are published
+        if (threadIdx.x < 64) {
+            const int j = threadIdx.x;
+            uint32_t m = 0;
+#pragma unroll
+            for (int k = 0; k < kQtCtas; ++k) m = max(m, *cluster.map_shared_rank(&part[it & 1][j], k));
+            const float a = __uint_as_float(m);
+            const float sj = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
+            sc[j] = sj;
+            if (rank == 0 && c0 + j < cols) {
+                scale_inv[c0 + j] = __fdiv_rn(1.0f, sj);
+                amax_out[c0 + j] = a;
+            }
+            const uint32_t b = __ballot_sync(0xFFFFFFFFu, __fmul_rn(a, sj) > fm);
+            if ((j & 31) == 0) maysat[j >> 5] = b;
+        }
+        __syncthreads();   // the scales
+        float s8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s8[j] = sc[cv * 8 + j];
+        const uint32_t cols8 = (maysat[cv >> 2] >> ((cv & 3) * 8)) & 0xFFu;
+        // pass 2: 128 x 64 tiles, thread (cv, rr) casts rows 4 rr .. + 3 of its 8 columns;
+        // the next tile's loads are issued before this tile is cast
+        auto load_tile = [&](int64_t r0, uint4 (&v)[4]) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int64_t gr = r0 + rr * 4 + k;
+                v[k] = (cok && gr < re) ? ld_hint(reinterpret_cast<const uint4 *>(x + gr * ld + gc), drop)
+                                        : make_uint4(0, 0, 0, 0);
+            }
+        };
+        uint4 nv[4];
+        if (rb < re) load_tile(rb, nv);
+        for (int64_t r0 = rb; r0 < re; r0 += kQtTile) {
+            uint4 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[k] = nv[k];
+            if (r0 + kQtTile < re) load_tile(r0 + kQtTile, nv);
+            if (counts) count_4x8<FMT>(v, s8, cols8, nf, sat);
+            uint32_t colw[8];
+            cast_transpose_4x8<FMT>(v, s8, colw);
+            // column line = 32 words (128 rows); 16-byte chunk rr >> 2 swizzled by cv = col >> 3
+#pragma unroll
+            for (int j = 0; j < 8; ++j) tile[(cv * 8 + j) * 32 + (((rr >> 2) ^ cv) * 4) + (rr & 3)] = colw[j];
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int q = threadIdx.x + kQtThreads * i;
+                const int col = q >> 3, ch = q & 7;   // output row c0 + col, rows r0 + 16 ch .. + 15
+                const int64_t go = c0 + col, gi = r0 + ch * 16;
+                const uint4 o = *reinterpret_cast<const uint4 *>(&tile[col * 32 + ((ch ^ (col >> 3)) * 4)]);
+                if (go < cols && gi < re) st_hint(reinterpret_cast<uint4 *>(qt + go * rows + gi), o, drop);
+            }
+            __syncthreads();   // the tile is rewritten by the next pass
+        }
+    }
+    if (counts) flush_counts(counts, nf, sat);
+    cluster.sync();   // no CTA leaves while a peer may still read its column maxima
+}
+
+// Clusters of k_qt_strip that fit on the device at once (cached per device).
+template <int FMT, bool POW2>
+static int qt_active_clusters() {
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cache[dev] > 0) return cache[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kQtCtas * 64);
+    cfg.blockDim = dim3(kQtThreads);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = kQtCtas;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_qt_strip<FMT, POW2>, &cfg) != cudaSuccess) return 0;
+    cache[dev] = n;
+    return n;
+}
+
+template <int FMT, bool POW2>
+static cudaError_t launch_qt_strip(cudaStream_t s, const uint16_t *x, uint8_t *qt, int64_t rows, int64_t cols,
+                                   int64_t ld, float *scale_inv, float *amax_out, uint32_t *counts) {
+    const int active = qt_active_clusters<FMT, POW2>();
+    if (active <= 0) return cudaErrorInvalidConfiguration;
+    // strips in flight (rows x 128 bytes each) within 64 MiB of L2, so pass 2 finds them there
+    const int64_t fit = std::max<int64_t>(1, ((int64_t)64 << 20) / std::max<int64_t>(1, rows * 128));
+    const int64_t nstrips = (cols + 63) / 64;
+    const int64_t ncl = std::min<int64_t>(std::min<int64_t>(nstrips, active), fit);
+    k_qt_strip<FMT, POW2><<<(unsigned)(ncl * kQtCtas), kQtThreads, 0, s>>>(x, qt, rows, cols, ld, scale_inv, amax_out,
+                                                                          counts);
+    return cudaPeekAtLastError();
 }
 
 // --------------------------------------------------------------- rowwise --
@@ -938,9 +1129,19 @@ extern "C" fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t
     if (st != FP8_OK) return st;
     if (rows == 0 || cols == 0) return FP8_OK;
     cudaStream_t s = as_stream(stream);
+    const uint16_t *xs = static_cast<const uint16_t *>(x_bf16);
+    if (rows <= kQtMaxRows) {   // one launch, one read of x from HBM
+        cudaError_t e;
+        if (fmt == FP8_E4M3)
+            e = pow2 ? launch_qt_strip<FP8_E4M3, true>(s, xs, qT, rows, cols, ld, scale_inv, amax_out, counts)
+                     : launch_qt_strip<FP8_E4M3, false>(s, xs, qT, rows, cols, ld, scale_inv, amax_out, counts);
+        else
+            e = pow2 ? launch_qt_strip<FP8_E5M2, true>(s, xs, qT, rows, cols, ld, scale_inv, amax_out, counts)
+                     : launch_qt_strip<FP8_E5M2, false>(s, xs, qT, rows, cols, ld, scale_inv, amax_out, counts);
+        return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    }
     uint32_t *amax_bits = reinterpret_cast<uint32_t *>(amax_out);
     if (cudaMemsetAsync(amax_bits, 0, (size_t)cols * sizeof(uint32_t), s) != cudaSuccess) return FP8_ERR_CUDA;
-    const uint16_t *xs = static_cast<const uint16_t *>(x_bf16);
     k_colamax<<<dim3((unsigned)((cols + 255) / 256), (unsigned)((rows + kColRows - 1) / kColRows)), 256, 0, s>>>(
         xs, rows, cols, ld, amax_bits);
     const dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));

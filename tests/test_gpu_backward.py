@@ -51,6 +51,41 @@ def test_rowwise_transpose_matches_oracle(orc, fmt, pow2, shape):
     assert_f32_equal(to_np(am), ref_am, "column amax")
 
 
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("shape", [(16384, 2112), (2064, 16400), (16400, 48)])
+def test_rowwise_transpose_schedules_strided(orc, fmt, shape):
+    """Both schedules of the transposed per-row quantizer against the oracle
+    ("FP8训练与QAT…Soup", section "FP8 三种缩放配方怎么选": rowwise scales of
+    the backward GEMMs' K-major operands): the single-pass strip kernel with
+    clusters that each take several strips (16384 rows: the strips in flight
+    are capped by L2; 16400 columns: more strips than clusters, a ragged last
+    strip and ranks with no rows) and the two-pass path for columns longer
+    than 16384 rows, on a strided input whose padding columns hold +Inf and
+    NaN, with the non-finite and saturation counts."""
+    rows, cols = shape
+    pad = 24
+    wide = inputs.bf16_bits(inputs.outlier_activations_bf16((rows, cols + pad), seed=rows + fmt, frac=0.01)).copy()
+    wide[:, cols::2] = 0x7F80
+    wide[:, cols + 1::2] = 0x7FC0
+    wide[rows // 3, 7] = 0xFF80        # -Inf in the data
+    wide[rows - 1, cols - 16] = 0x7FC1  # NaN in the last row
+    bits = np.ascontiguousarray(wide[:, :cols])
+    x = inputs.from_bf16_bits(wide, "cuda")   # [rows, cols + pad]; the quantizer reads cols of each row
+    for pow2 in (True, False):
+        c = torch.zeros(2, dtype=torch.int32, device="cuda")
+        qT = torch.empty((cols, rows), dtype=torch.uint8, device="cuda")
+        sinv = torch.empty(cols, dtype=torch.float32, device="cuda")
+        am = torch.empty(cols, dtype=torch.float32, device="cuda")
+        fp8q.fp8_quantize_rowwise_transpose(x, rows, cols, cols + pad, fmt, pow2, qT, sinv, am, counts=c)
+        rq, rs, rc = orc.quantize_rowwise_transpose(bits, fmt, pow2, counts=True)
+        assert_codes_equal(to_np(qT), rq, fmt)
+        assert_f32_equal(to_np(sinv), rs)
+        assert (int(c[0]), int(c[1])) == rc
+        xf = bf16_to_f64(inputs.from_bf16_bits(bits))
+        ref_am = np.where(np.isfinite(xf), np.abs(xf), 0).max(axis=0).astype(np.float32)
+        assert_f32_equal(to_np(am), ref_am, "column amax")
+
+
 def _tol_check(got, ref, mag, T, what):
     err = np.abs(got - ref)
     bound = T * 2.0 ** -22 * mag + 1e-30
