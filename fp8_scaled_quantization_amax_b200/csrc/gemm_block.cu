@@ -34,7 +34,8 @@
 //   warps 4-11  epilogue: warp w promotes TMEM lane quarter w % 4 (32 rows)
 //               and column half g = (w - 4) / 4 (tile columns g * 128 .. +
 //               127, one 128-row block of B, so one B scale) -- two 64-column
-//               round trips, scalar fp32 FMAs (fma.rn, one rounding per
+//               round trips, fp32 FMAs two columns per instruction
+//               (fma.rn.f32x2: each column its own fma, one rounding per
 //               term); then bf16 RNE and coalesced stores.
 // Summation order per output is fixed (K blocks in order, each block's
 // partial from the tensor core, then one FMA), so results are bit-identical
@@ -285,14 +286,24 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tmem_ld64_async(tsrc + q * 256, r);
                 tmem_wait64(r);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) acc[j] = fmaf(__uint_as_float(r[j]), sc, acc[j]);
+                for (int j = 0; j < 64; j += 2) {
+                    const float2 o = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), make_float2(sc, sc),
+                                                make_float2(acc[j], acc[j + 1]));
+                    acc[j] = o.x;
+                    acc[j + 1] = o.y;
+                }
                 tmem_ld64_async(tsrc + q * 256 + 64, r);
                 tmem_wait64(r);
                 // the partial is in registers: the release warp hands the buffer back to the MMA
                 tc_fence_before();
                 named_arrive(1 + q, blk::kReleaseThreads);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) acc[64 + j] = fmaf(__uint_as_float(r[j]), sc, acc[64 + j]);
+                for (int j = 0; j < 64; j += 2) {
+                    const float2 o = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), make_float2(sc, sc),
+                                                make_float2(acc[64 + j], acc[64 + j + 1]));
+                    acc[64 + j] = o.x;
+                    acc[64 + j + 1] = o.y;
+                }
                 ++it;
             };
             for (int kc = 0; kc < nk; kc += blk::PF) {
