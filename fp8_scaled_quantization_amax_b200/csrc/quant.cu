@@ -12,6 +12,7 @@
 #include <algorithm>
 
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -483,9 +484,26 @@ k_qt_strip(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t row
     for (int64_t strip = cid; strip < nstrips; strip += ncl, ++it) {
         const int64_t c0 = strip * 64, gc = c0 + cv * 8;
         const bool cok = gc < cols;   // cols % 16 == 0: a vector of 8 columns is all in or all out
-        // pass 1: column maxima of this CTA's rows
-        uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
-        if (cok) {
+        // pass 1: column maxima of this CTA's rows.  Fast form: |x| by the
+        // sign mask and a NaN-propagating bf16x2 max; if any column saw a
+        // NaN or Inf the CTA redoes its rows with the finite-only maximum.
+        uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;   // packed per-column maxima (bf16 magnitude bits)
+        auto pass1 = [&](auto EXACT) {
+            constexpr bool exact = decltype(EXACT)::value;
+            auto acc4 = [&](const uint4 &v) {
+                if (exact) {
+                    m0 = __vmaxu2(m0, abs_finite2(v.x));
+                    m1 = __vmaxu2(m1, abs_finite2(v.y));
+                    m2 = __vmaxu2(m2, abs_finite2(v.z));
+                    m3 = __vmaxu2(m3, abs_finite2(v.w));
+                } else {
+                    m0 = amax_fast_word(m0, v.x);
+                    m1 = amax_fast_word(m1, v.y);
+                    m2 = amax_fast_word(m2, v.z);
+                    m3 = amax_fast_word(m3, v.w);
+                }
+            };
+            if (!cok) return;
             const uint16_t *xc = x + gc;
             int64_t r = rb + rr;
             for (; r + 7 * 32 < re; r += 8 * 32) {
@@ -493,20 +511,16 @@ k_qt_strip(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t row
 #pragma unroll
                 for (int u = 0; u < 8; ++u) v[u] = ld_hint(reinterpret_cast<const uint4 *>(xc + (r + 32 * u) * ld), keep);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    m0 = __vmaxu2(m0, abs_finite2(v[u].x));
-                    m1 = __vmaxu2(m1, abs_finite2(v[u].y));
-                    m2 = __vmaxu2(m2, abs_finite2(v[u].z));
-                    m3 = __vmaxu2(m3, abs_finite2(v[u].w));
-                }
+                for (int u = 0; u < 8; ++u) acc4(v[u]);
             }
-            for (; r < re; r += 32) {
-                const uint4 v = ld_hint(reinterpret_cast<const uint4 *>(xc + r * ld), keep);
-                m0 = __vmaxu2(m0, abs_finite2(v.x));
-                m1 = __vmaxu2(m1, abs_finite2(v.y));
-                m2 = __vmaxu2(m2, abs_finite2(v.z));
-                m3 = __vmaxu2(m3, abs_finite2(v.w));
-            }
+            for (; r < re; r += 32) acc4(ld_hint(reinterpret_cast<const uint4 *>(xc + r * ld), keep));
+        };
+        pass1(std::false_type{});
+        const uint32_t hmax = max(max(m0 & 0xFFFFu, m0 >> 16), max(max(m1 & 0xFFFFu, m1 >> 16),
+                                  max(max(m2 & 0xFFFFu, m2 >> 16), max(m3 & 0xFFFFu, m3 >> 16))));
+        if (__syncthreads_or(hmax >= 0x7F80u)) {   // a NaN or Inf in this CTA's rows (rare)
+            m0 = m1 = m2 = m3 = 0;
+            pass1(std::true_type{});
         }
         red[rr][cv] = make_uint4(m0, m1, m2, m3);
         __syncthreads();
