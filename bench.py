@@ -392,7 +392,7 @@ class Workload:
         self.flops = 2 * 2.0 * T * N_out * K_in
         self.unit, self.bound = "TFLOP/s", "tensor"
         self.peak_dtype = "bf16"   # the dominant kernel is the bf16 weight-gradient GEMM
-        self.launches = 5          # + one memset (the column-amax buffer), not a kernel
+        self.launches = 4          # dY rowwise, W^T single-pass transposed rowwise, dgrad GEMM, wgrad GEMM
         self.config = config_of(self.name, self.profile)
         self.host_inputs = [("dY", self.dY), ("X", self.X)]
         self.host_output = self.DX

@@ -168,16 +168,18 @@ FP8Q_API fp8_status fp8_quantize_blockwise(const void *x_bf16, int64_t rows, int
  * the finite entries of the column; 0 gives 1).
  *   qT         [cols, rows] FP8, dense: qT[c][r] = sat_RNE(fp32(x[r][c]) * s_c).
  *   scale_inv  [cols] fp32, 1 / s_c.
- *   amax_out   [cols] fp32, the column amax (also used as the kernels'
- *              reduction buffer; overwritten).
+ *   amax_out   [cols] fp32, the column amax (on the three-launch path also
+ *              the kernels' reduction buffer; overwritten).
  *   counts     [2] uint32 or NULL: [0] += non-finite inputs (NaN, +-Inf),
  *              [1] += saturated elements (|fp32(x) * s| > fmax: +-Inf and
  *              values whose scaled magnitude rounds past fmax; NaN is not
  *              saturated) -- [DeepL] §5.1: overflow and NaN are the failures
  *              to detect.  Added to, never reset; 4-byte aligned.
  *   Shapes: rows % 16 == 0, cols % 16 == 0, ld % 8 == 0, ld >= cols,
- *   ceil(rows / 64) <= 65535.  Three launches: a memset of amax_out, the
- *   column reduction, the transposing cast.
+ *   ceil(rows / 64) <= 65535.  One launch when rows <= 16384 (x read once: an
+ *   8-CTA cluster per 64-column strip combines its partial column maxima
+ *   through distributed shared memory); longer columns take three launches:
+ *   a memset of amax_out, the column reduction, the transposing cast.
  */
 FP8Q_API fp8_status fp8_quantize_rowwise_transpose(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                           fp8_format fmt, int pow2, uint8_t *qT, float *scale_inv,
