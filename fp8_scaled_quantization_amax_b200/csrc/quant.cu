@@ -342,8 +342,10 @@ __device__ __forceinline__ void cast_transpose_4x8(const uint4 (&v)[4], const fl
         const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
         uint32_t c2[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            c2[j] = cvt2<FMT>(__fmul_rn(bf_lo(w[j]), s8[2 * j]), __fmul_rn(bf_hi(w[j]), s8[2 * j + 1]));
+        for (int j = 0; j < 4; ++j) {   // one rounded fp32 multiply per element, two per instruction
+            const float2 y = __fmul2_rn(make_float2(bf_lo(w[j]), bf_hi(w[j])), make_float2(s8[2 * j], s8[2 * j + 1]));
+            c2[j] = cvt2<FMT>(y.x, y.y);
+        }
         lo[k] = c2[0] | (c2[1] << 16);
         hi[k] = c2[2] | (c2[3] << 16);
     }
@@ -454,6 +456,11 @@ k_cast_transpose_col(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, i
 // earlier) and casts and transposes them in 128 x 64 tiles.  x crosses HBM
 // once; clusters loop over strips.  The grid is capped so that the strips
 // in flight fit in L2 together.
+// Split cluster barrier (every thread of every CTA of the cluster; arrive and
+// wait alternate): release on arrive, acquire on wait.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
 constexpr int kQtCtas = 8;
 constexpr int kQtThreads = 256;
 constexpr int kQtTile = 128;                      // rows per cast tile (4 per thread)
@@ -464,8 +471,8 @@ __global__ void __cluster_dims__(kQtCtas, 1, 1) __launch_bounds__(kQtThreads, 4)
 k_qt_strip(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t rows, int64_t cols, int64_t ld,
            float *__restrict__ scale_inv, float *__restrict__ amax_out, uint32_t *__restrict__ counts) {
     __shared__ __align__(16) uint32_t tile[64 * 32];   // [column][32 words = 128 rows of codes], swizzled
-    __shared__ uint4 red[32][8];                       // per row lane: packed maxima of 8 x 8 columns
-    __shared__ uint32_t part[2][64];                   // this CTA's column maxima (fp32 bits), by strip parity
+    __shared__ uint4 red[8][8];                        // per warp: packed maxima of 8 x 8 columns
+    __shared__ uint32_t part[64];                      // this CTA's column maxima (fp32 bits)
     __shared__ float sc[64];
     __shared__ uint32_t maysat[2];
     constexpr float fm = fmax_of<FMT>();
@@ -522,25 +529,36 @@ k_qt_strip(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t row
             m0 = m1 = m2 = m3 = 0;
             pass1(std::true_type{});
         }
-        red[rr][cv] = make_uint4(m0, m1, m2, m3);
+        // the four lanes of a warp with the same cv (lanes cv + 8i) first, by shuffles
+#pragma unroll
+        for (int o = 8; o < 32; o <<= 1) {
+            m0 = __vmaxu2(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, o));
+            m1 = __vmaxu2(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
+            m2 = __vmaxu2(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, o));
+            m3 = __vmaxu2(m3, __shfl_xor_sync(0xFFFFFFFFu, m3, o));
+        }
+        if ((threadIdx.x & 31) < 8) red[threadIdx.x >> 5][cv] = make_uint4(m0, m1, m2, m3);
+        // the previous strip's peers have read part[] (their "reads done" arrive)
+        if (it > 0) cluster_wait();
         __syncthreads();
         if (threadIdx.x < 64) {   // column j = 8 * (j >> 3) + (j & 7): word (j & 7) >> 1, half j & 1
             const int j = threadIdx.x, sh = (j & 1) * 16;
             uint32_t m = 0;
-#pragma unroll 8
-            for (int k = 0; k < 32; ++k) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
                 const uint4 w = red[k][j >> 3];
                 const uint32_t wj = ((j & 7) >> 1) == 0 ? w.x : ((j & 7) >> 1) == 1 ? w.y : ((j & 7) >> 1) == 2 ? w.z : w.w;
                 m = max(m, (wj >> sh) & 0xFFFFu);
             }
-            part[it & 1][j] = m << 16;   // bf16 magnitude bits << 16 = the fp32 bits of the same value
+            part[j] = m << 16;   // bf16 magnitude bits << 16 = the fp32 bits of the same value
         }
-        cluster.sync();   // every CTA's column maxima of this strip are published
+        cluster_arrive();   // every CTA's column maxima of this strip are published
+        cluster_wait();
         if (threadIdx.x < 64) {
             const int j = threadIdx.x;
             uint32_t m = 0;
 #pragma unroll
-            for (int k = 0; k < kQtCtas; ++k) m = max(m, *cluster.map_shared_rank(&part[it & 1][j], k));
+            for (int k = 0; k < kQtCtas; ++k) m = max(m, *cluster.map_shared_rank(&part[j], k));
             const float a = __uint_as_float(m);
             const float sj = POW2 ? pow2_scale_from_amax(a, fm) : scale_from_amax(a, fm);
             sc[j] = sj;
@@ -551,48 +569,56 @@ k_qt_strip(const uint16_t *__restrict__ x, uint8_t *__restrict__ qt, int64_t row
             const uint32_t b = __ballot_sync(0xFFFFFFFFu, __fmul_rn(a, sj) > fm);
             if ((j & 31) == 0) maysat[j >> 5] = b;
         }
+        cluster_arrive();   // this CTA has read its peers' part[] ("reads done"; waited before the next write)
         __syncthreads();   // the scales
         float s8[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) s8[j] = sc[cv * 8 + j];
         const uint32_t cols8 = (maysat[cv >> 2] >> ((cv & 3) * 8)) & 0xFFu;
         // pass 2: 128 x 64 tiles, thread (cv, rr) casts rows 4 rr .. + 3 of its 8 columns;
-        // the next tile's loads are issued before this tile is cast
-        auto load_tile = [&](int64_t r0, uint4 (&v)[4]) {
+        // the next tile's loads are issued before this tile is cast.  re is a
+        // multiple of 16, so a thread's four rows are all in or all out.
+        const uint16_t *xp = x + (rb + rr * 4) * ld + gc;   // + k * ld: row k of this thread's group
+        const int64_t tstep = (int64_t)kQtTile * ld;
+        auto load_tile = [&](int64_t r0, const uint16_t *p, uint4 (&v)[4]) {
+            const bool in = cok && r0 + rr * 4 < re;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int64_t gr = r0 + rr * 4 + k;
-                v[k] = (cok && gr < re) ? ld_hint(reinterpret_cast<const uint4 *>(x + gr * ld + gc), drop)
-                                        : make_uint4(0, 0, 0, 0);
-            }
+            for (int k = 0; k < 4; ++k)
+                v[k] = in ? ld_hint(reinterpret_cast<const uint4 *>(p + k * ld), drop) : make_uint4(0, 0, 0, 0);
+        };
+        // output row c0 + col (col = q >> 3), bytes r0 + 16 (q & 7) .. + 15, for q = t and t + 256
+        const int col0 = threadIdx.x >> 3, col1 = col0 + 32, ch = threadIdx.x & 7;
+        uint8_t *qp = qt + (c0 + col0) * rows + rb + ch * 16;   // + 32 rows: output row c0 + col1
+        const bool ok0 = c0 + col0 < cols, ok1 = c0 + col1 < cols;
+        const int tl0 = col0 * 32 + ((ch ^ (col0 >> 3)) * 4), tl1 = col1 * 32 + ((ch ^ (col1 >> 3)) * 4);
+        const int tw = (cv * 8) * 32 + (((rr >> 2) ^ cv) * 4) + (rr & 3);   // + 32 j: column cv * 8 + j
+        auto cast_tile = [&](int64_t r0, const uint4 (&v)[4]) {
+            if (counts) count_4x8<FMT>(v, s8, cols8, nf, sat);
+            uint32_t colw[8];
+            cast_transpose_4x8<FMT>(v, s8, colw);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) tile[tw + 32 * j] = colw[j];
+            __syncthreads();
+            const bool rin = r0 + ch * 16 < re;
+            const uint4 o0 = *reinterpret_cast<const uint4 *>(&tile[tl0]), o1 = *reinterpret_cast<const uint4 *>(&tile[tl1]);
+            if (rin && ok0) st_hint(reinterpret_cast<uint4 *>(qp), o0, drop);
+            if (rin && ok1) st_hint(reinterpret_cast<uint4 *>(qp + 32 * rows), o1, drop);
+            qp += kQtTile;
+            __syncthreads();   // the tile is rewritten by the next pass
         };
         uint4 nv[4];
-        if (rb < re) load_tile(rb, nv);
+        if (rb < re) load_tile(rb, xp, nv);
         for (int64_t r0 = rb; r0 < re; r0 += kQtTile) {
             uint4 v[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) v[k] = nv[k];
-            if (r0 + kQtTile < re) load_tile(r0 + kQtTile, nv);
-            if (counts) count_4x8<FMT>(v, s8, cols8, nf, sat);
-            uint32_t colw[8];
-            cast_transpose_4x8<FMT>(v, s8, colw);
-            // column line = 32 words (128 rows); 16-byte chunk rr >> 2 swizzled by cv = col >> 3
-#pragma unroll
-            for (int j = 0; j < 8; ++j) tile[(cv * 8 + j) * 32 + (((rr >> 2) ^ cv) * 4) + (rr & 3)] = colw[j];
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int q = threadIdx.x + kQtThreads * i;
-                const int col = q >> 3, ch = q & 7;   // output row c0 + col, rows r0 + 16 ch .. + 15
-                const int64_t go = c0 + col, gi = r0 + ch * 16;
-                const uint4 o = *reinterpret_cast<const uint4 *>(&tile[col * 32 + ((ch ^ (col >> 3)) * 4)]);
-                if (go < cols && gi < re) st_hint(reinterpret_cast<uint4 *>(qt + go * rows + gi), o, drop);
-            }
-            __syncthreads();   // the tile is rewritten by the next pass
+            xp += tstep;
+            if (r0 + kQtTile < re) load_tile(r0 + kQtTile, xp, nv);
+            cast_tile(r0, v);
         }
     }
     if (counts) flush_counts(counts, nf, sat);
-    cluster.sync();   // no CTA leaves while a peer may still read its column maxima
+    if (it > 0) cluster_wait();   // no CTA leaves while a peer may still read its column maxima
 }
 
 // Clusters of k_qt_strip that fit on the device at once (cached per device).
