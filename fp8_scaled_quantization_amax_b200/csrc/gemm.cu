@@ -895,7 +895,7 @@ using namespace fp8q_host;
 // The block-scaled GEMM on CTA pairs lives in gemm_block.cu.
 fp8_status fp8q_gemm_block_pair(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int64_t M,
                                 int64_t N, int64_t K, const float *sa, const float *sb, void *D_bf16, int64_t ldd,
-                                cudaStream_t s);
+                                fp8_format qfmt, uint8_t *qo, float *qsinv, uint32_t *counts, cudaStream_t s);
 
 namespace {
 std::atomic<uint32_t> g_split_epoch[64];   // per device; a split launch publishes with a fresh value
@@ -947,7 +947,8 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
     // otherwise one CTA per 128-row tile.
     if (M > BM && !one_sm_cluster_split(M, N, K, sms)) {
         if (mode == FP8_SCALE_BLOCK)
-            return fp8q_gemm_block_pair(A, fa, B, fb, M, N, K, a_scale_inv, b_scale_inv, D_bf16, ldd, s);
+            return fp8q_gemm_block_pair(A, fa, B, fb, M, N, K, a_scale_inv, b_scale_inv, D_bf16, ldd, FP8_E4M3,
+                                        nullptr, nullptr, nullptr, s);
         CUtensorMap ta, tb;
         if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
         const uint32_t idesc = make_idesc(fa, fb, 256, 256);
@@ -987,6 +988,43 @@ extern "C" fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uin
     else
         e = launch_gemm<kModeBlock>(s, sms, ta, tb, (int)M, (int)N, (int)K, idesc, a_scale_inv, b_scale_inv, D_bf16, ldd);
     return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+// Block-scaled GEMM whose output is requantized with 1 x 128 blocks for the
+// next GEMM (the MLP chain: H = up(X) in bf16, requantized for the down
+// projection).  With M > 128 and K > 0 one launch: the pair kernel's epilogue
+// rounds each output to bf16 and quantizes its 128-column blocks in
+// registers.  Otherwise the GEMM into D_bf16, then fp8_quantize_blockwise on
+// it.  Either way the codes and scales equal fp8_quantize_blockwise(D).
+extern "C" fp8_status fp8_gemm_block_requant(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
+                                             int64_t M, int64_t N, int64_t K, const float *a_scale_inv,
+                                             const float *b_scale_inv, void *D_bf16, int64_t ldd, fp8_format fo,
+                                             uint8_t *q, float *q_scale_inv, uint32_t *counts, void *stream) {
+    if ((fa != FP8_E4M3 && fa != FP8_E5M2) || (fb != FP8_E4M3 && fb != FP8_E5M2)) return FP8_ERR_INVALID_ARG;
+    if (fo != FP8_E4M3 && fo != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0) return FP8_ERR_SHAPE;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP8_ERR_SHAPE;
+    if (K % 16 || N % 16) return FP8_ERR_SHAPE;
+    if (D_bf16 && ldd < N) return FP8_ERR_SHAPE;
+    if (D_bf16 && (ldd % 8 || !aligned16(D_bf16))) return FP8_ERR_ALIGNMENT;
+    const bool fused = M > BM && K > 0;
+    if (M > 0 && N > 0) {
+        if (!q || !q_scale_inv || (!fused && !D_bf16)) return FP8_ERR_INVALID_ARG;
+        if (K > 0 && (!A || !B || !a_scale_inv || !b_scale_inv)) return FP8_ERR_INVALID_ARG;
+    }
+    if ((q && !aligned16(q)) || (A && !aligned16(A)) || (B && !aligned16(B))) return FP8_ERR_ALIGNMENT;
+    if (counts && (reinterpret_cast<uintptr_t>(counts) & 3u)) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (M == 0 || N == 0) return FP8_OK;
+    if (fused)
+        return fp8q_gemm_block_pair(A, fa, B, fb, M, N, K, a_scale_inv, b_scale_inv, D_bf16, ldd, fo, q,
+                                    q_scale_inv, counts, as_stream(stream));
+    st = fp8_gemm_scaled(A, fa, B, fb, M, N, K, FP8_SCALE_BLOCK, a_scale_inv, b_scale_inv, D_bf16, ldd, nullptr, 0,
+                         stream);
+    if (st != FP8_OK) return st;
+    return fp8_quantize_blockwise(D_bf16, M, N, ldd, fo, 1, q, q_scale_inv, counts, stream);
 }
 
 // The E8M0, the block-scaled pair and the bf16 weight-gradient GEMMs keep

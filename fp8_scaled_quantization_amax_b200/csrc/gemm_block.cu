@@ -93,10 +93,19 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// QFMT < 0: D = bf16(promoted sum).  QFMT = FP8_E4M3 / FP8_E5M2: the
+// epilogue also requantizes its output with 1 x 128 blocks, as the 1x128
+// block quantizer would quantize D (H of an MLP, requantized for the next
+// GEMM): each thread holds one row of one 128-column block, so the block's
+// amax, scale and cast happen in registers; D (optional) gets the bf16 values
+// the codes were cast from, qo [M, N] the codes, qsinv [ceil(N / 128), M]
+// the block scales' inverses, counts the non-finite / saturated counts.
+template <int QFMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
 k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                  int K, uint32_t idesc, const float *__restrict__ sa, const float *__restrict__ sb,
-                 __nv_bfloat16 *__restrict__ D, int64_t ldd) {
+                 __nv_bfloat16 *__restrict__ D, int64_t ldd, uint8_t *__restrict__ qo, float *__restrict__ qsinv,
+                 uint32_t *__restrict__ counts) {
     constexpr int STG = blk::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -239,6 +248,7 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int sp = warp & 3;
         const int g = (warp - 4) >> 2;                  // column half: tile columns g * 128 .. + 127
         const uint32_t tsrc = tmem + ((uint32_t)(sp * 32) << 16) + (uint32_t)(g * 128);   // this warp's lanes and columns
+        uint32_t nf_q = 0, sat_q = 0;   // requantization counters
         uint32_t it = 0;
         bool ok = true;
         for (int i = 0; ok && i < n_items; ++i) {
@@ -318,13 +328,72 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 break;
             }
             uint8_t *ebuf = smem + blk::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
+            const int colb = n_blk * 256 + g * 128;   // this warp's 128 columns: one 1 x 128 block
+            if constexpr (QFMT < 0) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(acc[h * 64 + 2 * j], acc[h * 64 + 2 * j + 1]);
-                store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, (int64_t)M, n_blk * 256 + g * 128 + h * 64, N);
+                    for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(acc[h * 64 + 2 * j], acc[h * 64 + 2 * j + 1]);
+                    store_rows_coalesced(ebuf, pk, lane, D, ldd, row0, (int64_t)M, colb + h * 64, N);
+                }
+            } else {
+                constexpr float fm = fmax_of<QFMT>();
+                uint32_t hb[2][32];   // the row's 128 outputs in bf16, RNE: the values the codes come from
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) hb[h][j] = pack_bf16x2(acc[h * 64 + 2 * j], acc[h * 64 + 2 * j + 1]);
+                if (D != nullptr) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) store_rows_coalesced(ebuf, hb[h], lane, D, ldd, row0, (int64_t)M, colb + h * 64, N);
+                }
+                // amax over the finite values of the block's columns below N (N % 16 == 0)
+                const int nvalid = N - colb;
+                uint32_t m2 = 0;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) m2 = amax_fast_word(m2, (h * 64 + 2 * j < nvalid) ? hb[h][j] : 0u);
+                uint32_t m = amax_fast_final(m2);
+                const bool nonfin = m == 0xFFFFFFFFu;
+                if (nonfin) {
+                    uint32_t bad = 0;
+                    m = 0;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (h * 64 + 2 * j < nvalid) m = amax_exact_word(m, hb[h][j], bad);
+                }
+                const float amax = bf16bits_to_float(m);
+                const float s = scale_from_amax(amax, fm);
+                const bool row_ok = row0 + lane < M;
+                if (row_ok && nvalid > 0) qsinv[(int64_t)(colb / 128) * M + row0 + lane] = __fdiv_rn(1.0f, s);
+                if (counts != nullptr && row_ok && may_saturate(nonfin, amax, s, fm)) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            if (h * 64 + 2 * j >= nvalid) continue;
+                            const uint32_t w = hb[h][j];
+                            nf_q += ((w & 0x7F80u) == 0x7F80u) + ((w & 0x7F800000u) == 0x7F800000u);
+                            sat_q += (fabsf(__fmul_rn(bf_lo(w), s)) > fm) + (fabsf(__fmul_rn(bf_hi(w), s)) > fm);
+                        }
+                }
+                uint32_t qw[32];   // 128 codes, four per word, column order
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t w0 = hb[j >> 4][2 * (j & 15)], w1 = hb[j >> 4][2 * (j & 15) + 1];
+                    const uint32_t c0 = cvt2<QFMT>(__fmul_rn(bf_lo(w0), s), __fmul_rn(bf_hi(w0), s));
+                    const uint32_t c1 = cvt2<QFMT>(__fmul_rn(bf_lo(w1), s), __fmul_rn(bf_hi(w1), s));
+                    qw[j] = c0 | (c1 << 16);
+                }
+                store_rows_coalesced(ebuf, qw, lane, qo, (int64_t)N, row0, (int64_t)M, colb, N);
             }
+        }
+        if constexpr (QFMT >= 0) {
+            if (counts != nullptr) flush_counts(counts, nf_q, sat_q);
         }
     }
 
@@ -338,7 +407,9 @@ k_gemm_block_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 }
 
 // Pairs of the block-scaled kernel that fit on the device at once (cached per
-// device); 0 when the kernel cannot be launched as the register split needs.
+// device and variant); 0 when the kernel cannot be launched as the register
+// split needs.
+template <int QFMT>
 int block_pair_capacity() {
     static int cache[64];
     static std::mutex mu;
@@ -346,11 +417,11 @@ int block_pair_capacity() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     std::lock_guard<std::mutex> lk(mu);
     if (cache[dev] > 0) return cache[dev];
-    if (cudaFuncSetAttribute(k_gemm_block_2sm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)blk::SMEM) !=
+    if (cudaFuncSetAttribute(k_gemm_block_2sm<QFMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)blk::SMEM) !=
         cudaSuccess)
         return 0;
     cudaFuncAttributes fa;   // the setmaxnreg split assumes this launch register count
-    if (cudaFuncGetAttributes(&fa, k_gemm_block_2sm) != cudaSuccess || fa.numRegs != sm2::REGS_LAUNCH) return 0;
+    if (cudaFuncGetAttributes(&fa, k_gemm_block_2sm<QFMT>) != cudaSuccess || fa.numRegs != sm2::REGS_LAUNCH) return 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 64);
     cfg.blockDim = dim3(sm2::THREADS);
@@ -363,9 +434,24 @@ int block_pair_capacity() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_block_2sm, &cfg) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_block_2sm<QFMT>, &cfg) != cudaSuccess) return 0;
     cache[dev] = n;
     return n;
+}
+
+template <int QFMT>
+fp8_status launch_block_pair(const CUtensorMap &ta, const CUtensorMap &tb, int64_t M, int64_t N, int64_t K,
+                             uint32_t idesc, const float *sa, const float *sb, void *D_bf16, int64_t ldd, uint8_t *qo,
+                             float *qsinv, uint32_t *counts, cudaStream_t s) {
+    const int cap = block_pair_capacity<QFMT>();
+    if (cap <= 0) return FP8_ERR_CUDA;
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
+    return pdl_launch(k_gemm_block_2sm<QFMT>, dim3(2 * pairs), dim3(sm2::THREADS), blk::SMEM, s, ta, tb, (int)M,
+                      (int)N, (int)K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D_bf16), ldd, qo, qsinv,
+                      counts) == cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_CUDA;
 }
 
 }  // namespace
@@ -373,24 +459,22 @@ int block_pair_capacity() {
 using namespace fp8q_host;
 
 // The block-scaled GEMM on CTA pairs (M > 128 rows); arguments validated by
-// fp8_gemm_scaled.  Returns FP8_ERR_CUDA when a map cannot be encoded or the
-// launch fails.
+// the entry points.  qo == NULL: D only.  qo != NULL: the output is also
+// requantized with 1 x 128 blocks of format qfmt (D may then be NULL).
+// Returns FP8_ERR_CUDA when a map cannot be encoded or the launch fails.
 fp8_status fp8q_gemm_block_pair(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int64_t M,
                                 int64_t N, int64_t K, const float *sa, const float *sb, void *D_bf16, int64_t ldd,
-                                cudaStream_t s) {
+                                fp8_format qfmt, uint8_t *qo, float *qsinv, uint32_t *counts, cudaStream_t s) {
     CUtensorMap ta, tb;
     if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
-    const int cap = block_pair_capacity();
-    if (cap <= 0) return FP8_ERR_CUDA;
-    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
     // fp32 accumulator, A/B formats, K-major A and B, N = 256 (>> 3), M = 256 (>> 4)
     const uint32_t idesc = (1u << 4) | ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(256 >> 3) << 17) |
                            ((uint32_t)(256 >> 4) << 24);
-    return pdl_launch(k_gemm_block_2sm, dim3(2 * pairs), dim3(sm2::THREADS), blk::SMEM, s, ta, tb, (int)M, (int)N,
-                      (int)K, idesc, sa, sb, static_cast<__nv_bfloat16 *>(D_bf16), ldd) == cudaSuccess
-               ? FP8_OK
-               : FP8_ERR_CUDA;
+    if (qo == nullptr)
+        return launch_block_pair<-1>(ta, tb, M, N, K, idesc, sa, sb, D_bf16, ldd, nullptr, nullptr, nullptr, s);
+    if (qfmt == FP8_E4M3)
+        return launch_block_pair<FP8_E4M3>(ta, tb, M, N, K, idesc, sa, sb, D_bf16, ldd, qo, qsinv, counts, s);
+    return launch_block_pair<FP8_E5M2>(ta, tb, M, N, K, idesc, sa, sb, D_bf16, ldd, qo, qsinv, counts, s);
 }
 
 // This file's device error word (read and optionally cleared by

@@ -40,6 +40,7 @@ SIGNATURES = {
     "fp8_gemm_workspace_size": (_S, [_I64, _I64, _I64, _I, _P]),
     "fp8_gemm_grouped": (_S, [_P, _I, _P, _I, _I, _P, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
     "fp8_gemm_scaled_noalloc": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _I, _P, _P, _P, _I64, _P]),
+    "fp8_gemm_block_requant": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _P, _P, _P, _I64, _I, _P, _P, _P, _P]),
     "fp8_amax_history_update": (_S, [_P, _P, _I, _P, _I, _P, _P, _P, _P]),
     "fp8_kv_quant": (_S, [_P, _I64, _I64, _I64, _I64, _I, _P, _P, _P, _P]),
     "fp8_kv_dequant": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P]),
@@ -166,6 +167,16 @@ def fp8_gemm_scaled_noalloc(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_in
     _check("fp8_gemm_scaled_noalloc", lib().fp8_gemm_scaled_noalloc(
         _ptr(A), fa, _ptr(B), fb, M, N, K, mode, _ptr(a_scale_inv), _ptr(b_scale_inv), _ptr(D), ldd,
         _stream(stream)))
+
+
+def fp8_gemm_block_requant(A, fa, B, fb, M, N, K, a_scale_inv, b_scale_inv, D, ldd, fo, q, q_scale_inv,
+                           counts=None, stream=None):
+    _dev(A, torch.uint8, "A"); _dev(B, torch.uint8, "B"); _dev(D, torch.bfloat16, "D")
+    _dev(a_scale_inv, torch.float32, "a_scale_inv"); _dev(b_scale_inv, torch.float32, "b_scale_inv")
+    _dev(q, torch.uint8, "q"); _dev(q_scale_inv, torch.float32, "q_scale_inv"); _dev(counts, torch.int32, "counts")
+    _check("fp8_gemm_block_requant", lib().fp8_gemm_block_requant(
+        _ptr(A), fa, _ptr(B), fb, M, N, K, _ptr(a_scale_inv), _ptr(b_scale_inv), _ptr(D), ldd, fo, _ptr(q),
+        _ptr(q_scale_inv), _ptr(counts), _stream(stream)))
 
 
 def fp8_gemm_grouped(A, fa, B, fb, G, group_offsets, total_M, N, K, mode, a_scale_inv, b_scale_inv, D, ldd,
@@ -386,6 +397,18 @@ def gemm(A, fa, B, fb, mode, a_scale_inv, b_scale_inv, out=None, workspace=None)
     D = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     fp8_gemm_scaled(A, fa, B, fb, M, N, K, mode, a_scale_inv, b_scale_inv, D, D.stride(0), workspace)
     return D
+
+
+def gemm_block_requant(A, fa, B, fb, a_scale_inv, b_scale_inv, fo, store_d=False, counts=None):
+    """(q [M, N] codes of format fo, q_scale_inv [ceil(N/128), M], D [M, N] bf16 or None): the block-scaled
+    GEMM's output requantized with 1 x 128 blocks, as quantize_blockwise(D, fo, 1) would."""
+    M, K = A.shape
+    N = B.shape[0]
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if store_d else None
+    q = torch.empty((M, N), dtype=torch.uint8, device=A.device)
+    qs = torch.empty(((N + 127) // 128, M), dtype=torch.float32, device=A.device)
+    fp8_gemm_block_requant(A, fa, B, fb, M, N, K, a_scale_inv, b_scale_inv, D, N, fo, q, qs, counts)
+    return q, qs, D
 
 
 def gemm_grouped(A, fa, B, fb, group_offsets, mode, a_scale_inv, b_scale_inv, out=None):

@@ -258,6 +258,37 @@ FP8Q_API fp8_status fp8_gemm_scaled(const uint8_t *A, fp8_format fa, const uint8
                            int64_t ldd, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Block-scaled GEMM whose output is requantized for the next GEMM ([DeepL]
+ * §2.3: per-block scales on every GEMM operand; an MLP's second GEMM takes
+ * the first one's output, H = bf16(up(X)), quantized with 1 x 128 blocks).
+ *   A, fa, B, fb, M, N, K, a_scale_inv, b_scale_inv: as fp8_gemm_scaled
+ *       with mode FP8_SCALE_BLOCK (fp32 scales, 1 x 128 blocks of A,
+ *       128 x 128 blocks of B).
+ *   D_bf16 [M, N] bf16, leading dimension ldd, device: the GEMM output
+ *       (RNE); may be NULL when M > 128 and K > 0, otherwise required.
+ *   fo:          format of the requantized output.
+ *   q            [M, N] FP8 (fo), dense, device, 16-byte aligned:
+ *                q = fp8_quantize_blockwise(D, block_rows = 1, fo) code for
+ *                code, whether or not D is stored.
+ *   q_scale_inv  [ceil(N / 128), M] fp32, device: 1 / s of each row's
+ *                128-column block (the layout fp8_quantize_blockwise
+ *                writes for block_rows = 1).
+ *   counts       [2] uint32 or NULL: non-finite and saturated elements of
+ *                the requantization, as fp8_quantize_blockwise counts them.
+ *   M > 128 and K > 0: one launch -- the CTA-pair kernel's epilogue rounds
+ *   each output to bf16 and quantizes its 128-column blocks in registers
+ *   (one thread holds one row of one block).  Otherwise two launches (the
+ *   GEMM into D_bf16, then fp8_quantize_blockwise on it).
+ *   Shapes: as fp8_gemm_scaled, and N % 16 == 0.  Errors as
+ *   fp8_gemm_scaled; FP8_ERR_INVALID_ARG also for a NULL q or q_scale_inv,
+ *   or a NULL D_bf16 where it is required.
+ */
+FP8Q_API fp8_status fp8_gemm_block_requant(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
+                                  int64_t M, int64_t N, int64_t K, const float *a_scale_inv,
+                                  const float *b_scale_inv, void *D_bf16, int64_t ldd, fp8_format fo,
+                                  uint8_t *q, float *q_scale_inv, uint32_t *counts, void *stream);
+
+/*
  * Weight-gradient GEMM kept in high precision ([Soup] section "FP8 三种缩放
  * 配方怎么选": the rowwise_with_gw_hp recipe keeps the weight gradient out of
  * FP8):

@@ -94,6 +94,13 @@ def test_validation_before_device_access():
     assert L.fp8_gemm_block_e8m0(FAKE, 2, FAKE, 0, 64, 64, 64, FAKE, FAKE, FAKE, 64, n) == INVALID
     assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 64, None, FAKE, FAKE, 64, n) == INVALID
     assert L.fp8_gemm_block_e8m0(FAKE, 0, FAKE, 0, 64, 64, 64, FAKE_ODD, FAKE, FAKE, 64, n) == ALIGN
+    # block-scaled GEMM with its output requantized 1x128
+    assert L.fp8_gemm_block_requant(FAKE, 0, FAKE, 0, 256, 264, 256, FAKE, FAKE, None, 264, 0, FAKE, FAKE, None, n) == SHAPE   # N % 16
+    assert L.fp8_gemm_block_requant(FAKE, 0, FAKE, 0, 256, 256, 256, FAKE, FAKE, None, 256, 3, FAKE, FAKE, None, n) == INVALID  # fo
+    assert L.fp8_gemm_block_requant(FAKE, 0, FAKE, 0, 256, 256, 256, FAKE, FAKE, None, 256, 0, None, FAKE, None, n) == INVALID  # q
+    assert L.fp8_gemm_block_requant(FAKE, 0, FAKE, 0, 64, 256, 256, FAKE, FAKE, None, 256, 0, FAKE, FAKE, None, n) == INVALID   # D needed
+    assert L.fp8_gemm_block_requant(FAKE, 0, FAKE, 0, 256, 256, 256, FAKE, FAKE, FAKE, 128, 0, FAKE, FAKE, None, n) == SHAPE   # ldd < N
+    assert L.fp8_gemm_block_requant(FAKE, 0, FAKE, 0, 256, 256, 256, FAKE, FAKE, None, 256, 0, FAKE, FAKE, FAKE_ODD, n) == ALIGN
     # backward operands and the bf16 weight gradient
     assert L.fp8_quantize_rowwise_transpose(FAKE, 24, 32, 32, 0, 1, FAKE, FAKE, FAKE, None, n) == SHAPE   # rows % 16
     assert L.fp8_quantize_rowwise_transpose(FAKE, 32, 32, 32, 0, 1, FAKE, FAKE, None, None, n) == INVALID
