@@ -41,6 +41,22 @@ __device__ __forceinline__ float pow2_scale_from_amax(float amax, float fm) {
     return __uint_as_float(e);
 }
 
+// E8M0 scale image (the operand layout of the hardware block-scaled MMA,
+// which reads one byte per row for every 32-wide K slice; a 32-bit word holds
+// four such bytes).  Here a byte carries a whole 128-wide K block, so one word
+// covers four K blocks: for K block kb and row r the byte at
+//   ((kb / 4) * ceil(rows / 128) + r / 128) * 512 + (r % 32) * 16
+//     + ((r % 128) / 32) * 4 + kb % 4
+// holds the biased exponent e of the dequantization factor 2^(e - 127).  For
+// a power-of-two scale s = 2^k the factor is 2^-k, so e = 127 - k
+// = 254 - (biased exponent of s).
+__device__ __forceinline__ uint8_t e8m0_of_scale(float s) {
+    return (uint8_t)(254u - ((__float_as_uint(s) >> 23) & 0xFFu));
+}
+__device__ __forceinline__ int64_t e8m0_offset(int64_t kb, int64_t rt, int64_t r) {
+    return ((kb >> 2) * rt + (r >> 7)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (kb & 3);
+}
+
 // Two bf16 in a 32-bit word -> two fp32 (exact).
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

@@ -80,10 +80,18 @@ __device__ __forceinline__ void tc_mma_pair_mx(uint32_t d_tmem, uint64_t adesc, 
         : "memory");
 }
 
+// QFMT < 0: D = bf16(sum).  QFMT = FP8_E4M3 / FP8_E5M2: the epilogue also
+// requantizes its output with 1 x 128 blocks and power-of-two scales, as
+// fp8_quantize_blockwise_e8m0 would quantize D: each thread holds one row of
+// one 128-column block; D (optional) gets the bf16 values, qo [M, N] the
+// codes, qsf the E8M0 image of the next GEMM's A operand (rows past M in the
+// last 128-row group: e = 127), counts the non-finite / saturated counts.
+template <int QFMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(sm2::THREADS, 1)
 k_gemm_mx_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, int M, int N,
-              int K, uint32_t idesc, __nv_bfloat16 *__restrict__ D, int64_t ldd) {
+              int K, uint32_t idesc, __nv_bfloat16 *__restrict__ D, int64_t ldd, uint8_t *__restrict__ qo,
+              uint8_t *__restrict__ qsf, uint32_t *__restrict__ counts) {
     constexpr int STG = mx::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -222,6 +230,7 @@ k_gemm_mx_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const int sp = warp & 3;
         const int ch = (warp - 4) >> 2;
         const uint32_t src = tmem + ((uint32_t)(sp * 32) << 16) + ch * 128;
+        uint32_t nf_q = 0, sat_q = 0;   // requantization counters
         for (int i = 0; i < n_items; ++i) {
             const int t = pair + i * npairs;
             const int m_blk = t % num_m, n_blk = t / num_m;
@@ -244,14 +253,75 @@ k_gemm_mx_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar, 0));
             uint8_t *ebuf = smem + mx::EPI_OFF + (size_t)(warp - 4) * kEpiBufBytes;
+            if constexpr (QFMT < 0) {
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const uint32_t *r = h2 ? r1 : r0;
-                uint32_t pk[32];
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const uint32_t *r = h2 ? r1 : r0;
+                    uint32_t pk[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-                store_rows_coalesced(ebuf, pk, lane, D, ldd, m - lane, M, n_base + h2 * 64, N);
+                    for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                    store_rows_coalesced(ebuf, pk, lane, D, ldd, m - lane, M, n_base + h2 * 64, N);
+                }
+            } else {
+                constexpr float fm = fmax_of<QFMT>();
+                uint32_t hb[2][32];   // the row's 128 outputs in bf16, RNE: the values the codes come from
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    hb[0][j] = pack_bf16x2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+                    hb[1][j] = pack_bf16x2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
+                }
+                if (D != nullptr) {
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) store_rows_coalesced(ebuf, hb[h2], lane, D, ldd, m - lane, M, n_base + h2 * 64, N);
+                }
+                // amax over the finite values of the block's columns below N (N % 16 == 0)
+                const int nvalid = N - n_base;
+                uint32_t m2 = 0;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) m2 = amax_fast_word(m2, (h * 64 + 2 * j < nvalid) ? hb[h][j] : 0u);
+                uint32_t mx16 = amax_fast_final(m2);
+                const bool nonfin = mx16 == 0xFFFFFFFFu;
+                if (nonfin) {
+                    uint32_t bad = 0;
+                    mx16 = 0;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (h * 64 + 2 * j < nvalid) mx16 = amax_exact_word(mx16, hb[h][j], bad);
+                }
+                const float amax = bf16bits_to_float(mx16);
+                const float sc = pow2_scale_from_amax(amax, fm);
+                const bool row_ok = m < M;
+                const int64_t rt = ((int64_t)M + 127) / 128;
+                if (nvalid > 0 && m < rt * 128)   // rows past M in the last 128-row group: factor 1
+                    qsf[e8m0_offset(n_base / 128, rt, m)] = row_ok ? e8m0_of_scale(sc) : (uint8_t)127;
+                if (counts != nullptr && row_ok && may_saturate(nonfin, amax, sc, fm)) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            if (h * 64 + 2 * j >= nvalid) continue;
+                            const uint32_t w = hb[h][j];
+                            nf_q += ((w & 0x7F80u) == 0x7F80u) + ((w & 0x7F800000u) == 0x7F800000u);
+                            sat_q += (fabsf(__fmul_rn(bf_lo(w), sc)) > fm) + (fabsf(__fmul_rn(bf_hi(w), sc)) > fm);
+                        }
+                }
+                uint32_t qw[32];   // 128 codes, four per word, column order
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t w0 = hb[j >> 4][2 * (j & 15)], w1 = hb[j >> 4][2 * (j & 15) + 1];
+                    const uint32_t c0 = cvt2<QFMT>(__fmul_rn(bf_lo(w0), sc), __fmul_rn(bf_hi(w0), sc));
+                    const uint32_t c1 = cvt2<QFMT>(__fmul_rn(bf_lo(w1), sc), __fmul_rn(bf_hi(w1), sc));
+                    qw[j] = c0 | (c1 << 16);
+                }
+                store_rows_coalesced(ebuf, qw, lane, qo, (int64_t)N, m - lane, (int64_t)M, n_base, N);
             }
+        }
+        if constexpr (QFMT >= 0) {
+            if (counts != nullptr) flush_counts(counts, nf_q, sat_q);
         }
     }
 
@@ -278,7 +348,9 @@ bool make_sf_map(CUtensorMap *map, const void *base, int64_t rows16, uint32_t bo
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Pairs of the E8M0 kernel that fit on the device at once (cached per device).
+// Pairs of the E8M0 kernel that fit on the device at once (cached per device
+// and variant).
+template <int QFMT>
 int mx_pair_capacity() {
     static int cache[64];
     static std::mutex mu;
@@ -286,7 +358,7 @@ int mx_pair_capacity() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     std::lock_guard<std::mutex> lk(mu);
     if (cache[dev] > 0) return cache[dev];
-    if (cudaFuncSetAttribute(k_gemm_mx_2sm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mx::SMEM) !=
+    if (cudaFuncSetAttribute(k_gemm_mx_2sm<QFMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mx::SMEM) !=
         cudaSuccess)
         return 0;
     cudaLaunchConfig_t cfg = {};
@@ -301,7 +373,7 @@ int mx_pair_capacity() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_mx_2sm, &cfg) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)k_gemm_mx_2sm<QFMT>, &cfg) != cudaSuccess) return 0;
     cache[dev] = n;
     return n;
 }
@@ -312,6 +384,37 @@ int mx_pair_capacity() {
 uint32_t make_idesc_mx(fp8_format fa, fp8_format fb, int mma_m, int mma_n) {
     return ((uint32_t)fa << 7) | ((uint32_t)fb << 10) | ((uint32_t)(mma_n >> 3) << 17) | (1u << 23) |
            ((uint32_t)(mma_m >> 4) << 24);
+}
+
+template <int QFMT>
+fp8_status launch_mx_q(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
+                       int64_t M, int64_t N, int64_t K, uint32_t idesc, void *D_bf16, int64_t ldd, uint8_t *qo,
+                       uint8_t *qsf, uint32_t *counts, cudaStream_t s) {
+    const int cap = mx_pair_capacity<QFMT>();
+    if (cap <= 0) return FP8_ERR_CUDA;
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
+    return pdl_launch(k_gemm_mx_2sm<QFMT>, dim3(2 * pairs), dim3(sm2::THREADS), mx::SMEM, s, ta, tb, tsa, tsb,
+                      (int)M, (int)N, (int)K, idesc, static_cast<__nv_bfloat16 *>(D_bf16), ldd, qo, qsf,
+                      counts) == cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_CUDA;
+}
+
+// Maps and launch; qo == NULL: bf16 output only.
+fp8_status launch_mx(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb, int64_t M, int64_t N,
+                     int64_t K, const uint8_t *a_sf, const uint8_t *b_sf, void *D_bf16, int64_t ldd, fp8_format fo,
+                     uint8_t *qo, uint8_t *qsf, uint32_t *counts, cudaStream_t s) {
+    const int64_t ng = (K + 4 * BK - 1) / (4 * BK);   // groups of four K blocks in the images
+    CUtensorMap ta, tb, tsa, tsb;
+    if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
+    if (!make_sf_map(&tsa, a_sf, ng * ((M + 127) / 128) * 32, 32) ||
+        !make_sf_map(&tsb, b_sf, ng * ((N + 127) / 128) * 32, 64))
+        return FP8_ERR_CUDA;
+    const uint32_t idesc = make_idesc_mx(fa, fb, 256, 256);
+    if (qo == nullptr) return launch_mx_q<-1>(ta, tb, tsa, tsb, M, N, K, idesc, D_bf16, ldd, nullptr, nullptr, nullptr, s);
+    if (fo == FP8_E4M3) return launch_mx_q<FP8_E4M3>(ta, tb, tsa, tsb, M, N, K, idesc, D_bf16, ldd, qo, qsf, counts, s);
+    return launch_mx_q<FP8_E5M2>(ta, tb, tsa, tsb, M, N, K, idesc, D_bf16, ldd, qo, qsf, counts, s);
 }
 
 }  // namespace
@@ -342,20 +445,46 @@ extern "C" fp8_status fp8_gemm_block_e8m0(const uint8_t *A, fp8_format fa, const
     if (K == 0)
         return cudaMemset2DAsync(D_bf16, (size_t)ldd * 2, 0, (size_t)N * 2, (size_t)M, s) == cudaSuccess ? FP8_OK
                                                                                                        : FP8_ERR_CUDA;
-    CUtensorMap ta, tb, tsa, tsb;
-    if (!make_map(&ta, A, K, M, 128) || !make_map(&tb, B, K, N, 128)) return FP8_ERR_CUDA;
-    if (!make_sf_map(&tsa, a_sf, ng * ((M + 127) / 128) * 32, 32) ||
-        !make_sf_map(&tsb, b_sf, ng * ((N + 127) / 128) * 32, 64))
-        return FP8_ERR_CUDA;
-    const int cap = mx_pair_capacity();
-    if (cap <= 0) return FP8_ERR_CUDA;
-    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, cap));
-    return pdl_launch(k_gemm_mx_2sm, dim3(2 * pairs), dim3(sm2::THREADS), mx::SMEM, s, ta, tb, tsa, tsb, (int)M,
-                      (int)N, (int)K, make_idesc_mx(fa, fb, 256, 256), static_cast<__nv_bfloat16 *>(D_bf16), ldd) ==
-                   cudaSuccess
-               ? FP8_OK
-               : FP8_ERR_CUDA;
+    return launch_mx(A, fa, B, fb, M, N, K, a_sf, b_sf, D_bf16, ldd, FP8_E4M3, nullptr, nullptr, nullptr, s);
+}
+
+// The E8M0 GEMM with its output requantized 1 x 128 (power-of-two scales)
+// in the epilogue; see include/fp8q.h.
+extern "C" fp8_status fp8_gemm_block_e8m0_requant(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
+                                                  int64_t M, int64_t N, int64_t K, const uint8_t *a_sf,
+                                                  const uint8_t *b_sf, void *D_bf16, int64_t ldd, fp8_format fo,
+                                                  uint8_t *q, uint8_t *q_sf, uint32_t *counts, void *stream) {
+    if ((fa != FP8_E4M3 && fa != FP8_E5M2) || (fb != FP8_E4M3 && fb != FP8_E5M2)) return FP8_ERR_INVALID_ARG;
+    if (fo != FP8_E4M3 && fo != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0) return FP8_ERR_SHAPE;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP8_ERR_SHAPE;
+    if (K % 16 || N % 16) return FP8_ERR_SHAPE;
+    if (D_bf16 && ldd < N) return FP8_ERR_SHAPE;
+    if (D_bf16 && (ldd % 8 || !aligned16(D_bf16))) return FP8_ERR_ALIGNMENT;
+    const int64_t ng = (K + 4 * BK - 1) / (4 * BK);
+    if (ng * ((M + 127) / 128) * 32 >= (1ll << 31) || ng * ((N + 127) / 128) * 32 >= (1ll << 31)) return FP8_ERR_SHAPE;
+    if (M > 0 && N > 0) {
+        if (!q || !q_sf) return FP8_ERR_INVALID_ARG;
+        if (K > 0 && (!A || !B || !a_sf || !b_sf)) return FP8_ERR_INVALID_ARG;
+    }
+    if ((q && !aligned16(q)) || (A && !aligned16(A)) || (B && !aligned16(B)) || (a_sf && !aligned16(a_sf)) ||
+        (b_sf && !aligned16(b_sf)))
+        return FP8_ERR_ALIGNMENT;
+    if (counts && (reinterpret_cast<uintptr_t>(counts) & 3u)) return FP8_ERR_ALIGNMENT;
+    int sms;
+    fp8_status st = check_device(&sms);
+    if (st != FP8_OK) return st;
+    if (M == 0 || N == 0) return FP8_OK;
+    cudaStream_t s = as_stream(stream);
+    if (K == 0) {   // D = 0: codes 0, every block's factor 1 (e = 127)
+        const size_t img = (size_t)((N + 511) / 512) * (size_t)((M + 127) / 128) * 512;
+        if (D_bf16 && cudaMemset2DAsync(D_bf16, (size_t)ldd * 2, 0, (size_t)N * 2, (size_t)M, s) != cudaSuccess)
+            return FP8_ERR_CUDA;
+        if (cudaMemsetAsync(q, 0, (size_t)M * N, s) != cudaSuccess || cudaMemsetAsync(q_sf, 127, img, s) != cudaSuccess)
+            return FP8_ERR_CUDA;
+        return FP8_OK;
+    }
+    return launch_mx(A, fa, B, fb, M, N, K, a_sf, b_sf, D_bf16, ldd, fo, q, q_sf, counts, s);
 }
 
 // This file's device error word (read and optionally cleared by

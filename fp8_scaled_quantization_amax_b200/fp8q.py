@@ -49,6 +49,7 @@ SIGNATURES = {
     "fp8_quantize_rowwise_transpose": (_S, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P]),
     "fp8_gemm_bf16_wgrad": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _I, _P]),
     "fp8_gemm_block_e8m0": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _P, _P, _P, _I64, _P]),
+    "fp8_gemm_block_e8m0_requant": (_S, [_P, _I, _P, _I, _I64, _I64, _I64, _P, _P, _P, _I64, _I, _P, _P, _P, _P]),
     "fp8_paged_kv_write": (_S, [_P, _P, _I64, _I64, _I64, _I64, _I, _P, _P, _P]),
     "fp8_paged_kv_gather": (_S, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P]),
     "fp8_scale_stats": (_S, [_P, _P, _I64, _P, _I64, _F, _P, _P, _P]),
@@ -301,6 +302,27 @@ def quantize_blockwise_e8m0(x, fmt, block_rows, counts=None):
     img = torch.empty(e8m0_image_bytes(rows, cols), dtype=torch.uint8, device=x.device)
     fp8_quantize_blockwise_e8m0(x, rows, cols, x.stride(0), fmt, block_rows, q, img, counts)
     return q, img
+
+
+def fp8_gemm_block_e8m0_requant(A, fa, B, fb, M, N, K, a_sf, b_sf, D, ldd, fo, q, q_sf, counts=None, stream=None):
+    _dev(A, torch.uint8, "A"); _dev(B, torch.uint8, "B"); _dev(D, torch.bfloat16, "D")
+    _dev(a_sf, torch.uint8, "a_sf"); _dev(b_sf, torch.uint8, "b_sf")
+    _dev(q, torch.uint8, "q"); _dev(q_sf, torch.uint8, "q_sf"); _dev(counts, torch.int32, "counts")
+    _check("fp8_gemm_block_e8m0_requant", lib().fp8_gemm_block_e8m0_requant(
+        _ptr(A), fa, _ptr(B), fb, M, N, K, _ptr(a_sf), _ptr(b_sf), _ptr(D), ldd, fo, _ptr(q), _ptr(q_sf),
+        _ptr(counts), _stream(stream)))
+
+
+def gemm_block_e8m0_requant(A, fa, B, fb, a_sf, b_sf, fo, store_d=False, counts=None):
+    """(q [M, N], q_sf E8M0 image, D or None): the E8M0 GEMM's output requantized 1 x 128 with
+    power-of-two scales, as quantize_blockwise_e8m0(D, fo, 1) would."""
+    M, K = A.shape
+    N = B.shape[0]
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if store_d else None
+    q = torch.empty((M, N), dtype=torch.uint8, device=A.device)
+    q_sf = torch.empty(e8m0_image_bytes(M, N), dtype=torch.uint8, device=A.device)
+    fp8_gemm_block_e8m0_requant(A, fa, B, fb, M, N, K, a_sf, b_sf, D, N, fo, q, q_sf, counts)
+    return q, q_sf, D
 
 
 def gemm_block_e8m0(A, fa, B, fb, a_sf, b_sf, out=None):

@@ -326,6 +326,28 @@ FP8Q_API fp8_status fp8_gemm_block_e8m0(const uint8_t *A, fp8_format fa, const u
                                void *D_bf16, int64_t ldd, void *stream);
 
 /*
+ * fp8_gemm_block_e8m0 whose output is requantized for the next GEMM with
+ * 1 x 128 blocks and power-of-two scales ([DeepL] §2.3 per-block scales;
+ * [Soup]'s power-of-two scales): q and q_sf equal
+ * fp8_quantize_blockwise_e8m0(D, block_rows = 1, fo) on D = bf16(GEMM),
+ * code for code and byte for byte (rows past M in the last 128-row group:
+ * e = 127; bytes of K blocks past the last one are not written).
+ *   A, fa, B, fb, M, N, K, a_sf, b_sf: as fp8_gemm_block_e8m0.
+ *   D_bf16 [M, N] bf16 (leading dimension ldd) or NULL: the GEMM output.
+ *   q [M, N] FP8 (fo), dense, 16-byte aligned; q_sf the E8M0 image of q
+ *   (fp8_quantize_blockwise_e8m0's layout and size for M x N), 16-byte
+ *   aligned; counts [2] or NULL as the quantizers count.
+ *   One launch: the epilogue rounds each output to bf16 and quantizes its
+ *   row's 128-column block in registers.  K == 0: D = 0, codes 0, e = 127.
+ *   Shapes: as fp8_gemm_block_e8m0, and N % 16 == 0.  Errors as
+ *   fp8_gemm_block_e8m0; FP8_ERR_INVALID_ARG for a NULL q or q_sf.
+ */
+FP8Q_API fp8_status fp8_gemm_block_e8m0_requant(const uint8_t *A, fp8_format fa, const uint8_t *B, fp8_format fb,
+                                       int64_t M, int64_t N, int64_t K, const uint8_t *a_sf,
+                                       const uint8_t *b_sf, void *D_bf16, int64_t ldd, fp8_format fo,
+                                       uint8_t *q, uint8_t *q_sf, uint32_t *counts, void *stream);
+
+/*
  * Grouped FP8 GEMM for mixture-of-experts layers ("DeepL押注FP8：…" §3.2: the
  * tokens routed to each expert form a group, and one grouped GEMM multiplies
  * every group by its own expert weight):

@@ -117,3 +117,31 @@ def test_requant_needs_d_where_it_does_not_fuse():
     qs = torch.empty((2, M), dtype=torch.float32, device="cuda")
     with pytest.raises(fp8q.Fp8Error):
         fp8q.fp8_gemm_block_requant(_cuda(A), 0, _cuda(B), 0, M, N, K, _cuda(da), _cuda(db), None, N, 0, q, qs)
+
+
+@pytest.mark.parametrize("fo", [0, 1])
+@pytest.mark.parametrize("shape", [(300, 272, 400), (520, 784, 640), (64, 272, 256), (1024, 1040, 896)])
+def test_e8m0_requant_equals_the_oracle_chain(orc, fo, shape):
+    """The E8M0 GEMM (power-of-two block scales in the MMA) with its output
+    requantized 1x128 with power-of-two scales into the next GEMM's E8M0
+    image, against the oracle's exact GEMM -> bf16 -> power-of-two 1x128
+    quantizer: codes, every image byte the quantizer defines (rows past M in
+    the last 128-row group hold e = 127), counts and the bf16 output."""
+    from tests.test_gpu_block_e8m0 import _image, _written
+    M, N, K = shape
+    va, A, da, vb, B, db = _operands(M, N, K, 2, seed=M + 7 * N + K + fo)
+    img_a, img_b = _image(da, M, K, 1), _image(db, N, K, 128)
+    SA, SB = _scale_maps(2, M, N, K, da, db)
+    ref = _exact_bf16(va, vb, SA, SB)
+    rq, rs, rc = orc.quantize_blockwise(_bits(ref), fo, 1, pow2=True, counts=True)
+    want, mask = _image(rs, M, N, 1), _written(M, N)
+    for store_d in (True, False):
+        c = torch.zeros(2, dtype=torch.int32, device="cuda")
+        q, qsf, D = fp8q.gemm_block_e8m0_requant(_cuda(A), 0, _cuda(B), 0, _cuda(img_a), _cuda(img_b), fo,
+                                                 store_d=store_d, counts=c)
+        if store_d:
+            assert torch.equal(D.cpu(), ref)
+        assert_codes_equal(to_np(q), rq, fo)
+        got = to_np(qsf)
+        assert np.array_equal(got[mask], want[mask]), f"{int((got[mask] != want[mask]).sum())} image bytes differ"
+        assert (int(c[0]), int(c[1])) == rc
