@@ -148,3 +148,39 @@ def test_gemm_e8m0_mlp_down_sampled(orc):
     ref, mag = orc.gemm_scaled_sampled(A, 0, B, 0, orc.SCALE_BLOCK, da, db, im, inn)
     got = bf16_to_f64(D[_cuda(im), _cuda(inn)])
     assert_gemm_close(got, ref, mag, "e8m0 mlp down sampled")
+
+
+def test_e8m0_accuracy_against_fp32_block_scales(orc):
+    """What power-of-two block scales cost in accuracy on the block MLP's up
+    projection ([8192, 4096] x W_up[11008, 4096]^T): both recipes' GPU
+    outputs on 64 sampled rows x every column, against the unquantized
+    product of the same bf16 inputs (fp64).  Power-of-two factors are up to
+    2x coarser than fp32 block scales (the codes use as little as half the
+    range below fmax, so values near the underflow end lose bits), but FP8's
+    relative precision does not depend on the scale elsewhere, so the two
+    errors must stay within a factor of two of each other.  FP8_ACCURACY_LOG, when set,
+    names a file that receives the two relative errors."""
+    import json
+    import os
+    M, N, K = 8192, 11008, 4096
+    x = inputs.bf16_bits(inputs.normal_bf16((M, K), 1.0, seed=5, device="cuda"))
+    w = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, seed=6, device="cuda"))
+    rows = np.sort(np.random.default_rng(3).choice(M, 64, replace=False))
+    truth = bf16_to_f64(inputs.from_bf16_bits(x[rows])) @ bf16_to_f64(inputs.from_bf16_bits(w)).T
+    err = {}
+    for name, pow2 in (("fp32 block scales", False), ("E8M0 block scales", True)):
+        A, da = orc.quantize_blockwise(x, 0, 1, pow2=pow2)
+        B, db = orc.quantize_blockwise(w, 0, 128, pow2=pow2)
+        if pow2:
+            D = fp8q.gemm_block_e8m0(_cuda(A), 0, _cuda(B), 0, _cuda(_image(da, M, K, 1)),
+                                     _cuda(_image(db, N, K, 128)))
+        else:
+            D = fp8q.gemm(_cuda(A), 0, _cuda(B), 0, 2, _cuda(da), _cuda(db))
+        got = bf16_to_f64(D[_cuda(rows)])
+        err[name] = float(np.linalg.norm(got - truth) / np.linalg.norm(truth))
+    e32, e8 = err["fp32 block scales"], err["E8M0 block scales"]
+    if os.environ.get("FP8_ACCURACY_LOG"):
+        with open(os.environ["FP8_ACCURACY_LOG"], "a") as f:
+            f.write(json.dumps({"shape": [M, N, K], "rows": 64, "relative_rms_error": err}) + "\n")
+    assert 0 < e32 < 0.1, err          # E4M3 keeps ~3 significand bits: a few % of the output norm
+    assert 0.5 * e32 <= e8 <= 2.0 * e32, err   # relative FP8 precision does not depend on the scale, except near underflow
