@@ -649,8 +649,9 @@ static cudaError_t launch_qt_strip(cudaStream_t s, const uint16_t *x, uint8_t *q
                                    int64_t ld, float *scale_inv, float *amax_out, uint32_t *counts) {
     const int active = qt_active_clusters<FMT, POW2>();
     if (active <= 0) return cudaErrorInvalidConfiguration;
-    // strips in flight (rows x 128 bytes each) within 64 MiB of L2, so pass 2 finds them there
-    const int64_t fit = std::max<int64_t>(1, ((int64_t)64 << 20) / std::max<int64_t>(1, rows * 128));
+    // strips in flight (rows x 128 bytes each) within 96 MiB of the 126 MB L2, so pass 2 finds them
+    // there (measured: 64 MiB starved long columns of clusters, 112 MiB gained nothing more)
+    const int64_t fit = std::max<int64_t>(1, ((int64_t)96 << 20) / std::max<int64_t>(1, rows * 128));
     const int64_t nstrips = (cols + 63) / 64;
     const int64_t ncl = std::min<int64_t>(std::min<int64_t>(nstrips, active), fit);
     k_qt_strip<FMT, POW2><<<(unsigned)(ncl * kQtCtas), kQtThreads, 0, s>>>(x, qt, rows, cols, ld, scale_inv, amax_out,
