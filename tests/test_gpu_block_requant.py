@@ -41,7 +41,8 @@ def _requant(A, B, da, db, fo, store_d):
 
 
 @pytest.mark.parametrize("fo", [0, 1])
-@pytest.mark.parametrize("shape", [(300, 272, 400), (520, 784, 640), (1024, 1040, 896), (64, 272, 256)])
+@pytest.mark.parametrize("shape", [(300, 272, 400), (520, 784, 640), (1024, 1040, 896), (64, 272, 256),
+                                   (129, 272, 144), (300, 272, 48)])
 def test_requant_equals_the_oracle_chain(orc, fo, shape):
     """Fused GEMM + 1x128 requantization against the oracle's exact GEMM
     rounded to bf16 and quantized by the oracle: codes, scales, counts and
@@ -120,7 +121,8 @@ def test_requant_needs_d_where_it_does_not_fuse():
 
 
 @pytest.mark.parametrize("fo", [0, 1])
-@pytest.mark.parametrize("shape", [(300, 272, 400), (520, 784, 640), (64, 272, 256), (1024, 1040, 896)])
+@pytest.mark.parametrize("shape", [(300, 272, 400), (520, 784, 640), (64, 272, 256), (1024, 1040, 896),
+                                   (129, 272, 144)])
 def test_e8m0_requant_equals_the_oracle_chain(orc, fo, shape):
     """The E8M0 GEMM (power-of-two block scales in the MMA) with its output
     requantized 1x128 with power-of-two scales into the next GEMM's E8M0

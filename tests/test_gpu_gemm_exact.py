@@ -116,7 +116,7 @@ def _check(D, va, vb, SA, SB, rows=None, what=""):
 # --------------------------------------------------- tensor and row modes --
 
 @pytest.mark.parametrize("mode", [0, 1])
-@pytest.mark.parametrize("shape", [(4096, 4096, 4096), (300, 272, 400), (520, 776, 640)])
+@pytest.mark.parametrize("shape", [(4096, 4096, 4096), (300, 272, 400), (520, 776, 640), (129, 272, 144), (300, 272, 48)])
 def test_exact_pair_kernel(mode, shape):
     """CTA-pair kernel: 4096^3 runs 256 tiles over several waves of pairs."""
     M, N, K = shape
@@ -170,10 +170,13 @@ def test_exact_dgrad_e5m2_times_e4m3():
 
 # ------------------------------------------------------ block-scaled mode --
 
-@pytest.mark.parametrize("shape", [(300, 272, 400), (520, 776, 640), (4096, 4096, 4096), (640, 1024, 896)])
+@pytest.mark.parametrize("shape", [(300, 272, 400), (520, 776, 640), (4096, 4096, 4096), (640, 1024, 896),
+                                   (129, 272, 144), (300, 272, 48), (520, 784, 16)])
 def test_exact_block_scaled_pair_kernel(shape):
     """fp32 per-block scales (1x128 of A, 128x128 of B): each K block's
-    partial promoted by the epilogue; ragged M, N and K."""
+    partial promoted by the epilogue; ragged M, N and K, K below one block
+    (48, 16: a single partial K block) and M = 129 (the odd CTA of the pair
+    holds one row)."""
     M, N, K = shape
     va, A, da, vb, B, db = _operands(M, N, K, 2, seed=31 + M)
     A_, B_, da_, db_ = _cuda(A), _cuda(B), _cuda(da), _cuda(db)
