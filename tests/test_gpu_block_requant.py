@@ -147,3 +147,47 @@ def test_e8m0_requant_equals_the_oracle_chain(orc, fo, shape):
         got = to_np(qsf)
         assert np.array_equal(got[mask], want[mask]), f"{int((got[mask] != want[mask]).sum())} image bytes differ"
         assert (int(c[0]), int(c[1])) == rc
+
+
+def test_block_mlp_step_replays_in_a_cuda_graph():
+    """The block-scaled MLP step -- X quantized 1x128, W_up and W_down
+    128x128, the up GEMM requantizing H in its epilogue, the down GEMM --
+    captured once in a CUDA graph (its launches use programmatic dependent
+    launch and thread-block clusters) and replayed with new inputs copied
+    into the captured buffers: every replay equals the eager step on the same
+    inputs, bit for bit."""
+    from fp8_scaled_quantization_amax_b200 import inputs
+    M, Dm, F = 512, 1024, 2816
+    X_ = torch.empty((M, Dm), dtype=torch.bfloat16, device="cuda")
+    Wu_ = torch.empty((F, Dm), dtype=torch.bfloat16, device="cuda")
+    Wd_ = torch.empty((Dm, F), dtype=torch.bfloat16, device="cuda")
+
+    def step(X, Wu, Wd):
+        qx, sx = fp8q.quantize_blockwise(X, 0, 1)
+        qwu, swu = fp8q.quantize_blockwise(Wu, 0, 128)
+        qh, sh, _ = fp8q.gemm_block_requant(qx, 0, qwu, 0, sx, swu, 0)
+        qwd, swd = fp8q.quantize_blockwise(Wd, 0, 128)
+        return fp8q.gemm(qh, 0, qwd, 0, fp8q.SCALE_BLOCK, sh, swd)
+
+    sets = [(inputs.normal_bf16((M, Dm), 1.0, seed=40 + i, device="cuda"),
+             inputs.normal_bf16((F, Dm), 0.02, seed=50 + i, device="cuda"),
+             inputs.normal_bf16((Dm, F), 0.02, seed=60 + i, device="cuda")) for i in range(3)]
+    for t, v in zip((X_, Wu_, Wd_), sets[0]):
+        t.copy_(v)
+    step(X_, Wu_, Wd_)   # warm-up outside the capture (per-device set-up of every kernel)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            Y_ = step(X_, Wu_, Wd_)
+    torch.cuda.current_stream().wait_stream(s)
+    for rep in range(6):
+        X, Wu, Wd = sets[rep % 3]
+        X_.copy_(X); Wu_.copy_(Wu); Wd_.copy_(Wd)
+        g.replay()
+        torch.cuda.synchronize()
+        ref = step(X, Wu, Wd)
+        torch.cuda.synchronize()
+        assert torch.equal(Y_, ref), rep
