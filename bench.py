@@ -24,6 +24,8 @@ bracketed by a barrier and a device synchronize; each step's kernels are
 timed with CUDA events on the launching stream, L2 is flushed (a 256 MiB write
 and a 256 MiB read)
 before every step outside the events; multi-GPU takes the max over ranks.
+Besides the mean the line carries the median and best per-step and
+dominant-kernel times (rank 0's).
 ``--impl reference`` times the CPU oracle (the only reference this project
 has) on a bounded sample of the same workload, on every host thread this
 process may use; the GPU line's ``cpu_baseline`` gives that figure and the
@@ -854,6 +856,9 @@ def main():
     ms_per_step = total_ms / steps
     value = world * wl.work() * steps / (total_ms * 1e-3)
     kern_avg_ms = max_over_ranks(statistics.mean(kern_ms))
+    # spread of the per-step device times (this rank's; the value above uses their sum)
+    step_med_ms, step_best_ms = statistics.median(step_ms), min(step_ms)
+    kern_med_ms, kern_best_ms = statistics.median(kern_ms), min(kern_ms)
 
     if args.profile:
         assert fp8q.fp8_device_error(clear=True) == 0, "a kernel gave up a bounded wait"
@@ -959,7 +964,8 @@ def main():
     cfg["l2"] = "flushed before every step (256 MiB write + 256 MiB read, outside the step's events)"
     line = {
         "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": world, "steps": steps, "warmup": warmup,
-        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": ms_per_step, "ms_per_step_median": step_med_ms, "ms_per_step_best": step_best_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": dtype, "data": "synthetic (seeded, per rank)", "config": cfg,
         "roofline": {"bound": wl.bound, "achieved": achieved, "peak": peak, "unit": wl.unit,
                      "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
@@ -969,7 +975,8 @@ def main():
                                 "blockmlp_e8m0": "fp8_gemm_block_e8m0_requant (up projection with its 1x128 requantization)",
                                 "blockmlp": "fp8_gemm_block_requant (up projection with its 1x128 requantization)"
                                 }.get(args.workload, "fp8_gemm_scaled"),
-                     "kernel_ms": kern_avg_ms, "peak_source": peak_src},
+                     "kernel_ms": kern_avg_ms, "kernel_ms_median": kern_med_ms, "kernel_ms_best": kern_best_ms,
+                     "peak_source": peak_src},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "steps": e2e_steps,
