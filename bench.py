@@ -64,6 +64,29 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, None, "fallback"
 
 
+def choose_peak(bound: str, peak_dtype: str, clocks: dict, pk) -> tuple:
+    """(peak, description) for the roofline of the dominant kernel.  pk is
+    peaks().  Tensor-bound kernels: the sustained (power-capped) figure when
+    the timed region ran under the power cap with the SM clock pulled down
+    (median below 90 % of max; the sustained figure was measured near
+    1.3 GHz), the burst figure otherwise; FP8 peaks are the bf16 figure times
+    the nominal dense ratio 2.  Memory-bound kernels: the HBM copy rate."""
+    hbm, bf16, bf16_sus, src = pk
+    if bound != "tensor":
+        return hbm, f"{src} HBM copy bandwidth {hbm} GB/s"
+    mhz, mhz_max = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    pulled_down = mhz is None or not mhz_max or mhz < 0.9 * mhz_max
+    capped = "sw_power_cap" in clocks.get("reasons", []) and pulled_down and bf16_sus is not None
+    base = bf16_sus if capped else bf16
+    kind = 'sustained' if capped else 'burst'
+    note = '; sw_power_cap was active in the timed region' if capped else ''
+    if peak_dtype == "bf16":
+        return base, (f"bf16 dense peak = {src} cuBLAS bf16 {kind} {base} TFLOP/s (MEASURED_PEAKS.json){note}"
+                      if src == "measured" else f"fallback bf16 {bf16}")
+    return base * FP8_OVER_BF16, (f"FP8 dense peak = {src} bf16 {kind} {base} TFLOP/s x nominal fp8/bf16 ratio 2 "
+                                  f"(MEASURED_PEAKS.json){note}" if src == "measured" else f"fallback bf16 {bf16} x 2")
+
+
 def recorded_traffic(workload: str):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary (profiles/roofline_traffic.json), or None when there is none or
@@ -918,30 +941,8 @@ def main():
     e2e_value = world * wl.work() / (e2e_ms * 1e-3)
     assert fp8q.fp8_device_error(clear=True) == 0, "a kernel gave up a bounded wait"
 
-    hbm, bf16, bf16_sus, src = peaks()
     clocks = clk.summary()
-    if wl.bound == "tensor":
-        # the sustained (power-capped) figure when the timed region ran under
-        # the power cap with the SM clock pulled down (median below 90 % of
-        # max; the sustained figure was measured near 1.3 GHz), the burst
-        # figure otherwise
-        mhz, mhz_max = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
-        pulled_down = mhz is None or not mhz_max or mhz < 0.9 * mhz_max
-        capped = "sw_power_cap" in clocks.get("reasons", []) and pulled_down and bf16_sus is not None
-        base = bf16_sus if capped else bf16
-        kind = 'sustained' if capped else 'burst'
-        note = '; sw_power_cap was active in the timed region' if capped else ''
-        if getattr(wl, "peak_dtype", "fp8") == "bf16":
-            peak = base
-            peak_src = (f"bf16 dense peak = {src} cuBLAS bf16 {kind} {base} TFLOP/s (MEASURED_PEAKS.json){note}"
-                        if src == "measured" else f"fallback bf16 {bf16}")
-        else:
-            peak = base * FP8_OVER_BF16
-            peak_src = (f"FP8 dense peak = {src} bf16 {kind} {base} TFLOP/s x nominal fp8/bf16 ratio 2 "
-                        f"(MEASURED_PEAKS.json){note}" if src == "measured" else f"fallback bf16 {bf16} x 2")
-    else:
-        peak = hbm
-        peak_src = f"{src} HBM copy bandwidth {hbm} GB/s"
+    peak, peak_src = choose_peak(wl.bound, getattr(wl, "peak_dtype", "fp8"), clocks, peaks())
     achieved = wl.kernel_work() / (kern_avg_ms * 1e-3)
 
     if rank != 0:

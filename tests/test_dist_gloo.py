@@ -44,7 +44,7 @@ def _worker(rank, world, port, results):
 
 def test_global_amax_scale_shared_by_all_ranks():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()   # no fork of a process that may hold threads
     results = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), results), nprocs=world, join=True)
     r0, r1 = results[0], results[1]
