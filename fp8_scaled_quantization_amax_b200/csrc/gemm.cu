@@ -476,12 +476,17 @@ k_gemm_fp8_2sm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
             return Item{pair + i * npairs, 0, nk, -1, t % mt, t / mt, e, r0, r1};
         } else {
-            if (i < n_full) {
-                const int t = pair + i * npairs;
+            // the first K half of a split tile runs before this pair's whole
+            // tiles and the second half after them, so the second half finds
+            // the first one's partial already published
+            const int h = pair & 1, kh = nk / 2, ts = full_tiles + pair / 2;
+            const bool first_half_first = pair < split_units && h == 0;
+            const int j = first_half_first ? i - 1 : i;
+            if (j >= 0 && j < n_full) {
+                const int t = pair + j * npairs;
                 return Item{t, 0, nk, -1, t % num_m, t / num_m, 0, 0, (int64_t)M};
             }
-            const int h = pair & 1, kh = nk / 2, t = full_tiles + pair / 2;
-            return Item{t, h ? kh : 0, h ? nk : kh, h, t % num_m, t / num_m, 0, 0, (int64_t)M};
+            return Item{ts, h ? kh : 0, h ? nk : kh, h, ts % num_m, ts / num_m, 0, 0, (int64_t)M};
         }
     };
 
@@ -830,13 +835,14 @@ int pair_capacity() {
     return n;
 }
 
-// Split-K plan for a grid of `cap` CTA pairs.  When all tiles fit in half
-// the pairs, each tile is computed as two K halves on two pairs (twice the
-// tensor cores on the problem).  The kernel also supports splitting only the
-// last wave of a multi-wave grid (full_tiles > 0), but measured at 4096^3 the
-// half-empty last wave already runs uncontended and faster than a full one,
-// so the fp32 hand-off did not pay (63.5 vs 61.4 us): the plan splits only
-// single-wave problems.
+// Split-K plan for a grid of `cap` CTA pairs.  The r tiles of the last wave
+// (all tiles, when they fit in half the pairs) are computed as two K halves
+// on two pairs, the first half handing its fp32 partial to the second
+// through the workspace.  With several waves the first halves run first and
+// the second halves last, so no pair waits for a partial; measured on
+// 4096 x 4096 tiles (L2 flushed, us): K = 8192 103.2 unsplit, 97.2 split;
+// K = 4096 59.4 either way (the half-empty last wave already runs faster
+// than a full one; with the halves run side by side it was 63.5).
 // The fp32 hand-off through global memory costs several microseconds, so a
 // pair split pays only for long K: measured on 16 tiles of 256 x 256, K =
 // 4096 (32 K blocks) ran 22.5 us unsplit and 24.6 split, K = 16384 53.2 and
@@ -847,8 +853,11 @@ struct SplitPlan { int full_tiles, units; size_t bytes; };
 SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int cap) {
     const int tiles = (int)(((M + 255) / 256) * ((N + 255) / 256));
     const int nk = (int)((K + BK - 1) / BK);
-    const int r = tiles % cap;
-    if (cap <= 0 || nk < kPairSplitMinKBlocks || r == 0 || tiles >= cap || 2 * r > cap) return SplitPlan{tiles, 0, 0};
+    const int r = cap > 0 ? tiles % cap : 0;
+    // r tiles in the last wave, split in K halves over 2r <= cap pairs; with
+    // several waves the first halves run before each pair's whole tiles and
+    // the second halves after them
+    if (cap <= 0 || r == 0 || 2 * r > cap || nk < kPairSplitMinKBlocks) return SplitPlan{tiles, 0, 0};
     const size_t flags_off = (size_t)r * 2 * sm2::kSplitPartialFloats * sizeof(float);
     return SplitPlan{tiles - r, 2 * r, flags_off + (((size_t)r * 2 * sizeof(uint32_t) + 255) & ~(size_t)255)};
 }

@@ -231,7 +231,10 @@ FP8Q_API fp8_status fp8_quantize_blockwise_e8m0(const void *x_bf16, int64_t rows
  *       of the GPU's CTA pairs, and that the cluster split below does not
  *       take, has each tile computed as two K halves on two CTA pairs, the
  *       first half handing its fp32 partial to the second through the
- *       workspace (TENSOR and ROW modes, M > 128).  The
+ *       workspace (TENSOR and ROW modes, M > 128); with several waves of
+ *       tiles whose last wave is at most half full, that wave's tiles are
+ *       split the same way (their first halves run first, their second
+ *       halves last).  The
  *       workspace must be zero-filled when first allocated; every call
  *       leaves it as it found it (its hand-off flags cleared), so the call
  *       may also be captured in a CUDA graph and replayed.  Calls that share

@@ -127,12 +127,14 @@ def test_exact_pair_kernel(mode, shape):
 
 
 @pytest.mark.parametrize("mode", [0, 1])
-@pytest.mark.parametrize("shape", [(1000, 1288, 8208), (1024, 1536, 16384)])
+@pytest.mark.parametrize("shape", [(1000, 1288, 8208), (1024, 1536, 16384), (4096, 4096, 8192)])
 def test_exact_pair_split_with_workspace(mode, shape):
     """Long K, few 256 x 256 tiles: each tile's K halves run on two pairs and
     the first hands its fp32 partial to the second through the workspace
-    (ragged K included: 8208 = 64 blocks + 16).  Repeated calls reuse the
-    workspace and must give the same exact result."""
+    (ragged K included: 8208 = 64 blocks + 16); 4096 x 4096 x 8192: only the
+    last wave's tiles are split (their first halves run first, their second halves
+    last).  Repeated calls reuse the workspace and must give the same exact
+    result."""
     M, N, K = shape
     va, A, da, vb, B, db = _operands(M, N, K, mode, seed=7 + mode, vmax=8)
     ws = fp8q.gemm_workspace(M, N, K, mode)

@@ -43,9 +43,11 @@ def _noalloc_via_c_abi(A, fa, B, fb, mode, da, db, D):
     assert st == 0, L.fp8_status_string(st)
 
 
-# (shape, uses the scratch): the pair split (few 256 x 256 tiles, K >= 64
-# blocks) needs it; multi-wave and cluster-split shapes do not.
-_SHAPES = [((1000, 1288, 8208), True), ((1024, 1536, 16384), True), ((4096, 4096, 4096), False),
+# (shape, uses the scratch): the pair split (K >= 64 blocks, with few 256 x
+# 256 tiles or a last wave of tiles at most half full) needs it; shorter K,
+# cluster-split shapes and grids of whole waves do not.
+_SHAPES = [((1000, 1288, 8208), True), ((1024, 1536, 16384), True), ((4096, 4096, 8192), True),
+           ((4096, 4096, 4096), False),
            ((1024, 1024, 16384), False), ((300, 272, 400), False)]
 
 
