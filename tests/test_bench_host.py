@@ -77,6 +77,9 @@ def test_every_workload_has_a_config():
         assert bench.config_of(w)["workload"]
 
 
-def test_cpu_sample_of_the_small_workload():
-    v, desc = bench.cpu_sample("tensor")
+@pytest.mark.parametrize("workload", list(bench.DEFAULT_STEPS))
+def test_cpu_sample_of_every_workload(workload):
+    """The oracle sample behind the reference arm and the GPU line's
+    cpu_baseline runs for every workload (one thread: a few seconds each)."""
+    v, desc = bench.cpu_sample(workload)
     assert v > 0 and desc
