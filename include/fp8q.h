@@ -5,6 +5,28 @@
  * delayed-scaling amax-history update and the FP8 KV-cache quantize /
  * dequantize.
  *
+ * Entry points, by step of the path
+ *   amax and quantizers   fp8_amax, fp8_quantize_tensorwise (current or
+ *                         delayed scale), fp8_quantize_rowwise (+ _pair for
+ *                         both GEMM operands in one launch),
+ *                         fp8_quantize_blockwise (1 x 128 / 128 x 128),
+ *                         fp8_quantize_blockwise_e8m0 (power-of-two block
+ *                         scales as the MMA's E8M0 image),
+ *                         fp8_quantize_rowwise_transpose (per-row codes of
+ *                         X^T for the bf16 weight-gradient recipe)
+ *   GEMMs                 fp8_gemm_scaled (tensor / row / block scales),
+ *                         fp8_gemm_block_e8m0, fp8_gemm_grouped (MoE groups),
+ *                         fp8_gemm_bf16_wgrad; fp8_gemm_block_requant and
+ *                         fp8_gemm_block_e8m0_requant quantize their own
+ *                         output 1 x 128 for the next GEMM in the epilogue;
+ *                         fp8_gemm_workspace_size / fp8_gemm_scaled_noalloc
+ *                         for the split-K scratch
+ *   delayed scaling       fp8_amax_history_update
+ *   KV cache              fp8_kv_quant / fp8_kv_dequant (per (b, h) slice),
+ *                         fp8_paged_kv_write / fp8_paged_kv_gather (pages)
+ *   health and errors     fp8_scale_stats, fp8_device_error,
+ *                         fp8_status_string
+ *
  * Sources (web pages on FP8 scaled quantization):
  *   [DeepL]  "DeepL押注FP8：大模型训练与推理统一精度实战解析"
  *   [H100]   "H100 FP8加速实测：新一代计算架构的飞跃"
@@ -15,7 +37,9 @@
  * Conventions shared by every entry point
  *   - Every pointer argument is DEVICE memory owned by the caller (allocate it
  *     with cudaMalloc, torch, ...).  The library allocates nothing on the
- *     device, keeps no per-call state and never synchronises the host.
+ *     device and never synchronises the host; its only device state is
+ *     static module memory: the sticky error words behind fp8_device_error
+ *     and the scratch array of fp8_gemm_scaled_noalloc.
  *   - bf16 tensors are raw 16-bit bfloat16 words; FP8 tensors are one byte per
  *     element (the format's code); scales are IEEE fp32.
  *   - "scale" s multiplies before the cast (q = cast(x * s)); "scale_inv"
