@@ -151,3 +151,19 @@ def test_header_compiles_as_plain_c_and_cpp(tmp_path, lang):
     r = subprocess.run([cc, *std, "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), "-c",
                         str(src), "-o", str(tmp_path / "use_header.o")], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_e8m0_image_size_and_layout_are_one_to_one():
+    """The E8M0 scale image that the GPU tests write for the block-scaled MMA
+    (tests/test_gpu_block_e8m0.py) and the binding's image size agree: every
+    (row, 128-column block) owns one byte of its own, the image holds nothing
+    else but the unused slots of a last group of fewer than four blocks, and
+    the exponent byte of a power-of-two factor 2^k is k + 127."""
+    from tests.test_gpu_block_e8m0 import _e8m0, _written
+    for rows, cols in [(1, 16), (128, 128), (300, 400), (257, 1040), (129, 2048), (8192, 11008)]:
+        nkb, rt = (cols + 127) // 128, (rows + 127) // 128
+        w = _written(rows, cols)
+        assert w.size == fp8q.e8m0_image_bytes(rows, cols)
+        assert int(w.sum()) == nkb * rt * 128          # no two (row, block) pairs share a byte
+        assert w.size - int(w.sum()) == (-nkb % 4) * rt * 128
+    assert list(_e8m0([1.0, 2.0, 0.5, 2.0 ** -126, 2.0 ** 127])) == [127, 128, 126, 1, 254]
